@@ -1,0 +1,239 @@
+"""CPU oracle for the fused short-convolution path -- TEST INFRASTRUCTURE ONLY.
+
+This package wraps ``sconv_oracle.c``: a plain, scalar, double-precision
+statement of what the path computes, written from the pages' definitions
+("vllm.models.inkling.nvidia.ops.sconv": module docstring, fused_sconv,
+sconv_seq_metadata; "core.ssm.ops.intermediate_extraction":
+scatter_intermediate_conv).  Only the tests, the smoke check and the
+benchmark's CPU-baseline leg may import it.  The CUDA library never calls it
+and shares no code with it; the product path fails loudly without its own
+extension instead of falling back here.
+
+Every function takes numpy arrays or CPU torch tensors.  bf16 data is passed
+as its raw 16-bit patterns (a torch bfloat16 tensor, or a numpy uint16 /
+int16 array together with ``dtype="bf16"``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sconv_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+# Plain build: no fast-math, no FMA contraction, so every double operation
+# rounds exactly once in source order.
+CFLAGS = ["-O2", "-std=c99", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math"]
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB) -> str:
+    """Compile the oracle C source into a shared library; returns its path."""
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        tmp = out + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *CFLAGS, "-o", tmp, src, "-lm"], check=True)
+        os.replace(tmp, out)
+    return out
+
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_INT = ctypes.c_int
+
+
+def _bind(path: str) -> ctypes.CDLL:
+    lib = ctypes.CDLL(path)
+    lib.oracle_fused.restype = _I64
+    lib.oracle_fused.argtypes = [
+        _INT, _P, _I64, _I64, _I64,            # dtype, x, x_row_stride, T, C
+        _P, _I64, _I64, _INT,                  # weight, w_stride_c, w_stride_k, W
+        _P, _P, _P, _I64, _I64, _I64, _I64,    # cache_in, cache_out, strides, nb, H, N, D
+        _P, _P, _P, _P,                        # positions, seq_idx, slot_mapping, query_start
+        _P, _I64, _I64, _I64,                  # block_table, bt_row_stride, num_reqs, max_blocks
+        _I64, _I64, _INT, _INT,                # off_s, ws, silu, residual
+        _I64, _I64, _P, _P,                    # t_begin, t_end, out_ref, row_state
+    ]
+    lib.oracle_seq_metadata.restype = None
+    lib.oracle_seq_metadata.argtypes = [_P, _I64, _I64, _I64, _P, _P]
+    lib.oracle_extract_windows.restype = None
+    lib.oracle_extract_windows.argtypes = [
+        _INT, _P, _I64, _I64, _I64, _I64, _P, _I64, _I64, _P, _I64, _I64]
+    lib.oracle_check_preconditions.restype = _INT
+    lib.oracle_check_preconditions.argtypes = [
+        _I64, _INT, _I64, _P, _P, _P, _P, _P, _I64, _I64]
+    return lib
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The oracle library.  SCONV_ORACLE_LIB names an alternative build
+    (the mutation tests point it at deliberately broken copies)."""
+    global _lib
+    if _lib is None:
+        alt = os.environ.get("SCONV_ORACLE_LIB")
+        _lib = _bind(alt if alt else build())
+    return _lib
+
+
+# --------------------------------------------------------------------------
+# array helpers
+
+def _np(a, dtype=None):
+    """Contiguous numpy view of a numpy array or CPU torch tensor."""
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            t = a.detach().cpu().contiguous()
+            if t.dtype == torch.bfloat16:
+                t = t.view(torch.int16)
+            a = t.numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    a = np.ascontiguousarray(a)
+    if dtype is not None:
+        if a.dtype != dtype:
+            raise TypeError(f"expected {dtype}, got {a.dtype}")
+    return a
+
+
+def _float_array(a, dtype: str):
+    """Raw element array for the oracle: float32 for 'f32', 16-bit for 'bf16'."""
+    arr = _np(a)
+    if dtype == "f32":
+        if arr.dtype != np.float32:
+            raise TypeError("f32 data must be float32")
+    elif dtype == "bf16":
+        if arr.dtype not in (np.int16, np.uint16):
+            raise TypeError("bf16 data must be passed as 16-bit patterns")
+        arr = arr.view(np.uint16)
+    else:
+        raise ValueError(dtype)
+    return arr
+
+
+def _ptr(a) -> int:
+    return a.ctypes.data if a is not None else 0
+
+
+_DT = {"f32": 0, "bf16": 1}
+
+
+def bf16_bits_to_f64(bits) -> np.ndarray:
+    """Exact decode of bf16 bit patterns to float64."""
+    b = _np(bits).view(np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def to_f64(a, dtype: str) -> np.ndarray:
+    arr = _float_array(a, dtype)
+    return arr.astype(np.float64) if dtype == "f32" else bf16_bits_to_f64(arr)
+
+
+# --------------------------------------------------------------------------
+# public oracle calls
+
+def fused(*, dtype, x, weight, cache, positions, block_table, seq_idx,
+          slot_mapping, query_start, off_s, ws, block_size, activation=None,
+          use_residual=True, t_range=None, write_cache=True):
+    """Oracle of fused_sconv ("vllm.models.inkling.nvidia.ops.sconv").
+
+    ``cache`` is [num_blocks, H, N, D] (any strides in elements, D stride 1
+    not required here).  Returns ``(out_ref, row_state, cache_out, skipped)``:
+    out_ref float64 [n, C] for the tokens in ``t_range`` (default all),
+    row_state uint8 [n] (1 computed, 0 PAD, 2 skipped), cache_out the cache
+    after the inserts (a new array) or None when ``write_cache`` is False.
+    """
+    xa = _float_array(x, dtype)
+    wa = _float_array(weight, dtype)
+    ca = _float_array(cache, dtype)
+    if xa.ndim != 2 or wa.ndim != 2 or ca.ndim != 4:
+        raise ValueError("x [T,C], weight [C,W], cache [nb,H,N,D] expected")
+    T, C = xa.shape
+    W = wa.shape[1]
+    nb, H, N, D = ca.shape
+    if N != block_size:
+        raise ValueError("cache.shape[2] must equal block_size")
+    pos = _np(positions, np.int64)
+    sid = _np(seq_idx, np.int32)
+    slot = _np(slot_mapping, np.int64)
+    qs = _np(query_start, np.int32)
+    bt = _np(block_table, np.int32)
+    t0, t1 = (0, T) if t_range is None else t_range
+    n = t1 - t0
+    out_ref = np.zeros((n, C), np.float64)
+    state = np.zeros(n, np.uint8)
+    cache_out = ca.copy() if write_cache else None
+    strides = np.array([s // ca.itemsize for s in ca.strides], np.int64)
+    skipped = lib().oracle_fused(
+        _DT[dtype], _ptr(xa), C, T, C, _ptr(wa), W, 1, W,
+        _ptr(ca), _ptr(cache_out), _ptr(strides), nb, H, N, D,
+        _ptr(pos), _ptr(sid), _ptr(slot), _ptr(qs),
+        _ptr(bt), bt.shape[1], bt.shape[0], bt.shape[1],
+        off_s, ws, int(activation in ("silu", "swish")), int(bool(use_residual)),
+        t0, t1, _ptr(out_ref), _ptr(state))
+    if skipped < 0:
+        raise ValueError("oracle_fused: malformed arguments")
+    return out_ref, state, cache_out, int(skipped)
+
+
+def update(*, dtype, x, weight, cache, positions, block_table, slot_mapping,
+           off_s, ws, block_size, activation=None, use_residual=True,
+           write_cache=True):
+    """Oracle of the single-token decode form (causal_conv1d_update in
+    "Implementation:Sgl project Sglang Mamba Ops"): token b is request b,
+    so the fused definition applies with seq_idx[b] = query_start[b] = b."""
+    B = _np(positions).shape[0]
+    ar = np.arange(B, dtype=np.int32)
+    return fused(dtype=dtype, x=x, weight=weight, cache=cache, positions=positions,
+                 block_table=block_table, seq_idx=ar, slot_mapping=slot_mapping,
+                 query_start=ar, off_s=off_s, ws=ws, block_size=block_size,
+                 activation=activation, use_residual=use_residual,
+                 write_cache=write_cache)
+
+
+def seq_metadata(query_start_loc, num_reqs, num_actual_tokens, num_padded_tokens=None):
+    """Oracle of sconv_seq_metadata; returns (seq_idx, query_start) int32."""
+    qsl = _np(query_start_loc, np.int32)
+    if num_padded_tokens is None:
+        num_padded_tokens = num_actual_tokens
+    si = np.zeros(num_padded_tokens, np.int32)
+    qs = np.zeros(num_padded_tokens, np.int32)
+    lib().oracle_seq_metadata(_ptr(qsl), num_reqs, num_actual_tokens,
+                              num_padded_tokens, _ptr(si), _ptr(qs))
+    return si, qs
+
+
+def extract_windows(*, dtype, src, abs_positions, real_count, out, d_conv):
+    """Oracle of scatter_intermediate_conv ("core.ssm.ops.intermediate_extraction").
+
+    ``src`` is [seq_len, conv_dim]; ``out`` [max_count, conv_dim, d_conv]
+    holds the prior bytes.  Returns a new array with the gathered windows.
+    """
+    sa = _float_array(src, dtype)
+    ap = _np(abs_positions, np.int32)
+    oa = _float_array(out, dtype).copy()
+    seq_len, conv_dim = sa.shape
+    max_count = oa.shape[0]
+    lib().oracle_extract_windows(
+        _DT[dtype], _ptr(sa), seq_len, conv_dim, conv_dim, 1, _ptr(ap),
+        int(real_count), max_count, _ptr(oa), conv_dim * d_conv, d_conv)
+    return oa
+
+
+def check_preconditions(*, W, block_size, positions, seq_idx, slot_mapping,
+                        query_start, block_table) -> int:
+    """0 if one launch is well defined on these metadata, else 1..3
+    (1 request rows not contiguous, 2 duplicate slots, 3 written slot read)."""
+    pos = _np(positions, np.int64)
+    sid = _np(seq_idx, np.int32)
+    slot = _np(slot_mapping, np.int64)
+    qs = _np(query_start, np.int32)
+    bt = _np(block_table, np.int32)
+    return int(lib().oracle_check_preconditions(
+        pos.shape[0], W, block_size, _ptr(pos), _ptr(sid), _ptr(slot), _ptr(qs),
+        _ptr(bt), bt.shape[1], bt.shape[1]))

@@ -1,0 +1,304 @@
+/*
+ * sconv_oracle.c -- TEST INFRASTRUCTURE, NOT PART OF THE PRODUCT.
+ *
+ * A plain, slow, scalar, double-precision CPU statement of what the fused
+ * short-convolution path computes.  It exists only so that the CUDA kernels
+ * can be checked against it: only the test suite, the smoke check and the
+ * CPU-baseline leg of the benchmark load it.  It shares no code, header,
+ * table or constant with the CUDA library, and the library never calls it.
+ *
+ * Sources followed (web pages, by title and section):
+ *   [P1] "vllm.models.inkling.nvidia.ops.sconv" -- module docstring (paged
+ *        sliding-window cache, stream D-sub-range, same-forward vs
+ *        pre-forward taps), fused_sconv (argument list and shapes),
+ *        sconv_seq_metadata (seq_idx / query_start buffers, padded rows).
+ *   [P2] "core.ssm.ops.intermediate_extraction" -- _scatter_intermediate_conv_kernel
+ *        and scatter_intermediate_conv (conditional, transposed window gather).
+ *   [P4] "Implementation:Sgl project Sglang Mamba Ops" -- causal_conv1d_update
+ *        (single-token decode form of the same convolution).
+ *
+ * Readings taken where the pages are silent (each one is a single place in
+ * this file):
+ *   - tap orientation: weight[c][W-1] multiplies the current position,
+ *     weight[c][0] the oldest one (the causal_conv1d convention that [P4]
+ *     names); see TAP_POSITION below.
+ *   - a tap is "inside the current forward" when its x row
+ *     (t + src - pos) is at or after query_start[t], the first x row of the
+ *     token's request ([P1] fused_sconv argument comments).
+ *   - epilogue order: out = act(conv) + x  (activation on the convolution,
+ *     residual added after); see EPILOGUE below.
+ *   - PAD rows (slot_mapping == -1) produce no output row and no cache write.
+ *   - window rows outside [0, seq_len) of an extraction read as zero.
+ *   - tokens whose indices fall outside the buffers they address are skipped
+ *     whole and counted (the library's documented bounds policy).
+ *
+ * Everything is computed in double.  Inputs are decoded exactly from their
+ * stored type (bf16 by a 16-bit shift into a float, float to double), and
+ * cache inserts / window gathers are byte copies.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+enum { ORACLE_F32 = 0, ORACLE_BF16 = 1 };
+
+static size_t elem_bytes(int dtype) { return dtype == ORACLE_F32 ? 4u : 2u; }
+
+/* Exact decode of one stored element to double. */
+static double load_value(const void *base, int dtype, int64_t index) {
+    if (dtype == ORACLE_F32) {
+        float f;
+        memcpy(&f, (const char *)base + index * 4, 4);
+        return (double)f;
+    }
+    uint16_t h;
+    memcpy(&h, (const char *)base + index * 2, 2);
+    uint32_t bits = (uint32_t)h << 16; /* bf16 is the top half of a float */
+    float f;
+    memcpy(&f, &bits, 4);
+    return (double)f;
+}
+
+static void copy_element(void *dst, int64_t dst_index, const void *src,
+                         int64_t src_index, int dtype) {
+    size_t e = elem_bytes(dtype);
+    memcpy((char *)dst + dst_index * (int64_t)e,
+           (const char *)src + src_index * (int64_t)e, e);
+}
+
+/* Reading of the tap orientation: tap k of a W-tap window ending at
+ * position pos sits at absolute position pos - (W-1) + k, so tap W-1 is the
+ * current token and tap 0 the oldest ([P4] causal_conv1d convention). */
+#define TAP_POSITION(pos, W, k) ((pos) - ((W) - 1) + (k))
+
+/* Reading of the epilogue order: activation on the convolution, then the
+ * residual input added ([P1] fused_sconv flags activation, use_residual). */
+#define EPILOGUE(conv, xv, silu, resid)                                       \
+    (((silu) ? (conv) / (1.0 + exp(-(conv))) : (conv)) + ((resid) ? (xv) : 0.0))
+
+enum tap_kind { TAP_X = 0, TAP_ZERO = 1, TAP_CACHE = 2 };
+
+/*
+ * oracle_fused -- [P1] fused_sconv: per token, insert x into its cache slot
+ * and convolve the W taps ending at its absolute position.
+ *
+ * Shapes and layouts follow [P1] fused_sconv's argument comments:
+ *   x            [T, C]  row stride x_row_stride, element stride 1, C = H*ws
+ *   weight       [C, W]  strides (w_stride_c, w_stride_k)
+ *   cache        [num_blocks, H, N, D]  strides cache_strides[0..3]
+ *   positions    [T] int64   absolute position of each token
+ *   seq_idx      [T] int32   request of each token
+ *   slot_mapping [T] int64   flat slot block*N + offset; -1 = PAD (skip)
+ *   query_start  [T] int32   first x row of the token's request
+ *   block_table  [num_reqs, max_blocks] int32, row stride bt_row_stride
+ * The stream owns cache lanes [off_s, off_s + ws) of every head; channel
+ * c = h*ws + j lives at lane off_s + j of head h.
+ *
+ * Pre-forward taps are read from cache_in (the cache as it was before the
+ * call).  If cache_out is not NULL the inserts of tokens in
+ * [t_begin, t_end) are written into it (the caller passes a copy of
+ * cache_in).  For every token t in [t_begin, t_end), row t - t_begin of
+ * out_ref [t_end - t_begin, C] receives the double-precision result and
+ * row_state[t - t_begin] is 1 (computed), 0 (PAD) or 2 (skipped: an index
+ * out of range).  Returns the number of skipped tokens, or -1 if an argument
+ * is malformed.
+ */
+int64_t oracle_fused(int dtype, const void *x, int64_t x_row_stride, int64_t T,
+                     int64_t C, const void *weight, int64_t w_stride_c,
+                     int64_t w_stride_k, int W, const void *cache_in,
+                     void *cache_out, const int64_t *cache_strides,
+                     int64_t num_blocks, int64_t H, int64_t N, int64_t D,
+                     const int64_t *positions, const int32_t *seq_idx,
+                     const int64_t *slot_mapping, const int32_t *query_start,
+                     const int32_t *block_table, int64_t bt_row_stride,
+                     int64_t num_reqs, int64_t max_blocks, int64_t off_s,
+                     int64_t ws, int silu, int residual, int64_t t_begin,
+                     int64_t t_end, double *out_ref, uint8_t *row_state) {
+    if (W < 1 || C != H * ws || off_s < 0 || off_s + ws > D || N < 1 ||
+        t_begin < 0 || t_end > T || t_begin > t_end)
+        return -1;
+    int64_t skipped = 0;
+    enum tap_kind kind[64];
+    int64_t tap_block[64];
+    if (W > 64) return -1;
+
+    for (int64_t t = t_begin; t < t_end; ++t) {
+        int64_t local = t - t_begin;
+        row_state[local] = 0;
+        int64_t slot = slot_mapping[t];
+        if (slot == -1) continue; /* PAD: [P1] "PAD = -1 => skip" */
+
+        int64_t pos = positions[t];
+        int64_t req = seq_idx[t];
+        int64_t q0 = query_start[t];
+        int bad = slot < 0 || slot >= num_blocks * N || req < 0 ||
+                  req >= num_reqs || q0 < 0 || q0 > t || pos < 0;
+
+        /* Resolve where each tap comes from ([P1] module docstring). */
+        for (int k = 0; k < W && !bad; ++k) {
+            int64_t src = TAP_POSITION(pos, W, k);
+            int64_t row = t + (src - pos);
+            if (row >= q0) {
+                kind[k] = TAP_X; /* same-forward tap: x row src - pos + t */
+            } else if (src < 0) {
+                kind[k] = TAP_ZERO; /* before position 0 */
+            } else {
+                int64_t logical = src / N;
+                if (logical >= max_blocks) { bad = 1; break; }
+                int64_t b = block_table[req * bt_row_stride + logical];
+                if (b < 0 || b >= num_blocks) { bad = 1; break; }
+                kind[k] = TAP_CACHE; /* pre-forward tap via block_table */
+                tap_block[k] = b;
+            }
+        }
+        if (bad) {
+            row_state[local] = 2;
+            ++skipped;
+            continue;
+        }
+        row_state[local] = 1;
+
+        for (int64_t c = 0; c < C; ++c) {
+            int64_t h = c / ws, j = c % ws;
+            int64_t x_index = t * x_row_stride + c;
+            if (cache_out) {
+                int64_t dst = (slot / N) * cache_strides[0] + h * cache_strides[1] +
+                              (slot % N) * cache_strides[2] +
+                              (off_s + j) * cache_strides[3];
+                copy_element(cache_out, dst, x, x_index, dtype);
+            }
+            double acc = 0.0;
+            for (int k = 0; k < W; ++k) {
+                int64_t src = TAP_POSITION(pos, W, k);
+                double v;
+                if (kind[k] == TAP_X) {
+                    v = load_value(x, dtype, (t + (src - pos)) * x_row_stride + c);
+                } else if (kind[k] == TAP_ZERO) {
+                    v = 0.0;
+                } else {
+                    int64_t idx = tap_block[k] * cache_strides[0] +
+                                  h * cache_strides[1] +
+                                  (src % N) * cache_strides[2] +
+                                  (off_s + j) * cache_strides[3];
+                    v = load_value(cache_in, dtype, idx);
+                }
+                acc += load_value(weight, dtype, c * w_stride_c + k * w_stride_k) * v;
+            }
+            out_ref[local * C + c] =
+                EPILOGUE(acc, load_value(x, dtype, x_index), silu, residual);
+        }
+    }
+    return skipped;
+}
+
+/*
+ * oracle_seq_metadata -- [P1] sconv_seq_metadata: for every token
+ * t < num_actual, seq_idx[t] is the last request r < num_reqs whose start
+ * query_start_loc[r] is <= t (so empty requests are never chosen) and
+ * query_start[t] = query_start_loc[seq_idx[t]]; rows
+ * [num_actual, num_padded) are filled with zero.  A plain linear scan.
+ */
+void oracle_seq_metadata(const int32_t *query_start_loc, int64_t num_reqs,
+                         int64_t num_actual, int64_t num_padded,
+                         int32_t *seq_idx_out, int32_t *query_start_out) {
+    for (int64_t t = 0; t < num_padded; ++t) {
+        if (t >= num_actual) {
+            seq_idx_out[t] = 0;
+            query_start_out[t] = 0;
+            continue;
+        }
+        int64_t found = 0;
+        for (int64_t r = 0; r < num_reqs; ++r)
+            if (query_start_loc[r] <= t) found = r;
+        seq_idx_out[t] = (int32_t)found;
+        query_start_out[t] = query_start_loc[found];
+    }
+}
+
+/*
+ * oracle_extract_windows -- [P2] scatter_intermediate_conv: for slot
+ * i < real_count, out[i][c][k] = src[abs_positions[i] - d_conv + k][c]
+ * (window [pos - d_conv, pos), written transposed), with rows outside
+ * [0, seq_len) reading as zero; slots i >= real_count are left untouched.
+ * `out` holds the caller's prior bytes on entry.  real_count is clamped to
+ * [0, max_count].
+ */
+void oracle_extract_windows(int dtype, const void *src, int64_t seq_len,
+                            int64_t conv_dim, int64_t src_stride_s,
+                            int64_t src_stride_c, const int32_t *abs_positions,
+                            int64_t real_count, int64_t max_count, void *out,
+                            int64_t out_slot_stride, int64_t d_conv) {
+    if (real_count > max_count) real_count = max_count;
+    size_t e = elem_bytes(dtype);
+    for (int64_t i = 0; i < real_count; ++i) {
+        for (int64_t c = 0; c < conv_dim; ++c) {
+            for (int64_t k = 0; k < d_conv; ++k) {
+                int64_t p = (int64_t)abs_positions[i] - d_conv + k;
+                int64_t dst = i * out_slot_stride + c * d_conv + k;
+                if (p >= 0 && p < seq_len)
+                    copy_element(out, dst, src, p * src_stride_s + c * src_stride_c,
+                                 dtype);
+                else
+                    memset((char *)out + dst * (int64_t)e, 0, e);
+            }
+        }
+    }
+}
+
+/* ---- precondition checks used by the tests' generator audit ---------- */
+
+static int cmp_i64(const void *a, const void *b) {
+    int64_t x = *(const int64_t *)a, y = *(const int64_t *)b;
+    return (x > y) - (x < y);
+}
+
+/*
+ * oracle_check_preconditions -- the conditions under which one launch is
+ * well defined ([P1] module docstring: the just-written slot is never read
+ * back in the same step; a request's rows are contiguous with positions
+ * rising by one):
+ *   1. within a request, positions[t] - t is constant and seq_idx agrees;
+ *   2. non-PAD slots are distinct;
+ *   3. no written slot is also read as a pre-forward tap.
+ * Returns 0 when all hold, else the number (1..3) of the first one broken.
+ */
+int oracle_check_preconditions(int64_t T, int W, int64_t N,
+                               const int64_t *positions, const int32_t *seq_idx,
+                               const int64_t *slot_mapping,
+                               const int32_t *query_start,
+                               const int32_t *block_table,
+                               int64_t bt_row_stride, int64_t max_blocks) {
+    for (int64_t t = 0; t < T; ++t) {
+        int64_t q0 = query_start[t];
+        if (q0 < 0 || q0 > t) return 1;
+        if (seq_idx[t] != seq_idx[q0]) return 1;
+        if (positions[t] - t != positions[q0] - q0) return 1;
+    }
+    int64_t *written = (int64_t *)malloc(sizeof(int64_t) * (size_t)(T + 1));
+    int64_t *read = (int64_t *)malloc(sizeof(int64_t) * (size_t)(T * W + 1));
+    int64_t nw = 0, nr = 0;
+    for (int64_t t = 0; t < T; ++t) {
+        if (slot_mapping[t] == -1) continue;
+        written[nw++] = slot_mapping[t];
+        int64_t pos = positions[t];
+        for (int k = 0; k < W; ++k) {
+            int64_t src = TAP_POSITION(pos, W, k);
+            if (t + (src - pos) >= query_start[t] || src < 0) continue;
+            int64_t logical = src / N;
+            if (logical >= max_blocks) continue;
+            int64_t b = block_table[(int64_t)seq_idx[t] * bt_row_stride + logical];
+            read[nr++] = b * N + src % N;
+        }
+    }
+    qsort(written, (size_t)nw, sizeof(int64_t), cmp_i64);
+    int result = 0;
+    for (int64_t i = 1; i < nw && !result; ++i)
+        if (written[i] == written[i - 1]) result = 2;
+    for (int64_t i = 0; i < nr && !result; ++i)
+        if (bsearch(&read[i], written, (size_t)nw, sizeof(int64_t), cmp_i64))
+            result = 3;
+    free(written);
+    free(read);
+    return result;
+}

@@ -1,0 +1,115 @@
+"""The pins must catch plausible mistakes in the oracle (CPU only).
+
+Each mutant is a copy of the oracle's C source with one plausible slip
+planted (a reversed or shifted tap, a wrong comparison, a swapped index, a
+dropped term, a transposed write).  It is compiled on the CPU, and the pin
+suite (tests/test_oracle_pins.py) is run against it in a child process; the
+suite must fail for every mutant.  Every planted slip keeps all memory
+accesses inside their buffers, so a mutant fails by assertion, not by crash.
+"""
+from __future__ import annotations
+
+import os
+import subprocess
+import sys
+import tempfile
+from concurrent.futures import ThreadPoolExecutor
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "sconv_oracle.c")
+
+# (name, text to replace, replacement); the first occurrence is replaced.
+MUTANTS = [
+    ("tap_orientation_reversed",
+     "#define TAP_POSITION(pos, W, k) ((pos) - ((W) - 1) + (k))",
+     "#define TAP_POSITION(pos, W, k) ((pos) - (k))"),
+    ("tap_window_shifted",
+     "#define TAP_POSITION(pos, W, k) ((pos) - ((W) - 1) + (k))",
+     "#define TAP_POSITION(pos, W, k) ((pos) - (W) + (k))"),
+    ("same_forward_strict",
+     "            if (row >= q0) {",
+     "            if (row > q0) {"),
+    ("logical_block_mod",
+     "                int64_t logical = src / N;",
+     "                int64_t logical = (src % N) % max_blocks;"),
+    ("block_offset_div",
+     "                                  (src % N) * cache_strides[2] +",
+     "                                  ((src / N) % N) * cache_strides[2] +"),
+    ("read_lane_ignores_off_s",
+     "                                  (off_s + j) * cache_strides[3];",
+     "                                  (j) * cache_strides[3];"),
+    ("read_head_dropped",
+     "                                  h * cache_strides[1] +\n                                  (src % N)",
+     "                                  0 * cache_strides[1] +\n                                  (src % N)"),
+    ("insert_offset_div",
+     "                              (slot % N) * cache_strides[2] +",
+     "                              ((slot / N) % N) * cache_strides[2] +"),
+    ("insert_lane_ignores_off_s",
+     "                              (off_s + j) * cache_strides[3];",
+     "                              (j) * cache_strides[3];"),
+    ("weight_taps_reversed",
+     "load_value(weight, dtype, c * w_stride_c + k * w_stride_k)",
+     "load_value(weight, dtype, c * w_stride_c + (W - 1 - k) * w_stride_k)"),
+    ("epilogue_residual_inside_act",
+     "(((silu) ? (conv) / (1.0 + exp(-(conv))) : (conv)) + ((resid) ? (xv) : 0.0))",
+     "(((silu) ? ((conv) + ((resid) ? (xv) : 0.0)) / (1.0 + exp(-((conv) + ((resid) ? (xv) : 0.0)))) : (conv) + ((resid) ? (xv) : 0.0)))"),
+    ("residual_dropped",
+     "+ ((resid) ? (xv) : 0.0))",
+     "+ 0.0)"),
+    ("silu_sign",
+     "(conv) / (1.0 + exp(-(conv)))",
+     "(conv) / (1.0 + exp((conv)))"),
+    ("pad_not_skipped",
+     "        if (slot == -1) continue; /* PAD",
+     "        if (slot == -2) continue; /* PAD"),
+    ("metadata_strict",
+     "            if (query_start_loc[r] <= t) found = r;",
+     "            if (query_start_loc[r] < t) found = r;"),
+    ("extract_window_shifted",
+     "int64_t p = (int64_t)abs_positions[i] - d_conv + k;",
+     "int64_t p = (int64_t)abs_positions[i] - d_conv + k + 1;"),
+    ("extract_not_transposed",
+     "int64_t dst = i * out_slot_stride + c * d_conv + k;",
+     "int64_t dst = i * out_slot_stride + k * conv_dim + c;"),
+    ("extract_ignores_real_count",
+     "    for (int64_t i = 0; i < real_count; ++i) {",
+     "    for (int64_t i = 0; i < max_count; ++i) {"),
+]
+
+
+def _run_mutant(tmp, name, old, new):
+    src = open(SRC).read()
+    assert old in src, f"mutant {name}: pattern not found"
+    mutated = src.replace(old, new, 1)
+    c_path = os.path.join(tmp, f"{name}.c")
+    so_path = os.path.join(tmp, f"lib{name}.so")
+    with open(c_path, "w") as f:
+        f.write(mutated)
+    oracle.build(force=True, src=c_path, out=so_path)
+    env = dict(os.environ, SCONV_ORACLE_LIB=so_path)
+    r = subprocess.run(
+        [sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+         os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    return name, r.returncode, r.stdout[-400:]
+
+
+def test_every_mutant_is_caught():
+    with tempfile.TemporaryDirectory() as tmp:
+        with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 2)) as ex:
+            results = list(ex.map(lambda m: _run_mutant(tmp, *m), MUTANTS))
+    survivors = [(n, out) for n, rc, out in results if rc != 1]
+    assert not survivors, f"mutants not caught by a failing assertion: {survivors}"
+
+
+def test_unmutated_oracle_passes_in_child():
+    """Control: the same child-process run passes on the real oracle."""
+    r = subprocess.run(
+        [sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+         os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+        cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-2000:]
