@@ -1,0 +1,17 @@
+"""B200-native (sm_100a) fused short-convolution step of hybrid/SSM inference.
+
+One launch per call: paged sliding-window cache insert, depthwise causal
+conv1d over the window ending at each token's absolute position, optional
+SiLU and residual ("vllm.models.inkling.nvidia.ops.sconv"), plus the decode
+update, prefix-caching window extraction
+("core.ssm.ops.intermediate_extraction") and per-token metadata builder.
+
+The kernels live in ``libsconv.so`` (C ABI: include/sconv.h), built by
+``python -m hybrid_sconv_b200.build``; importing this package without it
+raises ImportError.
+"""
+from .binding import (  # noqa: F401
+    EFLAG_BLOCK, EFLAG_LOGICAL, EFLAG_POSITION, EFLAG_QUERY_START, EFLAG_REQUEST,
+    EFLAG_SLOT, LIB_PATH, SconvError, fused_sconv, scatter_intermediate_conv,
+    sconv_extract_windows, sconv_fused, sconv_seq_metadata, sconv_update,
+)

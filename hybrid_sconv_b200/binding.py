@@ -1,0 +1,282 @@
+"""Thin Python binding of ``libsconv.so`` (the C ABI in include/sconv.h).
+
+Argument marshalling only: each function checks tensor ranks and dtypes,
+passes raw device pointers, element strides and the current CUDA stream to
+the C entry point of the same name, and turns a non-zero status into an
+exception.  Every step of the computation runs in the library's kernels; if
+the library is missing the import fails loudly -- there is no fallback.
+PyTorch provides device memory and streams only.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsconv.so")
+
+SCONV_OK, SCONV_ERR_INVALID, SCONV_ERR_UNSUPPORTED, SCONV_ERR_LAUNCH = 0, 1, 2, 3
+SCONV_F32, SCONV_BF16 = 0, 1
+SCONV_ACT_NONE, SCONV_ACT_SILU = 0, 1
+
+# err_flag bits (SCONV_EFLAG_* in sconv.h)
+EFLAG_SLOT, EFLAG_REQUEST, EFLAG_LOGICAL = 0x01, 0x02, 0x04
+EFLAG_BLOCK, EFLAG_QUERY_START, EFLAG_POSITION = 0x08, 0x10, 0x20
+
+_DTYPES = {torch.float32: SCONV_F32, torch.bfloat16: SCONV_BF16}
+
+
+class SconvError(RuntimeError):
+    """A libsconv entry point returned a non-zero status."""
+
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn}: {msg} (status {status})")
+        self.status = status
+
+
+_P, _I64, _INT = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+_I64P = ctypes.POINTER(ctypes.c_int64)
+
+_SIGNATURES = {
+    "sconv_fused": [
+        _P, _I64, _INT, _INT, _P, _I64, _I64, _INT,
+        _P, _I64P, _I64, _INT, _INT, _INT,
+        _P, _P, _P, _P,
+        _P, _I64, _INT, _INT,
+        _INT, _INT, _INT, _INT, _INT,
+        _P, _I64, _P, _P],
+    "sconv_update": [
+        _P, _I64, _INT, _INT, _P, _I64, _I64, _INT,
+        _P, _I64P, _I64, _INT, _INT, _INT,
+        _P, _P,
+        _P, _I64, _INT,
+        _INT, _INT, _INT, _INT, _INT,
+        _P, _I64, _P, _P],
+    "sconv_extract_windows": [
+        _P, _I64, _INT, _I64, _I64, _P, _P, _INT, _P, _I64, _INT, _INT, _P],
+    "sconv_seq_metadata": [_P, _INT, _INT, _INT, _P, _I64, _P, _I64, _P],
+}
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(
+            f"{_LIB_PATH} is not built; run `python -m hybrid_sconv_b200.build` "
+            "(the sconv ops have no fallback)")
+    lib = ctypes.CDLL(_LIB_PATH)
+    for name, args in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = _INT
+    lib.sconv_status_string.argtypes = [_INT]
+    lib.sconv_status_string.restype = ctypes.c_char_p
+    lib.sconv_abi_version.argtypes = []
+    lib.sconv_abi_version.restype = _INT
+    if lib.sconv_abi_version() != 1:
+        raise ImportError("libsconv.so ABI version mismatch; rebuild it")
+    return lib
+
+
+LIB = _load()
+LIB_PATH = _LIB_PATH
+
+
+def _check(fn: str, status: int, value_error: bool = False) -> None:
+    if status != SCONV_OK:
+        msg = LIB.sconv_status_string(status).decode()
+        if value_error and status == SCONV_ERR_INVALID:
+            raise ValueError(f"{fn}: {msg}")
+        raise SconvError(fn, status, msg)
+
+
+def _dev(*tensors: torch.Tensor) -> torch.device:
+    d = tensors[0].device
+    if d.type != "cuda":
+        raise ValueError("sconv ops take CUDA tensors")
+    for t in tensors[1:]:
+        if t is not None and t.device != d:
+            raise ValueError("all tensors must be on the same CUDA device")
+    return d
+
+
+def _ptr(t: Optional[torch.Tensor]) -> int:
+    return 0 if t is None else t.data_ptr()
+
+
+def _want(t: torch.Tensor, dtype: torch.dtype, name: str) -> None:
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _vector(t: torch.Tensor, dtype: torch.dtype, name: str, n: int) -> None:
+    _want(t, dtype, name)
+    if t.dim() != 1 or t.shape[0] < n or (n > 0 and t.stride(0) != 1):
+        raise ValueError(f"{name} must be a contiguous 1-D tensor of at least {n} elements")
+
+
+def _act(activation) -> int:
+    # As in fused_sconv: "silu" and "swish" select SiLU, anything else none.
+    return SCONV_ACT_SILU if activation in ("silu", "swish") else SCONV_ACT_NONE
+
+
+def _stream(device, stream) -> int:
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    return s.cuda_stream
+
+
+def _float_common(x, weight, cache):
+    dt = _DTYPES.get(x.dtype)
+    if dt is None:
+        raise TypeError("x must be float32 or bfloat16")
+    if weight.dtype != x.dtype or cache.dtype != x.dtype:
+        raise TypeError("x, weight and cache must share one dtype")
+    if x.dim() != 2 or weight.dim() != 2 or cache.dim() != 4:
+        raise ValueError("x [T, C], weight [C, W] and cache [num_blocks, H, N, D] expected")
+    if x.shape[0] > 0 and x.stride(1) != 1:
+        raise ValueError("x must have unit channel stride")
+    if weight.shape[0] != x.shape[1]:
+        raise ValueError("weight must be [C, W]")
+    return dt
+
+
+def sconv_fused(x, weight, cache, positions, block_table, seq_idx, slot_mapping,
+                query_start, off_s, ws, block_size, activation=None, use_residual=True, *,
+                out=None, err_flag=None, stream=None):
+    """Insert + depthwise causal conv1d over the paged cache in one launch
+    (fused_sconv, "vllm.models.inkling.nvidia.ops.sconv").  Returns ``out``
+    ([T, C], allocated like x when not given).  See sconv.h for layouts."""
+    dt = _float_common(x, weight, cache)
+    T, C = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    if T == 0:
+        return out
+    d = _dev(x, weight, cache, positions, block_table, seq_idx, slot_mapping, query_start,
+             out, err_flag)
+    _vector(positions, torch.int64, "positions", T)
+    _vector(seq_idx, torch.int32, "seq_idx", T)
+    _vector(slot_mapping, torch.int64, "slot_mapping", T)
+    _vector(query_start, torch.int32, "query_start", T)
+    _want(block_table, torch.int32, "block_table")
+    if block_table.dim() != 2 or block_table.stride(1) != 1:
+        raise ValueError("block_table must be [num_reqs, max_blocks] with unit inner stride")
+    if out.dtype != x.dtype or out.dim() != 2 or tuple(out.shape) != (T, C) or out.stride(1) != 1:
+        raise ValueError("out must be [T, C] like x with unit channel stride")
+    if err_flag is not None:
+        _vector(err_flag, torch.int32, "err_flag", 1)
+    if cache.shape[2] != block_size:
+        raise ValueError("cache.shape[2] must equal block_size")
+    nb, H, N, D = cache.shape
+    cs = (ctypes.c_int64 * 4)(*cache.stride())
+    with torch.cuda.device(d):
+        st = LIB.sconv_fused(
+            _ptr(x), x.stride(0), T, C, _ptr(weight), weight.stride(0), weight.stride(1),
+            weight.shape[1], _ptr(cache), cs, nb, H, N, D,
+            _ptr(positions), _ptr(seq_idx), _ptr(slot_mapping), _ptr(query_start),
+            _ptr(block_table), block_table.stride(0), block_table.shape[0],
+            block_table.shape[1], off_s, ws, _act(activation), int(bool(use_residual)), dt,
+            _ptr(out), out.stride(0), _ptr(err_flag), _stream(d, stream))
+    _check("sconv_fused", st)
+    return out
+
+
+def sconv_update(x, weight, cache, positions, block_table, slot_mapping, off_s, ws,
+                 block_size, activation=None, use_residual=True, *, out=None,
+                 err_flag=None, stream=None):
+    """Single-token decode: token b is request b (block_table row b).  Same
+    result as sconv_fused with seq_idx = query_start = arange(B)."""
+    dt = _float_common(x, weight, cache)
+    B, C = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    if B == 0:
+        return out
+    d = _dev(x, weight, cache, positions, block_table, slot_mapping, out, err_flag)
+    _vector(positions, torch.int64, "positions", B)
+    _vector(slot_mapping, torch.int64, "slot_mapping", B)
+    _want(block_table, torch.int32, "block_table")
+    if block_table.dim() != 2 or block_table.shape[0] < B or block_table.stride(1) != 1:
+        raise ValueError("block_table must be [>= B, max_blocks] with unit inner stride")
+    if out.dtype != x.dtype or tuple(out.shape) != (B, C) or out.stride(1) != 1:
+        raise ValueError("out must be [B, C] like x with unit channel stride")
+    if err_flag is not None:
+        _vector(err_flag, torch.int32, "err_flag", 1)
+    if cache.shape[2] != block_size:
+        raise ValueError("cache.shape[2] must equal block_size")
+    nb, H, N, D = cache.shape
+    cs = (ctypes.c_int64 * 4)(*cache.stride())
+    with torch.cuda.device(d):
+        st = LIB.sconv_update(
+            _ptr(x), x.stride(0), B, C, _ptr(weight), weight.stride(0), weight.stride(1),
+            weight.shape[1], _ptr(cache), cs, nb, H, N, D, _ptr(positions),
+            _ptr(slot_mapping), _ptr(block_table), block_table.stride(0),
+            block_table.shape[1], off_s, ws, _act(activation), int(bool(use_residual)), dt,
+            _ptr(out), out.stride(0), _ptr(err_flag), _stream(d, stream))
+    _check("sconv_update", st)
+    return out
+
+
+def sconv_extract_windows(src, abs_positions, real_count, out, d_conv, *, stream=None):
+    """Gather the d_conv-long windows [pos - d_conv, pos) of ``src`` for the
+    first ``real_count[0]`` slots into ``out[slot, conv_dim, d_conv]``
+    (scatter_intermediate_conv, "core.ssm.ops.intermediate_extraction").
+    ``src`` is [seq_len, conv_dim] or [batch, seq_len, conv_dim] (batch 0 is
+    read); ``real_count`` is a device int32[1]."""
+    if src.dim() == 3:
+        src = src[0]
+    if src.dim() != 2:
+        raise ValueError("src must be [seq_len, conv_dim] or [batch, seq_len, conv_dim]")
+    dt = _DTYPES.get(src.dtype)
+    if dt is None or out.dtype != src.dtype:
+        raise TypeError("src and out must share one dtype, float32 or bfloat16")
+    max_count = out.shape[0]
+    if max_count == 0:
+        return out
+    d = _dev(src, abs_positions, real_count, out)
+    _vector(abs_positions, torch.int32, "abs_positions", max_count)
+    _vector(real_count, torch.int32, "real_count", 1)
+    seq_len, conv_dim = src.shape
+    if out.dim() != 3 or out.shape[1] != conv_dim or out.shape[2] != d_conv or \
+            out.stride(2) != 1 or out.stride(1) != d_conv:
+        raise ValueError("out must be [max_count, conv_dim, d_conv] with dense inner dims")
+    with torch.cuda.device(d):
+        st = LIB.sconv_extract_windows(
+            _ptr(src), seq_len, conv_dim, src.stride(0), src.stride(1),
+            _ptr(abs_positions), _ptr(real_count), max_count, _ptr(out), out.stride(0),
+            d_conv, dt, _stream(d, stream))
+    _check("sconv_extract_windows", st)
+    return out
+
+
+def sconv_seq_metadata(query_start_loc, num_reqs, num_actual_tokens, seq_idx_out,
+                       query_start_out, num_padded_tokens=None, *, stream=None):
+    """Fill seq_idx_out / query_start_out for every token row in one launch
+    (sconv_seq_metadata, "vllm.models.inkling.nvidia.ops.sconv").  Raises
+    ValueError on the size errors the page names."""
+    if num_padded_tokens is None:
+        num_padded_tokens = num_actual_tokens
+    if num_padded_tokens < num_actual_tokens:
+        raise ValueError("num_padded_tokens must cover all actual tokens")
+    if num_padded_tokens > seq_idx_out.shape[0]:
+        raise ValueError("seq_idx_out is too small for the padded token count")
+    if num_padded_tokens > query_start_out.shape[0]:
+        raise ValueError("query_start_out is too small for the padded token count")
+    if num_padded_tokens == 0:
+        return
+    d = _dev(query_start_loc, seq_idx_out, query_start_out)
+    _vector(query_start_loc, torch.int32, "query_start_loc", num_reqs + 1)
+    _vector(seq_idx_out, torch.int32, "seq_idx_out", num_padded_tokens)
+    _vector(query_start_out, torch.int32, "query_start_out", num_padded_tokens)
+    with torch.cuda.device(d):
+        st = LIB.sconv_seq_metadata(
+            _ptr(query_start_loc), num_reqs, num_actual_tokens, num_padded_tokens,
+            _ptr(seq_idx_out), seq_idx_out.shape[0], _ptr(query_start_out),
+            query_start_out.shape[0], _stream(d, stream))
+    _check("sconv_seq_metadata", st, value_error=True)
+
+
+# Names used on the pages, for callers coming from them.
+fused_sconv = sconv_fused
+scatter_intermediate_conv = sconv_extract_windows

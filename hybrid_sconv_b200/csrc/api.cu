@@ -1,0 +1,221 @@
+// api.cu -- the extern "C" entry points declared in include/sconv.h.
+//
+// Every entry point validates its arguments on the host before it touches
+// the CUDA runtime, so a malformed call returns a status and enqueues
+// nothing.  Then it picks the 16-byte pack path when every pointer, stride
+// and lane offset allows it (else the one-element path) and launches.
+#include <stdint.h>
+
+#include "common.cuh"
+#include "sconv.h"
+
+namespace {
+
+using sconv::FusedArgs;
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int64_t elem_size(sconv_dtype dt) { return dt == SCONV_F32 ? 4 : 2; }
+
+// Half-open byte ranges [lo, hi) overlap?
+inline bool overlaps(const void *a, int64_t a_bytes, const void *b, int64_t b_bytes) {
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + static_cast<uintptr_t>(b_bytes) && b0 < a0 + static_cast<uintptr_t>(a_bytes);
+}
+
+// Shared checks of sconv_fused and sconv_update.  Returns SCONV_OK or the
+// status to report; on success fills `a` (except the metadata pointers
+// specific to one entry point) and `vec`.
+sconv_status check_fused(const void *x, int64_t x_rs, int T, int C, const void *weight,
+                         int64_t w_sc, int64_t w_sk, int W, void *cache, const int64_t *cs,
+                         int64_t num_blocks, int H, int N, int D, const int64_t *positions,
+                         const int64_t *slot_mapping, const int32_t *block_table, int64_t bt_rs,
+                         int num_reqs, int max_blocks, int off_s, int ws, sconv_act act,
+                         int use_residual, sconv_dtype dt, void *out, int64_t out_rs,
+                         int32_t *err_flag, FusedArgs &a, bool &vec) {
+    if (dt != SCONV_F32 && dt != SCONV_BF16) return SCONV_ERR_UNSUPPORTED;
+    if (W < 1) return SCONV_ERR_INVALID;
+    if (W > SCONV_MAX_W) return SCONV_ERR_UNSUPPORTED;
+    if (act != SCONV_ACT_NONE && act != SCONV_ACT_SILU) return SCONV_ERR_INVALID;
+    if (C < 1 || H < 1 || N < 1 || D < 1 || ws < 1 || off_s < 0) return SCONV_ERR_INVALID;
+    if (static_cast<int64_t>(off_s) + ws > D) return SCONV_ERR_INVALID;
+    if (static_cast<int64_t>(H) * ws != C) return SCONV_ERR_INVALID;
+    if (num_blocks < 1 || num_reqs < 1 || max_blocks < 1) return SCONV_ERR_INVALID;
+    if (!x || !weight || !cache || !cs || !positions || !slot_mapping || !block_table || !out)
+        return SCONV_ERR_INVALID;
+    if (cs[3] != 1 || cs[0] < 1 || cs[1] < 1 || cs[2] < 1) return SCONV_ERR_INVALID;
+    if (x_rs < C || out_rs < C || bt_rs < max_blocks) return SCONV_ERR_INVALID;
+    if (w_sc < 0 || w_sk < 0) return SCONV_ERR_INVALID;
+
+    const int64_t e = elem_size(dt);
+    const int64_t x_bytes = ((static_cast<int64_t>(T) - 1) * x_rs + C) * e;
+    const int64_t out_bytes = ((static_cast<int64_t>(T) - 1) * out_rs + C) * e;
+    const int64_t cache_bytes =
+        ((num_blocks - 1) * cs[0] + static_cast<int64_t>(H - 1) * cs[1] +
+         static_cast<int64_t>(N - 1) * cs[2] + D) * e;
+    if (overlaps(out, out_bytes, x, x_bytes) || overlaps(out, out_bytes, cache, cache_bytes))
+        return SCONV_ERR_INVALID;
+
+    const int64_t V = 16 / e;
+    vec = aligned16(x) && aligned16(out) && aligned16(cache) && x_rs % V == 0 &&
+          out_rs % V == 0 && cs[0] % V == 0 && cs[1] % V == 0 && cs[2] % V == 0 &&
+          off_s % V == 0 && ws % V == 0;
+
+    a.x = x;
+    a.x_rs = x_rs;
+    a.T = T;
+    a.C = C;
+    a.w = weight;
+    a.w_sc = w_sc;
+    a.w_sk = w_sk;
+    a.W = W;
+    a.cache = cache;
+    a.cs0 = cs[0];
+    a.cs1 = cs[1];
+    a.cs2 = cs[2];
+    a.num_blocks = num_blocks;
+    a.H = H;
+    a.N = N;
+    a.D = D;
+    a.positions = positions;
+    a.seq_idx = nullptr;
+    a.slot = slot_mapping;
+    a.qstart = nullptr;
+    a.bt = block_table;
+    a.bt_rs = bt_rs;
+    a.num_reqs = num_reqs;
+    a.max_blocks = max_blocks;
+    a.off_s = off_s;
+    a.ws = ws;
+    a.silu = act == SCONV_ACT_SILU;
+    a.resid = use_residual != 0;
+    a.out = out;
+    a.out_rs = out_rs;
+    a.err = err_flag;
+    return SCONV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sconv_abi_version(void) { return SCONV_ABI_VERSION; }
+
+const char *sconv_status_string(sconv_status s) {
+    switch (s) {
+        case SCONV_OK: return "ok";
+        case SCONV_ERR_INVALID: return "invalid argument";
+        case SCONV_ERR_UNSUPPORTED: return "unsupported argument";
+        case SCONV_ERR_LAUNCH: return "kernel launch failed";
+    }
+    return "unknown status";
+}
+
+sconv_status sconv_fused(const void *x, int64_t x_row_stride, int T, int C, const void *weight,
+                         int64_t w_stride_c, int64_t w_stride_k, int W, void *cache,
+                         const int64_t cache_strides[4], int64_t num_blocks, int H, int N, int D,
+                         const int64_t *positions, const int32_t *seq_idx,
+                         const int64_t *slot_mapping, const int32_t *query_start,
+                         const int32_t *block_table, int64_t bt_row_stride, int num_reqs,
+                         int max_blocks, int off_s, int ws, sconv_act act, int use_residual,
+                         sconv_dtype dt, void *out, int64_t out_row_stride, int32_t *err_flag,
+                         cudaStream_t stream) {
+    if (T < 0) return SCONV_ERR_INVALID;
+    if (T == 0) return SCONV_OK;
+    if (!seq_idx || !query_start) return SCONV_ERR_INVALID;
+    FusedArgs a;
+    bool vec = false;
+    const sconv_status st = check_fused(
+        x, x_row_stride, T, C, weight, w_stride_c, w_stride_k, W, cache, cache_strides,
+        num_blocks, H, N, D, positions, slot_mapping, block_table, bt_row_stride, num_reqs,
+        max_blocks, off_s, ws, act, use_residual, dt, out, out_row_stride, err_flag, a, vec);
+    if (st != SCONV_OK) return st;
+    a.seq_idx = seq_idx;
+    a.qstart = query_start;
+    return sconv::launch_fused(a, dt == SCONV_BF16, vec, false, stream) == cudaSuccess
+               ? SCONV_OK
+               : SCONV_ERR_LAUNCH;
+}
+
+sconv_status sconv_update(const void *x, int64_t x_row_stride, int B, int C, const void *weight,
+                          int64_t w_stride_c, int64_t w_stride_k, int W, void *cache,
+                          const int64_t cache_strides[4], int64_t num_blocks, int H, int N,
+                          int D, const int64_t *positions, const int64_t *slot_mapping,
+                          const int32_t *block_table, int64_t bt_row_stride, int max_blocks,
+                          int off_s, int ws, sconv_act act, int use_residual, sconv_dtype dt,
+                          void *out, int64_t out_row_stride, int32_t *err_flag,
+                          cudaStream_t stream) {
+    if (B < 0) return SCONV_ERR_INVALID;
+    if (B == 0) return SCONV_OK;
+    FusedArgs a;
+    bool vec = false;
+    const sconv_status st = check_fused(
+        x, x_row_stride, B, C, weight, w_stride_c, w_stride_k, W, cache, cache_strides,
+        num_blocks, H, N, D, positions, slot_mapping, block_table, bt_row_stride, B, max_blocks,
+        off_s, ws, act, use_residual, dt, out, out_row_stride, err_flag, a, vec);
+    if (st != SCONV_OK) return st;
+    return sconv::launch_fused(a, dt == SCONV_BF16, vec, true, stream) == cudaSuccess
+               ? SCONV_OK
+               : SCONV_ERR_LAUNCH;
+}
+
+sconv_status sconv_extract_windows(const void *src, int64_t seq_len, int conv_dim,
+                                   int64_t src_stride_s, int64_t src_stride_c,
+                                   const int32_t *abs_positions, const int32_t *real_count,
+                                   int max_count, void *out, int64_t out_slot_stride, int d_conv,
+                                   sconv_dtype dt, cudaStream_t stream) {
+    if (dt != SCONV_F32 && dt != SCONV_BF16) return SCONV_ERR_UNSUPPORTED;
+    if (max_count < 0 || conv_dim < 1 || seq_len < 0 || d_conv < 1) return SCONV_ERR_INVALID;
+    if (d_conv > SCONV_MAX_DCONV) return SCONV_ERR_UNSUPPORTED;
+    if (max_count == 0) return SCONV_OK;
+    if (!src || !abs_positions || !real_count || !out) return SCONV_ERR_INVALID;
+    if (src_stride_c != 1 || src_stride_s < conv_dim) return SCONV_ERR_INVALID;
+    if (out_slot_stride < static_cast<int64_t>(conv_dim) * d_conv) return SCONV_ERR_INVALID;
+    const int64_t e = elem_size(dt);
+    const int64_t out_bytes =
+        ((static_cast<int64_t>(max_count) - 1) * out_slot_stride +
+         static_cast<int64_t>(conv_dim) * d_conv) * e;
+    const int64_t src_bytes =
+        seq_len > 0 ? ((seq_len - 1) * src_stride_s + conv_dim) * e : 0;
+    if (src_bytes > 0 && overlaps(out, out_bytes, src, src_bytes)) return SCONV_ERR_INVALID;
+
+    const int64_t V = 16 / e;
+    const bool vec = aligned16(src) && aligned16(out) && src_stride_s % V == 0 &&
+                     conv_dim % V == 0 && out_slot_stride % V == 0;
+    sconv::ExtractArgs a;
+    a.src = src;
+    a.seq_len = seq_len;
+    a.conv_dim = conv_dim;
+    a.src_ss = src_stride_s;
+    a.abs_pos = abs_positions;
+    a.real_count = real_count;
+    a.max_count = max_count;
+    a.out = out;
+    a.out_ss = out_slot_stride;
+    a.d_conv = d_conv;
+    return sconv::launch_extract(a, dt == SCONV_BF16, vec, stream) == cudaSuccess
+               ? SCONV_OK
+               : SCONV_ERR_LAUNCH;
+}
+
+sconv_status sconv_seq_metadata(const int32_t *query_start_loc, int num_reqs,
+                                int num_actual_tokens, int num_padded_tokens,
+                                int32_t *seq_idx_out, int64_t seq_idx_cap,
+                                int32_t *query_start_out, int64_t query_start_cap,
+                                cudaStream_t stream) {
+    if (num_padded_tokens < 0) num_padded_tokens = num_actual_tokens;
+    if (num_actual_tokens < 0 || num_reqs < 0) return SCONV_ERR_INVALID;
+    if (num_padded_tokens < num_actual_tokens) return SCONV_ERR_INVALID;
+    if (num_padded_tokens > seq_idx_cap || num_padded_tokens > query_start_cap)
+        return SCONV_ERR_INVALID;
+    if (num_actual_tokens > 0 && num_reqs < 1) return SCONV_ERR_INVALID;
+    if (num_padded_tokens == 0) return SCONV_OK;
+    if (!query_start_loc || !seq_idx_out || !query_start_out) return SCONV_ERR_INVALID;
+    return sconv::launch_seq_metadata(query_start_loc, num_reqs, num_actual_tokens,
+                                      num_padded_tokens, seq_idx_out, query_start_out,
+                                      stream) == cudaSuccess
+               ? SCONV_OK
+               : SCONV_ERR_LAUNCH;
+}
+
+}  // extern "C"

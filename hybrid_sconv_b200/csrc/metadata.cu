@@ -1,0 +1,59 @@
+// metadata.cu -- per-token request index and request start in one launch
+// ("vllm.models.inkling.nvidia.ops.sconv", sconv_seq_metadata), sm_100a.
+//
+// One thread per token row.  The request is the last r < num_reqs with
+// query_start_loc[r] <= t, found by binary search; when the offsets table
+// is small each block first stages it in shared memory so the search's
+// dependent loads hit shared memory instead of L2.
+#include "common.cuh"
+
+namespace sconv {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kSmemReqs = 4096;  // stage query_start_loc when num_reqs <= this
+
+__global__ void __launch_bounds__(kThreads)
+seq_metadata_kernel(const int32_t *__restrict__ qsl, int num_reqs, int num_actual,
+                    int num_padded, int32_t *__restrict__ seq_idx,
+                    int32_t *__restrict__ query_start, int staged) {
+    extern __shared__ int32_t s_qsl[];
+    if (staged) {
+        for (int i = threadIdx.x; i < num_reqs; i += blockDim.x) s_qsl[i] = __ldg(qsl + i);
+        __syncthreads();
+    }
+    const int32_t *q = staged ? s_qsl : qsl;
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= num_padded) return;
+    if (t >= num_actual) {
+        seq_idx[t] = 0;
+        query_start[t] = 0;
+        return;
+    }
+    // Invariant: the answer lies in [lo, hi]; q[lo] <= t is assumed for lo = 0.
+    int lo = 0, hi = num_reqs - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (q[mid] <= t) lo = mid;
+        else hi = mid - 1;
+    }
+    seq_idx[t] = lo;
+    query_start[t] = q[lo];
+}
+
+}  // namespace
+
+cudaError_t launch_seq_metadata(const int32_t *qsl, int num_reqs, int num_actual, int num_padded,
+                                int32_t *seq_idx, int32_t *query_start, cudaStream_t stream) {
+    // With no actual tokens the search never runs; one entry keeps the
+    // staging loop and the search bounds well defined.
+    const int nr = num_reqs > 0 ? num_reqs : 1;
+    const int staged = nr <= kSmemReqs ? 1 : 0;
+    const size_t smem = staged ? static_cast<size_t>(nr) * sizeof(int32_t) : 0;
+    const int blocks = (num_padded + kThreads - 1) / kThreads;
+    seq_metadata_kernel<<<blocks, kThreads, smem, stream>>>(qsl, nr, num_actual, num_padded,
+                                                            seq_idx, query_start, staged);
+    return cudaGetLastError();
+}
+
+}  // namespace sconv

@@ -1,0 +1,198 @@
+/*
+ * sconv.h -- C ABI of the B200 (sm_100a) fused short-convolution library.
+ *
+ * The operation is the short-convolution step of hybrid attention/SSM
+ * inference described on the page "vllm.models.inkling.nvidia.ops.sconv"
+ * (module docstring and fused_sconv):
+ *
+ *   A layer's conv streams share one paged cache [num_blocks, H, N, D]
+ *   (head-major).  A stream owns the lanes [off_s, off_s + ws) of every head,
+ *   so its per-token channel count is C = H * ws and channel c = h*ws + j
+ *   lives at lane off_s + j of head h.  The cache holds the conv input at
+ *   every absolute position.  For each token one launch
+ *     1. writes the token's input row x[t, :] into its slot
+ *        (slot_mapping[t] = block * N + offset; -1 marks a PAD row, skipped);
+ *     2. convolves, per channel, the W taps ending at the token's absolute
+ *        position: a tap inside the current forward is read from x (row
+ *        t + src - pos), an earlier one from the cache through
+ *        block_table[request, src / N] at offset src % N, and a tap before
+ *        position 0 is zero;
+ *     3. applies the optional SiLU to the convolution and then adds the
+ *        residual x[t, c];
+ *   and is valid for prefill, decode and speculative tokens alike.
+ *
+ * Conventions shared by every entry point:
+ *   - All data pointers are DEVICE pointers owned by the caller.  Nothing is
+ *     allocated, freed or synchronised: work is enqueued on `stream`, the
+ *     grid depends only on the token count and channel count (or on
+ *     max_count), so every call can be captured in a CUDA graph.
+ *   - Strides are in ELEMENTS.  The innermost stride of x, out, src and the
+ *     cache D axis must be 1.
+ *   - Floating-point data (x, weight, cache, out, src) all have the one
+ *     dtype `dt`.  Accumulation is in fp32 over taps in order k = 0..W-1;
+ *     bf16 results are rounded to nearest even once.
+ *   - Tap orientation: weight[c][W-1] multiplies the current position and
+ *     weight[c][0] the position W-1 steps back (the causal_conv1d convention
+ *     of "Implementation:Sgl project Sglang Mamba Ops").
+ *   - Arguments are checked on the host before anything is enqueued; a bad
+ *     argument returns SCONV_ERR_INVALID or SCONV_ERR_UNSUPPORTED and
+ *     enqueues nothing.  The library never aborts the process.
+ *   - Indices read on the device (slots, requests, block-table entries,
+ *     query starts, positions) are range-checked per token.  A token with an
+ *     index out of range is skipped whole (no cache write, no output row)
+ *     and, if `err_flag` is not NULL, the matching SCONV_EFLAG_* bits are
+ *     OR-ed into *err_flag.  Nothing traps or waits.
+ *   - Preconditions not checked (behaviour is undefined when broken): the
+ *     rows of one request are contiguous in x with positions rising by one;
+ *     the non-PAD slots of a call are distinct; no slot written by a call is
+ *     also read by it as a pre-forward tap (the module docstring's argument
+ *     for why one launch has no write/read hazard).
+ */
+#ifndef SCONV_H
+#define SCONV_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sconv_status {
+    SCONV_OK = 0,
+    SCONV_ERR_INVALID = 1,     /* malformed argument (size, pointer, stride, overlap) */
+    SCONV_ERR_UNSUPPORTED = 2, /* well-formed but outside what is built (dtype, W, d_conv) */
+    SCONV_ERR_LAUNCH = 3       /* the CUDA launch itself failed */
+} sconv_status;
+
+typedef enum sconv_dtype { SCONV_F32 = 0, SCONV_BF16 = 1 } sconv_dtype;
+
+/* fused_sconv's activation: "silu" and "swish" both select SCONV_ACT_SILU. */
+typedef enum sconv_act { SCONV_ACT_NONE = 0, SCONV_ACT_SILU = 1 } sconv_act;
+
+/* Bits OR-ed into *err_flag by a token that is skipped. */
+#define SCONV_EFLAG_SLOT        0x01u /* slot_mapping not -1 and outside [0, num_blocks*N) */
+#define SCONV_EFLAG_REQUEST     0x02u /* seq_idx outside [0, num_reqs) */
+#define SCONV_EFLAG_LOGICAL     0x04u /* src / N >= max_blocks for a pre-forward tap */
+#define SCONV_EFLAG_BLOCK       0x08u /* block_table entry outside [0, num_blocks) */
+#define SCONV_EFLAG_QUERY_START 0x10u /* query_start[t] outside [0, t] */
+#define SCONV_EFLAG_POSITION    0x20u /* positions[t] < 0 */
+
+#define SCONV_MAX_W 8      /* taps supported by sconv_fused / sconv_update */
+#define SCONV_MAX_DCONV 8  /* window length supported by sconv_extract_windows */
+
+/*
+ * sconv_fused -- insert + depthwise causal conv1d over the paged cache, one
+ * launch ("vllm.models.inkling.nvidia.ops.sconv", fused_sconv).
+ *
+ *   x              [T, C] input rows, row stride x_row_stride (>= C).  Never
+ *                  written.  C must equal H * ws.
+ *   weight         [C, W] taps, strides (w_stride_c, w_stride_k).  1 <= W <= 8.
+ *   cache          [num_blocks, H, N, D], strides cache_strides[0..3] with
+ *                  cache_strides[3] == 1.  Read (pre-forward taps) and
+ *                  written (inserts) in place.  N is the block size.
+ *   positions      [T] int64 absolute position of each token.
+ *   seq_idx        [T] int32 request of each token (a block_table row).
+ *   slot_mapping   [T] int64 flat slot block*N + offset; -1 = PAD row (no
+ *                  cache write, no output row; its x is still read by the
+ *                  later tokens of its request).
+ *   query_start    [T] int32 first x row of the token's request.
+ *   block_table    [num_reqs, max_blocks] int32, row stride bt_row_stride.
+ *   off_s, ws      the stream's lanes [off_s, off_s + ws) within D.
+ *   act, use_residual   epilogue: out = act(conv) + (use_residual ? x : 0).
+ *   dt             dtype of x, weight, cache and out.
+ *   out            [T, C], row stride out_row_stride (>= C).  Must not
+ *                  overlap x or the cache.  PAD and skipped rows are left
+ *                  untouched.
+ *   err_flag       optional device int32; see SCONV_EFLAG_*.
+ * T == 0 returns SCONV_OK and enqueues nothing.
+ */
+sconv_status sconv_fused(
+    const void *x, int64_t x_row_stride, int T, int C,
+    const void *weight, int64_t w_stride_c, int64_t w_stride_k, int W,
+    void *cache, const int64_t cache_strides[4], int64_t num_blocks, int H, int N, int D,
+    const int64_t *positions, const int32_t *seq_idx, const int64_t *slot_mapping,
+    const int32_t *query_start,
+    const int32_t *block_table, int64_t bt_row_stride, int num_reqs, int max_blocks,
+    int off_s, int ws, sconv_act act, int use_residual, sconv_dtype dt,
+    void *out, int64_t out_row_stride, int32_t *err_flag, cudaStream_t stream);
+
+/*
+ * sconv_update -- single-token decode form: token b belongs to request b
+ * (seq_idx[b] = query_start[b] = b), so every pre-current tap comes from
+ * the cache or is zero.  Same computation as sconv_fused on those metadata
+ * (the decode update of causal_conv1d_update, "Implementation:Sgl project
+ * Sglang Mamba Ops", over the paged cache of the vllm sconv page).
+ *
+ *   x [B, C], positions [B], slot_mapping [B] (-1 = PAD), block_table
+ *   [B, max_blocks]; every other argument as in sconv_fused.
+ * B == 0 returns SCONV_OK and enqueues nothing.
+ */
+sconv_status sconv_update(
+    const void *x, int64_t x_row_stride, int B, int C,
+    const void *weight, int64_t w_stride_c, int64_t w_stride_k, int W,
+    void *cache, const int64_t cache_strides[4], int64_t num_blocks, int H, int N, int D,
+    const int64_t *positions, const int64_t *slot_mapping,
+    const int32_t *block_table, int64_t bt_row_stride, int max_blocks,
+    int off_s, int ws, sconv_act act, int use_residual, sconv_dtype dt,
+    void *out, int64_t out_row_stride, int32_t *err_flag, cudaStream_t stream);
+
+/*
+ * sconv_extract_windows -- conditional, transposed gather of the length-d_conv
+ * conv windows that prefix caching snapshots ("core.ssm.ops.intermediate_extraction",
+ * scatter_intermediate_conv and _scatter_intermediate_conv_kernel).
+ *
+ *   src            [seq_len, conv_dim], strides (src_stride_s, src_stride_c),
+ *                  src_stride_c == 1 (the pre-conv input of one sequence).
+ *   abs_positions  [max_count] int32 end position of each slot's window; the
+ *                  window is rows [pos - d_conv, pos).  Rows outside
+ *                  [0, seq_len) read as zero.
+ *   real_count     DEVICE int32[1]: slots i < *real_count are written, slots
+ *                  i >= *real_count return at once without touching out.
+ *                  The value is clamped to [0, max_count].  Read on the
+ *                  device, so the count may change between graph replays.
+ *   out            [max_count, conv_dim, d_conv]: out[i][c][k] at
+ *                  i*out_slot_stride + c*d_conv + k.  Must not overlap src.
+ *   d_conv         1..SCONV_MAX_DCONV.
+ * max_count == 0 returns SCONV_OK and enqueues nothing.
+ */
+sconv_status sconv_extract_windows(
+    const void *src, int64_t seq_len, int conv_dim, int64_t src_stride_s,
+    int64_t src_stride_c, const int32_t *abs_positions, const int32_t *real_count,
+    int max_count, void *out, int64_t out_slot_stride, int d_conv, sconv_dtype dt,
+    cudaStream_t stream);
+
+/*
+ * sconv_seq_metadata -- fill the per-token request index and request start
+ * in one launch ("vllm.models.inkling.nvidia.ops.sconv", sconv_seq_metadata).
+ *
+ *   query_start_loc  [num_reqs + 1] int32, non-decreasing, query_start_loc[0] == 0.
+ *   For t < num_actual_tokens:
+ *       seq_idx_out[t]     = the last r < num_reqs with query_start_loc[r] <= t
+ *                            (so an empty request is never chosen);
+ *       query_start_out[t] = query_start_loc[seq_idx_out[t]].
+ *   Rows [num_actual_tokens, num_padded_tokens) are set to 0 (such rows must
+ *   carry slot_mapping == -1 in the sconv_fused call that follows).
+ *   num_padded_tokens < 0 means num_padded_tokens = num_actual_tokens.
+ *   Returns SCONV_ERR_INVALID (and enqueues nothing) if num_padded_tokens <
+ *   num_actual_tokens, or if it exceeds seq_idx_cap or query_start_cap (the
+ *   element capacities of the two output buffers), or if num_reqs < 1 while
+ *   num_actual_tokens > 0.
+ */
+sconv_status sconv_seq_metadata(
+    const int32_t *query_start_loc, int num_reqs, int num_actual_tokens,
+    int num_padded_tokens, int32_t *seq_idx_out, int64_t seq_idx_cap,
+    int32_t *query_start_out, int64_t query_start_cap, cudaStream_t stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *sconv_status_string(sconv_status status);
+
+/* ABI version of this header; bumped on any incompatible change. */
+#define SCONV_ABI_VERSION 1
+int sconv_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SCONV_H */

@@ -54,7 +54,7 @@ def _bind(path: str) -> ctypes.CDLL:
         _P, _P, _P, _P,                        # positions, seq_idx, slot_mapping, query_start
         _P, _I64, _I64, _I64,                  # block_table, bt_row_stride, num_reqs, max_blocks
         _I64, _I64, _INT, _INT,                # off_s, ws, silu, residual
-        _I64, _I64, _P, _P,                    # t_begin, t_end, out_ref, row_state
+        _I64, _I64, _P, _P, _P,                # t_begin, t_end, out_ref, row_state, write_index
     ]
     lib.oracle_seq_metadata.restype = None
     lib.oracle_seq_metadata.argtypes = [_P, _I64, _I64, _I64, _P, _P]
@@ -139,7 +139,7 @@ def to_f64(a, dtype: str) -> np.ndarray:
 
 def fused(*, dtype, x, weight, cache, positions, block_table, seq_idx,
           slot_mapping, query_start, off_s, ws, block_size, activation=None,
-          use_residual=True, t_range=None, write_cache=True):
+          use_residual=True, t_range=None, write_cache=True, write_index=False):
     """Oracle of fused_sconv ("vllm.models.inkling.nvidia.ops.sconv").
 
     ``cache`` is [num_blocks, H, N, D] (any strides in elements, D stride 1
@@ -147,6 +147,8 @@ def fused(*, dtype, x, weight, cache, positions, block_table, seq_idx,
     out_ref float64 [n, C] for the tokens in ``t_range`` (default all),
     row_state uint8 [n] (1 computed, 0 PAD, 2 skipped), cache_out the cache
     after the inserts (a new array) or None when ``write_cache`` is False.
+    With ``write_index`` a fifth value is returned: int64 [n, C], the flat
+    cache element each (token, channel) is inserted at, -1 for none.
     """
     xa = _float_array(x, dtype)
     wa = _float_array(weight, dtype)
@@ -168,6 +170,7 @@ def fused(*, dtype, x, weight, cache, positions, block_table, seq_idx,
     out_ref = np.zeros((n, C), np.float64)
     state = np.zeros(n, np.uint8)
     cache_out = ca.copy() if write_cache else None
+    widx = np.empty((n, C), np.int64) if write_index else None
     strides = np.array([s // ca.itemsize for s in ca.strides], np.int64)
     skipped = lib().oracle_fused(
         _DT[dtype], _ptr(xa), C, T, C, _ptr(wa), W, 1, W,
@@ -175,9 +178,11 @@ def fused(*, dtype, x, weight, cache, positions, block_table, seq_idx,
         _ptr(pos), _ptr(sid), _ptr(slot), _ptr(qs),
         _ptr(bt), bt.shape[1], bt.shape[0], bt.shape[1],
         off_s, ws, int(activation in ("silu", "swish")), int(bool(use_residual)),
-        t0, t1, _ptr(out_ref), _ptr(state))
+        t0, t1, _ptr(out_ref), _ptr(state), _ptr(widx))
     if skipped < 0:
         raise ValueError("oracle_fused: malformed arguments")
+    if write_index:
+        return out_ref, state, cache_out, int(skipped), widx
     return out_ref, state, cache_out, int(skipped)
 
 

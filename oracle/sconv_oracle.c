@@ -22,9 +22,9 @@
  *   - tap orientation: weight[c][W-1] multiplies the current position,
  *     weight[c][0] the oldest one (the causal_conv1d convention that [P4]
  *     names); see TAP_POSITION below.
- *   - a tap is "inside the current forward" when its x row
- *     (t + src - pos) is at or after query_start[t], the first x row of the
- *     token's request ([P1] fused_sconv argument comments).
+ *   - a tap belongs to this step's forward (and is read from x) when its x
+ *     row t + src - pos is at or after query_start[t], the first x row of
+ *     the token's request ([P1] fused_sconv argument comments).
  *   - epilogue order: out = act(conv) + x  (activation on the convolution,
  *     residual added after); see EPILOGUE below.
  *   - PAD rows (slot_mapping == -1) produce no output row and no cache write.
@@ -101,8 +101,11 @@ enum tap_kind { TAP_X = 0, TAP_ZERO = 1, TAP_CACHE = 2 };
  * cache_in).  For every token t in [t_begin, t_end), row t - t_begin of
  * out_ref [t_end - t_begin, C] receives the double-precision result and
  * row_state[t - t_begin] is 1 (computed), 0 (PAD) or 2 (skipped: an index
- * out of range).  Returns the number of skipped tokens, or -1 if an argument
- * is malformed.
+ * out of range).  If write_index is not NULL, write_index[(t - t_begin)*C + c]
+ * receives the flat cache element index that token t's channel c is inserted
+ * at, or -1 when the token writes nothing (a sparse record of the inserts
+ * for caches too large to copy).  Returns the number of skipped tokens, or
+ * -1 if an argument is malformed.
  */
 int64_t oracle_fused(int dtype, const void *x, int64_t x_row_stride, int64_t T,
                      int64_t C, const void *weight, int64_t w_stride_c,
@@ -114,7 +117,8 @@ int64_t oracle_fused(int dtype, const void *x, int64_t x_row_stride, int64_t T,
                      const int32_t *block_table, int64_t bt_row_stride,
                      int64_t num_reqs, int64_t max_blocks, int64_t off_s,
                      int64_t ws, int silu, int residual, int64_t t_begin,
-                     int64_t t_end, double *out_ref, uint8_t *row_state) {
+                     int64_t t_end, double *out_ref, uint8_t *row_state,
+                     int64_t *write_index) {
     if (W < 1 || C != H * ws || off_s < 0 || off_s + ws > D || N < 1 ||
         t_begin < 0 || t_end > T || t_begin > t_end)
         return -1;
@@ -126,8 +130,10 @@ int64_t oracle_fused(int dtype, const void *x, int64_t x_row_stride, int64_t T,
     for (int64_t t = t_begin; t < t_end; ++t) {
         int64_t local = t - t_begin;
         row_state[local] = 0;
+        if (write_index)
+            for (int64_t c = 0; c < C; ++c) write_index[local * C + c] = -1;
         int64_t slot = slot_mapping[t];
-        if (slot == -1) continue; /* PAD: [P1] "PAD = -1 => skip" */
+        if (slot == -1) continue; /* PAD row: no write, no output ([P1]) */
 
         int64_t pos = positions[t];
         int64_t req = seq_idx[t];
@@ -162,12 +168,10 @@ int64_t oracle_fused(int dtype, const void *x, int64_t x_row_stride, int64_t T,
         for (int64_t c = 0; c < C; ++c) {
             int64_t h = c / ws, j = c % ws;
             int64_t x_index = t * x_row_stride + c;
-            if (cache_out) {
-                int64_t dst = (slot / N) * cache_strides[0] + h * cache_strides[1] +
-                              (slot % N) * cache_strides[2] +
-                              (off_s + j) * cache_strides[3];
-                copy_element(cache_out, dst, x, x_index, dtype);
-            }
+            int64_t dst = (slot / N) * cache_strides[0] + h * cache_strides[1] +
+                          (slot % N) * cache_strides[2] + (off_s + j) * cache_strides[3];
+            if (cache_out) copy_element(cache_out, dst, x, x_index, dtype);
+            if (write_index) write_index[local * C + c] = dst;
             double acc = 0.0;
             for (int k = 0; k < W; ++k) {
                 int64_t src = TAP_POSITION(pos, W, k);

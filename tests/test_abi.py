@@ -1,0 +1,149 @@
+"""The C ABI library loads, exports every entry point include/sconv.h
+declares, and rejects malformed arguments on the host (CPU only: no call
+here reaches a kernel launch)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sconv.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from hybrid_sconv_b200 import build
+    build.build()
+    from hybrid_sconv_b200 import binding
+    return binding.LIB
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sconv_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("sconv_fused", "sconv_update", "sconv_extract_windows", "sconv_seq_metadata"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert lib.sconv_abi_version() == 1
+    assert lib.sconv_status_string(0) == b"ok"
+
+
+FAKE = 1 << 20  # a non-null address; validation fails before anything is dereferenced
+
+
+def _strides(*s):
+    return (ctypes.c_int64 * 4)(*s)
+
+
+def _fused(lib, **over):
+    a = dict(x=FAKE, x_rs=8, T=4, C=8, w=FAKE + 4096, w_sc=4, w_sk=1, W=4,
+             cache=FAKE * 64, cs=_strides(512, 256, 16, 1), nb=8, H=2, N=16, D=16,
+             pos=FAKE, sid=FAKE, slot=FAKE, qs=FAKE, bt=FAKE, bt_rs=4, R=2, MB=4,
+             off_s=0, ws=4, act=0, res=1, dt=1, out=FAKE * 512, out_rs=8, err=0, stream=0)
+    a.update(over)
+    return lib.sconv_fused(a["x"], a["x_rs"], a["T"], a["C"], a["w"], a["w_sc"], a["w_sk"],
+                           a["W"], a["cache"], a["cs"], a["nb"], a["H"], a["N"], a["D"],
+                           a["pos"], a["sid"], a["slot"], a["qs"], a["bt"], a["bt_rs"],
+                           a["R"], a["MB"], a["off_s"], a["ws"], a["act"], a["res"], a["dt"],
+                           a["out"], a["out_rs"], a["err"], a["stream"])
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(T=0), 0),
+    (dict(T=-1), 1),
+    (dict(W=0), 1),
+    (dict(W=9), 2),
+    (dict(dt=7), 2),
+    (dict(act=5), 1),
+    (dict(C=6), 1),                      # C != H*ws
+    (dict(off_s=14), 1),                 # off_s + ws > D
+    (dict(cs=_strides(512, 256, 16, 2)), 1),  # D stride must be 1
+    (dict(x_rs=4), 1),                   # row stride < C
+    (dict(out_rs=4), 1),
+    (dict(bt_rs=2), 1),                  # block_table row stride < max_blocks
+    (dict(out=FAKE), 1),                 # out aliases x
+    (dict(out=FAKE * 64 + 64), 1),       # out inside the cache
+    (dict(x=0), 1),
+    (dict(sid=0), 1),
+    (dict(R=0), 1),
+    (dict(nb=0), 1),
+])
+def test_fused_host_validation(lib, over, status):
+    assert _fused(lib, **over) == status
+
+
+def test_update_host_validation(lib):
+    def call(B=4, W=4, dt=1, x=FAKE, out=FAKE * 512):
+        return lib.sconv_update(x, 8, B, 8, FAKE + 4096, 4, 1, W, FAKE * 64,
+                                _strides(512, 256, 16, 1), 8, 2, 16, 16, FAKE, FAKE, FAKE,
+                                4, 4, 0, 4, 0, 1, dt, out, 8, 0, 0)
+    assert call(B=0) == 0
+    assert call(B=-2) == 1
+    assert call(W=12) == 2
+    assert call(dt=3) == 2
+    assert call(out=FAKE) == 1
+
+
+def test_extract_host_validation(lib):
+    def call(max_count=4, d_conv=4, sc=1, out=FAKE * 64, ss=16, dt=1, oss=64, rc=FAKE):
+        return lib.sconv_extract_windows(FAKE, 100, 16, ss, sc, FAKE, rc, max_count, out,
+                                         oss, d_conv, dt, 0)
+    assert call(max_count=0) == 0
+    assert call(max_count=-1) == 1
+    assert call(d_conv=9) == 2
+    assert call(d_conv=0) == 1
+    assert call(sc=2) == 1
+    assert call(ss=8) == 1            # row stride < conv_dim
+    assert call(oss=32) == 1          # slot stride < conv_dim * d_conv
+    assert call(out=FAKE + 64) == 1   # overlaps src
+    assert call(dt=9) == 2
+    assert call(rc=0) == 1
+
+
+def test_seq_metadata_host_validation(lib):
+    def call(R=3, na=7, npad=10, cap_s=10, cap_q=10):
+        return lib.sconv_seq_metadata(FAKE, R, na, npad, FAKE * 2, cap_s, FAKE * 3, cap_q, 0)
+    assert call(na=0, npad=0) == 0
+    assert call(npad=5) == 1           # fewer padded than actual
+    assert call(cap_s=9) == 1
+    assert call(cap_q=9) == 1
+    assert call(R=0) == 1
+    assert call(na=-1) == 1
+
+
+def test_python_binding_size_errors_match_the_page():
+    """sconv_seq_metadata raises ValueError for the size errors the page
+    names before touching a device."""
+    import torch
+    from hybrid_sconv_b200 import sconv_seq_metadata
+    qsl = torch.zeros(4, dtype=torch.int32)
+    small = torch.zeros(3, dtype=torch.int32)
+    big = torch.zeros(10, dtype=torch.int32)
+    with pytest.raises(ValueError, match="cover all actual"):
+        sconv_seq_metadata(qsl, 3, 5, big, big, 4)
+    with pytest.raises(ValueError, match="seq_idx_out is too small"):
+        sconv_seq_metadata(qsl, 3, 5, small, big)
+    with pytest.raises(ValueError, match="query_start_out is too small"):
+        sconv_seq_metadata(qsl, 3, 5, big, small)
+
+
+def test_product_path_does_not_import_the_oracle():
+    """The package's sources never reference the CPU oracle."""
+    pkg = os.path.join(ROOT, "hybrid_sconv_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in text, f

@@ -46,11 +46,11 @@ MUTANTS = [
      "                                  h * cache_strides[1] +\n                                  (src % N)",
      "                                  0 * cache_strides[1] +\n                                  (src % N)"),
     ("insert_offset_div",
-     "                              (slot % N) * cache_strides[2] +",
-     "                              ((slot / N) % N) * cache_strides[2] +"),
+     "(slot % N) * cache_strides[2] + (off_s + j) * cache_strides[3];",
+     "((slot / N) % N) * cache_strides[2] + (off_s + j) * cache_strides[3];"),
     ("insert_lane_ignores_off_s",
-     "                              (off_s + j) * cache_strides[3];",
-     "                              (j) * cache_strides[3];"),
+     "(slot % N) * cache_strides[2] + (off_s + j) * cache_strides[3];",
+     "(slot % N) * cache_strides[2] + (j) * cache_strides[3];"),
     ("weight_taps_reversed",
      "load_value(weight, dtype, c * w_stride_c + k * w_stride_k)",
      "load_value(weight, dtype, c * w_stride_c + (W - 1 - k) * w_stride_k)"),
