@@ -58,6 +58,12 @@ def parse_args():
     p.add_argument("--no-extras", action="store_true",
                    help="skip the per-workload table, e2e and the CPU baseline")
     p.add_argument("--seed", type=int, default=1002)
+    p.add_argument("--only", choices=["chunked_prefill_bf16", "long_prefill_bf16",
+                                      "spec_decode_bf16"],
+                   help="time just this workload's kernels and print its table row")
+    p.add_argument("--max-hist", type=int, default=4096,
+                   help="longest cached history of the decode requests (smaller only for "
+                        "profiling captures; the workload itself uses 4096)")
     return p.parse_args()
 
 
@@ -261,8 +267,9 @@ class DecodeSets:
     cache; each has its own requests, histories, block permutation, x,
     metadata buffers and output."""
 
-    def __init__(self, n, seed, device):
-        self.wls = [workloads.decode_bf16(seed=seed + 7919 * i) for i in range(n)]
+    def __init__(self, n, seed, device, max_hist=4096):
+        self.wls = [workloads.decode_bf16(seed=seed + 7919 * i, max_hist=max_hist)
+                    for i in range(n)]
         self.device = device
         nb = max(w.num_blocks for w in self.wls)
         w0 = self.wls[0]
@@ -284,20 +291,16 @@ class DecodeSets:
             self.sets.append(s)
         self.alg_bytes = [algorithmic_bytes(wl) for wl in self.wls]
 
-    def step(self, i, fused=True, metadata=True, ev=None):
+    def step(self, i, fused=True, metadata=True):
         import hybrid_sconv_b200 as hs
         wl, s = self.wls[i], self.sets[i]
         if metadata:
             hs.sconv_seq_metadata(s["query_start_loc"], wl.R, wl.T, s["seq_idx"],
                                   s["query_start"])
         if fused:
-            if ev is not None:
-                ev[0].record()
             hs.sconv_fused(s["x"], self.weight, self.cache, s["positions"], s["block_table"],
                            s["seq_idx"], s["slot_mapping"], s["query_start"], out=s["out"],
                            **wl.kwargs())
-            if ev is not None:
-                ev[1].record()
 
 
 def run_steps_graphs(sets_obj, K, stream, **step_kw):
@@ -336,91 +339,97 @@ def time_region(full, tail, reps, stream, world, sampler=None):
     return start.elapsed_time(end) / 1e3, (w0, w1)  # seconds
 
 
-def fused_launch_durations(sets_obj, stream, n_sets):
-    """Per-launch durations of the fused kernel inside a graph replay: each
-    launch bracketed by event-record nodes on its stream."""
-    evs = [(torch.cuda.Event(enable_timing=True, external=True),
-            torch.cuda.Event(enable_timing=True, external=True)) for _ in range(n_sets)]
-
-    def body():
-        for i in range(n_sets):
-            sets_obj.step(i, ev=evs[i])
-
-    g = capture(body, stream)
+def fused_launch_duration(sets_obj, stream, reps=200):
+    """Average duration of one fused launch: a graph of the fused launches
+    alone (one per rotating set, metadata already built) replayed `reps`
+    times, timed by CUDA events on the launching stream, divided by the
+    number of launches."""
+    n = len(sets_obj.sets)
+    g = capture(lambda: [sets_obj.step(i, metadata=False) for i in range(n)], stream)
     for _ in range(3):
         g.replay()
     stream.synchronize()
-    durs = []
-    for _ in range(5):
-        g.replay()
-        stream.synchronize()
-        durs += [a.elapsed_time(b) * 1e-3 for a, b in evs]
-    return durs
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        s.record()
+        for _ in range(reps):
+            g.replay()
+        e.record()
+    e.synchronize()
+    del g
+    return s.elapsed_time(e) * 1e-3 / (reps * n)
 
 
 # --------------------------------------------------------------------------
 # other workloads: kernel-only throughput
 
-def per_workload_table(device, stream, peak):
+def _kernel_time(step_fns, reps, stream):
+    """Mean seconds per call of the launches in step_fns, replayed from one
+    CUDA graph and timed with CUDA events on the launching stream."""
+    g = capture(lambda: [f() for f in step_fns], stream)
+    g.replay()
+    stream.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        s.record()
+        for _ in range(reps):
+            g.replay()
+        e.record()
+    e.synchronize()
+    del g
+    return s.elapsed_time(e) * 1e-3 / (reps * len(step_fns))
+
+
+def _entry(wl, secs, nbytes, peak):
+    live = int((wl.slot_mapping != -1).sum())
+    gbs = nbytes / secs / 1e9
+    return {"kernel_us": round(secs * 1e6, 3), "mtokens_s": round(live / secs / 1e6, 2),
+            "alg_bytes": nbytes, "alg_gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
+
+
+def bench_prefill(name, device, stream, peak, reps=None):
+    """One prefill workload (a single set, larger than L2): the fused
+    kernel's throughput; for the long prefill also the window extraction
+    (48 rotating window sets, 48 x 5.2 MB > L2)."""
     import hybrid_sconv_b200 as hs
-    table = {}
+    out_table = {}
+    wl = workloads.NAMED[name]()
+    t = wl.tensors(device)
+    out = torch.empty_like(t["x"])
 
-    def kernel_time(step_fns, reps):
-        g = capture(lambda: [f() for f in step_fns], stream)
-        g.replay()
-        stream.synchronize()
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            s.record()
-            for _ in range(reps):
-                g.replay()
-            e.record()
-        e.synchronize()
-        del g
-        return s.elapsed_time(e) * 1e-3 / (reps * len(step_fns))
-
-    def entry(wl, secs, nbytes):
-        live = int((wl.slot_mapping != -1).sum())
+    def f():
+        hs.sconv_fused(t["x"], t["weight"], t["cache"], t["positions"], t["block_table"],
+                       t["seq_idx"], t["slot_mapping"], t["query_start"], out=out, **wl.kwargs())
+    reps = reps or (20 if name.startswith("long") else 100)
+    out_table[name] = _entry(wl, _kernel_time([f], reps, stream), algorithmic_bytes(wl), peak)
+    if name.startswith("long"):
+        e = wl.extra
+        rng = np.random.default_rng(wl.seed)
+        fns = []
+        rc = torch.tensor([e["real_count"]], dtype=torch.int32, device=device)
+        for _ in range(48):
+            pos = torch.from_numpy(rng.integers(e["d_conv"], wl.T + 1, size=e["max_count"])
+                                   .astype(np.int32)).to(device)
+            o = torch.empty((e["max_count"], wl.C, e["d_conv"]), dtype=torch.bfloat16,
+                            device=device)
+            fns.append(lambda pos=pos, o=o: hs.sconv_extract_windows(
+                t["x"], pos, rc, o, e["d_conv"]))
+        secs = _kernel_time(fns, 50, stream)
+        nbytes = 2 * e["real_count"] * e["d_conv"] * wl.C * wl.elem_bytes + 4 + 4 * e["max_count"]
         gbs = nbytes / secs / 1e9
-        return {"kernel_us": round(secs * 1e6, 3), "mtokens_s": round(live / secs / 1e6, 2),
-                "alg_bytes": nbytes, "alg_gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
+        out_table["extract_windows_long_prefill"] = {
+            "kernel_us": round(secs * 1e6, 3), "alg_bytes": nbytes,
+            "alg_gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
+    del t, out
+    torch.cuda.empty_cache()
+    return out_table
 
-    # chunked mixed prefill and long prefill: one set each, larger than L2
-    for name in ("chunked_prefill_bf16", "long_prefill_bf16"):
-        wl = workloads.NAMED[name]()
-        t = wl.tensors(device)
-        out = torch.empty_like(t["x"])
 
-        def f(wl=wl, t=t, out=out):
-            hs.sconv_fused(t["x"], t["weight"], t["cache"], t["positions"], t["block_table"],
-                           t["seq_idx"], t["slot_mapping"], t["query_start"], out=out,
-                           **wl.kwargs())
-        secs = kernel_time([f], 20 if name.startswith("long") else 100)
-        table[name] = entry(wl, secs, algorithmic_bytes(wl))
-        if name.startswith("long"):
-            e = wl.extra
-            rng = np.random.default_rng(wl.seed)
-            fns = []
-            rc = torch.tensor([e["real_count"]], dtype=torch.int32, device=device)
-            for j in range(48):  # rotate window sets: 48 x 5.2 MB > L2
-                pos = torch.from_numpy(rng.integers(e["d_conv"], wl.T + 1, size=e["max_count"])
-                                       .astype(np.int32)).to(device)
-                o = torch.empty((e["max_count"], wl.C, e["d_conv"]), dtype=torch.bfloat16,
-                                device=device)
-                fns.append(lambda pos=pos, o=o: hs.sconv_extract_windows(
-                    t["x"], pos, rc, o, e["d_conv"]))
-            secs = kernel_time(fns, 50)
-            nbytes = 2 * e["real_count"] * e["d_conv"] * wl.C * wl.elem_bytes + 4 + \
-                4 * e["max_count"]
-            gbs = nbytes / secs / 1e9
-            table["extract_windows_long_prefill"] = {
-                "kernel_us": round(secs * 1e6, 3), "alg_bytes": nbytes,
-                "alg_gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
-        del t, out
-        torch.cuda.empty_cache()
-
-    # speculative decode: rotating sets over one shared cache
-    wls = [workloads.spec_decode_bf16(seed=1004 + 7919 * i) for i in range(40)]
+def bench_spec_decode(device, stream, peak, n_sets=40):
+    """Speculative decode: rotating sets (each 7.5 MB, 40 sets > L2) over one
+    shared cache; the fused kernel's throughput."""
+    import hybrid_sconv_b200 as hs
+    wls = [workloads.spec_decode_bf16(seed=1004 + 7919 * i) for i in range(n_sets)]
     nb = max(w.num_blocks for w in wls)
     w0 = wls[0]
     g = torch.Generator(device=device).manual_seed(1004)
@@ -435,11 +444,19 @@ def per_workload_table(device, stream, peak):
         fns.append(lambda wl=wl, md=md, x=x, out=out: hs.sconv_fused(
             x, weight, cache, md["positions"], md["block_table"], md["seq_idx"],
             md["slot_mapping"], md["query_start"], out=out, **wl.kwargs()))
-    secs = kernel_time(fns, 200)
+    secs = _kernel_time(fns, 200, stream)
     nbytes = int(np.mean([algorithmic_bytes(w) for w in wls]))
-    table["spec_decode_bf16"] = entry(w0, secs, nbytes)
+    res = {"spec_decode_bf16": _entry(w0, secs, nbytes, peak)}
     del cache, fns
     torch.cuda.empty_cache()
+    return res
+
+
+def per_workload_table(device, stream, peak):
+    table = {}
+    table.update(bench_prefill("chunked_prefill_bf16", device, stream, peak))
+    table.update(bench_prefill("long_prefill_bf16", device, stream, peak))
+    table.update(bench_spec_decode(device, stream, peak))
     return table
 
 
@@ -577,11 +594,17 @@ def main():
     device = torch.device("cuda", local)
     stream = torch.cuda.Stream(device)
     peak, peak_kind = measured_hbm_peak()
+    if args.only:
+        if args.only == "spec_decode_bf16":
+            row = bench_spec_decode(device, stream, peak)
+        else:
+            row = bench_prefill(args.only, device, stream, peak, reps=max(3, args.steps))
+        print(json.dumps({"only": args.only, "peak_gbs": peak, "table": row}), flush=True)
+        return
     K, W = args.steps, max(3, args.warmup)
 
-    sets_obj = DecodeSets(args.sets, args.seed + 100003 * rank, device)
+    sets_obj = DecodeSets(args.sets, args.seed + 100003 * rank, device, args.max_hist)
     touched = sum(sets_obj.alg_bytes)
-    assert touched > L2_BYTES, "rotation too small to defeat L2"
 
     # warm-up, then exactly K timed steps
     wfull, wtail, wreps = run_steps_graphs(sets_obj, W, stream)
@@ -610,9 +633,8 @@ def main():
     value = tokens / secs / 1e6
     step_bytes = sum_over_ranks(float(np.mean(sets_obj.alg_bytes)) * K, world)
 
-    # the fused kernel's own launch durations (instrumented replay)
-    durs = fused_launch_durations(sets_obj, stream, len(sets_obj.sets))
-    avg = float(np.mean(durs))
+    # the fused kernel's own average launch duration
+    avg = fused_launch_duration(sets_obj, stream)
     bytes_per_launch = float(np.mean(sets_obj.alg_bytes))
     achieved = bytes_per_launch / avg / 1e9
     traffic = profiled_traffic(HEADLINE)
@@ -622,12 +644,14 @@ def main():
         "steps": K, "warmup": W, "ms_per_step": round(secs / K * 1e3, 6),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded generator; random-normal x, weight and cache)",
-        "config": config_block(world),
+        "config": dict(config_block(world), **({} if touched > L2_BYTES and args.max_hist == 4096
+                                                 else {"l2": "NOT defeated: profiling case",
+                                                       "max_hist": args.max_hist})),
         "hbm_gbs": round(step_bytes / secs / 1e9, 1),
         "gpu_launches": 2 * K,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": traffic, "kernel": "fused_sconv_kernel",
+                     "traffic": traffic, "kernel": "fused_token_kernel (sconv_fused, decode sizes)",
                      "alg_bytes_per_launch": int(bytes_per_launch),
                      "launch_us": round(avg * 1e6, 3),
                      "kernel_source_sha256_16": kernel_source_hash(),

@@ -24,6 +24,7 @@ SCONV_ACT_NONE, SCONV_ACT_SILU = 0, 1
 # err_flag bits (SCONV_EFLAG_* in sconv.h)
 EFLAG_SLOT, EFLAG_REQUEST, EFLAG_LOGICAL = 0x01, 0x02, 0x04
 EFLAG_BLOCK, EFLAG_QUERY_START, EFLAG_POSITION = 0x08, 0x10, 0x20
+EFLAG_TIMEOUT = 0x40
 
 _DTYPES = {torch.float32: SCONV_F32, torch.bfloat16: SCONV_BF16}
 

@@ -69,6 +69,7 @@ sconv_status check_fused(const void *x, int64_t x_rs, int T, int C, const void *
     a.w_sc = w_sc;
     a.w_sk = w_sk;
     a.W = W;
+    a.w_vec = (w_sc == W && w_sk == 1 && aligned16(weight)) ? 1 : 0;
     a.cache = cache;
     a.cs0 = cs[0];
     a.cs1 = cs[1];

@@ -113,6 +113,82 @@ __device__ __forceinline__ float load_weight(const bf16 *p) {
         static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short *>(p))) << 16);
 }
 
+// Unsigned 32-bit division by a divisor fixed for the whole launch, with one
+// multiply-high, a subtract, an add and two shifts: the round-up method of
+// Granlund and Montgomery, "Division by Invariant Integers using
+// Multiplication" (PLDI 1994), exact for every 32-bit dividend.  For d > 1,
+// with l = ceil(log2 d): m = floor(2^32 * (2^l - d) / d) + 1 and
+// q = (t + ((n - t) >> 1)) >> (l - 1), t = mulhi(m, n).  d == 1 uses
+// m = 0 and shifts 0, giving q = n.
+struct FastDiv {
+    uint32_t d, m, s1, s2;
+#ifndef __CUDACC_RTC__
+    __host__ static FastDiv make(uint32_t d) {
+        FastDiv f;
+        f.d = d;
+        if (d <= 1) {
+            f.m = 0;
+            f.s1 = 0;
+            f.s2 = 0;
+            return f;
+        }
+        uint32_t l = 0;
+        while ((1ull << l) < d) ++l;
+        f.m = static_cast<uint32_t>(((1ull << 32) * ((1ull << l) - d)) / d + 1);
+        f.s1 = 1;
+        f.s2 = l - 1;
+        return f;
+    }
+#endif
+    __device__ __forceinline__ uint32_t div(uint32_t n) const {
+        const uint32_t t = __umulhi(m, n);
+        return (t + ((n - t) >> s1)) >> s2;
+    }
+};
+
+// SiLU of the fp32 convolution, one formula per storage type so that every
+// kernel produces the same bits for the same token.  bf16 outputs: y *
+// sigmoid(y) written as h + h * tanh(h) with h = y / 2, one hardware tanh
+// (tanh.approx.f32, relative error near 2^-11, far below bf16's 2^-8
+// rounding step).  fp32 outputs: y / (1 + e^-y) with CUDA's fast exp and
+// divide (about 1e-6 relative).
+template <typename E>
+__device__ __forceinline__ float silu(float y);
+template <>
+__device__ __forceinline__ float silu<bf16>(float y) {
+    const float h = 0.5f * y;
+    float th;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(h));
+    return fmaf(h, th, h);
+}
+template <>
+__device__ __forceinline__ float silu<float>(float y) {
+    return __fdividef(y, 1.f + __expf(-y));
+}
+
+// Two independent fp32 FMAs (d_i = a_i * b_i + d_i, each rounded once) in
+// one packed sm_100 instruction.
+__device__ __forceinline__ void fma2(float &d0, float &d1, float a0, float a1, float b0,
+                                     float b1) {
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%0, %1};\n\t"
+        "fma.rn.f32x2 rc, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rc;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// Programmatic dependent launch (sm_90+): wait for the grids this one
+// depends on to finish and flush their memory, and let the grids that
+// depend on this one begin launching.  Both are no-ops when the launch did
+// not enable programmatic serialization.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Arguments of one fused launch, validated on the host.  Strides in elements.
 struct FusedArgs {
     const void *x;
@@ -121,10 +197,13 @@ struct FusedArgs {
     const void *w;
     int64_t w_sc, w_sk;
     int W;
+    int w_vec;  // 1: weight is [C, W] dense and 16-byte aligned (vector loads)
     void *cache;
     int64_t cs0, cs1, cs2;  // block, head, offset strides (D stride is 1)
     int64_t num_blocks;
     int H, N, D;
+    FastDiv divN;     // division by N for 32-bit positions and slots
+    int slots32;      // num_blocks * N < 2^31: slots divide in 32 bits
     const int64_t *positions;
     const int32_t *seq_idx;  // unused when every token is its own request
     const int64_t *slot;
@@ -137,6 +216,7 @@ struct FusedArgs {
     void *out;
     int64_t out_rs;
     int32_t *err;
+    int strip;        // tokens per thread in the strip kernel
 };
 
 struct ExtractArgs {
@@ -153,10 +233,30 @@ struct ExtractArgs {
 };
 
 // Host-side launchers (return the cudaError_t of the launch).
-cudaError_t launch_fused(const FusedArgs &a, bool bf16_data, bool vec, bool one_token_per_request,
+cudaError_t launch_fused(FusedArgs &a, bool bf16_data, bool vec, bool one_token_per_request,
                          cudaStream_t stream);
+// The TMA-pipelined prefill kernel; sets `used` false (and launches
+// nothing) when the call does not meet its layout requirements.
+cudaError_t launch_fused_tma(const FusedArgs &a, cudaStream_t stream, bool &used);
 cudaError_t launch_extract(const ExtractArgs &a, bool bf16_data, bool vec, cudaStream_t stream);
 cudaError_t launch_seq_metadata(const int32_t *qsl, int num_reqs, int num_actual, int num_padded,
                                 int32_t *seq_idx, int32_t *query_start, cudaStream_t stream);
+
+// Launch with programmatic stream serialization enabled.
+template <typename Kernel, typename... Args>
+inline cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 }  // namespace sconv

@@ -27,6 +27,8 @@ struct Raw<bf16> {
 };
 
 __device__ __forceinline__ int clamped_count(const ExtractArgs &a) {
+    pdl_wait();
+    pdl_trigger();
     int rc = __ldg(a.real_count);
     if (rc < 0) rc = 0;
     if (rc > a.max_count) rc = a.max_count;
@@ -100,21 +102,19 @@ cudaError_t launch_vec(const ExtractArgs &a, cudaStream_t stream) {
     dim3 grid(a.max_count, (nv + threads - 1) / threads);
     switch (a.d_conv) {
 #define SCONV_DC(n) \
-    case n: extract_windows_vec<E, n><<<grid, threads, 0, stream>>>(a); break;
+    case n: return launch_pdl(extract_windows_vec<E, n>, grid, dim3(threads), 0, stream, a);
         SCONV_DC(1) SCONV_DC(2) SCONV_DC(3) SCONV_DC(4)
         SCONV_DC(5) SCONV_DC(6) SCONV_DC(7) SCONV_DC(8)
 #undef SCONV_DC
         default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 template <typename E>
 cudaError_t launch_scalar(const ExtractArgs &a, int64_t src_sc, cudaStream_t stream) {
     const int threads = a.conv_dim >= 256 ? 256 : 64;
     dim3 grid(a.max_count, (a.conv_dim + threads - 1) / threads);
-    extract_windows_scalar<E><<<grid, threads, 0, stream>>>(a, src_sc);
-    return cudaGetLastError();
+    return launch_pdl(extract_windows_scalar<E>, grid, dim3(threads), 0, stream, a, src_sc);
 }
 
 }  // namespace

@@ -2,189 +2,270 @@
 // paged sliding-window cache ("vllm.models.inkling.nvidia.ops.sconv",
 // module docstring and fused_sconv), for sm_100a.
 //
-// Work split.  A thread owns one pack (VEC consecutive channels, one 16-byte
-// transaction) of TPT consecutive tokens.  A block is CV packs wide and TG
-// token groups tall (CV * TG = threads), so the grid is
-// (ceil(T / (TG*TPT)), ceil(C / (VEC*CV))): a function of T and C only, which
-// keeps every launch capturable in a CUDA graph.
+// Per token t (position pos, request r, first x row of the request q0,
+// slot s): a non-PAD token stores its x row into cache[s / N, h, s % N,
+// off_s + j] and convolves, per channel, the W taps ending at pos.  Tap at
+// lag d (position pos - d) is the x row t - d when that row is at or after
+// q0, zero before position 0, else the cache element at block
+// block_table[r, (pos - d) / N], offset (pos - d) % N.  out = act(conv) +
+// (residual ? x : 0), fp32 accumulation from the oldest tap to the newest.
 //
-// Data movement per thread:
-//   * the TPT x rows of its tokens are loaded once, up front, as independent
-//     16-byte loads, and kept in a register window; the W-1 rows before the
-//     tile (the halo) are loaded only when the tile's first token belongs to
-//     a request that began earlier (then every same-forward tap of the tile
-//     is a window register, so each x element is read from DRAM once);
-//   * taps that precede the token's request in x come from the cache via
-//     block_table[request, src / N], or are zero before position 0; they only
-//     occur for the first W-1 tokens of each request in this step;
-//   * each non-PAD token stores its x pack into its cache slot and its
-//     output pack into out -- two 16-byte stores.
-// The tap source (x, cache or zero) depends only on the token, so it is
-// uniform across the lanes of a warp.  Accumulation is fp32, oldest tap first.
+// A thread always owns one 16-byte channel pack (8 bf16 / 4 fp32, or one
+// element for unaligned layouts), so every load and store of x, out and the
+// cache is one 16-byte transaction and a warp covers 512 contiguous bytes of
+// a row.  Two kernels share that layout:
+//
+//  * fused_token_kernel -- one token per thread.  Used when there are few
+//    token-packs (decode, speculative decode): every load of a token
+//    (metadata, x, block-table entries, cache taps) is issued as early as
+//    its address is known, so a token costs three dependent DRAM round
+//    trips (metadata -> block table -> cache) and nothing more.
+//  * fused_strip_kernel -- a strip of L consecutive tokens per thread,
+//    streamed through a register ring: the x row and metadata of token
+//    t + PF are loaded while token t is computed, so loads are always in
+//    flight and each x element is read from DRAM once (the W-1 halo rows
+//    before the strip come from L2).  Used for prefill.
+//
+// The tap source (x, cache, zero) depends only on the token, so it is
+// uniform across a warp.  The grid of either kernel is a function of T and
+// C only, so every launch can be captured in a CUDA graph.  Both kernels
+// start with griddepcontrol.wait (programmatic dependent launch), so they
+// may be launched while the previous kernel in the stream drains.
 #include "common.cuh"
+#include "fused_common.cuh"
 #include "sconv.h"
 
 namespace sconv {
 namespace {
 
-template <typename E, int VEC, int MAXW, int TPT, bool ONE_TOKEN_PER_REQUEST>
-__global__ void __launch_bounds__(256)
-fused_sconv_kernel(const __grid_constant__ FusedArgs a) {
+constexpr int kThreads = 256;
+
+// Convolution, epilogue, output store and cache insert of one token.
+// tap_of(d, use) returns the tap at lag d and sets `use` false for a tap
+// that is zero (before position 0).
+template <typename E, int VEC, int MAXW, typename TapFn>
+__device__ __forceinline__ void conv_store(const FusedArgs &a, const float (&wr)[MAXW][VEC],
+                                           TapFn tap_of, const Pack<E, VEC> &cur, int t, int c,
+                                           int64_t slot, int64_t lane) {
+    float acc[VEC];
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
+#pragma unroll
+    for (int d = MAXW - 1; d >= 0; --d) {
+        if (d >= a.W) continue;
+        bool use = true;
+        const Pack<E, VEC> p = tap_of(d, use);
+        if (!use) continue;
+        float f[VEC];
+        p.to_float(f);
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) acc[v] = fmaf(wr[d][v], f[v], acc[v]);
+    }
+    float xc[VEC];
+    cur.to_float(xc);
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) {
+        float y = acc[v];
+        if (a.silu) y = silu<E>(y);
+        if (a.resid) y += xc[v];
+        acc[v] = y;
+    }
+    Pack<E, VEC> o;
+    o.from_float(acc);
+    o.store(static_cast<E *>(a.out) + static_cast<int64_t>(t) * a.out_rs + c);
+    int64_t blk, off;
+    split_n(a, slot, a.slots32 != 0, blk, off);
+    cur.store(static_cast<E *>(a.cache) + blk * a.cs0 + off * a.cs2 + lane);
+}
+
+template <typename E, int VEC, int MAXW, bool ONE>
+__global__ void __launch_bounds__(kThreads) fused_token_kernel(const __grid_constant__ FusedArgs a) {
     using P = Pack<E, VEC>;
-    const int nv = a.C / VEC;
+    pdl_wait();
+    pdl_trigger();
     const int pack = blockIdx.y * blockDim.x + threadIdx.x;
-    const int tok0 = (blockIdx.x * blockDim.y + threadIdx.y) * TPT;
-    if (pack >= nv || tok0 >= a.T) return;
-
-    const E *__restrict__ x = static_cast<const E *>(a.x);
-    const E *__restrict__ w = static_cast<const E *>(a.w);
-    E *__restrict__ cache = static_cast<E *>(a.cache);
-    E *__restrict__ out = static_cast<E *>(a.out);
-
+    const int t = blockIdx.x * blockDim.y + threadIdx.y;
+    if (pack >= a.C / VEC || t >= a.T) return;
+    const E *x = static_cast<const E *>(a.x);
     const int c = pack * VEC;
     const int h = c / a.ws;
     const int64_t lane = static_cast<int64_t>(h) * a.cs1 + a.off_s + (c - h * a.ws);
-    const int W = a.W;
 
-    // ---- per-token metadata (the same address across a warp's lanes) ----
-    int64_t pos[TPT], slot[TPT];
-    int req[TPT], q0[TPT];
-#pragma unroll
-    for (int i = 0; i < TPT; ++i) {
-        const int t = tok0 + i;
-        if (t < a.T) {
-            pos[i] = __ldg(a.positions + t);
-            slot[i] = __ldg(a.slot + t);
-            if (ONE_TOKEN_PER_REQUEST) {
-                req[i] = t;
-                q0[i] = t;
-            } else {
-                req[i] = __ldg(a.seq_idx + t);
-                q0[i] = __ldg(a.qstart + t);
-            }
-        } else {
-            pos[i] = 0;
-            slot[i] = -1;
-            req[i] = 0;
-            q0[i] = t;
-        }
-    }
-
-    // ---- x window: rows tok0-(MAXW-1) .. tok0+TPT-1 ----
-    P xs[TPT + MAXW - 1];
-#pragma unroll
-    for (int i = 0; i < TPT; ++i) {
-        const int t = tok0 + i;
-        if (t < a.T) xs[MAXW - 1 + i].load_nc(x + static_cast<int64_t>(t) * a.x_rs + c);
-    }
-    if (!ONE_TOKEN_PER_REQUEST) {
-        // Halo rows are same-forward taps only if the tile's first token's
-        // request began before the tile (a later token whose taps reach back
-        // past tok0 belongs to that same request).
-#pragma unroll
-        for (int m = 0; m < MAXW - 1; ++m) {
-            const int row = tok0 - (MAXW - 1) + m;
-            if (m >= MAXW - W && row >= q0[0] && row >= 0)
-                xs[m].load_nc(x + static_cast<int64_t>(row) * a.x_rs + c);
-        }
-    }
-
-    // ---- weights, indexed by lag d = W-1-k (d = 0 is the current token) ----
+    const Tok k = load_tok<ONE>(a, t);
+    P tap[MAXW];
+    tap[0].load_nc(x + static_cast<int64_t>(t) * a.x_rs + c);
     float wr[MAXW][VEC];
+    load_weights<E, VEC, MAXW>(a, c, wr);
+    if (k.slot == -1) return;  // PAD row
+
+    unsigned bad = check_tok<ONE>(a, k, t);
+    bool use[MAXW];
+    use[0] = true;
+    if (!bad) {
 #pragma unroll
-    for (int d = 0; d < MAXW; ++d) {
+        for (int d = 1; d < MAXW; ++d) {
+            use[d] = false;
+            if (d >= a.W) continue;
+            const int64_t src = k.pos - d;
+            if (t - d >= k.q0) {
+                tap[d].load_nc(x + static_cast<int64_t>(t - d) * a.x_rs + c);
+                use[d] = true;
+            } else if (src >= 0) {
+                bad |= load_cache_tap<E, VEC>(a, k.req, src, lane, tap[d]);
+                use[d] = true;
+            }
+        }
+    }
+    if (bad) {
+        if (a.err) atomicOr(a.err, static_cast<int>(bad));
+        return;
+    }
+    conv_store<E, VEC, MAXW>(
+        a, wr,
+        [&](int d, bool &u) {
+            u = use[d];
+            return tap[d];
+        },
+        tap[0], t, c, k.slot, lane);
+}
+
+// Ring of x rows: Q >= PF + MAXW slots, a power of two.
+template <int PF, int MAXW>
+struct Ring {
+    static constexpr int need = PF + MAXW;
+    static constexpr int Q = need <= 8 ? 8 : 16;
+};
+
+// Metadata of a 32-token chunk spread over a warp: lane l holds token
+// chunk_start + l, and each token's fields are broadcast by shuffle when it
+// is processed (one coalesced load per field per 32 tokens).
+struct ChunkMeta {
+    int64_t pos, slot;
+    int req, q0;
+};
+
+__device__ __forceinline__ ChunkMeta load_chunk(const FusedArgs &a, int t, int t_end) {
+    ChunkMeta m;
+    if (t < t_end) {
+        m.pos = __ldg(a.positions + t);
+        m.slot = __ldg(a.slot + t);
+        m.req = __ldg(a.seq_idx + t);
+        m.q0 = __ldg(a.qstart + t);
+    } else {
+        m.pos = 0;
+        m.slot = -1;
+        m.req = 0;
+        m.q0 = 0;
+    }
+    return m;
+}
+
+__device__ __forceinline__ Tok shfl_tok(const ChunkMeta &m, int src) {
+    Tok k;
+    k.pos = __shfl_sync(0xffffffffu, static_cast<long long>(m.pos), src);
+    k.slot = __shfl_sync(0xffffffffu, static_cast<long long>(m.slot), src);
+    k.req = __shfl_sync(0xffffffffu, m.req, src);
+    k.q0 = __shfl_sync(0xffffffffu, m.q0, src);
+    return k;
+}
+
+template <typename E, int VEC, int MAXW, int PF>
+__global__ void __launch_bounds__(kThreads, MAXW <= 4 ? 2 : 1) fused_strip_kernel(const __grid_constant__ FusedArgs a) {
+    using P = Pack<E, VEC>;
+    constexpr int Q = Ring<PF, MAXW>::Q;
+    static_assert(32 % Q == 0, "a metadata chunk holds whole ring turns");
+    pdl_wait();
+    pdl_trigger();
+    const int nv = a.C / VEC;
+    const int t_begin = (blockIdx.x * blockDim.y + threadIdx.y) * a.strip;
+    if (t_begin >= a.T) return;  // uniform across the warp (one strip per warp row)
+    // Lanes past the last channel pack stay in the loop (the metadata
+    // shuffles need the full warp) but load a valid pack and store nothing.
+    const int pack_raw = blockIdx.y * blockDim.x + threadIdx.x;
+    const bool active = pack_raw < nv;
+    const int pack = active ? pack_raw : nv - 1;
+    const int lid = threadIdx.x & 31;
+    const int t_end = t_begin + a.strip < a.T ? t_begin + a.strip : a.T;
+    const E *x = static_cast<const E *>(a.x) + pack * VEC;  // column of this pack
+    const int c = pack * VEC;
+    const int h = c / a.ws;
+    const int64_t lane = static_cast<int64_t>(h) * a.cs1 + a.off_s + (c - h * a.ws);
+
+    P ring[Q];  // ring[(row - t_begin) mod Q] holds x row `row`
 #pragma unroll
-        for (int v = 0; v < VEC; ++v)
-            wr[d][v] = d < W ? load_weight(w + static_cast<int64_t>(c + v) * a.w_sc +
-                                           static_cast<int64_t>(W - 1 - d) * a.w_sk)
-                             : 0.f;
+    for (int j = 0; j < PF; ++j)
+        if (t_begin + j < t_end) ring[j].load_nc(x + static_cast<int64_t>(t_begin + j) * a.x_rs);
+    ChunkMeta cur = load_chunk(a, t_begin + lid, t_end);
+    float wr[MAXW][VEC];
+    load_weights<E, VEC, MAXW>(a, c, wr);
+    // Halo rows before the strip are same-forward taps only if the strip's
+    // first token's request began earlier (a later token reaching back past
+    // t_begin belongs to that same request).
+    const int q0_first = __shfl_sync(0xffffffffu, cur.q0, 0);
+#pragma unroll
+    for (int d = 1; d < MAXW; ++d) {
+        const int row = t_begin - d;
+        if (d < a.W && row >= q0_first && row >= 0)
+            ring[Q - d].load_nc(x + static_cast<int64_t>(row) * a.x_rs);
     }
 
-    const int64_t slots_total = a.num_blocks * a.N;
+    for (int cb = t_begin; cb < t_end; cb += 32) {
+        const ChunkMeta nxt = load_chunk(a, cb + 32 + lid, t_end);
+        const int c_end = cb + 32 < t_end ? cb + 32 : t_end;
+        for (int base = cb; base < c_end; base += Q) {
 #pragma unroll
-    for (int i = 0; i < TPT; ++i) {
-        const int t = tok0 + i;
-        if (t >= a.T) break;
-        const int64_t s = slot[i];
-        if (s == -1) continue;  // PAD row: no insert, no output
+            for (int j = 0; j < Q; ++j) {
+                const int t = base + j;
+                if (t >= c_end) break;
+                const Tok k = shfl_tok(cur, t - cb);
+                const int tn = t + PF;  // prefetch the x row PF tokens ahead
+                if (tn < t_end) ring[(j + PF) % Q].load_nc(x + static_cast<int64_t>(tn) * a.x_rs);
+                if (k.slot == -1) continue;  // PAD row
 
-        unsigned bad = 0;
-        if (s < 0 || s >= slots_total) bad |= SCONV_EFLAG_SLOT;
-        if (!ONE_TOKEN_PER_REQUEST) {
-            if (req[i] < 0 || req[i] >= a.num_reqs) bad |= SCONV_EFLAG_REQUEST;
-            if (q0[i] < 0 || q0[i] > t) bad |= SCONV_EFLAG_QUERY_START;
-        }
-        if (pos[i] < 0) bad |= SCONV_EFLAG_POSITION;
-
-        // Pre-forward taps (lag d with row t-d before the request's first row).
-        P ct[MAXW];
-        if (!bad && t - q0[i] < W - 1) {
-            const int32_t *bt_row = a.bt + static_cast<int64_t>(req[i]) * a.bt_rs;
-#pragma unroll
-            for (int d = 1; d < MAXW; ++d) {
-                const int64_t src = pos[i] - d;
-                if (d < W && t - d < q0[i] && src >= 0) {
-                    const int64_t lb = src / a.N;
-                    if (lb >= a.max_blocks) {
-                        bad |= SCONV_EFLAG_LOGICAL;
-                        continue;
-                    }
-                    const int32_t b = __ldg(bt_row + lb);
-                    if (b < 0 || b >= a.num_blocks) {
-                        bad |= SCONV_EFLAG_BLOCK;
-                        continue;
-                    }
-                    ct[d].load_nc(cache + static_cast<int64_t>(b) * a.cs0 +
-                                  (src - lb * a.N) * a.cs2 + lane);
+                unsigned bad = check_tok<false>(a, k, t);
+                if (!bad && t - k.q0 >= a.W - 1) {
+                    // Every tap is an x row of this step, already in the ring.
+                    if (active)
+                        conv_store<E, VEC, MAXW>(
+                            a, wr,
+                            [&](int d, bool &u) {
+                                u = true;
+                                return ring[(j - d + Q) % Q];
+                            },
+                            ring[j], t, c, k.slot, lane);
+                    continue;
                 }
+                // The first W-1 tokens of a request: earlier taps from the
+                // cache (or zero before position 0).
+                P ct[MAXW];
+                bool from_x[MAXW], use[MAXW];
+#pragma unroll
+                for (int d = 1; d < MAXW; ++d) {
+                    from_x[d] = t - d >= k.q0;
+                    use[d] = from_x[d] || k.pos - d >= 0;
+                    if (d < a.W && !from_x[d] && k.pos - d >= 0 && !bad)
+                        bad |= load_cache_tap<E, VEC>(a, k.req, k.pos - d, lane, ct[d]);
+                }
+                if (bad) {
+                    if (a.err && active) atomicOr(a.err, static_cast<int>(bad));
+                    continue;
+                }
+                if (active)
+                    conv_store<E, VEC, MAXW>(
+                        a, wr,
+                        [&](int d, bool &u) {
+                            u = d == 0 || use[d];
+                            return (d == 0 || from_x[d]) ? ring[(j - d + Q) % Q] : ct[d];
+                        },
+                        ring[j], t, c, k.slot, lane);
             }
         }
-        if (bad) {
-            if (a.err) atomicOr(a.err, static_cast<int>(bad));
-            continue;
-        }
-
-        float acc[VEC];
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
-#pragma unroll
-        for (int d = MAXW - 1; d >= 0; --d) {
-            if (d >= W) continue;
-            float f[VEC];
-            if (t - d >= q0[i]) {
-                xs[MAXW - 1 + i - d].to_float(f);
-            } else if (pos[i] - d < 0) {
-#pragma unroll
-                for (int v = 0; v < VEC; ++v) f[v] = 0.f;
-            } else {
-                ct[d].to_float(f);
-            }
-#pragma unroll
-            for (int v = 0; v < VEC; ++v) acc[v] = fmaf(wr[d][v], f[v], acc[v]);
-        }
-
-        float xc[VEC];
-        xs[MAXW - 1 + i].to_float(xc);
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) {
-            float y = acc[v];
-            if (a.silu) y = y / (1.f + expf(-y));
-            if (a.resid) y += xc[v];
-            acc[v] = y;
-        }
-        P o;
-        o.from_float(acc);
-        o.store(out + static_cast<int64_t>(t) * a.out_rs + c);
-
-        const int64_t blk = s / a.N;
-        xs[MAXW - 1 + i].store(cache + blk * a.cs0 + (s - blk * a.N) * a.cs2 + lane);
+        cur = nxt;
     }
 }
 
-// Host-side choice of the tile: threads along channels (CV) and tokens per
-// thread (TPT) from T and C only.
-struct Tile {
-    int cv, tg, tpt;
+struct Shape {
+    int cv, tg;  // threads along channel packs, token rows (or strips) per block
 };
 
 inline int next_pow2(int v) {
@@ -193,71 +274,75 @@ inline int next_pow2(int v) {
     return p;
 }
 
-Tile choose_tile(int T, int nv, int maxw, bool one_token_per_request) {
-    Tile tl;
-    tl.cv = next_pow2(nv);
-    if (tl.cv < 32) tl.cv = 32;
-    if (tl.cv > 256) tl.cv = 256;
-    // Many token-packs: give each thread several tokens so halo rows and
-    // per-token addressing are amortised; few: one token per thread so the
-    // grid still covers every SM.
-    const int64_t work = static_cast<int64_t>(T) * nv;
-    const int64_t fill = 148LL * 2048;  // threads resident on a full B200
-    if (one_token_per_request) {
-        tl.tpt = 1;
-    } else if (work >= 8 * fill) {
-        tl.tpt = maxw <= 4 ? 8 : 4;
-    } else if (work >= 4 * fill) {
-        tl.tpt = 4;
-    } else {
-        tl.tpt = 1;
-    }
-    // Small grids: narrower blocks so more SMs get work.
-    int threads = 256;
-    const int64_t packs_per_block_row = tl.cv;
-    const int64_t blocks_256 =
-        ((T + (256 / tl.cv) * tl.tpt - 1) / ((256 / tl.cv) * tl.tpt)) *
-        ((nv + packs_per_block_row - 1) / packs_per_block_row);
-    if (blocks_256 < 2 * 148 && tl.cv <= 128) threads = 128;
-    if (threads < tl.cv) threads = tl.cv;
-    tl.tg = threads / tl.cv;
-    return tl;
+inline Shape block_shape(int nv, int64_t rows) {
+    Shape s;
+    s.cv = next_pow2(nv);
+    if (s.cv < 32) s.cv = 32;
+    if (s.cv > kThreads) s.cv = kThreads;
+    int threads = kThreads;
+    // Few rows: narrower blocks so more SMs get work.
+    const int64_t blocks = ((rows + kThreads / s.cv - 1) / (kThreads / s.cv)) *
+                           ((nv + s.cv - 1) / s.cv);
+    if (blocks < 2 * 148 && s.cv <= 128) threads = 128;
+    if (threads < s.cv) threads = s.cv;
+    s.tg = threads / s.cv;
+    return s;
 }
 
-template <typename E, int VEC, int MAXW, int TPT, bool ONE>
-cudaError_t launch_t(const FusedArgs &a, const Tile &tl, cudaStream_t stream) {
-    const int nv = a.C / VEC;
-    dim3 block(tl.cv, tl.tg);
-    const int64_t tokens_per_block = static_cast<int64_t>(tl.tg) * TPT;
-    dim3 grid(static_cast<unsigned>((a.T + tokens_per_block - 1) / tokens_per_block),
-              static_cast<unsigned>((nv + tl.cv - 1) / tl.cv));
-    fused_sconv_kernel<E, VEC, MAXW, TPT, ONE><<<grid, block, 0, stream>>>(a);
-    return cudaGetLastError();
-}
+// Strip kernel only when there is enough work to stream: T*C/VEC
+// token-packs above this many.
+constexpr int64_t kStripMinWork = 1 << 19;
+constexpr int kPF = 4;
 
 template <typename E, int VEC, int MAXW>
-cudaError_t launch_w(const FusedArgs &a, bool one, cudaStream_t stream) {
-    const Tile tl = choose_tile(a.T, a.C / VEC, MAXW, one);
-    if (one) return launch_t<E, VEC, MAXW, 1, true>(a, tl, stream);
-    switch (tl.tpt) {
-        case 8:
-            if constexpr (MAXW <= 4) return launch_t<E, VEC, MAXW, 8, false>(a, tl, stream);
-            else return launch_t<E, VEC, MAXW, 4, false>(a, tl, stream);
-        case 4: return launch_t<E, VEC, MAXW, 4, false>(a, tl, stream);
-        default: return launch_t<E, VEC, MAXW, 1, false>(a, tl, stream);
+cudaError_t launch_w(FusedArgs &a, bool one, cudaStream_t stream) {
+    const int nv = a.C / VEC;
+    const int64_t work = static_cast<int64_t>(a.T) * nv;
+    if (one || work < kStripMinWork || a.T < 64) {
+        const Shape s = block_shape(nv, a.T);
+        dim3 grid(static_cast<unsigned>((a.T + s.tg - 1) / s.tg),
+                  static_cast<unsigned>((nv + s.cv - 1) / s.cv));
+        if (one)
+            return launch_pdl(fused_token_kernel<E, VEC, MAXW, true>, grid, dim3(s.cv, s.tg), 0,
+                              stream, a);
+        return launch_pdl(fused_token_kernel<E, VEC, MAXW, false>, grid, dim3(s.cv, s.tg), 0,
+                          stream, a);
     }
+    if constexpr (sizeof(E) == 2 && VEC == 8) {
+        bool used = false;
+        const cudaError_t e = launch_fused_tma(a, stream, used);
+        if (used || e != cudaSuccess) return e;
+    }
+    // Strip length: a whole number of 32-token metadata chunks, the longest
+    // (up to 128 tokens) that still leaves about four waves of 256-thread
+    // blocks on 148 SMs.
+    int strip = 128;
+    while (strip > 32 && (static_cast<int64_t>((a.T + strip - 1) / strip) * nv) < 4 * 148 * 2 * 256)
+        strip /= 2;
+    a.strip = strip;
+    const int64_t strips = (a.T + strip - 1) / strip;
+    const Shape s = block_shape(nv, strips);
+    dim3 grid(static_cast<unsigned>((strips + s.tg - 1) / s.tg),
+              static_cast<unsigned>((nv + s.cv - 1) / s.cv));
+    return launch_pdl(fused_strip_kernel<E, VEC, MAXW, kPF>, grid, dim3(s.cv, s.tg), 0, stream, a);
 }
 
 template <typename E, int VEC>
-cudaError_t launch_v(const FusedArgs &a, bool one, cudaStream_t stream) {
-    if (a.W <= 4) return launch_w<E, VEC, 4>(a, one, stream);
+cudaError_t launch_v(FusedArgs &a, bool one, cudaStream_t stream) {
+    if (a.W <= 4) {
+        a.w_vec = a.w_vec && a.W == 4;
+        return launch_w<E, VEC, 4>(a, one, stream);
+    }
+    a.w_vec = a.w_vec && a.W == 8;
     return launch_w<E, VEC, 8>(a, one, stream);
 }
 
 }  // namespace
 
-cudaError_t launch_fused(const FusedArgs &a, bool bf16_data, bool vec, bool one,
-                         cudaStream_t stream) {
+cudaError_t launch_fused(FusedArgs &a, bool bf16_data, bool vec, bool one, cudaStream_t stream) {
+    a.divN = FastDiv::make(static_cast<uint32_t>(a.N));
+    a.slots32 = a.num_blocks * a.N < (1ll << 31);
+    a.strip = 1;
     if (bf16_data) {
         return vec ? launch_v<bf16, 8>(a, one, stream) : launch_v<bf16, 1>(a, one, stream);
     }

@@ -18,6 +18,8 @@ seq_metadata_kernel(const int32_t *__restrict__ qsl, int num_reqs, int num_actua
                     int num_padded, int32_t *__restrict__ seq_idx,
                     int32_t *__restrict__ query_start, int staged) {
     extern __shared__ int32_t s_qsl[];
+    pdl_wait();
+    pdl_trigger();
     if (staged) {
         for (int i = threadIdx.x; i < num_reqs; i += blockDim.x) s_qsl[i] = __ldg(qsl + i);
         __syncthreads();
@@ -51,9 +53,8 @@ cudaError_t launch_seq_metadata(const int32_t *qsl, int num_reqs, int num_actual
     const int staged = nr <= kSmemReqs ? 1 : 0;
     const size_t smem = staged ? static_cast<size_t>(nr) * sizeof(int32_t) : 0;
     const int blocks = (num_padded + kThreads - 1) / kThreads;
-    seq_metadata_kernel<<<blocks, kThreads, smem, stream>>>(qsl, nr, num_actual, num_padded,
-                                                            seq_idx, query_start, staged);
-    return cudaGetLastError();
+    return launch_pdl(seq_metadata_kernel, dim3(blocks), dim3(kThreads), smem, stream, qsl, nr,
+                      num_actual, num_padded, seq_idx, query_start, staged);
 }
 
 }  // namespace sconv

@@ -77,6 +77,8 @@ typedef enum sconv_act { SCONV_ACT_NONE = 0, SCONV_ACT_SILU = 1 } sconv_act;
 #define SCONV_EFLAG_BLOCK       0x08u /* block_table entry outside [0, num_blocks) */
 #define SCONV_EFLAG_QUERY_START 0x10u /* query_start[t] outside [0, t] */
 #define SCONV_EFLAG_POSITION    0x20u /* positions[t] < 0 */
+#define SCONV_EFLAG_TIMEOUT     0x40u /* a block's bulk copies did not arrive within its bounded
+                                         wait; that block wrote nothing further and returned */
 
 #define SCONV_MAX_W 8      /* taps supported by sconv_fused / sconv_update */
 #define SCONV_MAX_DCONV 8  /* window length supported by sconv_extract_windows */

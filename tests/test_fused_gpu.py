@@ -26,7 +26,7 @@ def test_random_small_cases(seed):
 
 @pytest.mark.parametrize("seed,dtype,ws,H,max_new", [
     (1, "bf16", 128, 32, 900),    # C = 4096, several tiles per request
-    (2, "bf16", 72, 9, 2500),     # C = 648: a ragged channel tail
+    (2, "bf16", 72, 9, 6000),     # C = 648: a ragged channel tail (TMA tiles past C)
     (3, "f32", 64, 16, 1500),     # fp32, 4-wide packs
     (4, "bf16", 32, 32, 3000),    # many token-packs: the 8-tokens-per-thread tile
     (5, "bf16", 8, 3, 400),       # C = 24: narrow blocks
@@ -49,6 +49,44 @@ def test_every_window_length(W, dtype):
     wl = workloads.build(f"w{W}", dtype=dtype, H=4, D=64, ws=32, off_s=16, W=W, N=4,
                          hist=rng.integers(0, 12, size=6), new=rng.integers(1, 300, size=6),
                          act="silu", residual=True, seed=W, num_pad=5, rng=rng)
+    check_small(wl, DEV)
+
+
+@pytest.mark.parametrize("W", range(1, 9))
+def test_strip_kernel_every_window_length(W):
+    """Enough token-packs (T*C/8 >= 2^19) for the streamed strip kernel,
+    with request starts, histories and PAD rows inside strips."""
+    rng = np.random.default_rng(100 + W)
+    wl = workloads.build(f"strip_w{W}", dtype="bf16", H=16, D=136, ws=128, off_s=8, W=W, N=16,
+                         hist=rng.integers(0, 30, size=4), new=rng.integers(600, 900, size=4),
+                         act="silu", residual=bool(W % 2), seed=W, num_pad=9, rng=rng)
+    assert wl.T * wl.C // 8 >= 1 << 19
+    check_small(wl, DEV)
+
+
+def test_unaligned_metadata_takes_the_strip_kernel():
+    """Metadata arrays that start 8 bytes past a 16-byte boundary cannot be
+    bulk-copied; the streamed strip kernel serves the same step."""
+    rng = np.random.default_rng(11)
+    wl = workloads.build("strip_unaligned", dtype="bf16", H=16, D=128, ws=128, off_s=0, W=4,
+                         N=16, hist=rng.integers(0, 30, size=4), new=rng.integers(600, 900, size=4),
+                         act="silu", residual=True, seed=11, num_pad=5, rng=rng)
+    t = wl.tensors(DEV)
+    for k in ("positions", "slot_mapping"):
+        buf = torch.empty(wl.T + 1, dtype=torch.int64, device=DEV)
+        buf[1:].copy_(t[k])
+        t[k] = buf[1:]
+    check_small(wl, DEV, t=t)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_strip_kernel_element_path(dtype):
+    """The strip kernel on a layout that is not 16-byte aligned (ws = 5)."""
+    rng = np.random.default_rng(7)
+    wl = workloads.build("strip_elem", dtype=dtype, H=100, D=10, ws=5, off_s=3, W=4, N=8,
+                         hist=rng.integers(0, 20, size=3), new=rng.integers(500, 600, size=3),
+                         act="silu", residual=True, seed=7, num_pad=4, rng=rng)
+    assert wl.T * wl.C >= 1 << 19
     check_small(wl, DEV)
 
 
