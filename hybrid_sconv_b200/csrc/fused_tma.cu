@@ -10,19 +10,24 @@
 //     and channels past C arrive as zeros), and
 //   * four 1-D tensor copies of the tile's positions, slot_mapping, seq_idx
 //     and query_start,
-// all completing on one mbarrier.  Tiles flow through a kStages-deep ring of
-// shared-memory stages, so up to kStages-1 tiles are in flight while one is
+// all completing on one mbarrier.  Tiles flow through a ring of STAGES
+// shared-memory stages, so up to STAGES-1 tiles are in flight while one is
 // computed: the memory system sees a steady stream of bulk copies whatever
-// the register budget of the compute threads.
+// the register budget of the compute threads.  The grid is persistent: one
+// block per resident slot (SMs x blocks per SM), each taking an equal
+// contiguous share of the (channel block, tile) units, so there is no
+// partial last wave.
 //
 // Compute.  Eight warps per block; warp g owns tokens 4g..4g+3 of the tile
-// and lane l the 16-byte pack of channels c0 + 8l .. c0 + 8l + 7.  A thread
-// reads the W+3 rows its four tokens need once from shared memory (16-byte
-// loads, conflict-free: a warp reads one contiguous 512-byte row), and per
-// token convolves, applies the epilogue and stores its output pack and its
-// cache insert straight to global memory.  Taps that precede the token's
-// request come from the cache through the block table (the first W-1
-// tokens of each request only).
+// and lane l the 16-byte pack of channels c0 + 8l .. c0 + 8l + 7.  Lanes
+// 0..3 classify the warp's four tokens (ordinary, PAD, or needing cache
+// taps / out of range) and compute their cache insert offsets once; when all
+// four are ordinary -- nearly always in prefill -- one straight-line block
+// convolves them from the W+3 shared-memory rows they need (16-byte loads,
+// conflict-free: a warp reads one contiguous 512-byte row).  Otherwise each
+// token takes the general path, where taps that precede the token's request
+// come from the cache through the block table.  Outputs and cache inserts
+// are 16-byte stores straight to global memory.
 //
 // Every wait on an mbarrier is bounded; a block whose copies do not arrive
 // in time sets SCONV_EFLAG_TIMEOUT, waits (bounded) for its other copies and
@@ -42,7 +47,6 @@ namespace {
 
 constexpr int kBC = 256;           // channels per tile
 constexpr int kBT = 32;            // tokens per tile
-constexpr int kStages = 4;         // shared-memory ring depth
 constexpr int kThreads = 256;      // 8 warps
 constexpr int kTokPerWarp = kBT / (kThreads / 32);  // 4
 constexpr int kMetaBytes = kBT * (8 + 8 + 4 + 4);   // positions, slots, seq_idx, query_start
@@ -53,8 +57,12 @@ struct Layout {
     static constexpr int rows = kBT + W - 1;
     static constexpr int x_bytes = rows * kBC * 2;  // multiple of 512: TMA destinations stay 128-B aligned
     static constexpr int stage = x_bytes + kMetaBytes;
-    static constexpr int smem = kStages * stage + kStages * 8;
 };
+
+template <int W, int STAGES>
+constexpr int kStages_smem() {
+    return STAGES * Layout<W>::stage + STAGES * 8;
+}
 
 struct TmaMaps {
     CUtensorMap x, pos, slot, sid, qs;
@@ -121,23 +129,28 @@ __device__ __forceinline__ void fma_pack(float (&acc)[8], const float (&w)[8], c
              __uint_as_float(q[i] & 0xffff0000u));
 }
 
-template <int W>
-__global__ void __launch_bounds__(kThreads, 2)
+// What a warp's lane u (< kTokPerWarp) knows about token u of its group.
+enum : int { kSkip = 0, kFast = 1, kSlow = 2 };
+
+template <int W, int STAGES, bool SILU, bool RESID>
+__global__ void __launch_bounds__(kThreads, STAGES <= 3 ? 3 : 2)
 fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ TmaMaps maps,
-                 int tiles_per_block) {
+                 int64_t units) {
     using L = Layout<W>;
     extern __shared__ __align__(128) unsigned char smem[];
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * L::stage);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * L::stage);
 
+    // Work units are (channel block, tile) pairs, channel-block major; this
+    // block takes an equal contiguous share of them.
     const int ntiles = (a.T + kBT - 1) / kBT;
-    const int tile0 = blockIdx.x * tiles_per_block;
-    const int my = min(tiles_per_block, ntiles - tile0);
+    const int64_t u_begin = units * blockIdx.x / gridDim.x;
+    const int64_t u_end = units * (blockIdx.x + 1) / gridDim.x;
+    const int my = static_cast<int>(u_end - u_begin);
     if (my <= 0) return;  // whole block
-    const int c0 = blockIdx.y * kBC;
 
     if (threadIdx.x == 0) {
 #pragma unroll
-        for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
@@ -145,9 +158,11 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
     pdl_trigger();
 
     auto issue = [&](int k) {
-        const int s = k % kStages;
+        const int s = k % STAGES;
         unsigned char *st = smem + s * L::stage;
-        const int t0 = (tile0 + k) * kBT;
+        const int64_t u = u_begin + k;
+        const int c0 = static_cast<int>(u / ntiles) * kBC;
+        const int t0 = static_cast<int>(u % ntiles) * kBT;
         mbar_expect_tx(&full[s], L::stage);
         tma_2d(st, &maps.x, c0, t0 - (W - 1), &full[s]);
         tma_1d(st + L::x_bytes, &maps.pos, t0, &full[s]);
@@ -156,28 +171,39 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
         tma_1d(st + L::x_bytes + kBT * 20, &maps.qs, t0, &full[s]);
     };
     if (threadIdx.x == 0)
-        for (int k = 0; k < kStages && k < my; ++k) issue(k);
+        for (int k = 0; k < STAGES && k < my; ++k) issue(k);
 
     const int lane_id = threadIdx.x & 31;
-    const int grp = threadIdx.x >> 5;
+    const int i0 = (threadIdx.x >> 5) * kTokPerWarp;
     const int nv = a.C / 8;
-    const int pack_raw = c0 / 8 + lane_id;
-    const bool active = pack_raw < nv;
-    const int c = (active ? pack_raw : nv - 1) * 8;
-    const int h = c / a.ws;
-    const int64_t lane = static_cast<int64_t>(h) * a.cs1 + a.off_s + (c - h * a.ws);
+    const int64_t slots_total = a.num_blocks * a.N;
+    int cur_cb = -1;
+    bool active = false;
+    int c = 0;
+    int64_t lane = 0;
     float wr[4][8];
-    load_weights<bf16, 8, 4>(a, c, wr);
 
     for (int k = 0; k < my; ++k) {
-        const int s = k % kStages;
-        const bool ok = mbar_wait(&full[s], (k / kStages) & 1);
+        const int s = k % STAGES;
+        const int64_t u = u_begin + k;
+        const int cb = static_cast<int>(u / ntiles);
+        const int t0 = static_cast<int>(u % ntiles) * kBT;
+        if (cb != cur_cb) {  // entering a new channel block: its taps and cache lanes
+            cur_cb = cb;
+            const int pack_raw = cb * (kBC / 8) + lane_id;
+            active = pack_raw < nv;
+            c = (active ? pack_raw : nv - 1) * 8;
+            const int h = c / a.ws;
+            lane = static_cast<int64_t>(h) * a.cs1 + a.off_s + (c - h * a.ws);
+            load_weights<bf16, 8, 4>(a, c, wr);
+        }
+        const bool ok = mbar_wait(&full[s], (k / STAGES) & 1);
         if (__syncthreads_or(!ok)) {
             // Copies did not arrive: report, let the others land, stop.
             if (threadIdx.x == 0) {
                 if (a.err) atomicOr(a.err, static_cast<int>(SCONV_EFLAG_TIMEOUT));
-                for (int j = k; j < my && j < k + kStages; ++j)
-                    mbar_wait(&full[j % kStages], (j / kStages) & 1);
+                for (int j = k; j < my && j < k + STAGES; ++j)
+                    mbar_wait(&full[j % STAGES], (j / STAGES) & 1);
             }
             __syncthreads();
             return;
@@ -188,8 +214,29 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
         const int64_t *mslot = mpos + kBT;
         const int32_t *msid = reinterpret_cast<const int32_t *>(st + L::x_bytes + kBT * 16);
         const int32_t *mqs = msid + kBT;
-        const int t0 = (tile0 + k) * kBT;
-        const int i0 = grp * kTokPerWarp;
+
+        // Lanes 0..3 classify the group's tokens and address their inserts.
+        int code = kSkip;
+        int64_t ins = 0;
+        if (lane_id < kTokPerWarp) {
+            const int i = i0 + lane_id;
+            const int t = t0 + i;
+            const int64_t slot = mslot[i];
+            if (t < a.T && slot != -1) {
+                const int64_t pos = mpos[i];
+                const int req = msid[i];
+                const int q0 = mqs[i];
+                const bool bad = slot < 0 || slot >= slots_total || req < 0 ||
+                                 req >= a.num_reqs || q0 < 0 || q0 > t || pos < 0;
+                code = (!bad && t - q0 >= W - 1) ? kFast : kSlow;
+                if (!bad) {
+                    int64_t blk, off;
+                    split_n(a, slot, a.slots32 != 0, blk, off);
+                    ins = blk * a.cs0 + off * a.cs2;
+                }
+            }
+        }
+        const unsigned fast_mask = __ballot_sync(0xffffffffu, code == kFast);
 
         // Shared-memory row r holds x row t0 - (W-1) + r; token i at lag d
         // reads row i + (W-1) - d.
@@ -197,68 +244,96 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
 #pragma unroll
         for (int r = 0; r < kTokPerWarp + W - 1; ++r) rows[r] = xs[(i0 + r) * 32];
 
+        bf16 *out = static_cast<bf16 *>(a.out);
+        bf16 *cache = static_cast<bf16 *>(a.cache);
+        if ((fast_mask & 0xfu) == 0xfu) {
+            // The common case: four ordinary tokens, straight-line code.
 #pragma unroll
-        for (int u = 0; u < kTokPerWarp; ++u) {
-            const int i = i0 + u;
-            const int t = t0 + i;
-            if (t >= a.T) break;
-            const int64_t slot = mslot[i];
-            if (slot == -1) continue;  // PAD row
-            const int64_t pos = mpos[i];
-            const int req = msid[i];
-            const int q0 = mqs[i];
-            unsigned bad = 0;
-            if (slot < 0 || slot >= a.num_blocks * a.N) bad |= SCONV_EFLAG_SLOT;
-            if (req < 0 || req >= a.num_reqs) bad |= SCONV_EFLAG_REQUEST;
-            if (q0 < 0 || q0 > t) bad |= SCONV_EFLAG_QUERY_START;
-            if (pos < 0) bad |= SCONV_EFLAG_POSITION;
-
-            float acc[8];
+            for (int uu = 0; uu < kTokPerWarp; ++uu) {
+                float acc[8];
 #pragma unroll
-            for (int v = 0; v < 8; ++v) acc[v] = 0.f;
-            if (!bad && t - q0 >= W - 1) {
-                // Every tap is an x row of this step, in shared memory.
+                for (int v = 0; v < 8; ++v) acc[v] = 0.f;
 #pragma unroll
-                for (int d = W - 1; d >= 0; --d) fma_pack(acc, wr[d], rows[u + W - 1 - d]);
-            } else {
-                // First W-1 tokens of a request: earlier taps from the cache
-                // (zero before position 0).
-                P ct[W];
+                for (int d = W - 1; d >= 0; --d) fma_pack(acc, wr[d], rows[uu + W - 1 - d]);
+                const int64_t ins_u = __shfl_sync(0xffffffffu, ins, uu);
+                float xc[8];
+                rows[uu + W - 1].to_float(xc);
 #pragma unroll
-                for (int d = 1; d < W; ++d)
-                    if (t - d < q0 && pos - d >= 0 && !bad)
-                        bad |= load_cache_tap<bf16, 8>(a, req, pos - d, lane, ct[d]);
-                if (bad) {
-                    if (a.err && active) atomicOr(a.err, static_cast<int>(bad));
-                    continue;
+                for (int v = 0; v < 8; ++v) {
+                    float y = acc[v];
+                    if (SILU) y = silu<bf16>(y);
+                    if (RESID) y += xc[v];
+                    acc[v] = y;
                 }
-#pragma unroll
-                for (int d = W - 1; d >= 0; --d) {
-                    if (d == 0 || t - d >= q0)
-                        fma_pack(acc, wr[d], rows[u + W - 1 - d]);
-                    else if (pos - d >= 0)
-                        fma_pack(acc, wr[d], ct[d]);
+                P o;
+                o.from_float(acc);
+                if (active) {
+                    o.store(out + static_cast<int64_t>(t0 + i0 + uu) * a.out_rs + c);
+                    rows[uu + W - 1].store(cache + ins_u + lane);
                 }
             }
-            if (!active) continue;
-            float xc[8];
-            rows[u + W - 1].to_float(xc);
+        } else {
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-                float y = acc[v];
-                if (a.silu) y = silu<bf16>(y);
-                if (a.resid) y += xc[v];
-                acc[v] = y;
+            for (int uu = 0; uu < kTokPerWarp; ++uu) {
+                const int code_u = __shfl_sync(0xffffffffu, code, uu);
+                const int64_t ins_u = __shfl_sync(0xffffffffu, ins, uu);
+                if (code_u == kSkip) continue;  // PAD row or past T
+                const int i = i0 + uu;
+                const int t = t0 + i;
+                float acc[8];
+#pragma unroll
+                for (int v = 0; v < 8; ++v) acc[v] = 0.f;
+                if (code_u == kFast) {
+#pragma unroll
+                    for (int d = W - 1; d >= 0; --d) fma_pack(acc, wr[d], rows[uu + W - 1 - d]);
+                } else {
+                    // Taps before the request's first row come from the cache
+                    // (zero before position 0), or an index is out of range.
+                    const int64_t slot = mslot[i];
+                    const int64_t pos = mpos[i];
+                    const int req = msid[i];
+                    const int q0 = mqs[i];
+                    unsigned bad = 0;
+                    if (slot < 0 || slot >= slots_total) bad |= SCONV_EFLAG_SLOT;
+                    if (req < 0 || req >= a.num_reqs) bad |= SCONV_EFLAG_REQUEST;
+                    if (q0 < 0 || q0 > t) bad |= SCONV_EFLAG_QUERY_START;
+                    if (pos < 0) bad |= SCONV_EFLAG_POSITION;
+                    P ct[W];
+#pragma unroll
+                    for (int d = 1; d < W; ++d)
+                        if (t - d < q0 && pos - d >= 0 && !bad)
+                            bad |= load_cache_tap<bf16, 8>(a, req, pos - d, lane, ct[d]);
+                    if (bad) {
+                        if (a.err && active) atomicOr(a.err, static_cast<int>(bad));
+                        continue;
+                    }
+#pragma unroll
+                    for (int d = W - 1; d >= 0; --d) {
+                        if (d == 0 || t - d >= q0)
+                            fma_pack(acc, wr[d], rows[uu + W - 1 - d]);
+                        else if (pos - d >= 0)
+                            fma_pack(acc, wr[d], ct[d]);
+                    }
+                }
+                float xc[8];
+                rows[uu + W - 1].to_float(xc);
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    float y = acc[v];
+                    if (SILU) y = silu<bf16>(y);
+                    if (RESID) y += xc[v];
+                    acc[v] = y;
+                }
+                P o;
+                o.from_float(acc);
+                if (active) {
+                    o.store(out + static_cast<int64_t>(t) * a.out_rs + c);
+                    rows[uu + W - 1].store(cache + ins_u + lane);
+                }
             }
-            P o;
-            o.from_float(acc);
-            o.store(static_cast<bf16 *>(a.out) + static_cast<int64_t>(t) * a.out_rs + c);
-            int64_t blk, off;
-            split_n(a, slot, a.slots32 != 0, blk, off);
-            rows[u + W - 1].store(static_cast<bf16 *>(a.cache) + blk * a.cs0 + off * a.cs2 + lane);
         }
         __syncthreads();  // every warp is done with stage s
-        if (threadIdx.x == 0 && k + kStages < my) issue(k + kStages);
+        if (threadIdx.x == 0 && k + STAGES < my) issue(k + STAGES);
     }
 }
 
@@ -288,25 +363,46 @@ bool encode_1d(CUtensorMap *m, CUtensorMapDataType type, const void *base, int64
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int W>
-cudaError_t launch_w(const FusedArgs &a, const TmaMaps &maps, cudaStream_t stream) {
-    using L = Layout<W>;
+constexpr int kLaunchStages = 4;
+
+template <int W, bool SILU, bool RESID>
+cudaError_t launch_flags(const FusedArgs &a, const TmaMaps &maps, cudaStream_t stream) {
+    constexpr int S = kLaunchStages;
+    constexpr int smem = kStages_smem<W, S>();
+    auto kernel = fused_tma_kernel<W, S, SILU, RESID>;
+    // Resident blocks per SM and the SM count, once per process and kernel
+    // (the grid is a function of the device and of T and C only).
     static std::once_flag once;
     static cudaError_t attr = cudaSuccess;
-    std::call_once(once, [] {
-        attr = cudaFuncSetAttribute(fused_tma_kernel<W>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, L::smem);
+    static int per_sm = 1, sms = 148;
+    std::call_once(once, [&] {
+        attr = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (attr != cudaSuccess) return;
+        int dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess)
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, smem) !=
+                cudaSuccess ||
+            per_sm < 1)
+            per_sm = 1;
     });
     if (attr != cudaSuccess) return attr;
-    const int ntiles = (a.T + kBT - 1) / kBT;
-    const int cblocks = (a.C + kBC - 1) / kBC;
-    // About three resident blocks per SM across the grid, each streaming a
-    // run of consecutive tiles of one channel block.
-    const int64_t target = 148LL * 3;
-    int per = static_cast<int>((static_cast<int64_t>(ntiles) * cblocks + target - 1) / target);
-    if (per < 1) per = 1;
-    const dim3 grid((ntiles + per - 1) / per, cblocks);
-    return launch_pdl(fused_tma_kernel<W>, grid, dim3(kThreads), L::smem, stream, a, maps, per);
+    const int64_t ntiles = (a.T + kBT - 1) / kBT;
+    const int64_t units = ntiles * ((a.C + kBC - 1) / kBC);
+    int64_t grid = static_cast<int64_t>(sms) * per_sm;
+    if (grid > units) grid = units;
+    return launch_pdl(kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem, stream, a,
+                      maps, units);
+}
+
+template <int W>
+cudaError_t launch_w(const FusedArgs &a, const TmaMaps &maps, cudaStream_t stream) {
+    if (a.silu) {
+        return a.resid ? launch_flags<W, true, true>(a, maps, stream)
+                       : launch_flags<W, true, false>(a, maps, stream);
+    }
+    return a.resid ? launch_flags<W, false, true>(a, maps, stream)
+                   : launch_flags<W, false, false>(a, maps, stream);
 }
 
 }  // namespace
