@@ -141,8 +141,10 @@ def measured_hbm_peak():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the sources of the fused token kernel (the one the decode
+    workload runs), to tell whether a committed ncu summary is current."""
     h = hashlib.sha256()
-    for name in ("fused.cu", "common.cuh"):
+    for name in ("fused.cu", "fused_common.cuh", "common.cuh"):
         with open(os.path.join(ROOT, "hybrid_sconv_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

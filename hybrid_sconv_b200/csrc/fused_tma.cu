@@ -61,7 +61,7 @@ struct Layout {
 
 template <int W, int STAGES>
 constexpr int kStages_smem() {
-    return STAGES * Layout<W>::stage + STAGES * 8;
+    return STAGES * Layout<W>::stage + 2 * STAGES * 8;
 }
 
 struct TmaMaps {
@@ -120,13 +120,59 @@ __device__ __forceinline__ void tma_1d(void *dst, const CUtensorMap *map, int x,
 
 using P = Pack<bf16, 8>;
 
-// acc += w * tap for one 8-channel pack, as four packed fp32 FMAs.
-__device__ __forceinline__ void fma_pack(float (&acc)[8], const float (&w)[8], const P &tap) {
+// acc += w * tap for one 8-channel pack: eight fp32-accumulating FMAs that
+// take bf16 operands directly (the product of two bf16 values is exact in
+// fp32, so this equals widening both and one fmaf, bit for bit).  w holds
+// the pack's weights for one lag as four bf16 pairs.
+__device__ __forceinline__ void fma_pack(float (&acc)[8], const uint32_t (&w)[4], const P &tap) {
     const uint32_t q[4] = {tap.u.x, tap.u.y, tap.u.z, tap.u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-        fma2(acc[2 * i], acc[2 * i + 1], w[2 * i], w[2 * i + 1], __uint_as_float(q[i] << 16),
-             __uint_as_float(q[i] & 0xffff0000u));
+        asm("{\n\t.reg .b16 wl, wh, tl, th;\n\t"
+            "mov.b32 {wl, wh}, %2;\n\t"
+            "mov.b32 {tl, th}, %3;\n\t"
+            "fma.rn.f32.bf16 %0, wl, tl, %0;\n\t"
+            "fma.rn.f32.bf16 %1, wh, th, %1;\n\t}"
+            : "+f"(acc[2 * i]), "+f"(acc[2 * i + 1])
+            : "r"(w[i]), "r"(q[i]));
+}
+
+// The pack's weights as bf16 pairs by lag (wb[d] multiplies position
+// pos - d, weight column W-1-d); lags >= W are zero.
+template <int W>
+__device__ __forceinline__ void load_weights_bf16(const FusedArgs &a, int c, uint32_t (&wb)[4][4]) {
+    const unsigned short *w = static_cast<const unsigned short *>(a.w);
+    unsigned short e[8][4];
+    if (a.w_vec) {  // dense [C, 4]: 32 contiguous elements
+        union {
+            uint4 u[4];
+            unsigned short h[32];
+        } raw;
+        const uint4 *p = reinterpret_cast<const uint4 *>(w + static_cast<int64_t>(c) * 4);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) raw.u[q] = __ldg(p + q);
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+#pragma unroll
+            for (int d = 0; d < 4; ++d) e[v][d] = raw.h[v * 4 + 3 - d];
+    } else {
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+#pragma unroll
+            for (int d = 0; d < 4; ++d)
+                e[v][d] = d < W ? __ldg(w + static_cast<int64_t>(c + v) * a.w_sc +
+                                        static_cast<int64_t>(W - 1 - d) * a.w_sk)
+                                : static_cast<unsigned short>(0);
+    }
+#pragma unroll
+    for (int d = 0; d < 4; ++d)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            wb[d][i] = static_cast<uint32_t>(e[2 * i][d]) | (static_cast<uint32_t>(e[2 * i + 1][d]) << 16);
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
 // What a warp's lane u (< kTokPerWarp) knows about token u of its group.
@@ -139,6 +185,7 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
     using L = Layout<W>;
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * L::stage);
+    uint64_t *empty = full + STAGES;
 
     // Work units are (channel block, tile) pairs, channel-block major; this
     // block takes an equal contiguous share of them.
@@ -150,14 +197,19 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
 
     if (threadIdx.x == 0) {
 #pragma unroll
-        for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kThreads / 32);
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
     pdl_wait();  // inputs may come from the previous kernel in the stream
     pdl_trigger();
 
+    int issued = 0;  // tiles issued so far (meaningful in thread 0, the producer)
     auto issue = [&](int k) {
+        ++issued;
         const int s = k % STAGES;
         unsigned char *st = smem + s * L::stage;
         const int64_t u = u_begin + k;
@@ -181,9 +233,12 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
     bool active = false;
     int c = 0;
     int64_t lane = 0;
-    float wr[4][8];
+    uint32_t wr[4][4];
+    bool alive = true;
+    int next = 0;  // the next tile this thread waits for
 
     for (int k = 0; k < my; ++k) {
+        next = k;
         const int s = k % STAGES;
         const int64_t u = u_begin + k;
         const int cb = static_cast<int>(u / ntiles);
@@ -195,18 +250,12 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
             c = (active ? pack_raw : nv - 1) * 8;
             const int h = c / a.ws;
             lane = static_cast<int64_t>(h) * a.cs1 + a.off_s + (c - h * a.ws);
-            load_weights<bf16, 8, 4>(a, c, wr);
+            load_weights_bf16<W>(a, c, wr);
         }
-        const bool ok = mbar_wait(&full[s], (k / STAGES) & 1);
-        if (__syncthreads_or(!ok)) {
-            // Copies did not arrive: report, let the others land, stop.
-            if (threadIdx.x == 0) {
-                if (a.err) atomicOr(a.err, static_cast<int>(SCONV_EFLAG_TIMEOUT));
-                for (int j = k; j < my && j < k + STAGES; ++j)
-                    mbar_wait(&full[j % STAGES], (j / STAGES) & 1);
-            }
-            __syncthreads();
-            return;
+        if (!mbar_wait(&full[s], (k / STAGES) & 1)) {  // copies did not arrive in time
+            if (a.err && lane_id == 0) atomicOr(a.err, static_cast<int>(SCONV_EFLAG_TIMEOUT));
+            alive = false;
+            break;
         }
         const unsigned char *st = smem + s * L::stage;
         const P *xs = reinterpret_cast<const P *>(st) + lane_id;  // row r at xs[r * 32]
@@ -332,8 +381,27 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
                 }
             }
         }
-        __syncthreads();  // every warp is done with stage s
-        if (threadIdx.x == 0 && k + STAGES < my) issue(k + STAGES);
+        // This warp is done with stage s.  The producer refills the stage
+        // of the previous tile once all eight warps have released it, so a
+        // warp never waits for the others to finish the tile it is on.
+        __syncwarp();
+        if (lane_id == 0) mbar_arrive(&empty[s]);
+        next = k + 1;
+        if (threadIdx.x == 0 && k >= 1 && k - 1 + STAGES < my) {
+            const int j = k - 1;
+            if (mbar_wait(&empty[j % STAGES], (j / STAGES) & 1)) {
+                issue(j + STAGES);
+            } else {
+                if (a.err) atomicOr(a.err, static_cast<int>(SCONV_EFLAG_TIMEOUT));
+                alive = false;
+                break;
+            }
+        }
+    }
+    if (!alive && threadIdx.x == 0) {
+        // Let the copies this block issued and has not consumed land before
+        // its shared memory is released (each wait bounded).
+        for (int j = next; j < issued; ++j) mbar_wait(&full[j % STAGES], (j / STAGES) & 1);
     }
 }
 
