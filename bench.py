@@ -91,22 +91,29 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(value: float, world: int) -> float:
+def _reduce(value: float, world: int, op_name: str) -> float:
+    """All-reduce one float over the ranks (timing and token counts only;
+    nothing on the data path is exchanged)."""
     if world == 1:
         return value
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=getattr(dist.ReduceOp, op_name))
     return float(t.item())
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    return _reduce(value, world, "MAX")
 
 
 def sum_over_ranks(value: float, world: int) -> float:
-    if world == 1:
-        return value
-    import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    return _reduce(value, world, "SUM")
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws its own requests (weak scaling: per-GPU work fixed)."""
+    return base + 100003 * rank
 
 
 # --------------------------------------------------------------------------
@@ -454,8 +461,24 @@ def bench_spec_decode(device, stream, peak, n_sets=40):
     return res
 
 
-def per_workload_table(device, stream, peak):
+def bench_update(sets_obj, stream, peak, reps=200):
+    """The decode workload through sconv_update (token b is request b; no
+    metadata build needed): one launch per rotating set."""
+    import hybrid_sconv_b200 as hs
+    fns = []
+    for wl, s in zip(sets_obj.wls, sets_obj.sets):
+        fns.append(lambda wl=wl, s=s: hs.sconv_update(
+            s["x"], sets_obj.weight, sets_obj.cache, s["positions"], s["block_table"],
+            s["slot_mapping"], out=s["out"], **wl.kwargs()))
+    secs = _kernel_time(fns, reps, stream)
+    nbytes = int(np.mean(sets_obj.alg_bytes)) - 8 * sets_obj.wls[0].T  # no seq_idx / query_start
+    return {"decode_bf16_update": _entry(sets_obj.wls[0], secs, nbytes, peak)}
+
+
+def per_workload_table(device, stream, peak, sets_obj=None):
     table = {}
+    if sets_obj is not None:
+        table.update(bench_update(sets_obj, stream, peak))
     table.update(bench_prefill("chunked_prefill_bf16", device, stream, peak))
     table.update(bench_prefill("long_prefill_bf16", device, stream, peak))
     table.update(bench_spec_decode(device, stream, peak))
@@ -491,34 +514,50 @@ def cpu_baseline(sets_obj, seconds=8.0):
 # e2e: the public API with host buffers
 
 def e2e(sets_obj, K, stream, world):
-    """Each step: H2D of the step's inputs from pinned host memory, the
-    metadata build and the fused step, D2H of the output."""
-    host, h2d, d2h = [], 0, 0
+    """End to end through the public API with host buffers.  Every step
+    copies its inputs (x, positions, slot_mapping, block_table,
+    query_start_loc) from pinned host memory to the device, builds the
+    metadata, runs the fused step and copies its output back to pinned host
+    memory.  As a serving engine does, the three run on their own streams
+    (joined by events), so step i+1's upload and step i-1's download overlap
+    step i's kernels; each step still moves all of its own bytes."""
+    keys = ("x", "positions", "slot_mapping", "block_table", "query_start_loc")
+    host = []
     for s in sets_obj.sets:
-        hs_ = {k: s[k].cpu().pin_memory() for k in
-               ("x", "positions", "slot_mapping", "block_table", "query_start_loc")}
-        hs_["out"] = torch.empty_like(s["out"], device="cpu").pin_memory()
-        host.append(hs_)
-    h2d = sum(host[0][k].numel() * host[0][k].element_size() for k in
-              ("x", "positions", "slot_mapping", "block_table", "query_start_loc"))
+        h = {k: s[k].cpu().pin_memory() for k in keys}
+        h["out"] = torch.empty_like(s["out"], device="cpu").pin_memory()
+        host.append(h)
+    h2d = sum(host[0][k].numel() * host[0][k].element_size() for k in keys)
     d2h = host[0]["out"].numel() * host[0]["out"].element_size()
     M = len(sets_obj.sets)
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
 
-    def step(i):
-        s, h = sets_obj.sets[i], host[i]
-        for k in ("x", "positions", "slot_mapping", "block_table", "query_start_loc"):
-            s[k].copy_(h[k], non_blocking=True)
-        sets_obj.step(i)
-        h["out"].copy_(s["out"], non_blocking=True)
+    def steps(n):
+        cur = torch.cuda.current_stream()
+        up.wait_stream(cur)
+        down.wait_stream(cur)
+        for i in range(n):
+            s, h = sets_obj.sets[i], host[i]
+            with torch.cuda.stream(up):
+                for k in keys:
+                    s[k].copy_(h[k], non_blocking=True)
+            cur.wait_stream(up)
+            sets_obj.step(i)
+            down.wait_stream(cur)
+            with torch.cuda.stream(down):
+                h["out"].copy_(s["out"], non_blocking=True)
+        cur.wait_stream(up)
+        cur.wait_stream(down)
 
-    full = capture(lambda: [step(i) for i in range(M)], stream)
-    tail = capture(lambda: [step(i) for i in range(K % M)], stream) if K % M else None
+    full = capture(lambda: steps(M), stream)
+    tail = capture(lambda: steps(K % M), stream) if K % M else None
     replay_steps(full, None, 2)
     secs = max_over_ranks(time_region(full, tail, K // M, stream, world)[0], world)
     del full, tail
     tokens = sum_over_ranks(float(sets_obj.wls[0].T * K), world)
     return {"value": round(tokens / secs / 1e6, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": K, "launch": "cuda_graph"}
+            "d2h_bytes_per_step": d2h, "steps": K,
+            "launch": "cuda_graph; upload, kernels and download on three streams"}
 
 
 # --------------------------------------------------------------------------
@@ -605,7 +644,7 @@ def main():
         return
     K, W = args.steps, max(3, args.warmup)
 
-    sets_obj = DecodeSets(args.sets, args.seed + 100003 * rank, device, args.max_hist)
+    sets_obj = DecodeSets(args.sets, rank_seed(args.seed, rank), device, args.max_hist)
     touched = sum(sets_obj.alg_bytes)
 
     # warm-up, then exactly K timed steps
@@ -665,7 +704,7 @@ def main():
     if not args.no_extras:
         line["e2e"] = e2e(sets_obj, min(K, 24000), stream, world)
         if rank == 0:
-            line["per_config"] = per_workload_table(device, stream, peak)
+            line["per_config"] = per_workload_table(device, stream, peak, sets_obj)
         if rank == 0 and world == 1:
             line["cpu_baseline"] = cpu_baseline(sets_obj)
     if rank == 0:

@@ -189,6 +189,14 @@ __device__ __forceinline__ void pdl_trigger() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Bring a line into L2 without reading it into registers.  Safe before
+// pdl_wait(): L2 is the device's point of coherence, so a write by the
+// preceding kernel that lands after the prefetch is still what the later
+// load sees.
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // Arguments of one fused launch, validated on the host.  Strides in elements.
 struct FusedArgs {
     const void *x;

@@ -27,6 +27,10 @@ struct Raw<bf16> {
 };
 
 __device__ __forceinline__ int clamped_count(const ExtractArgs &a) {
+    if (threadIdx.x == 0) {  // while the preceding kernel drains
+        prefetch_l2(a.real_count);
+        prefetch_l2(a.abs_pos + blockIdx.x);
+    }
     pdl_wait();
     pdl_trigger();
     int rc = __ldg(a.real_count);

@@ -81,13 +81,28 @@ __device__ __forceinline__ void conv_store(const FusedArgs &a, const float (&wr)
 template <typename E, int VEC, int MAXW, bool ONE>
 __global__ void __launch_bounds__(kThreads) fused_token_kernel(const __grid_constant__ FusedArgs a) {
     using P = Pack<E, VEC>;
-    pdl_wait();
-    pdl_trigger();
     const int pack = blockIdx.y * blockDim.x + threadIdx.x;
     const int t = blockIdx.x * blockDim.y + threadIdx.y;
-    if (pack >= a.C / VEC || t >= a.T) return;
+    const bool in_range = pack < a.C / VEC && t < a.T;
     const E *x = static_cast<const E *>(a.x);
     const int c = pack * VEC;
+    if (in_range) {
+        // While the preceding kernel drains: pull this token's metadata, its
+        // x pack and the pack's weights into L2 (a warp's lanes share t).
+        if ((threadIdx.x & 31) == 0) {
+            prefetch_l2(a.positions + t);
+            prefetch_l2(a.slot + t);
+            if (!ONE) {
+                prefetch_l2(a.seq_idx + t);
+                prefetch_l2(a.qstart + t);
+            }
+        }
+        prefetch_l2(x + static_cast<int64_t>(t) * a.x_rs + c);
+        if (a.w_vec) prefetch_l2(static_cast<const E *>(a.w) + static_cast<int64_t>(c) * a.W);
+    }
+    pdl_wait();
+    pdl_trigger();
+    if (!in_range) return;
     const int h = c / a.ws;
     const int64_t lane = static_cast<int64_t>(h) * a.cs1 + a.off_s + (c - h * a.ws);
 
