@@ -475,10 +475,40 @@ def bench_update(sets_obj, stream, peak, reps=200):
     return {"decode_bf16_update": _entry(sets_obj.wls[0], secs, nbytes, peak)}
 
 
+def bench_streams(sets_obj, stream, peak, reps=200):
+    """Two conv streams of the decode layer in one sconv_fused_streams
+    launch: the workload's stream (lanes 32..63) and a second stream on
+    lanes 0..31, sharing tokens, metadata and cache."""
+    import hybrid_sconv_b200 as hs
+    wl0 = sets_obj.wls[0]
+    g = torch.Generator(device=sets_obj.device).manual_seed(7)
+    w2 = workloads.normal((wl0.C, wl0.W), 0.5, torch.bfloat16, g, sets_obj.device)
+    fns = []
+    for wl, s in zip(sets_obj.wls, sets_obj.sets):
+        x2 = workloads.normal((wl.T, wl.C), 1.0, torch.bfloat16, g, sets_obj.device)
+        o2 = torch.empty_like(x2)
+        streams = [dict(x=s["x"], weight=sets_obj.weight, off_s=wl.off_s, ws=wl.ws,
+                        activation=wl.act, use_residual=wl.residual, out=s["out"]),
+                   dict(x=x2, weight=w2, off_s=0, ws=wl.ws, activation=wl.act,
+                        use_residual=wl.residual, out=o2)]
+        fns.append(lambda s=s, streams=streams, wl=wl: hs.sconv_fused_streams(
+            streams, sets_obj.cache, s["positions"], s["block_table"], s["seq_idx"],
+            s["slot_mapping"], s["query_start"], wl.N))
+    secs = _kernel_time(fns, reps, stream)
+    nbytes = 2 * int(np.mean(sets_obj.alg_bytes)) - 24 * wl0.T  # per-token metadata read once
+    gbs = nbytes / secs / 1e9
+    return {"decode_bf16_two_streams": {
+        "kernel_us": round(secs * 1e6, 3), "streams": 2,
+        "mtokens_s_per_stream": round(wl0.T / secs / 1e6, 2),
+        "stream_mtokens_s": round(2 * wl0.T / secs / 1e6, 2), "alg_bytes": nbytes,
+        "alg_gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}}
+
+
 def per_workload_table(device, stream, peak, sets_obj=None):
     table = {}
     if sets_obj is not None:
         table.update(bench_update(sets_obj, stream, peak))
+        table.update(bench_streams(sets_obj, stream, peak))
     table.update(bench_prefill("chunked_prefill_bf16", device, stream, peak))
     table.update(bench_prefill("long_prefill_bf16", device, stream, peak))
     table.update(bench_spec_decode(device, stream, peak))

@@ -13,5 +13,5 @@ raises ImportError.
 from .binding import (  # noqa: F401
     EFLAG_BLOCK, EFLAG_LOGICAL, EFLAG_POSITION, EFLAG_QUERY_START, EFLAG_REQUEST,
     EFLAG_SLOT, LIB_PATH, SconvError, fused_sconv, scatter_intermediate_conv,
-    sconv_extract_windows, sconv_fused, sconv_seq_metadata, sconv_update,
+    sconv_extract_windows, sconv_fused, sconv_fused_streams, sconv_seq_metadata, sconv_update,
 )

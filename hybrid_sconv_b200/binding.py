@@ -39,6 +39,15 @@ class SconvError(RuntimeError):
 
 _P, _I64, _INT = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
 _I64P = ctypes.POINTER(ctypes.c_int64)
+MAX_STREAMS = 4
+
+
+class StreamDesc(ctypes.Structure):
+    """sconv_stream_desc of sconv.h."""
+    _fields_ = [("x", _P), ("x_row_stride", _I64), ("weight", _P), ("w_stride_c", _I64),
+                ("w_stride_k", _I64), ("out", _P), ("out_row_stride", _I64), ("off_s", _INT),
+                ("ws", _INT), ("act", _INT), ("use_residual", _INT)]
+
 
 _SIGNATURES = {
     "sconv_fused": [
@@ -48,6 +57,12 @@ _SIGNATURES = {
         _P, _I64, _INT, _INT,
         _INT, _INT, _INT, _INT, _INT,
         _P, _I64, _P, _P],
+    "sconv_fused_streams": [
+        ctypes.POINTER(StreamDesc), _INT, _INT, _INT,
+        _P, _I64P, _I64, _INT, _INT, _INT,
+        _P, _P, _P, _P,
+        _P, _I64, _INT, _INT,
+        _INT, _P, _P],
     "sconv_update": [
         _P, _I64, _INT, _INT, _P, _I64, _I64, _INT,
         _P, _I64P, _I64, _INT, _INT, _INT,
@@ -181,6 +196,61 @@ def sconv_fused(x, weight, cache, positions, block_table, seq_idx, slot_mapping,
             _ptr(out), out.stride(0), _ptr(err_flag), _stream(d, stream))
     _check("sconv_fused", st)
     return out
+
+
+def sconv_fused_streams(streams, cache, positions, block_table, seq_idx, slot_mapping,
+                        query_start, block_size, *, err_flag=None, stream=None):
+    """Several conv streams of one layer in one call (sconv_fused_streams in
+    sconv.h): the same tokens, metadata and cache, disjoint lane ranges.
+    ``streams`` is a sequence of dicts with keys ``x``, ``weight``,
+    ``off_s``, ``ws`` and optionally ``activation``, ``use_residual``
+    (default True, as in fused_sconv) and ``out``.  Returns the outputs."""
+    if not 1 <= len(streams) <= MAX_STREAMS:
+        raise ValueError(f"1..{MAX_STREAMS} streams per call")
+    x0 = streams[0]["x"]
+    dt = _float_common(x0, streams[0]["weight"], cache)
+    T = x0.shape[0]
+    outs = []
+    descs = (StreamDesc * len(streams))()
+    for i, sd in enumerate(streams):
+        x, w = sd["x"], sd["weight"]
+        _float_common(x, w, cache)
+        if x.shape[0] != T or w.shape[1] != streams[0]["weight"].shape[1]:
+            raise ValueError("all streams share T and W")
+        out = sd.get("out")
+        if out is None:
+            out = torch.empty_like(x)
+        if out.dtype != x.dtype or tuple(out.shape) != tuple(x.shape) or (T and out.stride(1) != 1):
+            raise ValueError("out must be [T, C] like x with unit channel stride")
+        outs.append(out)
+        descs[i] = StreamDesc(_ptr(x), x.stride(0), _ptr(w), w.stride(0), w.stride(1), _ptr(out),
+                              out.stride(0), sd["off_s"], sd["ws"], _act(sd.get("activation")),
+                              int(bool(sd.get("use_residual", True))))
+    if T == 0:
+        return outs
+    d = _dev(x0, cache, positions, block_table, seq_idx, slot_mapping, query_start, err_flag,
+             *[sd["x"] for sd in streams], *[sd["weight"] for sd in streams], *outs)
+    _vector(positions, torch.int64, "positions", T)
+    _vector(seq_idx, torch.int32, "seq_idx", T)
+    _vector(slot_mapping, torch.int64, "slot_mapping", T)
+    _vector(query_start, torch.int32, "query_start", T)
+    _want(block_table, torch.int32, "block_table")
+    if block_table.dim() != 2 or block_table.stride(1) != 1:
+        raise ValueError("block_table must be [num_reqs, max_blocks] with unit inner stride")
+    if err_flag is not None:
+        _vector(err_flag, torch.int32, "err_flag", 1)
+    if cache.shape[2] != block_size:
+        raise ValueError("cache.shape[2] must equal block_size")
+    nb, H, N, D = cache.shape
+    cs = (ctypes.c_int64 * 4)(*cache.stride())
+    with torch.cuda.device(d):
+        st = LIB.sconv_fused_streams(
+            descs, len(streams), T, streams[0]["weight"].shape[1], _ptr(cache), cs, nb, H, N, D,
+            _ptr(positions), _ptr(seq_idx), _ptr(slot_mapping), _ptr(query_start),
+            _ptr(block_table), block_table.stride(0), block_table.shape[0],
+            block_table.shape[1], dt, _ptr(err_flag), _stream(d, stream))
+    _check("sconv_fused_streams", st)
+    return outs
 
 
 def sconv_update(x, weight, cache, positions, block_table, slot_mapping, off_s, ws,

@@ -138,6 +138,52 @@ sconv_status sconv_fused(const void *x, int64_t x_row_stride, int T, int C, cons
                : SCONV_ERR_LAUNCH;
 }
 
+sconv_status sconv_fused_streams(const sconv_stream_desc *streams, int n_streams, int T, int W,
+                                 void *cache, const int64_t cache_strides[4], int64_t num_blocks,
+                                 int H, int N, int D, const int64_t *positions,
+                                 const int32_t *seq_idx, const int64_t *slot_mapping,
+                                 const int32_t *query_start, const int32_t *block_table,
+                                 int64_t bt_row_stride, int num_reqs, int max_blocks,
+                                 sconv_dtype dt, int32_t *err_flag, cudaStream_t stream) {
+    if (T < 0 || n_streams < 1 || !streams) return SCONV_ERR_INVALID;
+    if (n_streams > SCONV_MAX_STREAMS) return SCONV_ERR_UNSUPPORTED;
+    if (T == 0) return SCONV_OK;
+    if (!seq_idx || !query_start) return SCONV_ERR_INVALID;
+    FusedArgs a[SCONV_MAX_STREAMS];
+    bool vec_all = true;
+    const int64_t e = elem_size(dt);
+    for (int i = 0; i < n_streams; ++i) {
+        const sconv_stream_desc &d = streams[i];
+        bool vec = false;
+        const sconv_status st = check_fused(
+            d.x, d.x_row_stride, T, H * d.ws, d.weight, d.w_stride_c, d.w_stride_k, W, cache,
+            cache_strides, num_blocks, H, N, D, positions, slot_mapping, block_table,
+            bt_row_stride, num_reqs, max_blocks, d.off_s, d.ws, d.act, d.use_residual, dt, d.out,
+            d.out_row_stride, err_flag, a[i], vec);
+        if (st != SCONV_OK) return st;
+        a[i].seq_idx = seq_idx;
+        a[i].qstart = query_start;
+        vec_all = vec_all && vec;
+        const int64_t out_bytes =
+            ((static_cast<int64_t>(T) - 1) * d.out_row_stride + H * d.ws) * e;
+        for (int j = 0; j < i; ++j) {
+            const sconv_stream_desc &o = streams[j];
+            // lane ranges disjoint
+            if (d.off_s < o.off_s + o.ws && o.off_s < d.off_s + d.ws) return SCONV_ERR_INVALID;
+            const int64_t o_out = ((static_cast<int64_t>(T) - 1) * o.out_row_stride + H * o.ws) * e;
+            const int64_t o_x = ((static_cast<int64_t>(T) - 1) * o.x_row_stride + H * o.ws) * e;
+            const int64_t d_x = ((static_cast<int64_t>(T) - 1) * d.x_row_stride + H * d.ws) * e;
+            if (overlaps(d.out, out_bytes, o.out, o_out) || overlaps(d.out, out_bytes, o.x, o_x) ||
+                overlaps(o.out, o_out, d.x, d_x))
+                return SCONV_ERR_INVALID;
+        }
+    }
+    return sconv::launch_fused_streams(a, n_streams, dt == SCONV_BF16, vec_all, stream) ==
+                   cudaSuccess
+               ? SCONV_OK
+               : SCONV_ERR_LAUNCH;
+}
+
 sconv_status sconv_update(const void *x, int64_t x_row_stride, int B, int C, const void *weight,
                           int64_t w_stride_c, int64_t w_stride_k, int W, void *cache,
                           const int64_t cache_strides[4], int64_t num_blocks, int H, int N,

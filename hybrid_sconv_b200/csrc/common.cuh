@@ -147,7 +147,8 @@ struct FastDiv {
 };
 
 // SiLU of the fp32 convolution, one formula per storage type so that every
-// kernel produces the same bits for the same token.  bf16 outputs: y *
+// kernel produces the same bits for the same token (the residual that
+// follows is added with __fadd_rn, so no kernel contracts it into an FMA).  bf16 outputs: y *
 // sigmoid(y) written as h + h * tanh(h) with h = y / 2, one hardware tanh
 // (tanh.approx.f32, relative error near 2^-11, far below bf16's 2^-8
 // rounding step).  fp32 outputs: y / (1 + e^-y) with CUDA's fast exp and
@@ -243,6 +244,10 @@ struct ExtractArgs {
 // Host-side launchers (return the cudaError_t of the launch).
 cudaError_t launch_fused(FusedArgs &a, bool bf16_data, bool vec, bool one_token_per_request,
                          cudaStream_t stream);
+// Several streams of one layer (same tokens, metadata and cache; disjoint
+// lane ranges) in one launch at decode sizes, else one launch per stream.
+cudaError_t launch_fused_streams(FusedArgs *s, int n, bool bf16_data, bool vec,
+                                 cudaStream_t stream);
 // The TMA-pipelined prefill kernel; sets `used` false (and launches
 // nothing) when the call does not meet its layout requirements.
 cudaError_t launch_fused_tma(const FusedArgs &a, cudaStream_t stream, bool &used);

@@ -67,7 +67,7 @@ __device__ __forceinline__ void conv_store(const FusedArgs &a, const float (&wr)
     for (int v = 0; v < VEC; ++v) {
         float y = acc[v];
         if (a.silu) y = silu<E>(y);
-        if (a.resid) y += xc[v];
+        if (a.resid) y = __fadd_rn(y, xc[v]);  // never contracted into an FMA
         acc[v] = y;
     }
     Pack<E, VEC> o;
@@ -78,31 +78,29 @@ __device__ __forceinline__ void conv_store(const FusedArgs &a, const float (&wr)
     cur.store(static_cast<E *>(a.cache) + blk * a.cs0 + off * a.cs2 + lane);
 }
 
+// Before the PDL wait: pull token t's metadata, its x pack and the pack's
+// weights into L2 while the preceding kernel drains (a warp's lanes share t).
+template <typename E, bool ONE>
+__device__ __forceinline__ void token_prefetch(const FusedArgs &a, int pack, int t, int vec) {
+    if ((threadIdx.x & 31) == 0) {
+        prefetch_l2(a.positions + t);
+        prefetch_l2(a.slot + t);
+        if (!ONE) {
+            prefetch_l2(a.seq_idx + t);
+            prefetch_l2(a.qstart + t);
+        }
+    }
+    const int c = pack * vec;
+    prefetch_l2(static_cast<const E *>(a.x) + static_cast<int64_t>(t) * a.x_rs + c);
+    if (a.w_vec) prefetch_l2(static_cast<const E *>(a.w) + static_cast<int64_t>(c) * a.W);
+}
+
+// One token-pack of the token kernel (after the PDL wait, in range).
 template <typename E, int VEC, int MAXW, bool ONE>
-__global__ void __launch_bounds__(kThreads) fused_token_kernel(const __grid_constant__ FusedArgs a) {
+__device__ __forceinline__ void token_body(const FusedArgs &a, int pack, int t) {
     using P = Pack<E, VEC>;
-    const int pack = blockIdx.y * blockDim.x + threadIdx.x;
-    const int t = blockIdx.x * blockDim.y + threadIdx.y;
-    const bool in_range = pack < a.C / VEC && t < a.T;
     const E *x = static_cast<const E *>(a.x);
     const int c = pack * VEC;
-    if (in_range) {
-        // While the preceding kernel drains: pull this token's metadata, its
-        // x pack and the pack's weights into L2 (a warp's lanes share t).
-        if ((threadIdx.x & 31) == 0) {
-            prefetch_l2(a.positions + t);
-            prefetch_l2(a.slot + t);
-            if (!ONE) {
-                prefetch_l2(a.seq_idx + t);
-                prefetch_l2(a.qstart + t);
-            }
-        }
-        prefetch_l2(x + static_cast<int64_t>(t) * a.x_rs + c);
-        if (a.w_vec) prefetch_l2(static_cast<const E *>(a.w) + static_cast<int64_t>(c) * a.W);
-    }
-    pdl_wait();
-    pdl_trigger();
-    if (!in_range) return;
     const int h = c / a.ws;
     const int64_t lane = static_cast<int64_t>(h) * a.cs1 + a.off_s + (c - h * a.ws);
 
@@ -142,6 +140,42 @@ __global__ void __launch_bounds__(kThreads) fused_token_kernel(const __grid_cons
             return tap[d];
         },
         tap[0], t, c, k.slot, lane);
+}
+
+template <typename E, int VEC, int MAXW, bool ONE>
+__global__ void __launch_bounds__(kThreads) fused_token_kernel(const __grid_constant__ FusedArgs a) {
+    const int pack = blockIdx.y * blockDim.x + threadIdx.x;
+    const int t = blockIdx.x * blockDim.y + threadIdx.y;
+    const bool in_range = pack < a.C / VEC && t < a.T;
+    if (in_range) token_prefetch<E, ONE>(a, pack, t, VEC);
+    pdl_wait();
+    pdl_trigger();
+    if (in_range) token_body<E, VEC, MAXW, ONE>(a, pack, t);
+}
+
+// Several conv streams of one layer (disjoint lane ranges of the same
+// cache, the same tokens and metadata) in one launch: the grid's y blocks
+// are the streams' channel blocks laid end to end.  Each block runs the
+// token kernel's work for its stream, so the latency-bound chain (metadata
+// -> block table -> cache) is paid once per launch for all streams.
+struct StreamSet {
+    FusedArgs s[SCONV_MAX_STREAMS];
+    int n;
+    int y0[SCONV_MAX_STREAMS + 1];  // first y block of each stream, y0[n] = total
+};
+
+template <typename E, int VEC, int MAXW>
+__global__ void __launch_bounds__(kThreads) fused_streams_kernel(const __grid_constant__ StreamSet m) {
+    int si = 0;
+    while (si + 1 < m.n && static_cast<int>(blockIdx.y) >= m.y0[si + 1]) ++si;
+    const FusedArgs &a = m.s[si];
+    const int pack = (blockIdx.y - m.y0[si]) * blockDim.x + threadIdx.x;
+    const int t = blockIdx.x * blockDim.y + threadIdx.y;
+    const bool in_range = pack < a.C / VEC && t < a.T;
+    if (in_range) token_prefetch<E, false>(a, pack, t, VEC);
+    pdl_wait();
+    pdl_trigger();
+    if (in_range) token_body<E, VEC, MAXW, false>(a, pack, t);
 }
 
 // Ring of x rows: Q >= PF + MAXW slots, a power of two.
@@ -352,7 +386,54 @@ cudaError_t launch_v(FusedArgs &a, bool one, cudaStream_t stream) {
     return launch_w<E, VEC, 8>(a, one, stream);
 }
 
+template <typename E, int VEC, int MAXW>
+cudaError_t launch_streams_t(FusedArgs *s, int n, cudaStream_t stream) {
+    StreamSet m;
+    m.n = n;
+    int nv_max = 0;
+    for (int i = 0; i < n; ++i) nv_max = s[i].C / VEC > nv_max ? s[i].C / VEC : nv_max;
+    const Shape sh = block_shape(nv_max, s[0].T);
+    m.y0[0] = 0;
+    for (int i = 0; i < n; ++i) {
+        s[i].w_vec = s[i].w_vec && s[i].W == MAXW;
+        m.s[i] = s[i];
+        m.y0[i + 1] = m.y0[i] + (s[i].C / VEC + sh.cv - 1) / sh.cv;
+    }
+    for (int i = n; i < SCONV_MAX_STREAMS; ++i) m.s[i] = s[0];  // never selected
+    dim3 grid(static_cast<unsigned>((s[0].T + sh.tg - 1) / sh.tg), static_cast<unsigned>(m.y0[n]));
+    return launch_pdl(fused_streams_kernel<E, VEC, MAXW>, grid, dim3(sh.cv, sh.tg), 0, stream, m);
+}
+
+template <typename E, int VEC>
+cudaError_t launch_streams_v(FusedArgs *s, int n, cudaStream_t stream) {
+    if (s[0].W <= 4) return launch_streams_t<E, VEC, 4>(s, n, stream);
+    return launch_streams_t<E, VEC, 8>(s, n, stream);
+}
+
 }  // namespace
+
+cudaError_t launch_fused_streams(FusedArgs *s, int n, bool bf16_data, bool vec,
+                                 cudaStream_t stream) {
+    // Prefill sizes are bandwidth-bound and nothing is gained by sharing
+    // the metadata: each stream takes its own (streamed or TMA) launch.
+    int64_t packs = 0;
+    for (int i = 0; i < n; ++i) packs += s[i].C / (vec ? (bf16_data ? 8 : 4) : 1);
+    if (static_cast<int64_t>(s[0].T) * packs >= kStripMinWork && s[0].T >= 64) {
+        for (int i = 0; i < n; ++i) {
+            const cudaError_t e = launch_fused(s[i], bf16_data, vec, false, stream);
+            if (e != cudaSuccess) return e;
+        }
+        return cudaSuccess;
+    }
+    for (int i = 0; i < n; ++i) {
+        s[i].divN = FastDiv::make(static_cast<uint32_t>(s[i].N));
+        s[i].slots32 = s[i].num_blocks * s[i].N < (1ll << 31);
+        s[i].strip = 1;
+    }
+    if (bf16_data)
+        return vec ? launch_streams_v<bf16, 8>(s, n, stream) : launch_streams_v<bf16, 1>(s, n, stream);
+    return vec ? launch_streams_v<float, 4>(s, n, stream) : launch_streams_v<float, 1>(s, n, stream);
+}
 
 cudaError_t launch_fused(FusedArgs &a, bool bf16_data, bool vec, bool one, cudaStream_t stream) {
     a.divN = FastDiv::make(static_cast<uint32_t>(a.N));

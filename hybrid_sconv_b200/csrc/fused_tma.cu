@@ -311,7 +311,7 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
                 for (int v = 0; v < 8; ++v) {
                     float y = acc[v];
                     if (SILU) y = silu<bf16>(y);
-                    if (RESID) y += xc[v];
+                    if (RESID) y = __fadd_rn(y, xc[v]);  // never contracted into an FMA
                     acc[v] = y;
                 }
                 P o;
@@ -370,7 +370,7 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
                 for (int v = 0; v < 8; ++v) {
                     float y = acc[v];
                     if (SILU) y = silu<bf16>(y);
-                    if (RESID) y += xc[v];
+                    if (RESID) y = __fadd_rn(y, xc[v]);  // never contracted into an FMA
                     acc[v] = y;
                 }
                 P o;

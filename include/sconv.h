@@ -81,6 +81,7 @@ typedef enum sconv_act { SCONV_ACT_NONE = 0, SCONV_ACT_SILU = 1 } sconv_act;
                                          wait; that block wrote nothing further and returned */
 
 #define SCONV_MAX_W 8      /* taps supported by sconv_fused / sconv_update */
+#define SCONV_MAX_STREAMS 4 /* conv streams per sconv_fused_streams call */
 #define SCONV_MAX_DCONV 8  /* window length supported by sconv_extract_windows */
 
 /*
@@ -118,6 +119,47 @@ sconv_status sconv_fused(
     const int32_t *block_table, int64_t bt_row_stride, int num_reqs, int max_blocks,
     int off_s, int ws, sconv_act act, int use_residual, sconv_dtype dt,
     void *out, int64_t out_row_stride, int32_t *err_flag, cudaStream_t stream);
+
+/*
+ * One conv stream of a layer for sconv_fused_streams: its input, taps,
+ * output, lane range and epilogue, each with the meaning it has in
+ * sconv_fused (C = H * ws).
+ */
+typedef struct sconv_stream_desc {
+    const void *x;          /* [T, C], row stride x_row_stride */
+    int64_t x_row_stride;
+    const void *weight;     /* [C, W], strides (w_stride_c, w_stride_k) */
+    int64_t w_stride_c, w_stride_k;
+    void *out;              /* [T, C], row stride out_row_stride */
+    int64_t out_row_stride;
+    int off_s, ws;          /* lanes [off_s, off_s + ws) of every head */
+    sconv_act act;
+    int use_residual;
+} sconv_stream_desc;
+
+/*
+ * sconv_fused_streams -- the fused step for several conv streams of one layer
+ * that share the paged cache, the tokens and all per-token metadata ("each
+ * layer's conv streams share one paged cache", vllm sconv page module
+ * docstring), in one call.  The result is exactly that of one sconv_fused per
+ * stream: the streams' lane ranges must be pairwise disjoint, so no stream
+ * reads or writes another's lanes.  At decode sizes one launch serves all
+ * streams (the metadata and block-table reads are shared); at prefill sizes
+ * each stream gets its own launch.
+ *
+ *   streams   HOST array of n_streams (1..SCONV_MAX_STREAMS) descriptors;
+ *             read during the call only.  Outputs must not overlap any x,
+ *             any other output or the cache.
+ *   every other argument as in sconv_fused, shared by all streams.
+ * T == 0 returns SCONV_OK and enqueues nothing.
+ */
+sconv_status sconv_fused_streams(
+    const sconv_stream_desc *streams, int n_streams, int T, int W,
+    void *cache, const int64_t cache_strides[4], int64_t num_blocks, int H, int N, int D,
+    const int64_t *positions, const int32_t *seq_idx, const int64_t *slot_mapping,
+    const int32_t *query_start,
+    const int32_t *block_table, int64_t bt_row_stride, int num_reqs, int max_blocks,
+    sconv_dtype dt, int32_t *err_flag, cudaStream_t stream);
 
 /*
  * sconv_update -- single-token decode form: token b belongs to request b

@@ -186,6 +186,32 @@ def fused(*, dtype, x, weight, cache, positions, block_table, seq_idx,
     return out_ref, state, cache_out, int(skipped)
 
 
+def fused_streams(*, dtype, streams, cache, positions, block_table, seq_idx, slot_mapping,
+                  query_start, block_size):
+    """Several conv streams of one layer over one cache: by definition one
+    fused_sconv per stream, every stream reading the cache as it was before
+    the call (their lane ranges are disjoint, so no stream sees another's
+    inserts).  ``streams``: dicts with x, weight, off_s, ws, activation,
+    use_residual.  Returns (outs, states, cache_out, skipped)."""
+    pre = _float_array(cache, dtype)
+    cache_out = pre.copy()
+    outs, states, skipped = [], [], 0
+    for sd in streams:
+        out, st, co, sk = fused(
+            dtype=dtype, x=sd["x"], weight=sd["weight"], cache=pre, positions=positions,
+            block_table=block_table, seq_idx=seq_idx, slot_mapping=slot_mapping,
+            query_start=query_start, off_s=sd["off_s"], ws=sd["ws"], block_size=block_size,
+            activation=sd.get("activation"), use_residual=sd.get("use_residual", True))
+        changed = co.view(np.uint8).reshape(co.shape + (-1,)) != pre.view(np.uint8).reshape(
+            pre.shape + (-1,))
+        mask = changed.any(axis=-1)
+        cache_out[mask] = co[mask]
+        outs.append(out)
+        states.append(st)
+        skipped += sk
+    return outs, states, cache_out, skipped
+
+
 def update(*, dtype, x, weight, cache, positions, block_table, slot_mapping,
            off_s, ws, block_size, activation=None, use_residual=True,
            write_cache=True):

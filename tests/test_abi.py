@@ -147,3 +147,26 @@ def test_product_path_does_not_import_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in text, f
+
+
+def test_streams_host_validation(lib):
+    """sconv_fused_streams rejects overlapping lane ranges, too many streams
+    and outputs that overlap another stream's buffers, before any launch."""
+    from hybrid_sconv_b200.binding import StreamDesc
+
+    def desc(x, out, off_s, ws=4, w=FAKE + 4096):
+        return StreamDesc(x, 8, w, 4, 1, out, 8, off_s, ws, 0, 1)
+
+    def call(descs, n=None, T=4):
+        arr = (StreamDesc * len(descs))(*descs)
+        return lib.sconv_fused_streams(arr, len(descs) if n is None else n, T, 4, FAKE * 64,
+                                       _strides(512, 256, 16, 1), 8, 2, 16, 16, FAKE, FAKE,
+                                       FAKE, FAKE, FAKE, 4, 2, 4, 1, 0, 0)
+    ok_a = desc(FAKE, FAKE * 512, 0)
+    ok_b = desc(FAKE * 2, FAKE * 1024, 8)
+    assert call([ok_a, ok_b], T=0) == 0
+    assert call([ok_a, desc(FAKE * 2, FAKE * 1024, 2)]) == 1          # lanes 0..3 and 2..5 overlap
+    assert call([ok_a, desc(FAKE * 2, FAKE * 512 + 16, 8)]) == 1      # outputs overlap
+    assert call([ok_a, desc(FAKE * 512, FAKE * 1024, 8)]) == 1        # output is another's x
+    assert call([ok_a] * 5) == 2                                       # more than 4 streams
+    assert call([ok_a], n=0) == 1

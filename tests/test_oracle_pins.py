@@ -431,3 +431,55 @@ def test_precondition_checker_detects_violations():
     pos[-1] += 1
     if wl.new[-1] >= 2:
         assert oracle.check_preconditions(**{**kw, "positions": pos}) == 1
+
+
+# --------------------------------------------------------------------------
+# several streams of one layer
+
+def _two_stream_case(seed, dtype="bf16"):
+    rng = np.random.default_rng(seed)
+    wl = workloads.build("kv", dtype=dtype, H=3, D=24, ws=8, off_s=0, W=4, N=4,
+                         hist=rng.integers(0, 12, size=3), new=rng.integers(1, 9, size=3),
+                         act="silu", residual=True, seed=seed, num_pad=2, rng=rng)
+    t = wl.tensors()
+    g = torch.Generator().manual_seed(seed + 1)
+    streams = [
+        dict(x=t["x"], weight=t["weight"], off_s=0, ws=8, activation="silu", use_residual=True),
+        dict(x=torch.randn(wl.T, 3 * 6, generator=g).to(t["x"].dtype),
+             weight=(torch.randn(18, 4, generator=g) * 0.5).to(t["x"].dtype),
+             off_s=10, ws=6, activation=None, use_residual=False),
+    ]
+    return wl, t, streams
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_streams_equal_sequential_single_stream_calls(seed):
+    """With disjoint lane ranges, applying the streams one after another
+    (each later stream reading the cache the earlier ones wrote) gives the
+    same outputs and cache as the combined definition."""
+    wl, t, streams = _two_stream_case(seed)
+    md = dict(positions=wl.positions, block_table=wl.block_table, seq_idx=wl.seq_idx,
+              slot_mapping=wl.slot_mapping, query_start=wl.query_start)
+    outs, states, cache_all, _ = oracle.fused_streams(
+        dtype=wl.dtype, streams=streams, cache=t["cache"], block_size=wl.N, **md)
+    cache = t["cache"]
+    for sd, out_c in zip(streams, outs):
+        out, st, cache_np, _ = oracle.fused(
+            dtype=wl.dtype, x=sd["x"], weight=sd["weight"], cache=cache, off_s=sd["off_s"],
+            ws=sd["ws"], block_size=wl.N, activation=sd["activation"],
+            use_residual=sd["use_residual"], **md)
+        np.testing.assert_array_equal(out, out_c)
+        cache = cache_np
+    np.testing.assert_array_equal(cache, cache_all)
+    # and every stream's written lanes hold its own x (read back by 4-D indexing)
+    for sd in streams:
+        xs = oracle._float_array(sd["x"], wl.dtype)
+        for row in range(wl.T):
+            if wl.slot_mapping[row] == -1:
+                continue
+            r, p = int(wl.seq_idx[row]), int(wl.positions[row])
+            b = int(wl.block_table[r, p // wl.N])
+            for h in range(wl.H):
+                np.testing.assert_array_equal(
+                    cache_all[b, h, p % wl.N, sd["off_s"]:sd["off_s"] + sd["ws"]],
+                    xs[row, h * sd["ws"]:(h + 1) * sd["ws"]])
