@@ -3,15 +3,27 @@
 One launch per call: paged sliding-window cache insert, depthwise causal
 conv1d over the window ending at each token's absolute position, optional
 SiLU and residual ("vllm.models.inkling.nvidia.ops.sconv"), plus the decode
-update, prefix-caching window extraction
-("core.ssm.ops.intermediate_extraction") and per-token metadata builder.
+update, several streams of a layer in one call, prefix-caching window
+extraction ("core.ssm.ops.intermediate_extraction") and the per-token
+metadata builder.
 
 The kernels live in ``libsconv.so`` (C ABI: include/sconv.h), built by
-``python -m hybrid_sconv_b200.build``; importing this package without it
-raises ImportError.
+``python -m hybrid_sconv_b200.build``.  The ops are loaded on first use;
+using one without the library raises ImportError (there is no fallback).
 """
-from .binding import (  # noqa: F401
-    EFLAG_BLOCK, EFLAG_LOGICAL, EFLAG_POSITION, EFLAG_QUERY_START, EFLAG_REQUEST,
-    EFLAG_SLOT, LIB_PATH, SconvError, fused_sconv, scatter_intermediate_conv,
-    sconv_extract_windows, sconv_fused, sconv_fused_streams, sconv_seq_metadata, sconv_update,
+
+_EXPORTS = (
+    "EFLAG_BLOCK", "EFLAG_LOGICAL", "EFLAG_POSITION", "EFLAG_QUERY_START", "EFLAG_REQUEST",
+    "EFLAG_SLOT", "EFLAG_TIMEOUT", "LIB_PATH", "SconvError", "fused_sconv",
+    "scatter_intermediate_conv", "sconv_extract_windows", "sconv_fused", "sconv_fused_streams",
+    "sconv_seq_metadata", "sconv_update",
 )
+
+__all__ = list(_EXPORTS)
+
+
+def __getattr__(name):
+    if name in _EXPORTS:
+        from . import binding  # loads libsconv.so, or raises ImportError
+        return getattr(binding, name)
+    raise AttributeError(f"module 'hybrid_sconv_b200' has no attribute {name!r}")

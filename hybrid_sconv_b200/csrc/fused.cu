@@ -78,9 +78,16 @@ __device__ __forceinline__ void conv_store(const FusedArgs &a, const float (&wr)
     cur.store(static_cast<E *>(a.cache) + blk * a.cs0 + off * a.cs2 + lane);
 }
 
-// Before the PDL wait: pull token t's metadata, its x pack and the pack's
-// weights into L2 while the preceding kernel drains (a warp's lanes share t).
-template <typename E, bool ONE>
+// Before the PDL wait, while the preceding kernel drains: pull token t's
+// metadata, its x pack and the pack's weights into L2 (a warp's lanes share
+// t), then go one step further.  The token's metadata and block-table
+// entries are read *speculatively* with L2-only loads (ld.global.cg, so no
+// line enters L1) -- the preceding kernel may still be writing them -- and
+// used only to choose which block-table lines and cache taps to prefetch
+// into L2.  Every speculative index is range-checked before it forms an
+// address.  After the wait the real loads run as usual; a stale value costs
+// a useless prefetch, never a wrong result.
+template <typename E, int MAXW, bool ONE>
 __device__ __forceinline__ void token_prefetch(const FusedArgs &a, int pack, int t, int vec) {
     if ((threadIdx.x & 31) == 0) {
         prefetch_l2(a.positions + t);
@@ -93,6 +100,25 @@ __device__ __forceinline__ void token_prefetch(const FusedArgs &a, int pack, int
     const int c = pack * vec;
     prefetch_l2(static_cast<const E *>(a.x) + static_cast<int64_t>(t) * a.x_rs + c);
     if (a.w_vec) prefetch_l2(static_cast<const E *>(a.w) + static_cast<int64_t>(c) * a.W);
+
+    const int64_t pos = __ldcg(a.positions + t);
+    const int req = ONE ? t : __ldcg(a.seq_idx + t);
+    const int q0 = ONE ? t : __ldcg(a.qstart + t);
+    if (req < 0 || req >= a.num_reqs || pos < 0 || pos >= (1ll << 31)) return;
+    const int h = c / a.ws;
+    const int64_t lane = static_cast<int64_t>(h) * a.cs1 + a.off_s + (c - h * a.ws);
+    const int32_t *bt_row = a.bt + static_cast<int64_t>(req) * a.bt_rs;
+#pragma unroll
+    for (int d = 1; d < MAXW; ++d) {
+        if (d >= a.W || t - d >= q0 || pos - d < 0) continue;
+        const uint32_t src = static_cast<uint32_t>(pos - d);
+        const uint32_t lb = a.divN.div(src);
+        if (lb >= static_cast<uint32_t>(a.max_blocks)) continue;
+        const int32_t b = __ldcg(bt_row + lb);
+        if (b < 0 || b >= a.num_blocks) continue;
+        prefetch_l2(static_cast<const E *>(a.cache) + static_cast<int64_t>(b) * a.cs0 +
+                    static_cast<int64_t>(src - lb * a.divN.d) * a.cs2 + lane);
+    }
 }
 
 // One token-pack of the token kernel (after the PDL wait, in range).
@@ -147,7 +173,7 @@ __global__ void __launch_bounds__(kThreads) fused_token_kernel(const __grid_cons
     const int pack = blockIdx.y * blockDim.x + threadIdx.x;
     const int t = blockIdx.x * blockDim.y + threadIdx.y;
     const bool in_range = pack < a.C / VEC && t < a.T;
-    if (in_range) token_prefetch<E, ONE>(a, pack, t, VEC);
+    if (in_range) token_prefetch<E, MAXW, ONE>(a, pack, t, VEC);
     pdl_wait();
     pdl_trigger();
     if (in_range) token_body<E, VEC, MAXW, ONE>(a, pack, t);
@@ -172,7 +198,7 @@ __global__ void __launch_bounds__(kThreads) fused_streams_kernel(const __grid_co
     const int pack = (blockIdx.y - m.y0[si]) * blockDim.x + threadIdx.x;
     const int t = blockIdx.x * blockDim.y + threadIdx.y;
     const bool in_range = pack < a.C / VEC && t < a.T;
-    if (in_range) token_prefetch<E, false>(a, pack, t, VEC);
+    if (in_range) token_prefetch<E, MAXW, false>(a, pack, t, VEC);
     pdl_wait();
     pdl_trigger();
     if (in_range) token_body<E, VEC, MAXW, false>(a, pack, t);
