@@ -87,7 +87,7 @@ __device__ __forceinline__ void conv_store(const FusedArgs &a, const float (&wr)
 // into L2.  Every speculative index is range-checked before it forms an
 // address.  After the wait the real loads run as usual; a stale value costs
 // a useless prefetch, never a wrong result.
-template <typename E, int MAXW, bool ONE>
+template <typename E, int MAXW, bool ONE, bool SPEC>
 __device__ __forceinline__ void token_prefetch(const FusedArgs &a, int pack, int t, int vec) {
     if ((threadIdx.x & 31) == 0) {
         prefetch_l2(a.positions + t);
@@ -100,6 +100,7 @@ __device__ __forceinline__ void token_prefetch(const FusedArgs &a, int pack, int
     const int c = pack * vec;
     prefetch_l2(static_cast<const E *>(a.x) + static_cast<int64_t>(t) * a.x_rs + c);
     if (a.w_vec) prefetch_l2(static_cast<const E *>(a.w) + static_cast<int64_t>(c) * a.W);
+    if (!SPEC) return;
 
     const int64_t pos = __ldcg(a.positions + t);
     const int req = ONE ? t : __ldcg(a.seq_idx + t);
@@ -168,12 +169,12 @@ __device__ __forceinline__ void token_body(const FusedArgs &a, int pack, int t) 
         tap[0], t, c, k.slot, lane);
 }
 
-template <typename E, int VEC, int MAXW, bool ONE>
+template <typename E, int VEC, int MAXW, bool ONE, bool SPEC>
 __global__ void __launch_bounds__(kThreads) fused_token_kernel(const __grid_constant__ FusedArgs a) {
     const int pack = blockIdx.y * blockDim.x + threadIdx.x;
     const int t = blockIdx.x * blockDim.y + threadIdx.y;
     const bool in_range = pack < a.C / VEC && t < a.T;
-    if (in_range) token_prefetch<E, MAXW, ONE>(a, pack, t, VEC);
+    if (in_range) token_prefetch<E, MAXW, ONE, SPEC>(a, pack, t, VEC);
     pdl_wait();
     pdl_trigger();
     if (in_range) token_body<E, VEC, MAXW, ONE>(a, pack, t);
@@ -190,7 +191,7 @@ struct StreamSet {
     int y0[SCONV_MAX_STREAMS + 1];  // first y block of each stream, y0[n] = total
 };
 
-template <typename E, int VEC, int MAXW>
+template <typename E, int VEC, int MAXW, bool SPEC>
 __global__ void __launch_bounds__(kThreads) fused_streams_kernel(const __grid_constant__ StreamSet m) {
     int si = 0;
     while (si + 1 < m.n && static_cast<int>(blockIdx.y) >= m.y0[si + 1]) ++si;
@@ -198,7 +199,7 @@ __global__ void __launch_bounds__(kThreads) fused_streams_kernel(const __grid_co
     const int pack = (blockIdx.y - m.y0[si]) * blockDim.x + threadIdx.x;
     const int t = blockIdx.x * blockDim.y + threadIdx.y;
     const bool in_range = pack < a.C / VEC && t < a.T;
-    if (in_range) token_prefetch<E, MAXW, false>(a, pack, t, VEC);
+    if (in_range) token_prefetch<E, MAXW, false, SPEC>(a, pack, t, VEC);
     pdl_wait();
     pdl_trigger();
     if (in_range) token_body<E, VEC, MAXW, false>(a, pack, t);
@@ -364,6 +365,11 @@ inline Shape block_shape(int nv, int64_t rows) {
     return s;
 }
 
+// Speculative prefetching before the PDL wait pays off only when this
+// launch's blocks can be resident while the preceding kernel still runs:
+// a launch of at most a quarter of the GPU's thread slots (148 SMs x 2048).
+inline bool speculate(int64_t threads) { return threads <= 148LL * 512; }
+
 // Strip kernel only when there is enough work to stream: T*C/VEC
 // token-packs above this many.
 constexpr int64_t kStripMinWork = 1 << 19;
@@ -377,11 +383,17 @@ cudaError_t launch_w(FusedArgs &a, bool one, cudaStream_t stream) {
         const Shape s = block_shape(nv, a.T);
         dim3 grid(static_cast<unsigned>((a.T + s.tg - 1) / s.tg),
                   static_cast<unsigned>((nv + s.cv - 1) / s.cv));
+        const bool spec =
+            speculate(static_cast<int64_t>(grid.x) * grid.y * s.cv * s.tg);
         if (one)
-            return launch_pdl(fused_token_kernel<E, VEC, MAXW, true>, grid, dim3(s.cv, s.tg), 0,
-                              stream, a);
-        return launch_pdl(fused_token_kernel<E, VEC, MAXW, false>, grid, dim3(s.cv, s.tg), 0,
-                          stream, a);
+            return spec ? launch_pdl(fused_token_kernel<E, VEC, MAXW, true, true>, grid,
+                                     dim3(s.cv, s.tg), 0, stream, a)
+                        : launch_pdl(fused_token_kernel<E, VEC, MAXW, true, false>, grid,
+                                     dim3(s.cv, s.tg), 0, stream, a);
+        return spec ? launch_pdl(fused_token_kernel<E, VEC, MAXW, false, true>, grid,
+                                 dim3(s.cv, s.tg), 0, stream, a)
+                    : launch_pdl(fused_token_kernel<E, VEC, MAXW, false, false>, grid,
+                                 dim3(s.cv, s.tg), 0, stream, a);
     }
     if constexpr (sizeof(E) == 2 && VEC == 8) {
         bool used = false;
@@ -427,7 +439,11 @@ cudaError_t launch_streams_t(FusedArgs *s, int n, cudaStream_t stream) {
     }
     for (int i = n; i < SCONV_MAX_STREAMS; ++i) m.s[i] = s[0];  // never selected
     dim3 grid(static_cast<unsigned>((s[0].T + sh.tg - 1) / sh.tg), static_cast<unsigned>(m.y0[n]));
-    return launch_pdl(fused_streams_kernel<E, VEC, MAXW>, grid, dim3(sh.cv, sh.tg), 0, stream, m);
+    if (speculate(static_cast<int64_t>(grid.x) * grid.y * sh.cv * sh.tg))
+        return launch_pdl(fused_streams_kernel<E, VEC, MAXW, true>, grid, dim3(sh.cv, sh.tg), 0,
+                          stream, m);
+    return launch_pdl(fused_streams_kernel<E, VEC, MAXW, false>, grid, dim3(sh.cv, sh.tg), 0,
+                      stream, m);
 }
 
 template <typename E, int VEC>

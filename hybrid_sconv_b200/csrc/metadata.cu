@@ -18,10 +18,13 @@ seq_metadata_kernel(const int32_t *__restrict__ qsl, int num_reqs, int num_actua
                     int num_padded, int32_t *__restrict__ seq_idx,
                     int32_t *__restrict__ query_start, int staged) {
     extern __shared__ int32_t s_qsl[];
-    // Pull the offsets table into L2 while the preceding kernel drains.
+    // Let the next kernel (typically the fused step that reads these
+    // buffers) launch at once: its own wait still orders it after this
+    // kernel, and it gets this kernel's whole wait to prefetch.  Then pull
+    // the offsets table into L2 while the preceding kernel drains.
+    pdl_trigger();
     for (int i = threadIdx.x * 32; i < num_reqs; i += blockDim.x * 32) prefetch_l2(qsl + i);
     pdl_wait();
-    pdl_trigger();
     if (staged) {
         for (int i = threadIdx.x; i < num_reqs; i += blockDim.x) s_qsl[i] = __ldg(qsl + i);
         __syncthreads();
