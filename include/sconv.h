@@ -207,6 +207,58 @@ sconv_status sconv_extract_windows(
     cudaStream_t stream);
 
 /*
+ * sconv_scatter_intermediate_ssm -- conditional row gather of SSM chunk-scan
+ * states for prefix caching ("core.ssm.ops.intermediate_extraction",
+ * _scatter_intermediate_ssm_kernel / scatter_intermediate_ssm): for slot
+ * i < *real_count, out row i = states row chunk_indices[i] (state_flat
+ * elements); slots i >= *real_count are left untouched and move no data.
+ *
+ *   states         [num_chunks, state_flat], row stride states_row_stride
+ *                  (elements), rows contiguous.
+ *   chunk_indices  [max_count] int64 per-slot row index.
+ *   real_count     DEVICE int32[1], clamped to [0, max_count], read on the
+ *                  device (may change between graph replays).
+ *   out            [max_count, state_flat], row stride out_row_stride; must
+ *                  not overlap states.
+ *   err_flag       optional device int32: a slot whose index is outside
+ *                  [0, num_chunks) is left untouched and sets
+ *                  SCONV_EFLAG_REQUEST.
+ * The copy is bit-exact (dt only fixes the element size).  max_count == 0
+ * returns SCONV_OK and enqueues nothing.
+ */
+sconv_status sconv_scatter_intermediate_ssm(
+    const void *states, int64_t num_chunks, int64_t state_flat, int64_t states_row_stride,
+    const int64_t *chunk_indices, const int32_t *real_count, int max_count, void *out,
+    int64_t out_row_stride, sconv_dtype dt, int32_t *err_flag, cudaStream_t stream);
+
+/*
+ * sconv_extract_windows_paged -- the window extraction of
+ * sconv_extract_windows with the conv input read from the paged cache of
+ * the vllm sconv page instead of a dense source: for slot i < *real_count,
+ * out[i][c][k] = cache[block_table[req, p / N], h, p % N, off_s + j] with
+ * req = request[i], p = abs_positions[i] - d_conv + k, c = h*ws + j, and
+ * zero for p < 0.  Slots i >= *real_count are untouched.
+ *
+ *   cache, cache_strides, num_blocks, H, N, D, off_s, ws: as in sconv_fused.
+ *   block_table    [num_reqs, max_blocks] int32, row stride bt_row_stride.
+ *   request        [max_count] int32 block-table row of each slot.
+ *   abs_positions  [max_count] int32 window end (exclusive) of each slot.
+ *   real_count     DEVICE int32[1], clamped to [0, max_count].
+ *   out            [max_count, C, d_conv] (C = H * ws), out[i][c][k] at
+ *                  i*out_slot_stride + c*d_conv + k; must not overlap the cache.
+ *   err_flag       optional: a slot whose request or block-table entry is
+ *                  out of range is left untouched and sets SCONV_EFLAG_REQUEST,
+ *                  SCONV_EFLAG_LOGICAL or SCONV_EFLAG_BLOCK.
+ * d_conv in 1..SCONV_MAX_DCONV.  max_count == 0 returns SCONV_OK.
+ */
+sconv_status sconv_extract_windows_paged(
+    const void *cache, const int64_t cache_strides[4], int64_t num_blocks, int H, int N, int D,
+    int off_s, int ws, const int32_t *block_table, int64_t bt_row_stride, int num_reqs,
+    int max_blocks, const int32_t *request, const int32_t *abs_positions,
+    const int32_t *real_count, int max_count, void *out, int64_t out_slot_stride, int d_conv,
+    sconv_dtype dt, int32_t *err_flag, cudaStream_t stream);
+
+/*
  * sconv_seq_metadata -- fill the per-token request index and request start
  * in one launch ("vllm.models.inkling.nvidia.ops.sconv", sconv_seq_metadata).
  *

@@ -61,6 +61,12 @@ def _bind(path: str) -> ctypes.CDLL:
     lib.oracle_extract_windows.restype = None
     lib.oracle_extract_windows.argtypes = [
         _INT, _P, _I64, _I64, _I64, _I64, _P, _I64, _I64, _P, _I64, _I64]
+    lib.oracle_scatter_ssm.restype = _I64
+    lib.oracle_scatter_ssm.argtypes = [_INT, _P, _I64, _I64, _I64, _P, _I64, _I64, _P, _I64]
+    lib.oracle_extract_windows_paged.restype = _I64
+    lib.oracle_extract_windows_paged.argtypes = [
+        _INT, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _I64, _I64, _I64, _P, _P, _I64,
+        _I64, _P, _I64, _I64]
     lib.oracle_check_preconditions.restype = _INT
     lib.oracle_check_preconditions.argtypes = [
         _I64, _INT, _I64, _P, _P, _P, _P, _P, _I64, _I64]
@@ -254,6 +260,42 @@ def extract_windows(*, dtype, src, abs_positions, real_count, out, d_conv):
         _DT[dtype], _ptr(sa), seq_len, conv_dim, conv_dim, 1, _ptr(ap),
         int(real_count), max_count, _ptr(oa), conv_dim * d_conv, d_conv)
     return oa
+
+
+def scatter_ssm(*, dtype, states, chunk_indices, real_count, out):
+    """Oracle of scatter_intermediate_ssm ("core.ssm.ops.intermediate_extraction").
+    ``states`` [num_chunks, ...] and ``out`` [max_count, ...] (same trailing
+    shape); returns (a new out array, slots skipped for a bad index)."""
+    sa = _float_array(states, dtype)
+    oa = _float_array(out, dtype).copy()
+    idx = _np(chunk_indices, np.int64)
+    num_chunks = sa.shape[0]
+    flat = int(np.prod(sa.shape[1:])) if sa.ndim > 1 else 1
+    skipped = lib().oracle_scatter_ssm(_DT[dtype], _ptr(sa), num_chunks, flat, flat, _ptr(idx),
+                                       int(real_count), oa.shape[0], _ptr(oa), flat)
+    return oa, int(skipped)
+
+
+def extract_windows_paged(*, dtype, cache, block_table, request, abs_positions, real_count,
+                          out, d_conv, off_s, ws):
+    """Window gather from the paged cache (sconv_extract_windows_paged):
+    out [max_count, H*ws, d_conv] holds the prior bytes.  Returns (a new
+    out array, slots skipped)."""
+    ca = _float_array(cache, dtype)
+    nb, H, N, D = ca.shape
+    strides = np.array([st // ca.itemsize for st in ca.strides], np.int64)
+    bt = _np(block_table, np.int32)
+    rq = _np(request, np.int32)
+    ap = _np(abs_positions, np.int32)
+    oa = _float_array(out, dtype).copy()
+    max_count = oa.shape[0]
+    skipped = lib().oracle_extract_windows_paged(
+        _DT[dtype], _ptr(ca), _ptr(strides), nb, H, N, off_s, ws, _ptr(bt), bt.shape[1],
+        bt.shape[0], bt.shape[1], _ptr(rq), _ptr(ap), int(real_count), max_count, _ptr(oa),
+        H * ws * d_conv, d_conv)
+    if skipped < 0:
+        raise ValueError("oracle_extract_windows_paged: malformed arguments")
+    return oa, int(skipped)
 
 
 def check_preconditions(*, W, block_size, positions, seq_idx, slot_mapping,

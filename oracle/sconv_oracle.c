@@ -306,3 +306,85 @@ int oracle_check_preconditions(int64_t T, int W, int64_t N,
     free(read);
     return result;
 }
+
+/*
+ * oracle_scatter_ssm -- [P2] scatter_intermediate_ssm: for slot
+ * i < real_count (clamped to [0, max_count]) out row i becomes states row
+ * chunk_indices[i] (state_flat elements, a byte copy).  Slots at or beyond
+ * real_count, and slots whose index is outside [0, num_chunks), keep their
+ * bytes.  Returns the number of slots skipped for a bad index.
+ */
+int64_t oracle_scatter_ssm(int dtype, const void *states, int64_t num_chunks,
+                           int64_t state_flat, int64_t states_row_stride,
+                           const int64_t *chunk_indices, int64_t real_count,
+                           int64_t max_count, void *out, int64_t out_row_stride) {
+    if (real_count > max_count) real_count = max_count;
+    int64_t skipped = 0;
+    for (int64_t i = 0; i < real_count; ++i) {
+        int64_t row = chunk_indices[i];
+        if (row < 0 || row >= num_chunks) {
+            ++skipped;
+            continue;
+        }
+        for (int64_t e = 0; e < state_flat; ++e)
+            copy_element(out, i * out_row_stride + e, states, row * states_row_stride + e,
+                         dtype);
+    }
+    return skipped;
+}
+
+/*
+ * oracle_extract_windows_paged -- the window gather of
+ * oracle_extract_windows with the conv input read from the paged cache of
+ * [P1]: for slot i < real_count, request r = request[i] and
+ * p = abs_positions[i] - d_conv + k,
+ *     out[i][c][k] = cache[block_table[r][p / N], h, p % N, off_s + j]
+ * (c = h*ws + j), zero for p < 0.  A slot whose request, logical block or
+ * block-table entry is out of range keeps its bytes and is counted.
+ */
+int64_t oracle_extract_windows_paged(int dtype, const void *cache,
+                                     const int64_t *cache_strides, int64_t num_blocks,
+                                     int64_t H, int64_t N, int64_t off_s, int64_t ws,
+                                     const int32_t *block_table, int64_t bt_row_stride,
+                                     int64_t num_reqs, int64_t max_blocks,
+                                     const int32_t *request, const int32_t *abs_positions,
+                                     int64_t real_count, int64_t max_count, void *out,
+                                     int64_t out_slot_stride, int64_t d_conv) {
+    if (real_count > max_count) real_count = max_count;
+    if (d_conv > 64) return -1;
+    size_t e = elem_bytes(dtype);
+    int64_t skipped = 0;
+    int64_t blk[64];
+    for (int64_t i = 0; i < real_count; ++i) {
+        int64_t r = request[i];
+        int bad = r < 0 || r >= num_reqs;
+        for (int64_t k = 0; k < d_conv && !bad; ++k) {
+            int64_t p = (int64_t)abs_positions[i] - d_conv + k;
+            blk[k] = -1;
+            if (p < 0) continue;
+            if (p / N >= max_blocks) { bad = 1; break; }
+            int64_t b = block_table[r * bt_row_stride + p / N];
+            if (b < 0 || b >= num_blocks) { bad = 1; break; }
+            blk[k] = b;
+        }
+        if (bad) {
+            ++skipped;
+            continue;
+        }
+        for (int64_t c = 0; c < H * ws; ++c) {
+            int64_t h = c / ws, j = c % ws;
+            for (int64_t k = 0; k < d_conv; ++k) {
+                int64_t p = (int64_t)abs_positions[i] - d_conv + k;
+                int64_t dst = i * out_slot_stride + c * d_conv + k;
+                if (p < 0) {
+                    memset((char *)out + dst * (int64_t)e, 0, e);
+                } else {
+                    int64_t src = blk[k] * cache_strides[0] + h * cache_strides[1] +
+                                  (p % N) * cache_strides[2] + (off_s + j) * cache_strides[3];
+                    copy_element(out, dst, cache, src, dtype);
+                }
+            }
+        }
+    }
+    return skipped;
+}

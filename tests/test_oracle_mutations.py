@@ -75,6 +75,18 @@ MUTANTS = [
     ("extract_not_transposed",
      "int64_t dst = i * out_slot_stride + c * d_conv + k;",
      "int64_t dst = i * out_slot_stride + k * conv_dim + c;"),
+    ("ssm_row_reversed",
+     "            copy_element(out, i * out_row_stride + e, states, row * states_row_stride + e,",
+     "            copy_element(out, i * out_row_stride + e, states, row * states_row_stride + (state_flat - 1 - e),"),
+    ("ssm_ignores_bad_index_check",
+     "        if (row < 0 || row >= num_chunks) {",
+     "        if (row < 0 || row >= num_chunks || row == 0) {"),
+    ("paged_offset_shifted",
+     "                                  (p % N) * cache_strides[2] + (off_s + j) * cache_strides[3];\n                    copy_element(out, dst, cache, src, dtype);",
+     "                                  ((p + 1) % N) * cache_strides[2] + (off_s + j) * cache_strides[3];\n                    copy_element(out, dst, cache, src, dtype);"),
+    ("paged_zero_at_position_0",
+     "                if (p < 0) {\n                    memset",
+     "                if (p < 1) {\n                    memset"),
     ("extract_ignores_real_count",
      "    for (int64_t i = 0; i < real_count; ++i) {",
      "    for (int64_t i = 0; i < max_count; ++i) {"),

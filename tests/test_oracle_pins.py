@@ -483,3 +483,99 @@ def test_streams_equal_sequential_single_stream_calls(seed):
                 np.testing.assert_array_equal(
                     cache_all[b, h, p % wl.N, sd["off_s"]:sd["off_s"] + sd["ws"]],
                     xs[row, h * sd["ws"]:(h + 1) * sd["ws"]])
+
+
+# --------------------------------------------------------------------------
+# SSM state gather and window extraction from the paged cache
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("real", [0, 3, 7, 20])
+def test_scatter_ssm_against_fancy_indexing(dtype, real):
+    rng = np.random.default_rng(real)
+    states = torch.randn(11, 3, 5).to(workloads.TORCH_DTYPE[dtype])
+    idx = rng.integers(0, 11, size=7).astype(np.int64)
+    idx[2] = 11  # out of range: that slot is skipped
+    out = workloads.sentinel((7, 3, 5), dtype)
+    got, skipped = oracle.scatter_ssm(dtype=dtype, states=states, chunk_indices=idx,
+                                      real_count=real, out=out)
+    raw_s = oracle._float_array(states, dtype)
+    raw_o = oracle._float_array(out, dtype)
+    expect = raw_o.copy()
+    rc = min(real, 7)
+    for i in range(rc):
+        if 0 <= idx[i] < 11:
+            expect[i] = raw_s[idx[i]]
+    np.testing.assert_array_equal(got.view(np.uint8), expect.view(np.uint8))
+    assert skipped == (1 if rc > 2 else 0)
+
+
+def _paged_windows_by_indexing(cache_raw, bt, req, pos, d_conv, off_s, ws, N, out_raw):
+    H = cache_raw.shape[1]
+    out = out_raw.copy()
+    for i, (r, p_end) in enumerate(zip(req, pos)):
+        for k in range(d_conv):
+            p = int(p_end) - d_conv + k
+            for h in range(H):
+                if p < 0:
+                    out[i, h * ws:(h + 1) * ws, k] = 0
+                else:
+                    out[i, h * ws:(h + 1) * ws, k] = cache_raw[bt[r, p // N], h, p % N,
+                                                               off_s:off_s + ws]
+    return out
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d_conv", [1, 4, 6])
+def test_extract_windows_paged_against_indexing(dtype, d_conv):
+    wl = workloads.random_case(61 + d_conv, dtype=dtype, max_hist=30)
+    t = wl.tensors()
+    rng = np.random.default_rng(d_conv)
+    n = 9
+    req = rng.integers(0, wl.R, size=n).astype(np.int32)
+    lengths = wl.hist + wl.new
+    pos = np.array([rng.integers(0, lengths[r] + 1) for r in req], np.int32)
+    out = workloads.sentinel((n, wl.C, d_conv), dtype)
+    got, skipped = oracle.extract_windows_paged(
+        dtype=dtype, cache=t["cache"], block_table=wl.block_table, request=req,
+        abs_positions=pos, real_count=6, out=out, d_conv=d_conv, off_s=wl.off_s, ws=wl.ws)
+    assert skipped == 0
+    raw_o = oracle._float_array(out, dtype)
+    expect = _paged_windows_by_indexing(oracle._float_array(t["cache"], dtype),
+                                        wl.block_table, req[:6], pos[:6], d_conv, wl.off_s,
+                                        wl.ws, wl.N, raw_o)
+    np.testing.assert_array_equal(got.view(np.uint8), expect.view(np.uint8))
+
+
+def test_extract_windows_paged_equals_dense_after_prefill():
+    """Prefill sequences from position 0 (the fused oracle inserts every
+    token into the paged cache); windows read back from the cache equal the
+    dense extraction from the same x rows."""
+    wl = workloads.build("pf", dtype="bf16", H=3, D=20, ws=6, off_s=7, W=4, N=4,
+                         hist=[0, 0], new=[13, 9], act="silu", residual=False, seed=5)
+    t = wl.tensors()
+    _, _, cache_after, _ = run_fused(wl, t)
+    d_conv, rng = 4, np.random.default_rng(5)
+    for r in range(2):
+        a, b = int(wl.query_start_loc[r]), int(wl.query_start_loc[r + 1])
+        pos = rng.integers(0, b - a + 1, size=5).astype(np.int32)
+        out = workloads.sentinel((5, wl.C, d_conv), "bf16")
+        paged, _ = oracle.extract_windows_paged(
+            dtype="bf16", cache=cache_after, block_table=wl.block_table,
+            request=np.full(5, r, np.int32), abs_positions=pos, real_count=5, out=out,
+            d_conv=d_conv, off_s=wl.off_s, ws=wl.ws)
+        dense = oracle.extract_windows(dtype="bf16", src=t["x"][a:b], abs_positions=pos,
+                                       real_count=5, out=out, d_conv=d_conv)
+        np.testing.assert_array_equal(paged, dense)
+
+
+def test_extract_windows_paged_bad_indices_skip_the_slot():
+    wl = workloads.random_case(70, dtype="f32", max_hist=20)
+    t = wl.tensors()
+    req = np.array([0, wl.R, 0], np.int32)  # slot 1: no such request
+    pos = np.array([1, 1, 1], np.int32)
+    out = workloads.sentinel((3, wl.C, 2), "f32")
+    got, skipped = oracle.extract_windows_paged(
+        dtype="f32", cache=t["cache"], block_table=wl.block_table, request=req,
+        abs_positions=pos, real_count=3, out=out, d_conv=2, off_s=wl.off_s, ws=wl.ws)
+    assert skipped == 1
+    assert (got[1].view(np.uint32) == 0xFFFFFFFF).all()
