@@ -429,6 +429,22 @@ def bench_prefill(name, device, stream, peak, reps=None):
         out_table["extract_windows_long_prefill"] = {
             "kernel_us": round(secs * 1e6, 3), "alg_bytes": nbytes,
             "alg_gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
+        # the same windows read through the block table from the paged cache
+        req = torch.zeros(e["max_count"], dtype=torch.int32, device=device)
+        pfns = []
+        for _ in range(48):
+            pos = torch.from_numpy(rng.integers(e["d_conv"], wl.T + 1, size=e["max_count"])
+                                   .astype(np.int32)).to(device)
+            o = torch.empty((e["max_count"], wl.C, e["d_conv"]), dtype=torch.bfloat16,
+                            device=device)
+            pfns.append(lambda pos=pos, o=o: hs.sconv_extract_windows_paged(
+                t["cache"], t["block_table"], req, pos, rc, o, e["d_conv"], wl.off_s, wl.ws))
+        secs = _kernel_time(pfns, 50, stream)
+        nbytes += 4 * e["max_count"] + 4 * 2 * e["real_count"]  # requests, block-table entries
+        gbs = nbytes / secs / 1e9
+        out_table["extract_windows_paged_long_prefill"] = {
+            "kernel_us": round(secs * 1e6, 3), "alg_bytes": nbytes,
+            "alg_gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
     del t, out
     torch.cuda.empty_cache()
     return out_table
@@ -504,6 +520,34 @@ def bench_streams(sets_obj, stream, peak, reps=200):
         "alg_gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}}
 
 
+def bench_ssm_gather(device, stream, peak, reps=50):
+    """Conditional SSM state gather: 256 chunk-scan states of [64, 64, 128]
+    fp32 (2 MB rows), 64 slots of which 40 real, 8 rotating index sets over
+    4 state tensors (1 GiB of distinct rows > L2)."""
+    import hybrid_sconv_b200 as hs
+    g = torch.Generator(device=device).manual_seed(11)
+    shape, nchunks, max_count, real = (64, 64, 128), 128, 64, 40
+    states = [workloads.normal((nchunks,) + shape, 1.0, torch.float32, g, device)
+              for _ in range(4)]
+    rng = np.random.default_rng(11)
+    rc = torch.tensor([real], dtype=torch.int32, device=device)
+    fns = []
+    for j in range(8):
+        idx = torch.from_numpy(rng.integers(0, nchunks, size=max_count)).to(device)
+        out = torch.empty((max_count,) + shape, dtype=torch.float32, device=device)
+        st = states[j % 4]
+        fns.append(lambda st=st, idx=idx, out=out: hs.sconv_scatter_intermediate_ssm(
+            st, idx, rc, out))
+    secs = _kernel_time(fns, reps, stream)
+    nbytes = 2 * real * int(np.prod(shape)) * 4 + 8 * max_count + 4
+    gbs = nbytes / secs / 1e9
+    del states, fns
+    torch.cuda.empty_cache()
+    return {"scatter_intermediate_ssm": {
+        "kernel_us": round(secs * 1e6, 3), "alg_bytes": nbytes, "alg_gbs": round(gbs, 1),
+        "frac": round(gbs / peak, 4)}}
+
+
 def per_workload_table(device, stream, peak, sets_obj=None):
     table = {}
     if sets_obj is not None:
@@ -512,6 +556,7 @@ def per_workload_table(device, stream, peak, sets_obj=None):
     table.update(bench_prefill("chunked_prefill_bf16", device, stream, peak))
     table.update(bench_prefill("long_prefill_bf16", device, stream, peak))
     table.update(bench_spec_decode(device, stream, peak))
+    table.update(bench_ssm_gather(device, stream, peak))
     return table
 
 

@@ -15,8 +15,9 @@ using one without the library raises ImportError (there is no fallback).
 _EXPORTS = (
     "EFLAG_BLOCK", "EFLAG_LOGICAL", "EFLAG_POSITION", "EFLAG_QUERY_START", "EFLAG_REQUEST",
     "EFLAG_SLOT", "EFLAG_TIMEOUT", "LIB_PATH", "SconvError", "fused_sconv",
-    "scatter_intermediate_conv", "sconv_extract_windows", "sconv_fused", "sconv_fused_streams",
-    "sconv_seq_metadata", "sconv_update",
+    "scatter_intermediate_conv", "scatter_intermediate_ssm", "sconv_extract_windows",
+    "sconv_extract_windows_paged", "sconv_fused", "sconv_fused_streams",
+    "sconv_scatter_intermediate_ssm", "sconv_seq_metadata", "sconv_update",
 )
 
 __all__ = list(_EXPORTS)

@@ -73,6 +73,11 @@ _SIGNATURES = {
     "sconv_extract_windows": [
         _P, _I64, _INT, _I64, _I64, _P, _P, _INT, _P, _I64, _INT, _INT, _P],
     "sconv_seq_metadata": [_P, _INT, _INT, _INT, _P, _I64, _P, _I64, _P],
+    "sconv_scatter_intermediate_ssm": [
+        _P, _I64, _I64, _I64, _P, _P, _INT, _P, _I64, _INT, _P, _P],
+    "sconv_extract_windows_paged": [
+        _P, _I64P, _I64, _INT, _INT, _INT, _INT, _INT, _P, _I64, _INT, _INT, _P, _P, _P, _INT,
+        _P, _I64, _INT, _INT, _P, _P],
 }
 
 
@@ -321,6 +326,72 @@ def sconv_extract_windows(src, abs_positions, real_count, out, d_conv, *, stream
     return out
 
 
+def sconv_scatter_intermediate_ssm(states, chunk_indices, real_count, out, *, err_flag=None,
+                                   stream=None):
+    """Gather rows of ``states`` [num_chunks, *state_shape] at
+    ``chunk_indices`` (int64 [max_count]) into ``out`` [max_count,
+    *state_shape] for the first ``real_count[0]`` slots only
+    (scatter_intermediate_ssm, "core.ssm.ops.intermediate_extraction")."""
+    dt = _DTYPES.get(states.dtype)
+    if dt is None or out.dtype != states.dtype:
+        raise TypeError("states and out must share one dtype, float32 or bfloat16")
+    max_count = out.shape[0]
+    if max_count == 0:
+        return out
+    if tuple(out.shape[1:]) != tuple(states.shape[1:]):
+        raise ValueError("out must be [max_count, *states.shape[1:]]")
+    st2 = states.reshape(states.shape[0], -1)
+    out2 = out.view(max_count, -1)
+    if st2.shape[0] and st2.stride(1) != 1 or out2.stride(1) != 1:
+        raise ValueError("state rows must be contiguous")
+    d = _dev(states, chunk_indices, real_count, out, err_flag)
+    _vector(chunk_indices, torch.int64, "chunk_indices", max_count)
+    _vector(real_count, torch.int32, "real_count", 1)
+    if err_flag is not None:
+        _vector(err_flag, torch.int32, "err_flag", 1)
+    with torch.cuda.device(d):
+        st = LIB.sconv_scatter_intermediate_ssm(
+            _ptr(st2), st2.shape[0], st2.shape[1], st2.stride(0) if st2.shape[0] else st2.shape[1],
+            _ptr(chunk_indices), _ptr(real_count), max_count, _ptr(out2), out2.stride(0), dt,
+            _ptr(err_flag), _stream(d, stream))
+    _check("sconv_scatter_intermediate_ssm", st)
+    return out
+
+
+def sconv_extract_windows_paged(cache, block_table, request, abs_positions, real_count, out,
+                                d_conv, off_s, ws, *, err_flag=None, stream=None):
+    """Windows [pos - d_conv, pos) of each slot's request read from the
+    paged cache [num_blocks, H, N, D] through ``block_table`` into ``out``
+    [max_count, H*ws, d_conv], for the first ``real_count[0]`` slots."""
+    dt = _DTYPES.get(cache.dtype)
+    if dt is None or out.dtype != cache.dtype:
+        raise TypeError("cache and out must share one dtype, float32 or bfloat16")
+    max_count = out.shape[0]
+    if max_count == 0:
+        return out
+    nb, H, N, D = cache.shape
+    if out.dim() != 3 or out.shape[1] != H * ws or out.shape[2] != d_conv or             out.stride(2) != 1 or out.stride(1) != d_conv:
+        raise ValueError("out must be [max_count, H*ws, d_conv] with dense inner dims")
+    d = _dev(cache, block_table, request, abs_positions, real_count, out, err_flag)
+    _vector(request, torch.int32, "request", max_count)
+    _vector(abs_positions, torch.int32, "abs_positions", max_count)
+    _vector(real_count, torch.int32, "real_count", 1)
+    _want(block_table, torch.int32, "block_table")
+    if block_table.dim() != 2 or block_table.stride(1) != 1:
+        raise ValueError("block_table must be [num_reqs, max_blocks] with unit inner stride")
+    if err_flag is not None:
+        _vector(err_flag, torch.int32, "err_flag", 1)
+    cs = (ctypes.c_int64 * 4)(*cache.stride())
+    with torch.cuda.device(d):
+        st = LIB.sconv_extract_windows_paged(
+            _ptr(cache), cs, nb, H, N, D, off_s, ws, _ptr(block_table), block_table.stride(0),
+            block_table.shape[0], block_table.shape[1], _ptr(request), _ptr(abs_positions),
+            _ptr(real_count), max_count, _ptr(out), out.stride(0), d_conv, dt, _ptr(err_flag),
+            _stream(d, stream))
+    _check("sconv_extract_windows_paged", st)
+    return out
+
+
 def sconv_seq_metadata(query_start_loc, num_reqs, num_actual_tokens, seq_idx_out,
                        query_start_out, num_padded_tokens=None, *, stream=None):
     """Fill seq_idx_out / query_start_out for every token row in one launch
@@ -351,3 +422,4 @@ def sconv_seq_metadata(query_start_loc, num_reqs, num_actual_tokens, seq_idx_out
 # Names used on the pages, for callers coming from them.
 fused_sconv = sconv_fused
 scatter_intermediate_conv = sconv_extract_windows
+scatter_intermediate_ssm = sconv_scatter_intermediate_ssm

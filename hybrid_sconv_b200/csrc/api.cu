@@ -245,6 +245,101 @@ sconv_status sconv_extract_windows(const void *src, int64_t seq_len, int conv_di
                : SCONV_ERR_LAUNCH;
 }
 
+sconv_status sconv_scatter_intermediate_ssm(const void *states, int64_t num_chunks,
+                                            int64_t state_flat, int64_t states_row_stride,
+                                            const int64_t *chunk_indices,
+                                            const int32_t *real_count, int max_count, void *out,
+                                            int64_t out_row_stride, sconv_dtype dt,
+                                            int32_t *err_flag, cudaStream_t stream) {
+    if (dt != SCONV_F32 && dt != SCONV_BF16) return SCONV_ERR_UNSUPPORTED;
+    if (max_count < 0 || num_chunks < 0 || state_flat < 1) return SCONV_ERR_INVALID;
+    if (max_count > 65535) return SCONV_ERR_UNSUPPORTED;  // one grid row per slot
+    if (max_count == 0) return SCONV_OK;
+    if (!states || !chunk_indices || !real_count || !out) return SCONV_ERR_INVALID;
+    if (states_row_stride < state_flat || out_row_stride < state_flat) return SCONV_ERR_INVALID;
+    const int64_t e = elem_size(dt);
+    const int64_t out_bytes = ((max_count - 1) * out_row_stride + state_flat) * e;
+    const int64_t st_bytes = num_chunks > 0 ? ((num_chunks - 1) * states_row_stride + state_flat) * e : 0;
+    if (st_bytes > 0 && overlaps(out, out_bytes, states, st_bytes)) return SCONV_ERR_INVALID;
+    const bool vec = aligned16(states) && aligned16(out) && (state_flat * e) % 16 == 0 &&
+                     (states_row_stride * e) % 16 == 0 && (out_row_stride * e) % 16 == 0;
+    sconv::SsmArgs a;
+    a.states = states;
+    a.num_chunks = num_chunks;
+    a.state_flat = state_flat;
+    a.states_rs = states_row_stride;
+    a.idx = chunk_indices;
+    a.real_count = real_count;
+    a.max_count = max_count;
+    a.out = out;
+    a.out_rs = out_row_stride;
+    a.err = err_flag;
+    return sconv::launch_scatter_ssm(a, static_cast<int>(e), vec, stream) == cudaSuccess
+               ? SCONV_OK
+               : SCONV_ERR_LAUNCH;
+}
+
+sconv_status sconv_extract_windows_paged(const void *cache, const int64_t cache_strides[4],
+                                         int64_t num_blocks, int H, int N, int D, int off_s,
+                                         int ws, const int32_t *block_table,
+                                         int64_t bt_row_stride, int num_reqs, int max_blocks,
+                                         const int32_t *request, const int32_t *abs_positions,
+                                         const int32_t *real_count, int max_count, void *out,
+                                         int64_t out_slot_stride, int d_conv, sconv_dtype dt,
+                                         int32_t *err_flag, cudaStream_t stream) {
+    if (dt != SCONV_F32 && dt != SCONV_BF16) return SCONV_ERR_UNSUPPORTED;
+    if (max_count < 0 || d_conv < 1) return SCONV_ERR_INVALID;
+    if (d_conv > SCONV_MAX_DCONV) return SCONV_ERR_UNSUPPORTED;
+    if (max_count == 0) return SCONV_OK;
+    if (H < 1 || N < 1 || D < 1 || ws < 1 || off_s < 0 || static_cast<int64_t>(off_s) + ws > D)
+        return SCONV_ERR_INVALID;
+    if (num_blocks < 1 || num_reqs < 1 || max_blocks < 1 || bt_row_stride < max_blocks)
+        return SCONV_ERR_INVALID;
+    if (!cache || !cache_strides || !block_table || !request || !abs_positions || !real_count ||
+        !out)
+        return SCONV_ERR_INVALID;
+    if (cache_strides[3] != 1 || cache_strides[0] < 1 || cache_strides[1] < 1 ||
+        cache_strides[2] < 1)
+        return SCONV_ERR_INVALID;
+    const int64_t C = static_cast<int64_t>(H) * ws;
+    if (out_slot_stride < C * d_conv) return SCONV_ERR_INVALID;
+    const int64_t e = elem_size(dt);
+    const int64_t out_bytes = ((max_count - 1) * out_slot_stride + C * d_conv) * e;
+    const int64_t cache_bytes = ((num_blocks - 1) * cache_strides[0] +
+                                 static_cast<int64_t>(H - 1) * cache_strides[1] +
+                                 static_cast<int64_t>(N - 1) * cache_strides[2] + D) * e;
+    if (overlaps(out, out_bytes, cache, cache_bytes)) return SCONV_ERR_INVALID;
+    const int64_t V = 16 / e;
+    const bool vec = aligned16(cache) && aligned16(out) && cache_strides[0] % V == 0 &&
+                     cache_strides[1] % V == 0 && cache_strides[2] % V == 0 && off_s % V == 0 &&
+                     ws % V == 0 && out_slot_stride % V == 0;
+    sconv::PagedExtractArgs a;
+    a.cache = cache;
+    a.cs0 = cache_strides[0];
+    a.cs1 = cache_strides[1];
+    a.cs2 = cache_strides[2];
+    a.num_blocks = num_blocks;
+    a.H = H;
+    a.N = N;
+    a.off_s = off_s;
+    a.ws = ws;
+    a.bt = block_table;
+    a.bt_rs = bt_row_stride;
+    a.num_reqs = num_reqs;
+    a.max_blocks = max_blocks;
+    a.request = request;
+    a.abs_pos = abs_positions;
+    a.real_count = real_count;
+    a.max_count = max_count;
+    a.out = out;
+    a.out_ss = out_slot_stride;
+    a.d_conv = d_conv;
+    a.err = err_flag;
+    return sconv::launch_extract_paged(a, dt == SCONV_BF16, vec, stream) == cudaSuccess
+               ? SCONV_OK
+               : SCONV_ERR_LAUNCH;
+}
+
 sconv_status sconv_seq_metadata(const int32_t *query_start_loc, int num_reqs,
                                 int num_actual_tokens, int num_padded_tokens,
                                 int32_t *seq_idx_out, int64_t seq_idx_cap,

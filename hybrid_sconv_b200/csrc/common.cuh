@@ -241,6 +241,34 @@ struct ExtractArgs {
     int d_conv;
 };
 
+// Conditional SSM state-row gather (scatter_intermediate_ssm).
+struct SsmArgs {
+    const void *states;
+    int64_t num_chunks, state_flat, states_rs;
+    const int64_t *idx;
+    const int32_t *real_count;
+    int max_count;
+    void *out;
+    int64_t out_rs;
+    int32_t *err;
+};
+
+// Window extraction from the paged cache.
+struct PagedExtractArgs {
+    const void *cache;
+    int64_t cs0, cs1, cs2, num_blocks;
+    int H, N, off_s, ws;
+    const int32_t *bt;
+    int64_t bt_rs;
+    int num_reqs, max_blocks;
+    const int32_t *request, *abs_pos, *real_count;
+    int max_count;
+    void *out;
+    int64_t out_ss;
+    int d_conv;
+    int32_t *err;
+};
+
 // Host-side launchers (return the cudaError_t of the launch).
 cudaError_t launch_fused(FusedArgs &a, bool bf16_data, bool vec, bool one_token_per_request,
                          cudaStream_t stream);
@@ -252,6 +280,9 @@ cudaError_t launch_fused_streams(FusedArgs *s, int n, bool bf16_data, bool vec,
 // nothing) when the call does not meet its layout requirements.
 cudaError_t launch_fused_tma(const FusedArgs &a, cudaStream_t stream, bool &used);
 cudaError_t launch_extract(const ExtractArgs &a, bool bf16_data, bool vec, cudaStream_t stream);
+cudaError_t launch_scatter_ssm(const SsmArgs &a, int elem_bytes, bool vec, cudaStream_t stream);
+cudaError_t launch_extract_paged(const PagedExtractArgs &a, bool bf16_data, bool vec,
+                                 cudaStream_t stream);
 cudaError_t launch_seq_metadata(const int32_t *qsl, int num_reqs, int num_actual, int num_padded,
                                 int32_t *seq_idx, int32_t *query_start, cudaStream_t stream);
 

@@ -170,3 +170,35 @@ def test_streams_host_validation(lib):
     assert call([ok_a, desc(FAKE * 512, FAKE * 1024, 8)]) == 1        # output is another's x
     assert call([ok_a] * 5) == 2                                       # more than 4 streams
     assert call([ok_a], n=0) == 1
+
+
+def test_gather_entry_points_host_validation(lib):
+    """Malformed calls of the SSM state gather and the paged window
+    extraction are rejected before any launch."""
+    def ssm(max_count=4, flat=64, srs=64, ors=64, dt=0, out=FAKE * 64, nchunks=8, rc=FAKE):
+        return lib.sconv_scatter_intermediate_ssm(FAKE, nchunks, flat, srs, FAKE * 2, rc,
+                                                  max_count, out, ors, dt, 0, 0)
+    assert ssm(max_count=0) == 0
+    assert ssm(max_count=-1) == 1
+    assert ssm(max_count=70000) == 2
+    assert ssm(flat=0) == 1
+    assert ssm(srs=32) == 1
+    assert ssm(ors=32) == 1
+    assert ssm(dt=4) == 2
+    assert ssm(out=FAKE + 16) == 1       # overlaps the states
+    assert ssm(rc=0) == 1
+
+    def paged(max_count=4, d_conv=4, off_s=0, ws=4, D=16, cs=None, oss=32, out=FAKE * 512,
+              bt_rs=4):
+        cs = cs or _strides(512, 256, 16, 1)
+        return lib.sconv_extract_windows_paged(FAKE * 64, cs, 8, 2, 16, D, off_s, ws, FAKE,
+                                               bt_rs, 2, 4, FAKE, FAKE, FAKE, max_count, out,
+                                               oss, d_conv, 1, 0, 0)
+    assert paged(max_count=0) == 0
+    assert paged(d_conv=9) == 2
+    assert paged(d_conv=0) == 1
+    assert paged(off_s=14) == 1          # off_s + ws > D
+    assert paged(cs=_strides(512, 256, 16, 2)) == 1
+    assert paged(oss=16) == 1            # slot stride < C * d_conv
+    assert paged(out=FAKE * 64 + 32) == 1  # inside the cache
+    assert paged(bt_rs=2) == 1
