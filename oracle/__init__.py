@@ -4,8 +4,10 @@ This package wraps ``sconv_oracle.c``: a plain, scalar, double-precision
 statement of what the path computes, written from the pages' definitions
 ("vllm.models.inkling.nvidia.ops.sconv": module docstring, fused_sconv,
 sconv_seq_metadata; "core.ssm.ops.intermediate_extraction":
-scatter_intermediate_conv).  Only the tests, the smoke check and the
-benchmark's CPU-baseline leg may import it.  The CUDA library never calls it
+scatter_intermediate_conv / scatter_intermediate_ssm; "Implementation:Sgl
+project Sglang Mamba Ops": causal_conv1d_fwd / causal_conv1d_update).
+Only the tests, the smoke check and the benchmark's CPU-baseline leg may
+import it.  The CUDA library never calls it
 and shares no code with it; the product path fails loudly without its own
 extension instead of falling back here.
 
@@ -67,6 +69,21 @@ def _bind(path: str) -> ctypes.CDLL:
     lib.oracle_extract_windows_paged.argtypes = [
         _INT, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _I64, _I64, _I64, _P, _P, _I64,
         _I64, _P, _I64, _I64]
+    lib.oracle_conv1d_fwd.restype = _I64
+    lib.oracle_conv1d_fwd.argtypes = [
+        _INT, _P, _I64, _I64, _I64, _I64,      # dtype, x, x_st, x_sc, total_tokens, dim
+        _P, _I64, _I64, _INT, _P,              # weight, w_sc, w_sk, W, bias
+        _P, _P, _I64, _I64, _I64, _I64, _I64,  # states in/out, strides, L, num_lines
+        _P, _I64, _P, _P,                      # qsl, batch, cache_indices, has_init
+        _INT, _I64, _P, _P,                    # silu, pad_slot_id, out_ref, row_state
+    ]
+    lib.oracle_conv1d_update.restype = _I64
+    lib.oracle_conv1d_update.argtypes = [
+        _INT, _P, _I64, _I64, _I64, _I64,      # dtype, x, x_sb, x_sc, batch, dim
+        _P, _I64, _I64, _INT, _P,              # weight, w_sc, w_sk, W, bias
+        _P, _P, _I64, _I64, _I64, _I64, _I64,  # states in/out, strides, L, num_lines
+        _P, _P, _INT, _I64, _P, _P,            # cache_seqlens, indices, silu, pad, out, state
+    ]
     lib.oracle_check_preconditions.restype = _INT
     lib.oracle_check_preconditions.argtypes = [
         _I64, _INT, _I64, _P, _P, _P, _P, _P, _I64, _I64]
@@ -296,6 +313,75 @@ def extract_windows_paged(*, dtype, cache, block_table, request, abs_positions, 
     if skipped < 0:
         raise ValueError("oracle_extract_windows_paged: malformed arguments")
     return oa, int(skipped)
+
+
+def _dense_states(conv_states, dtype):
+    """(states_in, states_out copy, L, num_lines) of a [num_lines, dim, L]
+    state buffer, contiguous; (None, None, 0, 0) for no states."""
+    if conv_states is None:
+        return None, None, 0, 0
+    sa = _float_array(conv_states, dtype)
+    if sa.ndim != 3:
+        raise ValueError("conv_states must be [num_lines, dim, state_len]")
+    return sa, sa.copy(), sa.shape[2], sa.shape[0]
+
+
+def conv1d_fwd(*, dtype, x, weight, bias=None, conv_states=None, query_start_loc,
+               cache_indices=None, has_initial_state=None, activation=None,
+               pad_slot_id=-1):
+    """Oracle of causal_conv1d_fwd ("Implementation:Sgl project Sglang Mamba
+    Ops") over x [total_tokens, dim] (token-major values; the layout the
+    kernel reads is immaterial here).  Returns ``(out_ref, row_state,
+    states_out, skipped)``: out_ref float64 [total_tokens, dim] (rows with
+    row_state != 1 are zero), row_state uint8 [total_tokens], states_out the
+    new [num_lines, dim, L] lines (None without conv_states)."""
+    xa = _float_array(x, dtype)
+    wa = _float_array(weight, dtype)
+    if xa.ndim != 2 or wa.ndim != 2:
+        raise ValueError("x [total_tokens, dim] and weight [dim, W] expected")
+    T, dim = xa.shape
+    W = wa.shape[1]
+    ba = None if bias is None else _float_array(bias, dtype)
+    s_in, s_out, L, lines = _dense_states(conv_states, dtype)
+    qsl = _np(query_start_loc, np.int32)
+    ci = None if cache_indices is None else _np(cache_indices, np.int32)
+    hi = None if has_initial_state is None else _np(has_initial_state).astype(np.uint8)
+    out_ref = np.zeros((T, dim), np.float64)
+    state = np.zeros(T, np.uint8)
+    skipped = lib().oracle_conv1d_fwd(
+        _DT[dtype], _ptr(xa), dim, 1, T, dim, _ptr(wa), W, 1, W, _ptr(ba),
+        _ptr(s_in), _ptr(s_out), dim * L, L, 1, L, lines,
+        _ptr(qsl), qsl.shape[0] - 1, _ptr(ci), _ptr(hi),
+        int(activation in ("silu", "swish")), int(pad_slot_id), _ptr(out_ref), _ptr(state))
+    if skipped < 0:
+        raise ValueError("oracle_conv1d_fwd: malformed arguments")
+    return out_ref, state, s_out, int(skipped)
+
+
+def conv1d_update(*, dtype, x, conv_state, weight, bias=None, activation=None,
+                  cache_seqlens=None, conv_state_indices=None, pad_slot_id=-1):
+    """Oracle of causal_conv1d_update ("Implementation:Sgl project Sglang
+    Mamba Ops"): x [batch, dim], one token per sequence.  Returns
+    ``(out_ref, row_state, states_out, skipped)``."""
+    xa = _float_array(x, dtype)
+    wa = _float_array(weight, dtype)
+    B, dim = xa.shape
+    W = wa.shape[1]
+    ba = None if bias is None else _float_array(bias, dtype)
+    s_in, s_out, L, lines = _dense_states(conv_state, dtype)
+    if s_in is None:
+        raise ValueError("conv_state is required")
+    cs = None if cache_seqlens is None else _np(cache_seqlens, np.int32)
+    ci = None if conv_state_indices is None else _np(conv_state_indices, np.int32)
+    out_ref = np.zeros((B, dim), np.float64)
+    state = np.zeros(B, np.uint8)
+    skipped = lib().oracle_conv1d_update(
+        _DT[dtype], _ptr(xa), dim, 1, B, dim, _ptr(wa), W, 1, W, _ptr(ba),
+        _ptr(s_in), _ptr(s_out), dim * L, L, 1, L, lines, _ptr(cs), _ptr(ci),
+        int(activation in ("silu", "swish")), int(pad_slot_id), _ptr(out_ref), _ptr(state))
+    if skipped < 0:
+        raise ValueError("oracle_conv1d_update: malformed arguments")
+    return out_ref, state, s_out, int(skipped)
 
 
 def check_preconditions(*, W, block_size, positions, seq_idx, slot_mapping,

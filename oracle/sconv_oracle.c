@@ -14,8 +14,10 @@
  *        sconv_seq_metadata (seq_idx / query_start buffers, padded rows).
  *   [P2] "core.ssm.ops.intermediate_extraction" -- _scatter_intermediate_conv_kernel
  *        and scatter_intermediate_conv (conditional, transposed window gather).
- *   [P4] "Implementation:Sgl project Sglang Mamba Ops" -- causal_conv1d_update
- *        (single-token decode form of the same convolution).
+ *   [P4] "Implementation:Sgl project Sglang Mamba Ops" -- causal_conv1d_fwd
+ *        and causal_conv1d_update (the same convolution over dense
+ *        per-sequence state lines: conv_states, cache_indices,
+ *        has_initial_state, bias, pad_slot_id; x and states in place).
  *
  * Readings taken where the pages are silent (each one is a single place in
  * this file):
@@ -383,6 +385,179 @@ int64_t oracle_extract_windows_paged(int dtype, const void *cache,
                                   (p % N) * cache_strides[2] + (off_s + j) * cache_strides[3];
                     copy_element(out, dst, cache, src, dtype);
                 }
+            }
+        }
+    }
+    return skipped;
+}
+
+/* ---------------------------------------------------------------------------
+ * The dense-state interface of [P4]: causal_conv1d_fwd and
+ * causal_conv1d_update, where a sequence's history is a dense state line
+ * (conv_states[line]) instead of the paged cache.
+ *
+ * Reading of the state line: it holds the last L inputs of its sequence,
+ * oldest first (entry L-1 is the most recent input), L >= W-1.  A sequence
+ * is convolved over its extended input e = (state line, or L zeros) followed
+ * by its x rows, so output t uses e entries L + TAP_POSITION(t, W, k), and
+ * the line afterwards holds the last L entries of e.
+ *
+ * Reading of the bias: added to the convolution before the activation.
+ */
+#define BIASED(conv, b) ((conv) + (b))
+
+/* Element index of entry i of a state line. */
+#define STATE_INDEX(line, c, i, s_line, s_c, s_k) \
+    ((line) * (s_line) + (c) * (s_c) + (i) * (s_k))
+
+/*
+ * oracle_conv1d_fwd -- [P4] causal_conv1d_fwd (varlen prefill).
+ *   x        [total_tokens, dim], strides (x_st, x_sc)
+ *   weight   [dim, W], strides (w_sc, w_sk);  bias [dim] or NULL
+ *   states_in / states_out: [num_lines, dim, L] with strides
+ *            (s_line, s_c, s_k); states_out is the caller's copy of
+ *            states_in and receives the new lines.  states_in NULL: zero
+ *            history, no state write.
+ *   qsl      [batch+1] sequence b is x rows qsl[b] .. qsl[b+1]-1
+ *   cache_indices [batch] state line of sequence b (NULL: b); a sequence
+ *            whose line equals pad_slot_id is skipped
+ *   has_init [batch] 1 = start from the state line, 0 = from zeros
+ *            (NULL: all 0)
+ * out_ref [total_tokens, dim] receives the double results of computed rows;
+ * row_state[t] is 1 (computed), 0 (not part of a computed sequence) or 2
+ * (skipped: the line is outside [0, num_lines)).  Returns the number of
+ * skipped sequences, or -1 if an argument is malformed.
+ */
+int64_t oracle_conv1d_fwd(int dtype, const void *x, int64_t x_st, int64_t x_sc,
+                          int64_t total_tokens, int64_t dim, const void *weight,
+                          int64_t w_sc, int64_t w_sk, int W, const void *bias,
+                          const void *states_in, void *states_out, int64_t s_line,
+                          int64_t s_c, int64_t s_k, int64_t L, int64_t num_lines,
+                          const int32_t *qsl, int64_t batch,
+                          const int32_t *cache_indices, const uint8_t *has_init,
+                          int silu, int64_t pad_slot_id, double *out_ref,
+                          uint8_t *row_state) {
+    if (W < 1 || batch < 0 || (states_in && (L < W - 1 || !states_out)))
+        return -1;
+    for (int64_t t = 0; t < total_tokens; ++t) row_state[t] = 0;
+    int64_t skipped = 0;
+    for (int64_t b = 0; b < batch; ++b) {
+        int64_t q0 = qsl[b], q1 = qsl[b + 1];
+        if (q0 < 0 || q1 < q0 || q1 > total_tokens) return -1;
+        int64_t line = cache_indices ? cache_indices[b] : b;
+        if (cache_indices && line == pad_slot_id) continue; /* padded entry */
+        if (states_in && (line < 0 || line >= num_lines)) {
+            for (int64_t t = q0; t < q1; ++t) row_state[t] = 2;
+            ++skipped;
+            continue;
+        }
+        int from_state = states_in && has_init && has_init[b];
+        int64_t Lh = states_in ? L : W - 1; /* history entries ahead of x */
+        int64_t n = q1 - q0;
+        for (int64_t c = 0; c < dim; ++c) {
+            for (int64_t t = 0; t < n; ++t) {
+                double acc = 0.0;
+                for (int k = 0; k < W; ++k) {
+                    int64_t i = Lh + TAP_POSITION(t, W, k); /* entry of e */
+                    double v;
+                    if (i >= Lh)
+                        v = load_value(x, dtype, (q0 + i - Lh) * x_st + c * x_sc);
+                    else if (from_state)
+                        v = load_value(states_in, dtype,
+                                       STATE_INDEX(line, c, i, s_line, s_c, s_k));
+                    else
+                        v = 0.0;
+                    acc += load_value(weight, dtype, c * w_sc + k * w_sk) * v;
+                }
+                double bv = bias ? load_value(bias, dtype, c) : 0.0;
+                out_ref[(q0 + t) * dim + c] = EPILOGUE(BIASED(acc, bv), 0.0, silu, 0);
+            }
+            if (!states_in) continue;
+            /* new line = the last L entries of e, i.e. entries n .. n+L-1 */
+            for (int64_t i = 0; i < L; ++i) {
+                int64_t j = n + i;
+                int64_t dst = STATE_INDEX(line, c, i, s_line, s_c, s_k);
+                if (j >= Lh)
+                    copy_element(states_out, dst, x, (q0 + j - Lh) * x_st + c * x_sc, dtype);
+                else if (from_state)
+                    copy_element(states_out, dst, states_in,
+                                 STATE_INDEX(line, c, j, s_line, s_c, s_k), dtype);
+                else
+                    memset((char *)states_out + dst * (int64_t)elem_bytes(dtype), 0,
+                           elem_bytes(dtype));
+            }
+        }
+        for (int64_t t = q0; t < q1; ++t) row_state[t] = 1;
+    }
+    return skipped;
+}
+
+/*
+ * oracle_conv1d_update -- [P4] causal_conv1d_update (one token per
+ * sequence).  x [batch, dim] strides (x_sb, x_sc); state lines as in
+ * oracle_conv1d_fwd; indices [batch] (NULL: b), pad_slot_id skips.
+ *
+ * cache_seqlens NULL: the line is shifted -- its entries are the last L
+ * inputs, the taps before the token are entries L-(W-1) .. L-1, and the new
+ * line is the last L entries of (line, x) -- exactly oracle_conv1d_fwd on a
+ * one-row sequence that starts from its state.
+ * cache_seqlens given (reading: a circular line): s = cache_seqlens[b] inputs
+ * were seen, input at position p is kept at entry p mod L; the taps before
+ * the token are positions s-(W-1) .. s-1 and the token is stored at entry
+ * s mod L, nothing else moves.
+ * out_ref [batch, dim]; row_state[b] 1 computed / 0 padded / 2 bad line.
+ */
+int64_t oracle_conv1d_update(int dtype, const void *x, int64_t x_sb, int64_t x_sc,
+                             int64_t batch, int64_t dim, const void *weight, int64_t w_sc,
+                             int64_t w_sk, int W, const void *bias, const void *states_in,
+                             void *states_out, int64_t s_line, int64_t s_c, int64_t s_k,
+                             int64_t L, int64_t num_lines, const int32_t *cache_seqlens,
+                             const int32_t *indices, int silu, int64_t pad_slot_id,
+                             double *out_ref, uint8_t *row_state) {
+    if (W < 2 || L < W - 1 || !states_in || !states_out) return -1;
+    int64_t skipped = 0;
+    for (int64_t b = 0; b < batch; ++b) {
+        row_state[b] = 0;
+        int64_t line = indices ? indices[b] : b;
+        if (indices && line == pad_slot_id) continue;
+        if (line < 0 || line >= num_lines) {
+            row_state[b] = 2;
+            ++skipped;
+            continue;
+        }
+        row_state[b] = 1;
+        int64_t s = cache_seqlens ? cache_seqlens[b] : 0;
+        for (int64_t c = 0; c < dim; ++c) {
+            double acc = 0.0;
+            for (int k = 0; k < W; ++k) {
+                double v;
+                if (k == W - 1) {
+                    v = load_value(x, dtype, b * x_sb + c * x_sc);
+                } else {
+                    int64_t i;
+                    if (cache_seqlens) {
+                        int64_t p = s + TAP_POSITION(0, W, k);
+                        i = ((p % L) + L) % L;
+                    } else {
+                        i = L + TAP_POSITION(0, W, k);
+                    }
+                    v = load_value(states_in, dtype, STATE_INDEX(line, c, i, s_line, s_c, s_k));
+                }
+                acc += load_value(weight, dtype, c * w_sc + k * w_sk) * v;
+            }
+            double bv = bias ? load_value(bias, dtype, c) : 0.0;
+            out_ref[b * dim + c] = EPILOGUE(BIASED(acc, bv), 0.0, silu, 0);
+            if (cache_seqlens) {
+                int64_t i = ((s % L) + L) % L;
+                copy_element(states_out, STATE_INDEX(line, c, i, s_line, s_c, s_k), x,
+                             b * x_sb + c * x_sc, dtype);
+            } else {
+                for (int64_t i = 0; i + 1 < L; ++i)
+                    copy_element(states_out, STATE_INDEX(line, c, i, s_line, s_c, s_k),
+                                 states_in, STATE_INDEX(line, c, i + 1, s_line, s_c, s_k),
+                                 dtype);
+                copy_element(states_out, STATE_INDEX(line, c, L - 1, s_line, s_c, s_k), x,
+                             b * x_sb + c * x_sc, dtype);
             }
         }
     }

@@ -3,8 +3,8 @@
 Each mutant is a copy of the oracle's C source with one plausible slip
 planted (a reversed or shifted tap, a wrong comparison, a swapped index, a
 dropped term, a transposed write).  It is compiled on the CPU, and the pin
-suite (tests/test_oracle_pins.py) is run against it in a child process; the
-suite must fail for every mutant.  Every planted slip keeps all memory
+suites (tests/test_oracle_pins.py and tests/test_oracle_pins_dense.py) are
+run against it in a child process; they must fail for every mutant.  Every planted slip keeps all memory
 accesses inside their buffers, so a mutant fails by assertion, not by crash.
 """
 from __future__ import annotations
@@ -90,7 +90,41 @@ MUTANTS = [
     ("extract_ignores_real_count",
      "    for (int64_t i = 0; i < real_count; ++i) {",
      "    for (int64_t i = 0; i < max_count; ++i) {"),
+    ("dense_bias_dropped",
+     "#define BIASED(conv, b) ((conv) + (b))",
+     "#define BIASED(conv, b) ((conv) + 0.0 * (b))"),
+    ("dense_bias_after_activation",
+     "out_ref[(q0 + t) * dim + c] = EPILOGUE(BIASED(acc, bv), 0.0, silu, 0);",
+     "out_ref[(q0 + t) * dim + c] = EPILOGUE(acc, 0.0, silu, 0) + bv;"),
+    ("dense_taps_from_oldest_entries",
+     "int64_t i = Lh + TAP_POSITION(t, W, k); /* entry of e */",
+     "int64_t i = (W - 1) + TAP_POSITION(t, W, k); /* entry of e */"),
+    ("dense_has_init_ignored",
+     "int from_state = states_in && has_init && has_init[b];",
+     "int from_state = states_in != NULL;"),
+    ("dense_line_not_shifted",
+     "            int64_t j = n + i;",
+     "            int64_t j = i;"),
+    ("dense_zero_line_not_zeroed",
+     "memset((char *)states_out + dst * (int64_t)elem_bytes(dtype), 0,",
+     "memset((char *)states_out + dst * (int64_t)elem_bytes(dtype), 0x3f,"),
+    ("dense_pad_not_skipped",
+     "if (cache_indices && line == pad_slot_id) continue; /* padded entry */",
+     "if (cache_indices && line == pad_slot_id - 1) continue; /* padded entry */"),
+    ("update_ring_taps_shifted",
+     "                        i = ((p % L) + L) % L;",
+     "                        i = (((p + 1) % L) + L) % L;"),
+    ("update_ring_store_shifted",
+     "                int64_t i = ((s % L) + L) % L;",
+     "                int64_t i = (((s + 1) % L) + L) % L;"),
+    ("update_line_not_shifted",
+     "                                 states_in, STATE_INDEX(line, c, i + 1, s_line, s_c, s_k),",
+     "                                 states_in, STATE_INDEX(line, c, i, s_line, s_c, s_k),"),
+    ("update_taps_from_oldest_entries",
+     "                        i = L + TAP_POSITION(0, W, k);",
+     "                        i = (W - 1) + TAP_POSITION(0, W, k);"),
 ]
+PIN_FILES = ["test_oracle_pins.py", "test_oracle_pins_dense.py"]
 
 
 def _run_mutant(tmp, name, old, new):
@@ -105,7 +139,7 @@ def _run_mutant(tmp, name, old, new):
     env = dict(os.environ, SCONV_ORACLE_LIB=so_path)
     r = subprocess.run(
         [sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-         os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+         *[os.path.join(ROOT, "tests", f) for f in PIN_FILES]],
         cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     return name, r.returncode, r.stdout[-400:]
 
@@ -122,6 +156,6 @@ def test_unmutated_oracle_passes_in_child():
     """Control: the same child-process run passes on the real oracle."""
     r = subprocess.run(
         [sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-         os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+         *[os.path.join(ROOT, "tests", f) for f in PIN_FILES]],
         cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stdout[-2000:]

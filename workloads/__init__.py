@@ -349,3 +349,97 @@ def sentinel(shape, dtype, device="cpu") -> torch.Tensor:
     raw = torch.full(shape, -1, dtype=torch.int16 if dtype == "bf16" else torch.int32,
                      device=device)
     return raw.view(dt)
+
+
+# --------------------------------------------------------------------------
+# the dense-state interface ("Implementation:Sgl project Sglang Mamba Ops":
+# causal_conv1d_fwd / causal_conv1d_update)
+
+def dense_conv_inputs(seed, *, dtype, dim, W, state_len, lens, num_lines=None, num_pad=0,
+                      init_frac=0.5, bias=True, x_layout="token_major",
+                      state_layout="k_contig", device="cpu", pad_slot_id=-1,
+                      w_sigma=0.5, x_sigma=1.0, state_sigma=1.0, has_init=None):
+    """Inputs of one varlen prefill over dense state lines.
+
+    Sequence b owns x rows [query_start_loc[b], query_start_loc[b+1]) with
+    lens[b] rows.  cache_indices are distinct lines drawn from a seeded
+    permutation of ``num_lines`` (default batch + 3) lines, ``num_pad`` of
+    them replaced by ``pad_slot_id``; has_initial_state is 1 with
+    probability ``init_frac`` (or the given array).  Storage layouts:
+      x_layout  "token_major": x [T, dim] contiguous;
+                "channel_major": a contiguous [dim, T] buffer seen as [T, dim].
+      state_layout "k_contig": conv_states [lines, dim, L] contiguous;
+                   "c_contig": a contiguous [lines, L, dim] buffer seen as
+                   [lines, dim, L].
+    Returns a dict of tensors on ``device`` (x, weight, bias or None,
+    conv_states, query_start_loc, cache_indices, has_initial_state).
+    """
+    rng = np.random.default_rng(seed)
+    lens = np.asarray(lens, np.int64)
+    batch = len(lens)
+    T = int(lens.sum())
+    num_lines = batch + 3 if num_lines is None else num_lines
+    qsl = np.zeros(batch + 1, np.int32)
+    qsl[1:] = np.cumsum(lens)
+    lines = rng.permutation(num_lines)[:batch].astype(np.int32)
+    if num_pad:
+        lines[rng.choice(batch, size=num_pad, replace=False)] = pad_slot_id
+    if has_init is None:
+        has_init = rng.random(batch) < init_frac
+    dt = TORCH_DTYPE[dtype]
+    big = (T + num_lines * state_len) * dim >= SMALL_ELEMS
+    gen_device = device if big else "cpu"
+    g = torch.Generator(device=gen_device).manual_seed(seed)
+    weight = normal((dim, W), w_sigma, dt, g, gen_device).to(device)
+    b = normal((dim,), w_sigma, dt, g, gen_device).to(device) if bias else None
+    if x_layout == "token_major":
+        x = torch.empty((T, dim), dtype=dt, device=device)
+    elif x_layout == "channel_major":
+        x = torch.empty((dim, T), dtype=dt, device=device).t()
+    else:
+        raise ValueError(x_layout)
+    fill_normal_(x if x.is_contiguous() else x.t(), x_sigma, g, gen_device)
+    if state_layout == "k_contig":
+        cs = torch.empty((num_lines, dim, state_len), dtype=dt, device=device)
+    elif state_layout == "c_contig":
+        cs = torch.empty((num_lines, state_len, dim), dtype=dt, device=device).transpose(1, 2)
+    else:
+        raise ValueError(state_layout)
+    fill_normal_(cs if cs.is_contiguous() else cs.transpose(1, 2), state_sigma, g, gen_device)
+    return {
+        "x": x, "weight": weight, "bias": b, "conv_states": cs,
+        "query_start_loc": torch.from_numpy(qsl).to(device),
+        "cache_indices": torch.from_numpy(lines).to(device),
+        "has_initial_state": torch.from_numpy(np.asarray(has_init, np.bool_)).to(device),
+        "pad_slot_id": pad_slot_id,
+    }
+
+
+def dense_update_inputs(seed, *, dtype, batch, dim, W, state_len, num_lines=None, num_pad=0,
+                        ring=False, bias=True, state_layout="k_contig", device="cpu",
+                        pad_slot_id=-1, max_seqlen=4096):
+    """Inputs of one decode step over dense state lines: x [batch, dim],
+    conv_state [lines, dim, L] (layouts as in dense_conv_inputs), distinct
+    conv_state_indices with ``num_pad`` padded entries, and for ``ring``
+    cache_seqlens uniform in 0..max_seqlen."""
+    rng = np.random.default_rng(seed)
+    num_lines = batch + 3 if num_lines is None else num_lines
+    lines = rng.permutation(num_lines)[:batch].astype(np.int32)
+    if num_pad:
+        lines[rng.choice(batch, size=num_pad, replace=False)] = pad_slot_id
+    seqlens = rng.integers(0, max_seqlen + 1, size=batch).astype(np.int32) if ring else None
+    dt = TORCH_DTYPE[dtype]
+    g = torch.Generator().manual_seed(seed)
+    weight = normal((dim, W), 0.5, dt, g, "cpu").to(device)
+    b = normal((dim,), 0.5, dt, g, "cpu").to(device) if bias else None
+    x = normal((batch, dim), 1.0, dt, g, "cpu").to(device)
+    if state_layout == "k_contig":
+        cs = normal((num_lines, dim, state_len), 1.0, dt, g, "cpu").to(device)
+    else:
+        cs = normal((num_lines, state_len, dim), 1.0, dt, g, "cpu").to(device).transpose(1, 2)
+    return {
+        "x": x, "weight": weight, "bias": b, "conv_state": cs,
+        "conv_state_indices": torch.from_numpy(lines).to(device),
+        "cache_seqlens": None if seqlens is None else torch.from_numpy(seqlens).to(device),
+        "pad_slot_id": pad_slot_id,
+    }
