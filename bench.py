@@ -59,7 +59,8 @@ def parse_args():
                    help="skip the per-workload table, e2e and the CPU baseline")
     p.add_argument("--seed", type=int, default=1002)
     p.add_argument("--only", choices=["chunked_prefill_bf16", "long_prefill_bf16",
-                                      "spec_decode_bf16"],
+                                      "spec_decode_bf16", "dense", "dense_prefill_bf16",
+                                      "dense_long_prefill_bf16", "dense_decode_bf16"],
                    help="time just this workload's kernels and print its table row")
     p.add_argument("--max-hist", type=int, default=4096,
                    help="longest cached history of the decode requests (smaller only for "
@@ -376,7 +377,8 @@ def _kernel_time(step_fns, reps, stream):
     """Mean seconds per call of the launches in step_fns, replayed from one
     CUDA graph and timed with CUDA events on the launching stream."""
     g = capture(lambda: [f() for f in step_fns], stream)
-    g.replay()
+    for _ in range(3):  # warm-up replays (clocks, caches, lazy module loads)
+        g.replay()
     stream.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
@@ -548,6 +550,80 @@ def bench_ssm_gather(device, stream, peak, reps=50):
         "frac": round(gbs / peak, 4)}}
 
 
+def dense_fwd_bytes(d) -> int:
+    """Bytes sconv_causal_conv1d_fwd must move: x read and out written for
+    every row of a computed sequence, each computed line read (when the
+    sequence starts from it) and written, weights, bias and metadata."""
+    T, dim = d["x"].shape
+    e = d["x"].element_size()
+    L = d["conv_states"].shape[2]
+    W = d["weight"].shape[1]
+    qsl = d["query_start_loc"].cpu().numpy()
+    lines = d["cache_indices"].cpu().numpy()
+    init = d["has_initial_state"].cpu().numpy()
+    live = lines != d["pad_slot_id"]
+    rows = int(((qsl[1:] - qsl[:-1]) * live).sum())
+    state = int((live * (1 + init)).sum()) * L * dim * e
+    meta = 4 * (len(qsl) + len(lines)) + len(init)
+    return 2 * rows * dim * e + state + (W + 1) * dim * e + meta
+
+
+def bench_dense_prefill(name, device, stream, peak):
+    """sconv_causal_conv1d_fwd (causal_conv1d_fwd of the Sglang Mamba ops
+    page) in place: the mixed prefill over 2 input sets (2 x 147 MB > L2),
+    or the long single-sequence prefill (1 GB)."""
+    import hybrid_sconv_b200 as hs
+    nsets, reps = (2, 50) if name == "dense_prefill_bf16" else (1, 10)
+    sets = [workloads.DENSE_NAMED[name](seed=1011 + 17 * i if name == "dense_prefill_bf16"
+                                        else 1012, device=device) for i in range(nsets)]
+    fns = [lambda d=d: hs.sconv_causal_conv1d_fwd(
+        d["x"], d["weight"], d["bias"], d["conv_states"], d["query_start_loc"],
+        d["cache_indices"], d["has_initial_state"], True) for d in sets]
+    secs = _kernel_time(fns, reps, stream)
+    nbytes = int(np.mean([dense_fwd_bytes(d) for d in sets]))
+    rows = int(sets[0]["query_start_loc"][-1])
+    gbs = nbytes / secs / 1e9
+    del sets, fns
+    torch.cuda.empty_cache()
+    return {name: {"kernel_us": round(secs * 1e6, 3), "mtokens_s": round(rows / secs / 1e6, 2),
+                   "alg_bytes": nbytes, "alg_gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}}
+
+
+def bench_dense_decode(device, stream, peak, nsets=96, reps=200):
+    """sconv_causal_conv1d_update (causal_conv1d_update) in place: 256
+    sequences, 96 rotating sets of 256 distinct lines each from a 151 MB
+    line pool (> L2)."""
+    import hybrid_sconv_b200 as hs
+    u0 = workloads.dense_decode_bf16(device=device)
+    B, dim = u0["x"].shape
+    g = torch.Generator(device=device).manual_seed(1013)
+    pool = torch.empty((nsets * B, dim, 3), dtype=torch.bfloat16, device=device)
+    workloads.fill_normal_(pool, 1.0, g, device)
+    perm = torch.randperm(nsets * B, generator=torch.Generator().manual_seed(1013))
+    fns = []
+    for i in range(nsets):
+        x = workloads.normal((B, dim), 1.0, torch.bfloat16, g, device)
+        idx = perm[i * B:(i + 1) * B].to(torch.int32).to(device)
+        fns.append(lambda x=x, idx=idx: hs.sconv_causal_conv1d_update(
+            x, pool, u0["weight"], u0["bias"], True, None, idx))
+    secs = _kernel_time(fns, reps, stream)
+    nbytes = 2 * B * dim * 2 + 2 * B * dim * 3 * 2 + 5 * dim * 2 + 4 * B
+    gbs = nbytes / secs / 1e9
+    del pool, fns
+    torch.cuda.empty_cache()
+    return {"dense_decode_bf16": {"kernel_us": round(secs * 1e6, 3),
+                                  "mtokens_s": round(B / secs / 1e6, 2), "alg_bytes": nbytes,
+                                  "alg_gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}}
+
+
+def bench_dense(device, stream, peak):
+    table = {}
+    for name in ("dense_prefill_bf16", "dense_long_prefill_bf16"):
+        table.update(bench_dense_prefill(name, device, stream, peak))
+    table.update(bench_dense_decode(device, stream, peak))
+    return table
+
+
 def per_workload_table(device, stream, peak, sets_obj=None):
     table = {}
     if sets_obj is not None:
@@ -557,6 +633,7 @@ def per_workload_table(device, stream, peak, sets_obj=None):
     table.update(bench_prefill("long_prefill_bf16", device, stream, peak))
     table.update(bench_spec_decode(device, stream, peak))
     table.update(bench_ssm_gather(device, stream, peak))
+    table.update(bench_dense(device, stream, peak))
     return table
 
 
@@ -713,6 +790,13 @@ def main():
     if args.only:
         if args.only == "spec_decode_bf16":
             row = bench_spec_decode(device, stream, peak)
+        elif args.only == "dense":
+            row = bench_dense(device, stream, peak)
+        elif args.only == "dense_decode_bf16":
+            row = bench_dense_decode(device, stream, peak, nsets=args.sets,
+                                     reps=max(3, args.steps))
+        elif args.only.startswith("dense"):
+            row = bench_dense_prefill(args.only, device, stream, peak)
         else:
             row = bench_prefill(args.only, device, stream, peak, reps=max(3, args.steps))
         print(json.dumps({"only": args.only, "peak_gbs": peak, "table": row}), flush=True)

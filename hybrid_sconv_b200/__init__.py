@@ -14,8 +14,10 @@ using one without the library raises ImportError (there is no fallback).
 
 _EXPORTS = (
     "EFLAG_BLOCK", "EFLAG_LOGICAL", "EFLAG_POSITION", "EFLAG_QUERY_START", "EFLAG_REQUEST",
-    "EFLAG_SLOT", "EFLAG_TIMEOUT", "LIB_PATH", "SconvError", "fused_sconv",
-    "scatter_intermediate_conv", "scatter_intermediate_ssm", "sconv_extract_windows",
+    "EFLAG_SLOT", "EFLAG_TIMEOUT", "LIB_PATH", "SconvError", "causal_conv1d_fwd",
+    "causal_conv1d_update", "fused_sconv", "scatter_intermediate_conv",
+    "scatter_intermediate_ssm", "sconv_causal_conv1d_fwd", "sconv_causal_conv1d_update",
+    "sconv_extract_windows",
     "sconv_extract_windows_paged", "sconv_fused", "sconv_fused_streams",
     "sconv_scatter_intermediate_ssm", "sconv_seq_metadata", "sconv_update",
 )

@@ -75,6 +75,12 @@ _SIGNATURES = {
     "sconv_seq_metadata": [_P, _INT, _INT, _INT, _P, _I64, _P, _I64, _P],
     "sconv_scatter_intermediate_ssm": [
         _P, _I64, _I64, _I64, _P, _P, _INT, _P, _I64, _INT, _P, _P],
+    "sconv_causal_conv1d_fwd": [
+        _P, _I64, _I64, _INT, _INT, _P, _I64, _I64, _INT, _P,
+        _P, _I64, _I64, _I64, _INT, _INT, _P, _INT, _P, _P, _INT, _INT, _P, _INT, _P, _P],
+    "sconv_causal_conv1d_update": [
+        _P, _I64, _I64, _INT, _INT, _P, _I64, _I64, _INT, _P,
+        _P, _I64, _I64, _I64, _INT, _INT, _P, _P, _INT, _INT, _P, _INT, _P, _P],
     "sconv_extract_windows_paged": [
         _P, _I64P, _I64, _INT, _INT, _INT, _INT, _INT, _P, _I64, _INT, _INT, _P, _P, _P, _INT,
         _P, _I64, _INT, _INT, _P, _P],
@@ -419,7 +425,105 @@ def sconv_seq_metadata(query_start_loc, num_reqs, num_actual_tokens, seq_idx_out
     _check("sconv_seq_metadata", st, value_error=True)
 
 
+def _dense_common(x, weight, bias, states, out, err_flag, states_name):
+    dt = _DTYPES.get(x.dtype)
+    if dt is None:
+        raise TypeError("x must be float32 or bfloat16")
+    for t, name in ((weight, "weight"), (bias, "bias"), (states, states_name), (out, "out")):
+        if t is not None and t.dtype != x.dtype:
+            raise TypeError(f"{name} must have x's dtype")
+    if x.dim() != 2 or weight.dim() != 2 or weight.shape[0] != x.shape[1]:
+        raise ValueError("x [rows, dim] and weight [dim, W] expected")
+    dim = x.shape[1]
+    if bias is not None and (bias.dim() != 1 or bias.shape[0] != dim or bias.stride(0) != 1):
+        raise ValueError("bias must be a contiguous [dim] tensor")
+    if states is not None and (states.dim() != 3 or states.shape[1] != dim):
+        raise ValueError(f"{states_name} must be [num_lines, dim, state_len]")
+    if out.shape != x.shape or out.stride() != x.stride():
+        raise ValueError("out must have x's shape and strides")
+    if err_flag is not None:
+        _vector(err_flag, torch.int32, "err_flag", 1)
+    return dt
+
+
+def sconv_causal_conv1d_fwd(x, weight, bias, conv_states, query_start_loc, cache_indices,
+                            has_initial_state, silu_activation, pad_slot_id=-1, *, out=None,
+                            err_flag=None, stream=None):
+    """Varlen prefill over dense state lines (causal_conv1d_fwd,
+    "Implementation:Sgl project Sglang Mamba Ops"), in place by default.
+
+    x [total_tokens, dim] with any strides (a channel-major [dim, T] buffer
+    is passed as its transpose view); weight [dim, W]; bias [dim] or None;
+    conv_states [num_lines, dim, state_len] (any strides) or None;
+    query_start_loc int32 [batch+1]; cache_indices int32 [batch] or None;
+    has_initial_state bool/uint8 [batch] or None.  Writes the outputs into
+    ``out`` (default: x itself) and the new lines into conv_states; returns
+    ``out``."""
+    if out is None:
+        out = x
+    dt = _dense_common(x, weight, bias, conv_states, out, err_flag, "conv_states")
+    batch = query_start_loc.shape[0] - 1
+    d = _dev(x, weight, bias, conv_states, query_start_loc, cache_indices, has_initial_state,
+             out, err_flag)
+    _vector(query_start_loc, torch.int32, "query_start_loc", batch + 1)
+    if cache_indices is not None:
+        _vector(cache_indices, torch.int32, "cache_indices", batch)
+    if has_initial_state is not None:
+        if has_initial_state.dtype not in (torch.bool, torch.uint8):
+            raise TypeError("has_initial_state must be bool or uint8")
+        if has_initial_state.dim() != 1 or has_initial_state.shape[0] < batch or (
+                batch > 0 and has_initial_state.stride(0) != 1):
+            raise ValueError("has_initial_state must be a contiguous [batch] tensor")
+    cs = conv_states
+    s_strides = cs.stride() if cs is not None else (0, 0, 0)
+    with torch.cuda.device(d):
+        st = LIB.sconv_causal_conv1d_fwd(
+            _ptr(x), x.stride(0), x.stride(1), x.shape[0], x.shape[1], _ptr(weight),
+            weight.stride(0), weight.stride(1), weight.shape[1], _ptr(bias), _ptr(cs),
+            s_strides[0], s_strides[1], s_strides[2], cs.shape[2] if cs is not None else 0,
+            cs.shape[0] if cs is not None else 0, _ptr(query_start_loc), batch,
+            _ptr(cache_indices), _ptr(has_initial_state),
+            SCONV_ACT_SILU if silu_activation else SCONV_ACT_NONE, int(pad_slot_id), _ptr(out),
+            dt, _ptr(err_flag), _stream(d, stream))
+    _check("sconv_causal_conv1d_fwd", st)
+    return out
+
+
+def sconv_causal_conv1d_update(x, conv_state, weight, bias, silu_activation, cache_seqlens=None,
+                               conv_state_indices=None, pad_slot_id=-1, *, out=None,
+                               err_flag=None, stream=None):
+    """One decode token per sequence over dense state lines
+    (causal_conv1d_update, "Implementation:Sgl project Sglang Mamba Ops"),
+    in place by default.  x [batch, dim]; conv_state [num_lines, dim,
+    state_len]; cache_seqlens int32 [batch] makes the lines circular;
+    conv_state_indices int32 [batch] or None.  Returns ``out`` (default x)."""
+    if out is None:
+        out = x
+    dt = _dense_common(x, weight, bias, conv_state, out, err_flag, "conv_state")
+    if conv_state is None:
+        raise ValueError("conv_state is required")
+    batch = x.shape[0]
+    d = _dev(x, conv_state, weight, bias, cache_seqlens, conv_state_indices, out, err_flag)
+    if cache_seqlens is not None:
+        _vector(cache_seqlens, torch.int32, "cache_seqlens", batch)
+    if conv_state_indices is not None:
+        _vector(conv_state_indices, torch.int32, "conv_state_indices", batch)
+    cs = conv_state
+    with torch.cuda.device(d):
+        st = LIB.sconv_causal_conv1d_update(
+            _ptr(x), x.stride(0), x.stride(1), batch, x.shape[1], _ptr(weight),
+            weight.stride(0), weight.stride(1), weight.shape[1], _ptr(bias), _ptr(cs),
+            cs.stride(0), cs.stride(1), cs.stride(2), cs.shape[2], cs.shape[0],
+            _ptr(cache_seqlens), _ptr(conv_state_indices),
+            SCONV_ACT_SILU if silu_activation else SCONV_ACT_NONE, int(pad_slot_id), _ptr(out),
+            dt, _ptr(err_flag), _stream(d, stream))
+    _check("sconv_causal_conv1d_update", st)
+    return out
+
+
 # Names used on the pages, for callers coming from them.
 fused_sconv = sconv_fused
 scatter_intermediate_conv = sconv_extract_windows
 scatter_intermediate_ssm = sconv_scatter_intermediate_ssm
+causal_conv1d_fwd = sconv_causal_conv1d_fwd
+causal_conv1d_update = sconv_causal_conv1d_update

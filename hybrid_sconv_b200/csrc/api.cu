@@ -96,6 +96,106 @@ sconv_status check_fused(const void *x, int64_t x_rs, int T, int C, const void *
     return SCONV_OK;
 }
 
+// Elements spanned by a strided tensor: the largest offset + 1 (0 if empty).
+int64_t span(const int64_t *ext, const int64_t *str, int nd) {
+    int64_t last = 0;
+    for (int i = 0; i < nd; ++i) {
+        if (ext[i] == 0) return 0;
+        last += (ext[i] - 1) * str[i];
+    }
+    return last + 1;
+}
+
+// True when no two index tuples of the strided tensor address the same
+// element: taken by increasing stride, every dimension of extent > 1 steps
+// past everything the smaller dimensions span.
+bool non_overlapping(const int64_t *ext, const int64_t *str, int nd) {
+    int order[4] = {0, 1, 2, 3};
+    for (int i = 0; i < nd; ++i) {
+        if (str[i] < 0) return false;
+        for (int j = i; j > 0 && str[order[j]] < str[order[j - 1]]; --j) {
+            const int t = order[j];
+            order[j] = order[j - 1];
+            order[j - 1] = t;
+        }
+    }
+    int64_t covered = 1;  // elements spanned by the dimensions taken so far
+    for (int i = 0; i < nd; ++i) {
+        const int d = order[i];
+        if (ext[d] <= 1) continue;
+        if (str[d] < covered) return false;
+        covered = str[d] * (ext[d] - 1) + covered;
+    }
+    return true;
+}
+
+// Shared checks of the dense-state entry points (T rows of x: the tokens of
+// the prefill, the sequences of the update).  Fills `a` and `vec`.
+sconv_status check_dense(const void *x, int64_t x_st, int64_t x_sc, int T, int dim,
+                         const void *weight, int64_t w_sc, int64_t w_sk, int W, const void *bias,
+                         void *states, int64_t s_line, int64_t s_c, int64_t s_k, int L,
+                         int num_lines, sconv_act act, void *out, sconv_dtype dt,
+                         sconv::DenseArgs &a, bool &vec) {
+    if (dt != SCONV_F32 && dt != SCONV_BF16) return SCONV_ERR_UNSUPPORTED;
+    if (act != SCONV_ACT_NONE && act != SCONV_ACT_SILU) return SCONV_ERR_INVALID;
+    if (W < 2) return SCONV_ERR_INVALID;
+    if (W > SCONV_MAX_W) return SCONV_ERR_UNSUPPORTED;
+    if (T < 0 || dim < 1 || !x || !weight || !out) return SCONV_ERR_INVALID;
+    if (w_sc < 0 || w_sk < 0) return SCONV_ERR_INVALID;
+    if (static_cast<int64_t>(dim) > 65535LL * 128) return SCONV_ERR_UNSUPPORTED;
+    const int64_t e = elem_size(dt);
+    const int64_t xe[2] = {T, dim}, xs[2] = {x_st, x_sc};
+    if (!non_overlapping(xe, xs, 2)) return SCONV_ERR_INVALID;
+    const int64_t x_bytes = span(xe, xs, 2) * e;
+    if (out != x && overlaps(out, x_bytes, x, x_bytes)) return SCONV_ERR_INVALID;
+    const int64_t we[2] = {dim, W}, wst[2] = {w_sc, w_sk};
+    const int64_t w_bytes = span(we, wst, 2) * e;
+    if (overlaps(weight, w_bytes, out, x_bytes)) return SCONV_ERR_INVALID;
+    if (bias && overlaps(bias, dim * e, out, x_bytes)) return SCONV_ERR_INVALID;
+    if (states) {
+        if (L < W - 1) return SCONV_ERR_INVALID;
+        if (L > SCONV_MAX_STATE_LEN) return SCONV_ERR_UNSUPPORTED;
+        if (num_lines < 1) return SCONV_ERR_INVALID;
+        const int64_t se[3] = {num_lines, dim, L}, ss[3] = {s_line, s_c, s_k};
+        if (!non_overlapping(se, ss, 3)) return SCONV_ERR_INVALID;
+        const int64_t s_bytes = span(se, ss, 3) * e;
+        if (overlaps(states, s_bytes, x, x_bytes) || overlaps(states, s_bytes, out, x_bytes) ||
+            overlaps(states, s_bytes, weight, w_bytes) ||
+            (bias && overlaps(states, s_bytes, bias, dim * e)))
+            return SCONV_ERR_INVALID;
+    }
+    const int64_t V = 16 / e;
+    vec = x_sc == 1 && aligned16(x) && aligned16(out) && (x_st * e) % 16 == 0 && dim % V == 0 &&
+          dim / V <= 65535;
+    a = sconv::DenseArgs{};
+    a.x = x;
+    a.out = out;
+    a.x_st = x_st;
+    a.x_sc = x_sc;
+    a.T = T;
+    a.dim = dim;
+    a.w = weight;
+    a.w_sc = w_sc;
+    a.w_sk = w_sk;
+    a.W = W;
+    a.bias = bias;
+    a.st = states;
+    a.s_line = s_line;
+    a.s_c = s_c;
+    a.s_k = s_k;
+    a.L = states ? L : 0;
+    a.num_lines = states ? num_lines : 0;
+    a.silu = act == SCONV_ACT_SILU;
+    a.st_mode = 0;
+    if (states && vec && aligned16(states) && (s_line * e) % 16 == 0) {
+        if (s_c == 1 && (s_k * e) % 16 == 0)
+            a.st_mode = 1;
+        else if (s_k == 1 && s_c == L)
+            a.st_mode = 2;
+    }
+    return SCONV_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -336,6 +436,60 @@ sconv_status sconv_extract_windows_paged(const void *cache, const int64_t cache_
     a.d_conv = d_conv;
     a.err = err_flag;
     return sconv::launch_extract_paged(a, dt == SCONV_BF16, vec, stream) == cudaSuccess
+               ? SCONV_OK
+               : SCONV_ERR_LAUNCH;
+}
+
+sconv_status sconv_causal_conv1d_fwd(
+    void *x, int64_t x_stride_t, int64_t x_stride_c, int total_tokens, int dim,
+    const void *weight, int64_t w_stride_c, int64_t w_stride_k, int W, const void *bias,
+    void *conv_states, int64_t s_stride_line, int64_t s_stride_c, int64_t s_stride_k,
+    int state_len, int num_lines, const int32_t *query_start_loc, int batch,
+    const int32_t *cache_indices, const uint8_t *has_initial_state, sconv_act act,
+    int pad_slot_id, void *out, sconv_dtype dt, int32_t *err_flag, cudaStream_t stream) {
+    if (batch < 0) return SCONV_ERR_INVALID;
+    sconv::DenseArgs a;
+    bool vec = false;
+    const sconv_status st = check_dense(
+        x, x_stride_t, x_stride_c, total_tokens, dim, weight, w_stride_c, w_stride_k, W, bias,
+        conv_states, s_stride_line, s_stride_c, s_stride_k, state_len, num_lines, act, out, dt,
+        a, vec);
+    if (st != SCONV_OK) return st;
+    if (batch == 0) return SCONV_OK;
+    if (!query_start_loc) return SCONV_ERR_INVALID;
+    a.qsl = query_start_loc;
+    a.batch = batch;
+    a.lines = cache_indices;
+    a.init = has_initial_state;
+    a.pad = pad_slot_id;
+    a.err = err_flag;
+    return sconv::launch_dense_fwd(a, dt == SCONV_BF16, vec, stream) == cudaSuccess
+               ? SCONV_OK
+               : SCONV_ERR_LAUNCH;
+}
+
+sconv_status sconv_causal_conv1d_update(
+    void *x, int64_t x_stride_b, int64_t x_stride_c, int batch, int dim,
+    const void *weight, int64_t w_stride_c, int64_t w_stride_k, int W, const void *bias,
+    void *conv_state, int64_t s_stride_line, int64_t s_stride_c, int64_t s_stride_k,
+    int state_len, int num_lines, const int32_t *cache_seqlens,
+    const int32_t *conv_state_indices, sconv_act act, int pad_slot_id, void *out,
+    sconv_dtype dt, int32_t *err_flag, cudaStream_t stream) {
+    if (batch < 0 || !conv_state) return SCONV_ERR_INVALID;
+    sconv::DenseArgs a;
+    bool vec = false;
+    const sconv_status st = check_dense(
+        x, x_stride_b, x_stride_c, batch, dim, weight, w_stride_c, w_stride_k, W, bias,
+        conv_state, s_stride_line, s_stride_c, s_stride_k, state_len, num_lines, act, out, dt,
+        a, vec);
+    if (st != SCONV_OK) return st;
+    if (batch == 0) return SCONV_OK;
+    a.batch = batch;
+    a.lines = conv_state_indices;
+    a.seqlens = cache_seqlens;
+    a.pad = pad_slot_id;
+    a.err = err_flag;
+    return sconv::launch_dense_update(a, dt == SCONV_BF16, vec, stream) == cudaSuccess
                ? SCONV_OK
                : SCONV_ERR_LAUNCH;
 }

@@ -269,6 +269,35 @@ struct PagedExtractArgs {
     int32_t *err;
 };
 
+// Dense-state conv (causal_conv1d_fwd / causal_conv1d_update).  Strides in
+// elements; for the update, T is the batch and x_st its row stride.
+struct DenseArgs {
+    const void *x;
+    void *out;
+    int64_t x_st, x_sc;
+    int T, dim;
+    const void *w;
+    int64_t w_sc, w_sk;
+    int W;
+    const void *bias;
+    void *st;  // conv state lines, or nullptr
+    int64_t s_line, s_c, s_k;
+    int L, num_lines;
+    const int32_t *qsl;     // [batch+1] (prefill)
+    int batch;
+    const int32_t *lines;   // [batch] or nullptr (line b)
+    const uint8_t *init;    // [batch] or nullptr (prefill)
+    const int32_t *seqlens; // [batch] or nullptr (update: circular line)
+    int silu;
+    int pad;
+    int32_t *err;
+    // Line layout for 16-byte packs of channels: 0 any (element access),
+    // 1 channel-contiguous entries (s_c == 1, one pack per entry),
+    // 2 entry-contiguous lines (s_k == 1, s_c == L: a pack's lines are one
+    // contiguous run of VEC*L elements).
+    int st_mode;
+};
+
 // Host-side launchers (return the cudaError_t of the launch).
 cudaError_t launch_fused(FusedArgs &a, bool bf16_data, bool vec, bool one_token_per_request,
                          cudaStream_t stream);
@@ -283,6 +312,10 @@ cudaError_t launch_extract(const ExtractArgs &a, bool bf16_data, bool vec, cudaS
 cudaError_t launch_scatter_ssm(const SsmArgs &a, int elem_bytes, bool vec, cudaStream_t stream);
 cudaError_t launch_extract_paged(const PagedExtractArgs &a, bool bf16_data, bool vec,
                                  cudaStream_t stream);
+// `vec`: x (and out) hold channels at unit stride in 16-byte aligned packs.
+cudaError_t launch_dense_fwd(const DenseArgs &a, bool bf16_data, bool vec, cudaStream_t stream);
+cudaError_t launch_dense_update(const DenseArgs &a, bool bf16_data, bool vec,
+                                cudaStream_t stream);
 cudaError_t launch_seq_metadata(const int32_t *qsl, int num_reqs, int num_actual, int num_padded,
                                 int32_t *seq_idx, int32_t *query_start, cudaStream_t stream);
 

@@ -1,0 +1,707 @@
+// dense.cu -- the dense-state interface of the short convolution, sm_100a
+// ("Implementation:Sgl project Sglang Mamba Ops": causal_conv1d_fwd and
+// causal_conv1d_update).  A sequence's history is a dense line of its last L
+// inputs (oldest first) instead of the paged cache, and x, out and the lines
+// may all be updated in place.
+//
+//  * dense_fwd_tile -- varlen prefill, x token-major in 16-byte channel
+//    packs.  One 256-thread block owns a (sequence, channel block) column of
+//    PP packs and walks it in tiles of TT = 256 / PP rows: each thread
+//    copies one pack of a tile ahead into a kStages-deep shared-memory ring
+//    with cp.async (only rows of this sequence, so nothing past its end is
+//    read), convolves one row of the current tile and stores it.  The W-1
+//    rows before a tile come from a shared-memory carry of the column's last
+//    L inputs, which starts as the state line and ends as the new line: no
+//    block re-reads x rows that another block may already have overwritten,
+//    so the in-place form needs no scratch memory and no ordering between
+//    blocks.  PP is chosen per call so that the grid covers the SMs: wide
+//    columns (fewer, longer blocks) for many sequences, narrow ones for a
+//    few long sequences.
+//  * dense_fwd_generic -- any x layout (channel-major included): a thread per
+//    (sequence, channel) walks the rows with the taps in registers.
+//  * dense_update -- one token per sequence; shifted or circular line.
+//
+// Every sum runs oldest tap first, starting from the bias, in fp32 FMAs, so
+// the three kernels agree bit for bit on the same token.  A sequence whose
+// line or row range is out of range is skipped and reported through the
+// optional error flag; nothing traps or waits.
+#include "common.cuh"
+#include "sconv.h"
+
+namespace sconv {
+namespace {
+
+constexpr int kRowsPerThread = 2;  // rows of a tile each thread convolves
+constexpr int kTileThreads = 256;
+constexpr int kStages = 8;
+constexpr int kLptMaxBatch = 64;   // longest-first block order up to this many sequences
+constexpr int kMaxL = SCONV_MAX_STATE_LEN;
+
+template <typename E>
+struct RawOf;
+template <>
+struct RawOf<bf16> {
+    using T = uint16_t;
+};
+template <>
+struct RawOf<float> {
+    using T = uint32_t;
+};
+
+__device__ __forceinline__ float raw_to_float(uint16_t v) {
+    return __uint_as_float(static_cast<uint32_t>(v) << 16);
+}
+__device__ __forceinline__ float raw_to_float(uint32_t v) { return __uint_as_float(v); }
+
+template <typename E>
+__device__ __forceinline__ typename RawOf<E>::T float_to_raw(float f);
+template <>
+__device__ __forceinline__ uint16_t float_to_raw<bf16>(float f) {
+    const bf16 h = __float2bfloat16_rn(f);
+    return *reinterpret_cast<const uint16_t *>(&h);
+}
+template <>
+__device__ __forceinline__ uint32_t float_to_raw<float>(float f) {
+    return __float_as_uint(f);
+}
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void flag(int32_t *err, unsigned bits) {
+    if (err) atomicOr(err, static_cast<int>(bits));
+}
+
+// Per-sequence checks shared by the prefill kernels.  Returns false (after
+// flagging, from one thread of the sequence) when the sequence is skipped;
+// otherwise sets the row range, the line and whether the history comes from
+// the line.
+__device__ __forceinline__ bool sequence_setup(const DenseArgs &a, int b, bool reporter,
+                                               int &q0, int &n, int64_t &line, bool &from) {
+    q0 = __ldg(a.qsl + b);
+    const int q1 = __ldg(a.qsl + b + 1);
+    if (q0 < 0 || q1 < q0 || q1 > a.T) {
+        if (reporter) flag(a.err, SCONV_EFLAG_QUERY_START);
+        return false;
+    }
+    n = q1 - q0;
+    line = a.lines ? __ldg(a.lines + b) : b;
+    if (a.lines && line == a.pad) return false;  // padded entry
+    if (a.st && (line < 0 || line >= a.num_lines)) {
+        if (reporter) flag(a.err, SCONV_EFLAG_SLOT);
+        return false;
+    }
+    from = a.st && a.init && __ldg(a.init + b);
+    return true;
+}
+
+// Weights of VEC channels from c, indexed by tap slot k' in 0..MAXW-1 with
+// tap k = k' - (MAXW - W); slots before the first tap hold zero.
+template <typename E, int VEC, int MAXW>
+__device__ __forceinline__ void load_taps(const DenseArgs &a, int c, float (&w)[MAXW][VEC]) {
+    const E *wp = static_cast<const E *>(a.w);
+#pragma unroll
+    for (int kk = 0; kk < MAXW; ++kk) {
+        const int k = kk - (MAXW - a.W);
+#pragma unroll
+        for (int v = 0; v < VEC; ++v)
+            w[kk][v] = k >= 0 ? load_weight(wp + (c + v) * a.w_sc + k * a.w_sk) : 0.f;
+    }
+}
+
+template <typename E, int VEC>
+__device__ __forceinline__ void load_bias(const DenseArgs &a, int c, float (&acc)[VEC]) {
+    const E *bp = static_cast<const E *>(a.bias);
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) acc[v] = bp ? load_weight(bp + c + v) : 0.f;
+}
+
+// State line entry i of VEC channels from c, as one raw pack (zero when the
+// history does not come from the line).
+template <typename E, int VEC>
+__device__ __forceinline__ uint4 line_pack(const DenseArgs &a, int64_t line, int c, int i,
+                                           bool from) {
+    using R = typename RawOf<E>::T;
+    union {
+        uint4 u;
+        R e[VEC];
+    } p;
+    p.u = make_uint4(0u, 0u, 0u, 0u);
+    if (from) {
+        const R *s = static_cast<const R *>(a.st) + line * a.s_line + i * a.s_k;
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) p.e[v] = s[static_cast<int64_t>(c + v) * a.s_c];
+    }
+    return p.u;
+}
+
+template <typename E, int VEC>
+__device__ __forceinline__ void store_line_pack(const DenseArgs &a, int64_t line, int c, int i,
+                                                uint4 u) {
+    using R = typename RawOf<E>::T;
+    union {
+        uint4 u;
+        R e[VEC];
+    } p;
+    p.u = u;
+    R *s = static_cast<R *>(a.st) + line * a.s_line + i * a.s_k;
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) s[static_cast<int64_t>(c + v) * a.s_c] = p.e[v];
+}
+
+// acc[v] += w[v] * tap[v] for the eight bf16 channels of a pack, with the
+// mixed-precision FMA that takes bf16 operands directly: the product of two
+// bf16 values is exact in fp32, so this equals widening both and one fmaf,
+// bit for bit.  w holds the weights of one tap as four bf16 pairs (channel
+// 2i in the low half), the same layout as the pack's words.
+__device__ __forceinline__ void fma_bf16x8(float (&acc)[8], const uint32_t (&w)[4], uint4 tap) {
+    const uint32_t q[4] = {tap.x, tap.y, tap.z, tap.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        asm("{\n\t.reg .b16 wl, wh, tl, th;\n\t"
+            "mov.b32 {wl, wh}, %2;\n\t"
+            "mov.b32 {tl, th}, %3;\n\t"
+            "fma.rn.f32.bf16 %0, wl, tl, %0;\n\t"
+            "fma.rn.f32.bf16 %1, wh, th, %1;\n\t}"
+            : "+f"(acc[2 * i]), "+f"(acc[2 * i + 1])
+            : "r"(w[i]), "r"(q[i]));
+}
+
+// Per-thread weights of the tiled kernel: bf16 pairs for bf16 data, floats
+// for fp32 data; tap slot k' as in load_taps.
+template <typename E, int MAXW>
+struct TileWeights {
+    float w[MAXW][4];
+    __device__ __forceinline__ void load(const DenseArgs &a, int c) {
+        load_taps<float, 4, MAXW>(a, c, w);
+    }
+    __device__ __forceinline__ void fma(float (&acc)[4], int kk, uint4 tap) const {
+        const float t[4] = {__uint_as_float(tap.x), __uint_as_float(tap.y),
+                            __uint_as_float(tap.z), __uint_as_float(tap.w)};
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[v] = fmaf(w[kk][v], t[v], acc[v]);
+    }
+};
+template <int MAXW>
+struct TileWeights<bf16, MAXW> {
+    uint32_t w[MAXW][4];
+    __device__ __forceinline__ void load(const DenseArgs &a, int c) {
+        const uint16_t *wp = static_cast<const uint16_t *>(a.w);
+#pragma unroll
+        for (int kk = 0; kk < MAXW; ++kk) {
+            const int k = kk - (MAXW - a.W);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint32_t lo = 0, hi = 0;
+                if (k >= 0) {
+                    lo = __ldg(wp + (c + 2 * i) * a.w_sc + k * a.w_sk);
+                    hi = __ldg(wp + (c + 2 * i + 1) * a.w_sc + k * a.w_sk);
+                }
+                w[kk][i] = lo | (hi << 16);
+            }
+        }
+    }
+    __device__ __forceinline__ void fma(float (&acc)[8], int kk, uint4 tap) const {
+        fma_bf16x8(acc, w[kk], tap);
+    }
+};
+
+// Prefill, token-major x.  Block i covers column y of sequence b (packs
+// y*PP .. y*PP+PP-1); with at most kLptMaxBatch sequences the blocks go
+// longest sequence first (so the long columns start in the first wave and
+// short ones fill the tail), else sequences interleave.  A tile is TT rows;
+// thread (g, p) = (threadIdx.x / PP, threadIdx.x % PP) convolves rows
+// g*RPT .. g*RPT+RPT-1 of pack p from a register window of W-1+RPT rows.
+// One barrier per tile: the carry is double-buffered (tile s reads
+// carry[s & 1] and writes the next carry into the other), and the ring
+// stage refilled at tile s was last read at tile s-1, before it.
+template <typename E, int PP, int MAXW, int THREADS>
+__global__ void __launch_bounds__(THREADS) dense_fwd_tile(const __grid_constant__ DenseArgs a, int ncb) {
+    constexpr int VEC = 16 / sizeof(E);
+    constexpr int RPT = kRowsPerThread;
+    constexpr int TT = THREADS / PP * RPT;
+    constexpr int NW = MAXW - 1 + RPT;  // window rows of one thread
+    extern __shared__ uint4 ring[];     // kStages * TT * PP packs
+    __shared__ uint4 carry[2][kMaxL * PP];
+    __shared__ int order[kLptMaxBatch];
+
+    pdl_wait();
+    pdl_trigger();
+    int b, y;
+    if (a.batch <= kLptMaxBatch) {
+        // Rank sequences by length, longest first (ties by index).
+        if (threadIdx.x < a.batch) {
+            const int t = threadIdx.x;
+            const int len = __ldg(a.qsl + t + 1) - __ldg(a.qsl + t);
+            int rank = 0;
+            for (int u = 0; u < a.batch; ++u) {
+                const int lu = __ldg(a.qsl + u + 1) - __ldg(a.qsl + u);
+                rank += (lu > len) || (lu == len && u < t);
+            }
+            order[rank] = t;
+        }
+        __syncthreads();
+        b = order[blockIdx.x / ncb];
+        y = blockIdx.x % ncb;
+    } else {
+        b = blockIdx.x % a.batch;
+        y = blockIdx.x / a.batch;
+    }
+    const int p = threadIdx.x % PP;
+    const int g = threadIdx.x / PP;
+    const int c = (y * PP + p) * VEC;
+    const bool cvalid = c < a.dim;
+
+    int q0, n;
+    int64_t line;
+    bool from;
+    if (!sequence_setup(a, b, threadIdx.x == 0 && y == 0, q0, n, line, from)) return;
+    const int Lc = a.st ? a.L : a.W - 1;  // entries of history ahead of x
+    const int ci = threadIdx.x / PP;      // carry entry this thread maintains (if < Lc)
+
+    // The carry starts as the history: the line, or zeros.
+    if (ci < Lc) carry[0][ci * PP + p] = cvalid ? line_pack<E, VEC>(a, line, c, ci, from)
+                                                : make_uint4(0u, 0u, 0u, 0u);
+
+    TileWeights<E, MAXW> wt;
+    float bias[VEC];
+    if (cvalid) {
+        wt.load(a, c);
+        load_bias<E, VEC>(a, c, bias);
+    }
+
+    const E *x = static_cast<const E *>(a.x) + static_cast<int64_t>(q0) * a.x_st + c;
+    E *out = static_cast<E *>(a.out) + static_cast<int64_t>(q0) * a.x_st + c;
+    const int ntiles = (n + TT - 1) / TT;
+    // Copies: thread (g, p) fetches rows g + j * TT / RPT of pack p, so a
+    // warp's copies cover whole rows.
+    auto issue = [&](int s) {
+#pragma unroll
+        for (int j = 0; j < RPT; ++j) {
+            const int r = g + j * (TT / RPT);
+            const int row = s * TT + r;
+            if (s < ntiles && row < n && cvalid)
+                cp_async16(&ring[((s % kStages) * TT + r) * PP + p], x + row * a.x_st);
+        }
+        cp_async_commit();
+    };
+#pragma unroll
+    for (int s = 0; s < kStages - 1; ++s) issue(s);
+
+    const int r0 = g * RPT;
+    for (int s = 0; s < ntiles; ++s) {
+        cp_async_wait<kStages - 2>();
+        __syncthreads();  // tile s and carry[s & 1] are complete; tile s-1 is no longer read
+        issue(s + kStages - 1);
+        const uint4 *tile = ring + (s % kStages) * TT * PP;
+        const uint4 *cin = carry[s & 1];
+        const int nv = min(TT, n - s * TT);
+        if (r0 < nv && cvalid) {
+            // win[j] holds row r0 - (MAXW-1) + j (from the carry when < 0).
+            uint4 win[NW];
+#pragma unroll
+            for (int j = 0; j < NW; ++j) {
+                const int rr = r0 - (MAXW - 1) + j;
+                if (j < MAXW - a.W) continue;  // before the first tap of row r0
+                win[j] = rr >= 0 ? tile[rr * PP + p] : cin[(Lc + rr) * PP + p];
+            }
+#pragma unroll
+            for (int u = 0; u < RPT; ++u) {
+                if (r0 + u >= nv) break;
+                float acc[VEC];
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) acc[v] = bias[v];
+#pragma unroll
+                for (int kk = 0; kk < MAXW; ++kk)
+                    if (kk >= MAXW - a.W) wt.fma(acc, kk, win[u + kk]);
+                if (a.silu) {
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) acc[v] = silu<E>(acc[v]);
+                }
+                Pack<E, VEC> o;
+                o.from_float(acc);
+                o.store(out + static_cast<int64_t>(s * TT + r0 + u) * a.x_st);
+            }
+        }
+        // Next carry: the last Lc entries of (carry, the tile's nv rows).
+        if (ci < Lc) {
+            const int src = nv + ci;
+            carry[(s + 1) & 1][ci * PP + p] =
+                src >= Lc ? tile[(src - Lc) * PP + p] : cin[src * PP + p];
+        }
+    }
+    cp_async_wait<0>();
+    // Each thread stores the carry entry it wrote itself: no barrier needed.
+    if (a.st && ci < Lc && cvalid)
+        store_line_pack<E, VEC>(a, line, c, ci, carry[ntiles & 1][ci * PP + p]);
+}
+
+// Prefill, any x layout: thread (b, c) walks sequence b's rows of channel c.
+// prev[j-1] holds the input j rows back; lag-j weight wl[j] = weight[c][W-1-j].
+template <typename E, int MAXW>
+__global__ void __launch_bounds__(128) dense_fwd_generic(const __grid_constant__ DenseArgs a) {
+    using R = typename RawOf<E>::T;
+    const int b = blockIdx.x;
+    const int c = blockIdx.y * blockDim.x + threadIdx.x;
+    pdl_wait();
+    pdl_trigger();
+    int q0, n;
+    int64_t line;
+    bool from;
+    if (!sequence_setup(a, b, threadIdx.x == 0 && blockIdx.y == 0, q0, n, line, from)) return;
+    if (c >= a.dim) return;
+
+    const int W = a.W;
+    const E *wp = static_cast<const E *>(a.w) + c * a.w_sc;
+    float wl[MAXW];
+#pragma unroll
+    for (int j = 0; j < MAXW; ++j) wl[j] = j < W ? load_weight(wp + (W - 1 - j) * a.w_sk) : 0.f;
+    const float bias = a.bias ? load_weight(static_cast<const E *>(a.bias) + c) : 0.f;
+
+    R *st = a.st ? static_cast<R *>(a.st) + line * a.s_line + c * a.s_c : nullptr;
+    const int L = a.L;
+    float prev[MAXW - 1];
+#pragma unroll
+    for (int j = 1; j < MAXW; ++j)
+        prev[j - 1] = (from && j < W) ? raw_to_float(st[(L - j) * a.s_k]) : 0.f;
+    // Line entries that survive the call: new entry i = old entry n + i.
+    if (st) {
+        for (int i = 0; i < L && n + i < L; ++i) st[i * a.s_k] = from ? st[(n + i) * a.s_k] : R(0);
+    }
+
+    const R *x = static_cast<const R *>(a.x) + static_cast<int64_t>(q0) * a.x_st +
+                 static_cast<int64_t>(c) * a.x_sc;
+    R *out = static_cast<R *>(a.out) + static_cast<int64_t>(q0) * a.x_st +
+             static_cast<int64_t>(c) * a.x_sc;
+    for (int t = 0; t < n; ++t) {
+        const R xr = x[static_cast<int64_t>(t) * a.x_st];
+        const float xf = raw_to_float(xr);
+        float acc = bias;
+#pragma unroll
+        for (int j = MAXW - 1; j >= 1; --j)
+            if (j < W) acc = fmaf(wl[j], prev[j - 1], acc);
+        acc = fmaf(wl[0], xf, acc);
+#pragma unroll
+        for (int j = MAXW - 2; j >= 1; --j) prev[j] = prev[j - 1];
+        prev[0] = xf;
+        if (a.silu) acc = silu<E>(acc);
+        out[static_cast<int64_t>(t) * a.x_st] = float_to_raw<E>(acc);
+        if (st && t >= n - L) st[(t - (n - L)) * a.s_k] = xr;
+    }
+}
+
+// VEC raw elements moved as one load or store of VEC * sizeof(R) bytes.
+template <int BYTES>
+struct RawVec;
+template <>
+struct RawVec<2> {
+    using T = uint16_t;
+};
+template <>
+struct RawVec<4> {
+    using T = uint32_t;
+};
+template <>
+struct RawVec<8> {
+    using T = uint2;
+};
+template <>
+struct RawVec<16> {
+    using T = uint4;
+};
+template <typename R, int VEC>
+union Lanes {
+    typename RawVec<VEC * sizeof(R)>::T v;
+    R e[VEC];
+};
+
+// Decode: thread (b, j) updates channels c .. c+VEC-1 of sequence b (VEC * 2
+// or 4 bytes: many threads, little serial work each, since one decode step
+// is bound by memory latency, not bandwidth).  The block's weights are
+// staged in shared memory before the wait for the preceding kernel (they
+// are constant).  Every line entry the update needs is read before the
+// first write, so the line costs one memory round trip.  Line access by
+// layout (MODE = DenseArgs::st_mode): 0 single elements; 1 one VEC-element
+// vector per entry; 2 the block's whole run of lines (VEC*L contiguous
+// elements per thread) staged through shared memory with 16-byte copies,
+// updated there by each thread for its own channels, and copied back.
+template <typename E, int VEC, int MAXW, int LMAX, int MODE>
+__global__ void __launch_bounds__(128) dense_update(const __grid_constant__ DenseArgs a) {
+    using R = typename RawOf<E>::T;
+    using LV = Lanes<R, VEC>;
+    extern __shared__ uint4 smem16[];
+    const int b = blockIdx.x;
+    const int c0 = blockIdx.y * blockDim.x * VEC;  // first channel of the block
+    const int nch = min(static_cast<int>(blockDim.x) * VEC, a.dim - c0);
+    const int c = c0 + threadIdx.x * VEC;
+    const bool active = c < a.dim;
+    const int L = a.L, W = a.W;
+
+    // weights of the block's channels, [nch][W]
+    R *wsm = reinterpret_cast<R *>(smem16);
+    {
+        const R *wg = static_cast<const R *>(a.w);
+        for (int j = threadIdx.x; j < nch * W; j += blockDim.x) {
+            const int ch = j / W, k = j - ch * W;
+            wsm[j] = __ldg(wg + static_cast<int64_t>(c0 + ch) * a.w_sc +
+                           static_cast<int64_t>(k) * a.w_sk);
+        }
+    }
+    float acc[VEC];
+    if (active) load_bias<E, VEC>(a, c, acc);
+    if (threadIdx.x == 0 && a.lines) prefetch_l2(a.lines + b);
+    pdl_wait();
+    pdl_trigger();
+    const int64_t line = a.lines ? __ldg(a.lines + b) : b;
+    if (a.lines && line == a.pad) return;
+    if (line < 0 || line >= a.num_lines) {
+        if (threadIdx.x == 0 && blockIdx.y == 0) flag(a.err, SCONV_EFLAG_SLOT);
+        return;
+    }
+    // x (issued before the line, which waits on the index): plain loads,
+    // since with out == x this kernel writes it.
+    R xr[VEC];
+    if (active) {
+        const R *xp = static_cast<const R *>(a.x) + static_cast<int64_t>(b) * a.x_st +
+                      static_cast<int64_t>(c) * a.x_sc;
+        if constexpr (VEC > 1) {
+            LV xin;
+            xin.v = *reinterpret_cast<const typename RawVec<VEC * sizeof(R)>::T *>(xp);
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) xr[v] = xin.e[v];
+        } else {
+            xr[0] = *xp;
+        }
+    }
+    const bool ring = a.seqlens != nullptr;
+    const int64_t s = ring ? __ldg(a.seqlens + b) : 0;
+    R *st = static_cast<R *>(a.st) + line * a.s_line + static_cast<int64_t>(c) * a.s_c;
+
+    // MODE 2: stage this block's contiguous run of lines after the weights.
+    uint4 *run16 = smem16 + (nch * W * static_cast<int>(sizeof(R)) + 15) / 16;
+    R *mine = reinterpret_cast<R *>(run16) + threadIdx.x * VEC * L;
+    int n16 = 0;
+    uint4 *grun = nullptr;
+    if constexpr (MODE == 2) {
+        n16 = nch * L * static_cast<int>(sizeof(R)) / 16;
+        grun = reinterpret_cast<uint4 *>(static_cast<R *>(a.st) + line * a.s_line +
+                                         static_cast<int64_t>(c0) * L);
+        for (int j = threadIdx.x; j < n16; j += blockDim.x) run16[j] = grun[j];
+    }
+    __syncthreads();  // weights (and lines) staged
+
+    // Entry i of the thread's VEC channels.
+    auto get = [&](int64_t i, R (&e)[VEC]) {
+        if constexpr (MODE == 1) {
+            LV p;
+            p.v = *reinterpret_cast<const typename RawVec<VEC * sizeof(R)>::T *>(st + i * a.s_k);
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) e[v] = p.e[v];
+        } else if constexpr (MODE == 2) {
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) e[v] = mine[v * L + i];
+        } else {
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) e[v] = st[v * a.s_c + i * a.s_k];
+        }
+    };
+    auto put = [&](int64_t i, const R (&e)[VEC]) {
+        if constexpr (MODE == 1) {
+            LV p;
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) p.e[v] = e[v];
+            *reinterpret_cast<typename RawVec<VEC * sizeof(R)>::T *>(st + i * a.s_k) = p.v;
+        } else if constexpr (MODE == 2) {
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) mine[v * L + i] = e[v];
+        } else {
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) st[v * a.s_c + i * a.s_k] = e[v];
+        }
+    };
+
+    if (active) {
+        // The W-1 taps before the token, by tap slot, and (shifted line) the
+        // entries 1..L-1 that move down one place.
+        R tap[MAXW - 1][VEC];
+#pragma unroll
+        for (int kk = 0; kk < MAXW - 1; ++kk) {
+            const int k = kk - (MAXW - W);
+            if (k < 0) continue;
+            int64_t i = L - (W - 1) + k;
+            if (ring) {
+                i = (s - (W - 1) + k) % L;
+                if (i < 0) i += L;
+            }
+            get(i, tap[kk]);
+        }
+        R keep[LMAX - 1][VEC];
+        if (!ring) {
+#pragma unroll
+            for (int i = 0; i < LMAX - 1; ++i)
+                if (i + 1 < L) get(i + 1, keep[i]);
+        }
+
+        const R *wt = wsm + threadIdx.x * VEC * W;
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) {
+#pragma unroll
+            for (int kk = 0; kk < MAXW - 1; ++kk) {
+                const int k = kk - (MAXW - W);
+                if (k >= 0)
+                    acc[v] = fmaf(raw_to_float(wt[v * W + k]), raw_to_float(tap[kk][v]), acc[v]);
+            }
+            acc[v] = fmaf(raw_to_float(wt[v * W + W - 1]), raw_to_float(xr[v]), acc[v]);
+            if (a.silu) acc[v] = silu<E>(acc[v]);
+        }
+
+        if (ring) {
+            int64_t i = s % L;
+            if (i < 0) i += L;
+            put(i, xr);
+        } else {
+#pragma unroll
+            for (int i = 0; i < LMAX - 1; ++i)
+                if (i + 1 < L) put(i, keep[i]);
+            put(L - 1, xr);
+        }
+        R *op = static_cast<R *>(a.out) + static_cast<int64_t>(b) * a.x_st +
+                static_cast<int64_t>(c) * a.x_sc;
+        if constexpr (VEC > 1) {
+            LV o;
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) o.e[v] = float_to_raw<E>(acc[v]);
+            *reinterpret_cast<typename RawVec<VEC * sizeof(R)>::T *>(op) = o.v;
+        } else {
+            *op = float_to_raw<E>(acc[0]);
+        }
+    }
+    if constexpr (MODE == 2) {
+        __syncthreads();
+        for (int j = threadIdx.x; j < n16; j += blockDim.x) grun[j] = run16[j];
+    }
+}
+
+int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0, v = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+            n = v;
+        else
+            n = 148;
+    }
+    return n;
+}
+
+// Packs per block: the widest column (up to 8 packs, 128 bytes of a row)
+// that still gives at least 1.5 blocks per SM.  Every block streams a whole
+// column, so wide columns read whole 128-byte lines and keep the DRAM
+// accesses of a row together, while a few long sequences need narrower
+// columns to spread their channels over the chip.
+int pick_pp(int batch, int packs) {
+    const int64_t want = 3LL * sm_count() / 2;
+    int pp = 8;
+    while (pp > 1 && pp > packs) pp /= 2;
+    for (; pp > 1; pp /= 2)
+        if (static_cast<int64_t>(batch) * ((packs + pp - 1) / pp) >= want) return pp;
+    return 1;
+}
+
+template <typename E, int PP, int MAXW, int THREADS>
+cudaError_t launch_tile_pp(const DenseArgs &a, int packs, cudaStream_t stream) {
+    constexpr int TT = THREADS / PP * kRowsPerThread;
+    constexpr size_t kSmem = static_cast<size_t>(kStages) * TT * PP * sizeof(uint4);
+    static bool configured = false;
+    if (!configured) {
+        const cudaError_t e = cudaFuncSetAttribute(
+            dense_fwd_tile<E, PP, MAXW, THREADS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            static_cast<int>(kSmem));
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    const int ncb = (packs + PP - 1) / PP;
+    return launch_pdl(dense_fwd_tile<E, PP, MAXW, THREADS>,
+                      dim3(static_cast<unsigned>(static_cast<int64_t>(a.batch) * ncb)),
+                      dim3(THREADS), kSmem, stream, a, ncb);
+}
+
+template <typename E, int MAXW>
+cudaError_t launch_tile(const DenseArgs &a, cudaStream_t stream) {
+    constexpr int VEC = 16 / sizeof(E);
+    const int packs = a.dim / VEC;
+    const int pp = pick_pp(a.batch, packs);
+    switch (pp) {
+        case 8: return launch_tile_pp<E, 8, MAXW, kTileThreads>(a, packs, stream);
+        case 4: return launch_tile_pp<E, 4, MAXW, kTileThreads>(a, packs, stream);
+        case 2: return launch_tile_pp<E, 2, MAXW, kTileThreads>(a, packs, stream);
+        default: return launch_tile_pp<E, 1, MAXW, kTileThreads>(a, packs, stream);
+    }
+}
+
+template <typename E, int MAXW>
+cudaError_t launch_fwd_t(const DenseArgs &a, bool vec, cudaStream_t stream) {
+    if (vec) return launch_tile<E, MAXW>(a, stream);
+    return launch_pdl(dense_fwd_generic<E, MAXW>, dim3(a.batch, (a.dim + 127) / 128), dim3(128),
+                      0, stream, a);
+}
+
+// Decode threads own 4 bytes of channels (2 bf16 or 1 fp32) on the vector
+// path, one channel otherwise.
+template <typename E, int MAXW, int LMAX>
+cudaError_t launch_update_l(const DenseArgs &a, bool vec, cudaStream_t stream) {
+    constexpr int VEC = 4 / sizeof(E);
+    const int v = vec ? VEC : 1;
+    const int per_block = 128 * v;
+    const dim3 grid(a.T, (a.dim + per_block - 1) / per_block);
+    const int nch = a.dim < per_block ? a.dim : per_block;
+    size_t smem = (static_cast<size_t>(nch) * a.W * sizeof(E) + 15) / 16 * 16;
+    if (!vec)
+        return launch_pdl(dense_update<E, 1, MAXW, LMAX, 0>, grid, dim3(128), smem, stream, a);
+    switch (a.st_mode) {
+        case 1:
+            return launch_pdl(dense_update<E, VEC, MAXW, LMAX, 1>, grid, dim3(128), smem, stream, a);
+        case 2:
+            smem += static_cast<size_t>(nch) * a.L * sizeof(E);
+            return launch_pdl(dense_update<E, VEC, MAXW, LMAX, 2>, grid, dim3(128), smem, stream, a);
+        default:
+            return launch_pdl(dense_update<E, VEC, MAXW, LMAX, 0>, grid, dim3(128), smem, stream, a);
+    }
+}
+
+template <typename E, int MAXW>
+cudaError_t launch_update_t(const DenseArgs &a, bool vec, cudaStream_t stream) {
+    return a.L <= 4 ? launch_update_l<E, MAXW, 4>(a, vec, stream)
+                    : launch_update_l<E, MAXW, kMaxL>(a, vec, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_dense_fwd(const DenseArgs &a, bool bf16_data, bool vec, cudaStream_t stream) {
+    if (a.batch == 0) return cudaSuccess;
+    if (bf16_data)
+        return a.W <= 4 ? launch_fwd_t<bf16, 4>(a, vec, stream) : launch_fwd_t<bf16, 8>(a, vec, stream);
+    return a.W <= 4 ? launch_fwd_t<float, 4>(a, vec, stream) : launch_fwd_t<float, 8>(a, vec, stream);
+}
+
+cudaError_t launch_dense_update(const DenseArgs &a, bool bf16_data, bool vec,
+                                cudaStream_t stream) {
+    if (a.T == 0) return cudaSuccess;
+    if (bf16_data)
+        return a.W <= 4 ? launch_update_t<bf16, 4>(a, vec, stream)
+                        : launch_update_t<bf16, 8>(a, vec, stream);
+    return a.W <= 4 ? launch_update_t<float, 4>(a, vec, stream)
+                    : launch_update_t<float, 8>(a, vec, stream);
+}
+
+}  // namespace sconv

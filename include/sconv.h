@@ -83,6 +83,7 @@ typedef enum sconv_act { SCONV_ACT_NONE = 0, SCONV_ACT_SILU = 1 } sconv_act;
 #define SCONV_MAX_W 8      /* taps supported by sconv_fused / sconv_update */
 #define SCONV_MAX_STREAMS 4 /* conv streams per sconv_fused_streams call */
 #define SCONV_MAX_DCONV 8  /* window length supported by sconv_extract_windows */
+#define SCONV_MAX_STATE_LEN 16 /* dense state line of sconv_causal_conv1d_fwd / _update */
 
 /*
  * sconv_fused -- insert + depthwise causal conv1d over the paged cache, one
@@ -256,6 +257,86 @@ sconv_status sconv_extract_windows_paged(
     int off_s, int ws, const int32_t *block_table, int64_t bt_row_stride, int num_reqs,
     int max_blocks, const int32_t *request, const int32_t *abs_positions,
     const int32_t *real_count, int max_count, void *out, int64_t out_slot_stride, int d_conv,
+    sconv_dtype dt, int32_t *err_flag, cudaStream_t stream);
+
+/*
+ * sconv_causal_conv1d_fwd -- varlen prefill over dense per-sequence state
+ * lines: the interface of causal_conv1d_fwd ("Implementation:Sgl project
+ * Sglang Mamba Ops", Signature and I/O Contract).  The same depthwise causal
+ * convolution as sconv_fused, with a sequence's history kept as a dense
+ * line of its last state_len inputs instead of a paged cache.
+ *
+ * For sequence b (x rows query_start_loc[b] .. query_start_loc[b+1]-1, n of
+ * them) with line = cache_indices[b] (b when cache_indices is NULL):
+ *   - line == pad_slot_id (only when cache_indices is given): the sequence is
+ *     skipped; its out rows and its line are untouched;
+ *   - e = conv_states[line] (state_len entries, oldest first) when
+ *     has_initial_state[b] is 1, else state_len zeros, followed by the n x
+ *     rows (with conv_states NULL: W-1 zeros followed by the x rows);
+ *   - out row t = act(sum_k weight[c][k] * e[t + k + state_len - (W-1)] +
+ *     bias[c]): weight[c][W-1] multiplies the current row;
+ *   - conv_states[line] = the last state_len entries of e (with n == 0 and
+ *     has_initial_state 0 that is a line of zeros).
+ *
+ *   x                [total_tokens, dim], element strides (x_stride_t,
+ *                    x_stride_c): token-major (x_stride_c == 1) or
+ *                    channel-major (x_stride_t == 1) storage, or any other
+ *                    layout whose elements do not overlap.
+ *   weight           [dim, W], strides (w_stride_c, w_stride_k); 2 <= W <= 8.
+ *   bias             [dim] contiguous, or NULL.
+ *   conv_states      [num_lines, dim, state_len], strides (s_stride_line,
+ *                    s_stride_c, s_stride_k), read and written in place; or
+ *                    NULL (no history, nothing written).
+ *                    W-1 <= state_len <= SCONV_MAX_STATE_LEN.
+ *   query_start_loc  [batch+1] int32, 0 <= q[b] <= q[b+1] <= total_tokens.
+ *   cache_indices    [batch] int32, or NULL.  Lines of different sequences
+ *                    must differ.
+ *   has_initial_state [batch] uint8 0/1 (a torch bool tensor), or NULL (0).
+ *   out              [total_tokens, dim] with x's strides: either x itself
+ *                    (the page's in-place form) or a buffer that does not
+ *                    overlap x.  Rows of no computed sequence are untouched.
+ *   All floating data (x, weight, bias, conv_states, out) has type dt.
+ *   err_flag         optional device int32: a sequence whose line is outside
+ *                    [0, num_lines) sets SCONV_EFLAG_SLOT, one whose
+ *                    query_start_loc entries are out of order or range sets
+ *                    SCONV_EFLAG_QUERY_START; such a sequence is skipped.
+ * One thread block owns a (sequence, channel block) column and walks it in
+ * row order, so the in-place form needs no scratch memory and no ordering
+ * between blocks.  Asynchronous; no allocation; CUDA-graph capturable.
+ */
+sconv_status sconv_causal_conv1d_fwd(
+    void *x, int64_t x_stride_t, int64_t x_stride_c, int total_tokens, int dim,
+    const void *weight, int64_t w_stride_c, int64_t w_stride_k, int W, const void *bias,
+    void *conv_states, int64_t s_stride_line, int64_t s_stride_c, int64_t s_stride_k,
+    int state_len, int num_lines, const int32_t *query_start_loc, int batch,
+    const int32_t *cache_indices, const uint8_t *has_initial_state, sconv_act act,
+    int pad_slot_id, void *out, sconv_dtype dt, int32_t *err_flag, cudaStream_t stream);
+
+/*
+ * sconv_causal_conv1d_update -- one decode token per sequence over dense
+ * state lines: the interface of causal_conv1d_update ("Implementation:Sgl
+ * project Sglang Mamba Ops").  For sequence b with line =
+ * conv_state_indices[b] (b when NULL; skipped when it equals pad_slot_id):
+ *   - cache_seqlens NULL (shifted line): the taps before the token are line
+ *     entries state_len-(W-1) .. state_len-1; afterwards the line holds its
+ *     last state_len-1 entries followed by x[b] -- exactly
+ *     sconv_causal_conv1d_fwd on a one-row sequence with has_initial_state 1;
+ *   - cache_seqlens given (circular line): s = cache_seqlens[b] inputs were
+ *     seen, the input at position p sits at entry p mod state_len, the taps
+ *     before the token are positions s-(W-1) .. s-1, and x[b] is stored at
+ *     entry s mod state_len, nothing else moving;
+ *   out[b, c] = act(sum_k weight[c][k] * tap_k + bias[c]), tap_{W-1} = x[b, c].
+ *
+ *   x [batch, dim] (strides x_stride_b, x_stride_c); out has x's strides and
+ *   is x itself or does not overlap it.  conv_state is required.  Other
+ *   arguments and errors as in sconv_causal_conv1d_fwd.
+ */
+sconv_status sconv_causal_conv1d_update(
+    void *x, int64_t x_stride_b, int64_t x_stride_c, int batch, int dim,
+    const void *weight, int64_t w_stride_c, int64_t w_stride_k, int W, const void *bias,
+    void *conv_state, int64_t s_stride_line, int64_t s_stride_c, int64_t s_stride_k,
+    int state_len, int num_lines, const int32_t *cache_seqlens,
+    const int32_t *conv_state_indices, sconv_act act, int pad_slot_id, void *out,
     sconv_dtype dt, int32_t *err_flag, cudaStream_t stream);
 
 /*

@@ -202,3 +202,43 @@ def test_gather_entry_points_host_validation(lib):
     assert paged(oss=16) == 1            # slot stride < C * d_conv
     assert paged(out=FAKE * 64 + 32) == 1  # inside the cache
     assert paged(bt_rs=2) == 1
+
+
+def test_dense_entry_points_host_validation(lib):
+    """Malformed calls of sconv_causal_conv1d_fwd / _update are rejected
+    before any launch (every call here either fails validation or has an
+    empty batch)."""
+    def fwd(batch=2, W=4, dt=1, act=1, L=3, x_st=16, x_sc=1, T=8, dim=16, out=FAKE,
+            states=FAKE * 64, s_c=3, s_k=1, lines=4, qsl=FAKE * 3, w=FAKE * 2):
+        return lib.sconv_causal_conv1d_fwd(
+            FAKE, x_st, x_sc, T, dim, w, 4, 1, W, 0, states, 48, s_c, s_k, L, lines, qsl,
+            batch, 0, 0, act, -1, out, dt, 0, 0)
+    assert fwd(batch=0) == 0
+    assert fwd(batch=0, x_st=1, x_sc=8) == 0       # channel-major x
+    assert fwd(batch=0, states=0) == 0              # no state lines
+    assert fwd(batch=-1) == 1
+    assert fwd(W=1) == 1
+    assert fwd(W=9) == 2
+    assert fwd(dt=5) == 2
+    assert fwd(act=3) == 1
+    assert fwd(L=2) == 1                            # state_len < W-1
+    assert fwd(L=17) == 2
+    assert fwd(x_st=8) == 1                         # rows of x overlap
+    assert fwd(out=FAKE + 2) == 1                   # out overlaps x without being x
+    assert fwd(states=FAKE + 4) == 1                # lines overlap x
+    assert fwd(s_c=2) == 1                          # line entries overlap
+    assert fwd(lines=0) == 1
+    assert fwd(qsl=0) == 1
+    assert fwd(dim=0) == 1
+    assert fwd(w=FAKE + 32) == 1                    # weight inside x (written in place)
+
+    def upd(batch=2, W=4, L=3, st=FAKE * 64, dt=1):
+        return lib.sconv_causal_conv1d_update(
+            FAKE, 16, 1, batch, 16, FAKE * 2, 4, 1, W, 0, st, 48, 3, 1, L, 4, 0, 0, 1, -1,
+            FAKE, dt, 0, 0)
+    assert upd(batch=0) == 0
+    assert upd(st=0) == 1
+    assert upd(batch=-3) == 1
+    assert upd(L=17) == 2
+    assert upd(W=9) == 2
+    assert upd(dt=9) == 2

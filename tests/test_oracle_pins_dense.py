@@ -339,3 +339,20 @@ def test_empty_sequence_line():
     assert rs.size == 0
     assert np.array_equal(new[l0], d["conv_states"][l0].numpy())
     assert not new[l1].any()
+
+
+@pytest.mark.parametrize("name", ["dense_prefill_bf16", "dense_decode_bf16"])
+def test_dense_named_workloads_are_well_formed(name):
+    d = workloads.DENSE_NAMED[name]()
+    if "query_start_loc" in d:
+        qsl = d["query_start_loc"].numpy()
+        assert qsl[0] == 0 and (np.diff(qsl) >= 1).all() and qsl[-1] == d["x"].shape[0]
+        lines = d["cache_indices"].numpy()
+        states = d["conv_states"]
+    else:
+        lines = d["conv_state_indices"].numpy()
+        states = d["conv_state"]
+    live = lines[lines != d["pad_slot_id"]]
+    assert len(set(live.tolist())) == len(live)
+    assert ((live >= 0) & (live < states.shape[0])).all()
+    assert states.shape[1] == d["x"].shape[1] and d["weight"].shape == (d["x"].shape[1], 4)

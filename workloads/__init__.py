@@ -443,3 +443,36 @@ def dense_update_inputs(seed, *, dtype, batch, dim, W, state_len, num_lines=None
         "cache_seqlens": None if seqlens is None else torch.from_numpy(seqlens).to(device),
         "pad_slot_id": pad_slot_id,
     }
+
+
+def dense_prefill_bf16(seed=1011, device="cpu"):
+    """Mixed varlen prefill over dense lines, the shapes of the chunked
+    prefill step: 16 sequences of uniform 1-2048 new tokens, each resuming
+    from its line when its cached prefix (uniform 0-2048) is non-empty;
+    dim = 4096, W = 4, L = 3, bias, SiLU, lines drawn from a pool of 64."""
+    rng = np.random.default_rng(seed)
+    prefix = rng.integers(0, 2049, size=16)
+    lens = rng.integers(1, 2049, size=16)
+    return dense_conv_inputs(seed, dtype="bf16", dim=4096, W=4, state_len=3, lens=lens,
+                             num_lines=64, has_init=prefix > 0, device=device)
+
+
+def dense_long_prefill_bf16(seed=1012, device="cpu"):
+    """One sequence of 65536 tokens from an empty line; dim = 8192 (the long
+    SSM-style prefill), W = 4, L = 3, weight N(0, 0.3), bias, SiLU."""
+    return dense_conv_inputs(seed, dtype="bf16", dim=8192, W=4, state_len=3, lens=[65536],
+                             num_lines=1, has_init=[False], w_sigma=0.3, device=device)
+
+
+def dense_decode_bf16(seed=1013, device="cpu"):
+    """One decode token for each of 256 sequences, dim = 1024, W = 4, L = 3,
+    shifted lines from a pool of 512, bias, SiLU."""
+    return dense_update_inputs(seed, dtype="bf16", batch=256, dim=1024, W=4, state_len=3,
+                               num_lines=512, device=device)
+
+
+DENSE_NAMED = {
+    "dense_prefill_bf16": dense_prefill_bf16,
+    "dense_long_prefill_bf16": dense_long_prefill_bf16,
+    "dense_decode_bf16": dense_decode_bf16,
+}
