@@ -215,22 +215,65 @@ struct TileWeights<bf16, MAXW> {
     }
 };
 
+// Two independent fp32 products (d_i = a_i * b_i, each rounded once) in one
+// packed sm_100 instruction.
+__device__ __forceinline__ void mul2(float &d0, float &d1, float a0, float a1, float b0,
+                                     float b1) {
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// The activation of VEC accumulators in place.  bf16 data: the operations
+// of silu<bf16> (h = y/2, then h + h*tanh(h)) with the multiply and the FMA
+// done two at a time in packed fp32 instructions -- the same roundings, so
+// the same bits as the scalar form the other kernels use.
+template <typename E, int VEC>
+__device__ __forceinline__ void silu_pack(float (&acc)[VEC]) {
+    if constexpr (sizeof(E) == 2) {
+        float h[VEC], t[VEC];
+#pragma unroll
+        for (int v = 0; v < VEC; v += 2) mul2(h[v], h[v + 1], acc[v], acc[v + 1], 0.5f, 0.5f);
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) asm("tanh.approx.f32 %0, %1;" : "=f"(t[v]) : "f"(h[v]));
+#pragma unroll
+        for (int v = 0; v < VEC; v += 2) {
+            acc[v] = h[v];
+            acc[v + 1] = h[v + 1];
+            fma2(acc[v], acc[v + 1], h[v], h[v + 1], t[v], t[v + 1]);
+        }
+    } else {
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) acc[v] = silu<E>(acc[v]);
+    }
+}
+
 // Prefill, token-major x.  Block i covers column y of sequence b (packs
 // y*PP .. y*PP+PP-1); with at most kLptMaxBatch sequences the blocks go
 // longest sequence first (so the long columns start in the first wave and
 // short ones fill the tail), else sequences interleave.  A tile is TT rows;
 // thread (g, p) = (threadIdx.x / PP, threadIdx.x % PP) convolves rows
 // g*RPT .. g*RPT+RPT-1 of pack p from a register window of W-1+RPT rows.
-// One barrier per tile: the carry is double-buffered (tile s reads
-// carry[s & 1] and writes the next carry into the other), and the ring
-// stage refilled at tile s was last read at tile s-1, before it.
-template <typename E, int PP, int MAXW, int THREADS>
+// Each ring stage holds HALO = WT-1 rows ahead of its tile: the rows before
+// the tile, written into the stage while the previous tile is computed (the
+// first from the state line), so every tap is a plain shared-memory read.
+// The last L inputs (the new state line) ride along in a double-buffered
+// carry.  One barrier per tile: tile s reads carry[s & 1] and writes the
+// next into the other, and the stage refilled at tile s was last read at
+// tile s-1.  WT is the exact tap count (2..4), or 8 for any W up to 8.
+template <typename E, int PP, int WT, int THREADS>
 __global__ void __launch_bounds__(THREADS) dense_fwd_tile(const __grid_constant__ DenseArgs a, int ncb) {
     constexpr int VEC = 16 / sizeof(E);
     constexpr int RPT = kRowsPerThread;
     constexpr int TT = THREADS / PP * RPT;
-    constexpr int NW = MAXW - 1 + RPT;  // window rows of one thread
-    extern __shared__ uint4 ring[];     // kStages * TT * PP packs
+    constexpr int HALO = WT - 1;
+    constexpr int SR = HALO + TT;       // rows of one ring stage
+    constexpr int NW = WT - 1 + RPT;    // window rows of one thread
+    extern __shared__ uint4 ring[];     // kStages * SR * PP packs
     __shared__ uint4 carry[2][kMaxL * PP];
     __shared__ int order[kLptMaxBatch];
 
@@ -260,19 +303,27 @@ __global__ void __launch_bounds__(THREADS) dense_fwd_tile(const __grid_constant_
     const int g = threadIdx.x / PP;
     const int c = (y * PP + p) * VEC;
     const bool cvalid = c < a.dim;
+    const int W = WT == 8 ? a.W : WT;
 
     int q0, n;
     int64_t line;
     bool from;
     if (!sequence_setup(a, b, threadIdx.x == 0 && y == 0, q0, n, line, from)) return;
-    const int Lc = a.st ? a.L : a.W - 1;  // entries of history ahead of x
-    const int ci = threadIdx.x / PP;      // carry entry this thread maintains (if < Lc)
+    const int L = a.L;
+    const int ci = threadIdx.x / PP;  // carry entry / halo row this thread maintains
 
-    // The carry starts as the history: the line, or zeros.
-    if (ci < Lc) carry[0][ci * PP + p] = cvalid ? line_pack<E, VEC>(a, line, c, ci, from)
-                                                : make_uint4(0u, 0u, 0u, 0u);
+    // The history: the line (or zeros) is the first carry, and its last
+    // HALO entries are the first stage's halo (zeros before the line).
+    if (a.st && ci < L)
+        carry[0][ci * PP + p] = cvalid ? line_pack<E, VEC>(a, line, c, ci, from)
+                                       : make_uint4(0u, 0u, 0u, 0u);
+    if (ci < HALO) {
+        const int e = L - HALO + ci;
+        ring[ci * PP + p] = (cvalid && a.st && e >= 0) ? line_pack<E, VEC>(a, line, c, e, from)
+                                                       : make_uint4(0u, 0u, 0u, 0u);
+    }
 
-    TileWeights<E, MAXW> wt;
+    TileWeights<E, WT> wt;
     float bias[VEC];
     if (cvalid) {
         wt.load(a, c);
@@ -290,7 +341,7 @@ __global__ void __launch_bounds__(THREADS) dense_fwd_tile(const __grid_constant_
             const int r = g + j * (TT / RPT);
             const int row = s * TT + r;
             if (s < ntiles && row < n && cvalid)
-                cp_async16(&ring[((s % kStages) * TT + r) * PP + p], x + row * a.x_st);
+                cp_async16(&ring[((s % kStages) * SR + HALO + r) * PP + p], x + row * a.x_st);
         }
         cp_async_commit();
     };
@@ -300,20 +351,19 @@ __global__ void __launch_bounds__(THREADS) dense_fwd_tile(const __grid_constant_
     const int r0 = g * RPT;
     for (int s = 0; s < ntiles; ++s) {
         cp_async_wait<kStages - 2>();
-        __syncthreads();  // tile s and carry[s & 1] are complete; tile s-1 is no longer read
+        __syncthreads();  // tile s, its halo and carry[s & 1] are complete
         issue(s + kStages - 1);
-        const uint4 *tile = ring + (s % kStages) * TT * PP;
-        const uint4 *cin = carry[s & 1];
+        const uint4 *stage = ring + (s % kStages) * SR * PP;  // row -HALO of the tile
         const int nv = min(TT, n - s * TT);
         if (r0 < nv && cvalid) {
-            // win[j] holds row r0 - (MAXW-1) + j (from the carry when < 0).
+            // win[j] holds tile row r0 - (WT-1) + j.
             uint4 win[NW];
 #pragma unroll
             for (int j = 0; j < NW; ++j) {
-                const int rr = r0 - (MAXW - 1) + j;
-                if (j < MAXW - a.W) continue;  // before the first tap of row r0
-                win[j] = rr >= 0 ? tile[rr * PP + p] : cin[(Lc + rr) * PP + p];
+                if (j < WT - W) continue;  // before the first tap of row r0
+                win[j] = stage[(r0 + j) * PP + p];
             }
+            E *orow = out + static_cast<int64_t>(s * TT + r0) * a.x_st;
 #pragma unroll
             for (int u = 0; u < RPT; ++u) {
                 if (r0 + u >= nv) break;
@@ -321,27 +371,28 @@ __global__ void __launch_bounds__(THREADS) dense_fwd_tile(const __grid_constant_
 #pragma unroll
                 for (int v = 0; v < VEC; ++v) acc[v] = bias[v];
 #pragma unroll
-                for (int kk = 0; kk < MAXW; ++kk)
-                    if (kk >= MAXW - a.W) wt.fma(acc, kk, win[u + kk]);
-                if (a.silu) {
-#pragma unroll
-                    for (int v = 0; v < VEC; ++v) acc[v] = silu<E>(acc[v]);
-                }
+                for (int kk = 0; kk < WT; ++kk)
+                    if (kk >= WT - W) wt.fma(acc, kk, win[u + kk]);
+                if (a.silu) silu_pack<E, VEC>(acc);
                 Pack<E, VEC> o;
                 o.from_float(acc);
-                o.store(out + static_cast<int64_t>(s * TT + r0 + u) * a.x_st);
+                o.store(orow + u * a.x_st);
             }
         }
-        // Next carry: the last Lc entries of (carry, the tile's nv rows).
-        if (ci < Lc) {
+        // The next stage's halo: the last HALO rows of this (full) tile.
+        if (ci < HALO && s + 1 < ntiles)
+            ring[((s + 1) % kStages) * SR * PP + ci * PP + p] = stage[(TT + ci) * PP + p];
+        // Next carry: the last L entries of (carry, the tile's nv rows).
+        if (a.st && ci < L) {
+            const uint4 *cin = carry[s & 1];
             const int src = nv + ci;
             carry[(s + 1) & 1][ci * PP + p] =
-                src >= Lc ? tile[(src - Lc) * PP + p] : cin[src * PP + p];
+                src >= L ? stage[(HALO + src - L) * PP + p] : cin[src * PP + p];
         }
     }
     cp_async_wait<0>();
     // Each thread stores the carry entry it wrote itself: no barrier needed.
-    if (a.st && ci < Lc && cvalid)
+    if (a.st && ci < L && cvalid)
         store_line_pack<E, VEC>(a, line, c, ci, carry[ntiles & 1][ci * PP + p]);
 }
 
@@ -618,40 +669,50 @@ int pick_pp(int batch, int packs) {
     return 1;
 }
 
-template <typename E, int PP, int MAXW, int THREADS>
+template <typename E, int PP, int WT, int THREADS>
 cudaError_t launch_tile_pp(const DenseArgs &a, int packs, cudaStream_t stream) {
     constexpr int TT = THREADS / PP * kRowsPerThread;
-    constexpr size_t kSmem = static_cast<size_t>(kStages) * TT * PP * sizeof(uint4);
+    constexpr size_t kSmem = static_cast<size_t>(kStages) * (WT - 1 + TT) * PP * sizeof(uint4);
     static bool configured = false;
     if (!configured) {
         const cudaError_t e = cudaFuncSetAttribute(
-            dense_fwd_tile<E, PP, MAXW, THREADS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            dense_fwd_tile<E, PP, WT, THREADS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
             static_cast<int>(kSmem));
         if (e != cudaSuccess) return e;
         configured = true;
     }
     const int ncb = (packs + PP - 1) / PP;
-    return launch_pdl(dense_fwd_tile<E, PP, MAXW, THREADS>,
+    return launch_pdl(dense_fwd_tile<E, PP, WT, THREADS>,
                       dim3(static_cast<unsigned>(static_cast<int64_t>(a.batch) * ncb)),
                       dim3(THREADS), kSmem, stream, a, ncb);
 }
 
-template <typename E, int MAXW>
+template <typename E, int WT>
+cudaError_t launch_tile_w(const DenseArgs &a, int packs, int pp, cudaStream_t stream) {
+    switch (pp) {
+        case 8: return launch_tile_pp<E, 8, WT, kTileThreads>(a, packs, stream);
+        case 4: return launch_tile_pp<E, 4, WT, kTileThreads>(a, packs, stream);
+        case 2: return launch_tile_pp<E, 2, WT, kTileThreads>(a, packs, stream);
+        default: return launch_tile_pp<E, 1, WT, kTileThreads>(a, packs, stream);
+    }
+}
+
+template <typename E>
 cudaError_t launch_tile(const DenseArgs &a, cudaStream_t stream) {
     constexpr int VEC = 16 / sizeof(E);
     const int packs = a.dim / VEC;
     const int pp = pick_pp(a.batch, packs);
-    switch (pp) {
-        case 8: return launch_tile_pp<E, 8, MAXW, kTileThreads>(a, packs, stream);
-        case 4: return launch_tile_pp<E, 4, MAXW, kTileThreads>(a, packs, stream);
-        case 2: return launch_tile_pp<E, 2, MAXW, kTileThreads>(a, packs, stream);
-        default: return launch_tile_pp<E, 1, MAXW, kTileThreads>(a, packs, stream);
+    switch (a.W) {
+        case 2: return launch_tile_w<E, 2>(a, packs, pp, stream);
+        case 3: return launch_tile_w<E, 3>(a, packs, pp, stream);
+        case 4: return launch_tile_w<E, 4>(a, packs, pp, stream);
+        default: return launch_tile_w<E, 8>(a, packs, pp, stream);
     }
 }
 
 template <typename E, int MAXW>
 cudaError_t launch_fwd_t(const DenseArgs &a, bool vec, cudaStream_t stream) {
-    if (vec) return launch_tile<E, MAXW>(a, stream);
+    if (vec) return launch_tile<E>(a, stream);
     return launch_pdl(dense_fwd_generic<E, MAXW>, dim3(a.batch, (a.dim + 127) / 128), dim3(128),
                       0, stream, a);
 }
