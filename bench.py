@@ -356,9 +356,10 @@ def fused_launch_duration(sets_obj, stream, reps=200):
     number of launches."""
     n = len(sets_obj.sets)
     g = capture(lambda: [sets_obj.step(i, metadata=False) for i in range(n)], stream)
-    for _ in range(3):
-        g.replay()
-    stream.synchronize()
+    with torch.cuda.stream(stream):  # on the timed stream, finished before timing
+        for _ in range(3):
+            g.replay()
+    torch.cuda.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         s.record()
@@ -377,9 +378,13 @@ def _kernel_time(step_fns, reps, stream):
     """Mean seconds per call of the launches in step_fns, replayed from one
     CUDA graph and timed with CUDA events on the launching stream."""
     g = capture(lambda: [f() for f in step_fns], stream)
-    for _ in range(3):  # warm-up replays (clocks, caches, lazy module loads)
-        g.replay()
-    stream.synchronize()
+    # Warm-up replays (clocks, caches, lazy module loads) on the timed stream,
+    # finished device-wide before the first event: a warm-up left running on
+    # another stream would overlap the timed replays and inflate them.
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+    torch.cuda.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         s.record()
