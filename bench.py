@@ -60,7 +60,8 @@ def parse_args():
     p.add_argument("--seed", type=int, default=1002)
     p.add_argument("--only", choices=["chunked_prefill_bf16", "long_prefill_bf16",
                                       "spec_decode_bf16", "dense", "dense_prefill_bf16",
-                                      "dense_long_prefill_bf16", "dense_decode_bf16"],
+                                      "dense_long_prefill_bf16", "dense_decode_bf16",
+                                      "decode_chain"],
                    help="time just this workload's kernels and print its table row")
     p.add_argument("--max-hist", type=int, default=4096,
                    help="longest cached history of the decode requests (smaller only for "
@@ -527,6 +528,73 @@ def bench_streams(sets_obj, stream, peak, reps=200):
         "alg_gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}}
 
 
+def decode_chain_step(hs, sets_obj, i, layers, pdl, side):
+    """One decode step through a stack of layers: sconv_seq_metadata, then
+    one sconv_fused per layer (its own cache and weight), layer l+1
+    convolving layer l's output.  pdl: every launch on the current stream
+    (programmatic dependent launch between neighbours).  Otherwise the
+    layers alternate between the current stream and `side`, joined by
+    events, so each launch waits for its predecessor to finish."""
+    wl, s = sets_obj.wls[i], sets_obj.sets[i]
+    main = torch.cuda.current_stream()
+    hs.sconv_seq_metadata(s["query_start_loc"], wl.R, wl.T, s["seq_idx"], s["query_start"])
+    x, cur = s["x"], main
+    for l, (cache, weight, out) in enumerate(layers):
+        target = main if (pdl or l % 2 == 0) else side
+        if target is not cur:
+            ev = torch.cuda.Event()
+            ev.record(cur)
+            target.wait_event(ev)
+        with torch.cuda.stream(target):
+            hs.sconv_fused(x, weight, cache, s["positions"], s["block_table"], s["seq_idx"],
+                           s["slot_mapping"], s["query_start"], out=out, **wl.kwargs())
+        cur, x = target, out
+    if cur is not main:
+        ev = torch.cuda.Event()
+        ev.record(cur)
+        main.wait_event(ev)
+
+
+def bench_decode_chain(sets_obj, stream, peak, n_layers=4, reps=50):
+    """The decode workload through a stack of n_layers layers (each its own
+    4.2 GB cache and weight; layer l+1 convolves layer l's output, the chain
+    a model's decode step runs, without the projections between), over the
+    96 rotating sets.  Timed with every launch on one stream (PDL: a launch
+    becomes resident while its predecessor runs and prefetches its
+    metadata, block-table lines and cache taps before waiting) and with the
+    layers alternating between two streams joined by events (each launch
+    starts only when its predecessor has finished)."""
+    import hybrid_sconv_b200 as hs
+    dev = sets_obj.device
+    w0 = sets_obj.wls[0]
+    g = torch.Generator(device=dev).manual_seed(4242)
+    layers = []
+    for l in range(n_layers):
+        if l == 0:
+            cache, weight = sets_obj.cache, sets_obj.weight
+        else:
+            cache = torch.empty_like(sets_obj.cache)
+            workloads.fill_normal_(cache, 1.0, g, dev)
+            weight = workloads.normal((w0.C, w0.W), w0.w_sigma, torch.bfloat16, g, dev)
+        layers.append((cache, weight, torch.zeros((w0.T, w0.C), dtype=torch.bfloat16, device=dev)))
+    side = torch.cuda.Stream(dev)
+    n = len(sets_obj.sets)
+    res = {}
+    for mode, pdl in (("pdl", True), ("serialised", False)):
+        secs = _kernel_time([lambda i=i: decode_chain_step(hs, sets_obj, i, layers, pdl, side)
+                             for i in range(n)], reps, stream)
+        res[mode] = secs
+    del layers
+    torch.cuda.empty_cache()
+    return {f"decode_chain_{n_layers}_layers": {
+        "step_us_pdl": round(res["pdl"] * 1e6, 3),
+        "step_us_serialised": round(res["serialised"] * 1e6, 3),
+        "layer_us_pdl": round(res["pdl"] * 1e6 / n_layers, 3),
+        "layer_us_serialised": round(res["serialised"] * 1e6 / n_layers, 3),
+        "mtokens_s_layers": round(w0.T * n_layers / res["pdl"] / 1e6, 2),
+        "launches_per_step": 1 + n_layers}}
+
+
 def bench_ssm_gather(device, stream, peak, reps=50):
     """Conditional SSM state gather: 256 chunk-scan states of [64, 64, 128]
     fp32 (2 MB rows), 64 slots of which 40 real, 8 rotating index sets over
@@ -634,6 +702,7 @@ def per_workload_table(device, stream, peak, sets_obj=None):
     if sets_obj is not None:
         table.update(bench_update(sets_obj, stream, peak))
         table.update(bench_streams(sets_obj, stream, peak))
+        table.update(bench_decode_chain(sets_obj, stream, peak))
     table.update(bench_prefill("chunked_prefill_bf16", device, stream, peak))
     table.update(bench_prefill("long_prefill_bf16", device, stream, peak))
     table.update(bench_spec_decode(device, stream, peak))
@@ -797,6 +866,9 @@ def main():
             row = bench_spec_decode(device, stream, peak)
         elif args.only == "dense":
             row = bench_dense(device, stream, peak)
+        elif args.only == "decode_chain":
+            sets_obj = DecodeSets(args.sets, rank_seed(args.seed, rank), device, args.max_hist)
+            row = bench_decode_chain(sets_obj, stream, peak)
         elif args.only == "dense_decode_bf16":
             row = bench_dense_decode(device, stream, peak, nsets=args.sets,
                                      reps=max(3, args.steps))
