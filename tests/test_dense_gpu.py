@@ -303,3 +303,10 @@ def test_benchmark_sizes_on_channel_slices(name):
     chans = [(0, 24), (dim // 2 - 8, dim // 2 + 24), (dim - 40, dim)]
     _slice_check(d, "bf16", True, chans, x_before, states_before, d["x"].cpu(),
                  d["conv_states"].cpu())
+
+
+def test_decode_benchmark_size_full():
+    """The benchmark's decode update (256 sequences, dim 1024, L 3) against
+    the oracle element by element, lines bit-exact."""
+    u = workloads.dense_decode_bf16()
+    assert _run_update(u, "bf16", silu=True) == 0
