@@ -5,18 +5,18 @@
 // may all be updated in place.
 //
 //  * dense_fwd_tile -- varlen prefill, x token-major in 16-byte channel
-//    packs.  One 256-thread block owns a (sequence, channel block) column of
-//    PP packs and walks it in tiles of TT = 256 / PP rows: each thread
-//    copies one pack of a tile ahead into a kStages-deep shared-memory ring
-//    with cp.async (only rows of this sequence, so nothing past its end is
-//    read), convolves one row of the current tile and stores it.  The W-1
-//    rows before a tile come from a shared-memory carry of the column's last
-//    L inputs, which starts as the state line and ends as the new line: no
-//    block re-reads x rows that another block may already have overwritten,
-//    so the in-place form needs no scratch memory and no ordering between
-//    blocks.  PP is chosen per call so that the grid covers the SMs: wide
-//    columns (fewer, longer blocks) for many sequences, narrow ones for a
-//    few long sequences.
+//    packs.  One 256-thread block owns a (sequence, column of PP packs) and
+//    walks it in tiles of TT = 2 * 256 / PP rows: each thread copies two
+//    packs of a tile seven tiles ahead into a shared-memory ring with
+//    cp.async (only rows of this sequence, so nothing past its end is read)
+//    and convolves two rows of the current tile.  Each ring stage holds the
+//    W-1 rows before its tile, written while the previous tile is computed;
+//    the column's last L inputs ride along in a carry that starts as the
+//    state line and ends as the new line.  No block re-reads x rows that
+//    another block may already have overwritten, so the in-place form needs
+//    no scratch memory and no ordering between blocks.  PP is chosen per
+//    call: the widest column that still gives the SMs 1.5 blocks each, and
+//    blocks run longest sequence first.
 //  * dense_fwd_generic -- any x layout (channel-major included): a thread per
 //    (sequence, channel) walks the rows with the taps in registers.
 //  * dense_update -- one token per sequence; shifted or circular line.
