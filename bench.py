@@ -26,6 +26,7 @@ import argparse
 import hashlib
 import json
 import os
+import platform
 import re
 import statistics
 import subprocess
@@ -733,7 +734,22 @@ def cpu_baseline(sets_obj, seconds=8.0):
     return {"value": round(n * wl.T / el / 1e6, 6), "unit": UNIT, "cores": 1,
             "kind": "oracle",
             "sample": f"{n} full decode steps ({wl.T} tokens each, C={wl.C}) on one core, "
-                      f"{el:.1f} s"}
+                      f"{el:.1f} s",
+            "host": host_cpu()}
+
+
+def host_cpu() -> dict:
+    """The host's logical CPU count and model name (for the CPU baseline)."""
+    model = platform.processor() or "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "model": model}
 
 
 # --------------------------------------------------------------------------
@@ -874,7 +890,7 @@ def main_reference(args, rank, world):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_block(1),
             "cpu_baseline": {"value": round(v, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample, "host": host_cpu()},
             "e2e": {"value": round(v, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
