@@ -315,13 +315,48 @@ class DecodeSets:
                            **wl.kwargs())
 
 
-def run_steps_graphs(sets_obj, K, stream, **step_kw):
-    """Graphs that together replay exactly K steps over the rotating sets."""
+def pipelined_steps(sets_obj, idxs, side):
+    """Steps idxs in order, each sconv_seq_metadata + sconv_fused over its
+    batch, with the next step's metadata built beside the current step's
+    convolution, as a serving engine prepares step i+1's inputs while step
+    i runs: metadata(i+1) goes to `side` once conv(i-1) has finished (its
+    buffers are the next batch's own), and conv(i+1) waits for both
+    conv(i) (its cache inserts are the next step's history) and
+    metadata(i+1).  Each step still launches both kernels."""
+    main = torch.cuda.current_stream()
+    side.wait_stream(main)
+    with torch.cuda.stream(side):
+        sets_obj.step(idxs[0], fused=False)
+    meta_done = torch.cuda.Event()
+    meta_done.record(side)
+    for j, i in enumerate(idxs):
+        main.wait_event(meta_done)
+        before = torch.cuda.Event()
+        before.record(main)  # everything up to conv(i-1)
+        sets_obj.step(i, metadata=False)
+        if j + 1 < len(idxs):
+            side.wait_event(before)
+            with torch.cuda.stream(side):
+                sets_obj.step(idxs[j + 1], fused=False)
+            meta_done = torch.cuda.Event()
+            meta_done.record(side)
+    main.wait_stream(side)
+
+
+def run_steps_graphs(sets_obj, K, stream, pipeline=False, **step_kw):
+    """Graphs that together replay exactly K steps over the rotating sets
+    (pipelined: next-step metadata beside the current convolution)."""
     M = len(sets_obj.sets)
-    full = capture(lambda: [sets_obj.step(i, **step_kw) for i in range(M)], stream)
-    tail = None
-    if K % M:
-        tail = capture(lambda: [sets_obj.step(i, **step_kw) for i in range(K % M)], stream)
+    side = torch.cuda.Stream(stream.device)
+
+    def steps(n):
+        if pipeline:
+            pipelined_steps(sets_obj, list(range(n)), side)
+        else:
+            for i in range(n):
+                sets_obj.step(i, **step_kw)
+    full = capture(lambda: steps(M), stream)
+    tail = capture(lambda: steps(K % M), stream) if K % M else None
     return full, tail, K // M
 
 
@@ -484,6 +519,21 @@ def bench_spec_decode(device, stream, peak, n_sets=40):
     del cache, fns
     torch.cuda.empty_cache()
     return res
+
+
+def bench_serial_step(sets_obj, stream, peak, reps=200):
+    """The decode step without pipelining: metadata then convolution, each
+    step's metadata waiting for the previous step's convolution."""
+    full, _, _ = run_steps_graphs(sets_obj, len(sets_obj.sets), stream, pipeline=False)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            full.replay()
+    torch.cuda.synchronize()
+    secs, _ = time_region(full, None, reps, stream, 1)
+    del full
+    per = secs / (reps * len(sets_obj.sets))
+    return {"decode_step_serial": {"step_us": round(per * 1e6, 3),
+                                   "mtokens_s": round(sets_obj.wls[0].T / per / 1e6, 2)}}
 
 
 def bench_update(sets_obj, stream, peak, reps=200):
@@ -701,6 +751,7 @@ def bench_dense(device, stream, peak):
 def per_workload_table(device, stream, peak, sets_obj=None):
     table = {}
     if sets_obj is not None:
+        table.update(bench_serial_step(sets_obj, stream, peak))
         table.update(bench_update(sets_obj, stream, peak))
         table.update(bench_streams(sets_obj, stream, peak))
         table.update(bench_decode_chain(sets_obj, stream, peak))
@@ -842,6 +893,9 @@ def config_block(world):
             "global_batch": 256 * world, "seq_len": 1,
             "parallelism": f"dp{world}" if world > 1 else "single",
             "step": "sconv_seq_metadata + sconv_fused",
+            "pipelining": "the next step's sconv_seq_metadata runs beside the current "
+                          "step's sconv_fused (engine-style input preparation); the "
+                          "convolutions run in order, each waiting for the previous one",
             "l2": "rotating input sets (each touching its own cache blocks), combined "
                   "footprint > 126 MB L2"}
 
@@ -931,11 +985,12 @@ def main():
     touched = sum(sets_obj.alg_bytes)
 
     # warm-up, then exactly K timed steps
-    wfull, wtail, wreps = run_steps_graphs(sets_obj, W, stream)
-    replay_steps(wfull, wtail, wreps)
+    wfull, wtail, wreps = run_steps_graphs(sets_obj, W, stream, pipeline=True)
+    with torch.cuda.stream(stream):
+        replay_steps(wfull, wtail, wreps)
     torch.cuda.synchronize()
     del wfull, wtail
-    full, tail, reps = run_steps_graphs(sets_obj, K, stream)
+    full, tail, reps = run_steps_graphs(sets_obj, K, stream, pipeline=True)
     sampler = ClockSampler(local) if rank == 0 else None
     secs, (w0, w1) = time_region(full, tail, reps, stream, world, sampler)
     secs = max_over_ranks(secs, world)

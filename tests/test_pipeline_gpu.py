@@ -1,0 +1,67 @@
+"""The benchmark's pipelined decode steps compute exactly what the plain
+sequence of steps computes.
+
+Pipelining builds step i+1's metadata (sconv_seq_metadata,
+"vllm.models.inkling.nvidia.ops.sconv") on a second stream while step i's
+sconv_fused runs; the convolutions keep their order, since step i+1 reads
+as history what step i inserted.  Several batches share one paged cache
+here, so any reordering of the convolutions or a metadata buffer read
+before it is complete would change the bits.
+"""
+from __future__ import annotations
+
+import pytest
+import torch
+
+import bench
+from tests._gpu import raw
+
+pytestmark = pytest.mark.gpu
+
+
+def _snapshot(sets_obj):
+    return raw(sets_obj.cache).clone(), [raw(s["out"]).clone() for s in sets_obj.sets]
+
+
+def _reset(sets_obj, cache0):
+    raw(sets_obj.cache).copy_(cache0)
+    for s in sets_obj.sets:
+        raw(s["out"]).fill_(-1)
+        s["seq_idx"].fill_(-7)
+        s["query_start"].fill_(-7)
+
+
+@pytest.mark.parametrize("n", [1, 2, 6])
+def test_pipelined_steps_equal_plain_steps(n):
+    dev = torch.device("cuda", 0)
+    sets_obj = bench.DecodeSets(n, 5151, dev, max_hist=64)
+    cache0 = raw(sets_obj.cache).clone()
+
+    _reset(sets_obj, cache0)
+    for i in range(n):
+        sets_obj.step(i)
+    torch.cuda.synchronize()
+    plain_cache, plain_outs = _snapshot(sets_obj)
+
+    side = torch.cuda.Stream(dev)
+    _reset(sets_obj, cache0)
+    bench.pipelined_steps(sets_obj, list(range(n)), side)
+    torch.cuda.synchronize()
+    cache, outs = _snapshot(sets_obj)
+    assert torch.equal(cache, plain_cache)
+    for a, b in zip(outs, plain_outs):
+        assert torch.equal(a, b)
+
+    # the same from the benchmark's graphs (two rounds over the batches)
+    stream = torch.cuda.Stream(dev)
+    _reset(sets_obj, cache0)
+    full, tail, reps = bench.run_steps_graphs(sets_obj, n, stream, pipeline=True)
+    _reset(sets_obj, cache0)
+    with torch.cuda.stream(stream):
+        bench.replay_steps(full, tail, reps)
+    torch.cuda.synchronize()
+    cache, outs = _snapshot(sets_obj)
+    assert torch.equal(cache, plain_cache)
+    for a, b in zip(outs, plain_outs):
+        assert torch.equal(a, b)
+    del full, tail
