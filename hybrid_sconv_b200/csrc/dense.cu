@@ -17,8 +17,11 @@
 //    no scratch memory and no ordering between blocks.  PP is chosen per
 //    call: the widest column that still gives the SMs 1.5 blocks each, and
 //    blocks run longest sequence first.
-//  * dense_fwd_generic -- any x layout (channel-major included): a thread per
-//    (sequence, channel) walks the rows with the taps in registers.
+//  * dense_fwd_cm -- channel-major x (token stride 1): a warp per (sequence,
+//    channel) walks the channel's contiguous tokens, four per lane, with the
+//    taps before a lane's tokens shuffled from the lanes below.
+//  * dense_fwd_generic -- any other layout: a thread per (sequence, channel)
+//    walks the rows with the taps in registers.
 //  * dense_update -- one token per sequence; shifted or circular line.
 //
 // Every sum runs oldest tap first, starting from the bias, in fp32 FMAs, so
@@ -46,6 +49,31 @@ struct RawOf<bf16> {
 template <>
 struct RawOf<float> {
     using T = uint32_t;
+};
+
+// VEC raw elements moved as one load or store of VEC * sizeof(R) bytes.
+template <int BYTES>
+struct RawVec;
+template <>
+struct RawVec<2> {
+    using T = uint16_t;
+};
+template <>
+struct RawVec<4> {
+    using T = uint32_t;
+};
+template <>
+struct RawVec<8> {
+    using T = uint2;
+};
+template <>
+struct RawVec<16> {
+    using T = uint4;
+};
+template <typename R, int VEC>
+union Lanes {
+    typename RawVec<VEC * sizeof(R)>::T v;
+    R e[VEC];
 };
 
 __device__ __forceinline__ float raw_to_float(uint16_t v) {
@@ -396,6 +424,173 @@ __global__ void __launch_bounds__(THREADS) dense_fwd_tile(const __grid_constant_
         store_line_pack<E, VEC>(a, line, c, ci, carry[ntiles & 1][ci * PP + p]);
 }
 
+// Prefill, channel-major x (token stride 1).  Warp (b, c) walks channel c of
+// sequence b in chunks of 32 * TOK tokens, lane l holding TOK consecutive
+// tokens (one 16-byte vector) of a chunk.  The chunks are aligned to 16-byte
+// boundaries of the row, so a sequence that starts mid-vector has its first
+// `skew` slots masked: those read the state line (or zero) instead of x, and
+// are not written.  The W-1 tokens before a lane's first come from the lanes
+// below it (for the lowest lanes, from the previous chunk, or from the state
+// line for the first) by shuffles.  Chunks are loaded kCmAhead ahead.  A warp
+// reads a chunk before it writes it and never reads a chunk it has written,
+// so the in-place form is safe; masked slots may belong to a neighbouring
+// sequence, whose warp may be writing them, and are never used.  The sums
+// run oldest tap first from the bias, as in the other kernels.
+constexpr int kCmAhead = 4;  // chunks loaded ahead
+
+template <typename E, int MAXW>
+__global__ void __launch_bounds__(256) dense_fwd_cm(const __grid_constant__ DenseArgs a) {
+    using R = typename RawOf<E>::T;
+    constexpr int TOK = 16 / sizeof(R);  // tokens per lane
+    constexpr int CHUNK = 32 * TOK;      // tokens per warp chunk
+    constexpr unsigned kFull = 0xffffffffu;
+    const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const bool live = gw < static_cast<int64_t>(a.batch) * a.dim;
+    const int b = static_cast<int>(gw / a.dim);
+    const int c = static_cast<int>(gw - static_cast<int64_t>(b) * a.dim);
+    const int W = a.W, L = a.L;
+    // The weights are constant: loaded while the preceding kernel drains.
+    // wl[d] multiplies the token d back (weight column W-1-d).
+    float wl[MAXW];
+    float bias = 0.f;
+    if (live) {
+        const E *wp = static_cast<const E *>(a.w) + static_cast<int64_t>(c) * a.w_sc;
+#pragma unroll
+        for (int d = 0; d < MAXW; ++d) wl[d] = d < W ? load_weight(wp + (W - 1 - d) * a.w_sk) : 0.f;
+        if (a.bias) bias = load_weight(static_cast<const E *>(a.bias) + c);
+    }
+    pdl_wait();
+    pdl_trigger();
+    if (!live) return;
+    int q0, n;
+    int64_t line;
+    bool from;
+    if (!sequence_setup(a, b, lane == 0 && c == 0, q0, n, line, from)) return;
+
+    R *st = a.st ? static_cast<R *>(a.st) + line * a.s_line + static_cast<int64_t>(c) * a.s_c
+                 : nullptr;
+    // Token t of the sequence (t < 0: the history) as it enters the taps.
+    auto history = [&](int t) -> float {
+        const int h = L + t;  // line entry
+        return (from && h >= 0) ? raw_to_float(st[static_cast<int64_t>(h) * a.s_k]) : 0.f;
+    };
+
+    const int64_t base = static_cast<int64_t>(c) * a.x_sc + static_cast<int64_t>(q0) * a.x_st;
+    const R *xrow = static_cast<const R *>(a.x) + base;
+    R *orow = static_cast<R *>(a.out) + base;
+    // Slots of the first vector before the sequence's first token (x itself
+    // is 16-byte aligned: the host sends other layouts elsewhere).
+    const int skew = static_cast<int>((reinterpret_cast<uintptr_t>(xrow) / sizeof(R)) % TOK);
+    const bool aligned_out = ((reinterpret_cast<uintptr_t>(orow) / sizeof(R)) % TOK) == skew &&
+                             (reinterpret_cast<uintptr_t>(orow) % sizeof(R)) == 0;
+    const int nchunks = (n + skew + CHUNK - 1) / CHUNK;
+    const R *xv = xrow - skew;  // 16-byte aligned
+    R *ov = orow - skew;
+
+    // This lane's vector of chunk k.  A whole 16-byte load only when the
+    // vector ends inside the sequence (its start may lie before it: those
+    // slots are still inside x, since x is 16-byte aligned, and are replaced
+    // by the history); otherwise single elements of the sequence only, so
+    // nothing past the sequence's last token is read.
+    auto fetch = [&](int k) -> uint4 {
+        const int t0 = k * CHUNK - skew + TOK * lane;
+        if (t0 + TOK <= n) return *reinterpret_cast<const uint4 *>(xv + k * CHUNK + TOK * lane);
+        Lanes<R, TOK> v;
+        v.v = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int i = 0; i < TOK; ++i)
+            if (t0 + i >= 0 && t0 + i < n) v.e[i] = xrow[t0 + i];
+        return v.v;
+    };
+    // x first: its loads do not wait for the line's.
+    uint4 buf[kCmAhead];
+#pragma unroll
+    for (int u = 0; u < kCmAhead; ++u)
+        if (u < nchunks) buf[u] = fetch(u);
+    // Every read of the old line comes before any write to it.  prv: this
+    // lane's slots of the previous chunk (before the first chunk, the
+    // history); head: the first chunk's slots before the sequence (the
+    // history); keep: the entries that survive the call (n < L: new entry i
+    // = old entry n + i).
+    float prv[TOK], head[TOK];
+#pragma unroll
+    for (int i = 0; i < TOK; ++i) {
+        prv[i] = history(TOK * lane + i - CHUNK - skew);
+        const int t = TOK * lane + i - skew;
+        head[i] = t < 0 ? history(t) : 0.f;
+    }
+    if (st) {
+        const bool mine = lane < L && n + lane < L;
+        R keep = R(0);
+        if (mine && from) keep = st[static_cast<int64_t>(n + lane) * a.s_k];
+        __syncwarp();  // the old line is read (by every lane) before any entry is written
+        if (mine) st[static_cast<int64_t>(lane) * a.s_k] = keep;
+    }
+
+    for (int k0 = 0; k0 < nchunks; k0 += kCmAhead) {
+#pragma unroll
+        for (int u = 0; u < kCmAhead; ++u) {
+            const int k = k0 + u;
+            if (k >= nchunks) break;
+            Lanes<R, TOK> cur;
+            cur.v = buf[u];
+            if (k + kCmAhead < nchunks) buf[u] = fetch(k + kCmAhead);  // never a chunk it wrote
+            const int t0 = k * CHUNK - skew + TOK * lane;  // sequence index of slot 0
+            const bool full = k * CHUNK >= skew && (k + 1) * CHUNK - skew <= n;  // warp-uniform
+            float xf[TOK];
+#pragma unroll
+            for (int i = 0; i < TOK; ++i) xf[i] = raw_to_float(cur.e[i]);
+            if (!full) {
+#pragma unroll
+                for (int i = 0; i < TOK; ++i)
+                    if (t0 + i < 0) xf[i] = head[i];  // only in the first chunk
+            }
+            // p[j] = slot -j relative to this lane's first, from lane
+            // l - ceil(j/TOK) of this chunk or (below lane 0) of the previous.
+            float p[MAXW];
+#pragma unroll
+            for (int j = 1; j < MAXW; ++j) {
+                if (j >= W) break;  // uniform across the warp
+                const int src = lane - (j + TOK - 1) / TOK;
+                const int e = (TOK - j % TOK) % TOK;
+                const float vc = __shfl_sync(kFull, xf[e], src & 31);
+                const float vp = __shfl_sync(kFull, prv[e], src & 31);
+                p[j] = src >= 0 ? vc : vp;
+            }
+            Lanes<R, TOK> y;
+#pragma unroll
+            for (int i = 0; i < TOK; ++i) {
+                float acc = bias;
+#pragma unroll
+                for (int d = MAXW - 1; d >= 0; --d) {
+                    if (d >= W) continue;
+                    acc = fmaf(wl[d], d <= i ? xf[i - d] : p[d - i], acc);
+                }
+                if (a.silu) acc = silu<E>(acc);
+                y.e[i] = float_to_raw<E>(acc);
+            }
+            if (aligned_out && t0 >= 0 && t0 + TOK <= n) {
+                *reinterpret_cast<uint4 *>(ov + k * CHUNK + TOK * lane) = y.v;
+            } else {
+#pragma unroll
+                for (int i = 0; i < TOK; ++i)
+                    if (t0 + i >= 0 && t0 + i < n) orow[t0 + i] = y.e[i];
+            }
+            if (st && (k + 1) * CHUNK - skew > n - L) {  // the chunk holds part of the last L
+#pragma unroll
+                for (int i = 0; i < TOK; ++i) {
+                    const int t = t0 + i;
+                    if (t >= 0 && t < n && t >= n - L)
+                        st[static_cast<int64_t>(t - (n - L)) * a.s_k] = cur.e[i];
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < TOK; ++i) prv[i] = xf[i];
+        }
+    }
+}
+
 // Prefill, any x layout: thread (b, c) walks sequence b's rows of channel c.
 // prev[j-1] holds the input j rows back; lag-j weight wl[j] = weight[c][W-1-j].
 template <typename E, int MAXW>
@@ -450,30 +645,6 @@ __global__ void __launch_bounds__(128) dense_fwd_generic(const __grid_constant__
     }
 }
 
-// VEC raw elements moved as one load or store of VEC * sizeof(R) bytes.
-template <int BYTES>
-struct RawVec;
-template <>
-struct RawVec<2> {
-    using T = uint16_t;
-};
-template <>
-struct RawVec<4> {
-    using T = uint32_t;
-};
-template <>
-struct RawVec<8> {
-    using T = uint2;
-};
-template <>
-struct RawVec<16> {
-    using T = uint4;
-};
-template <typename R, int VEC>
-union Lanes {
-    typename RawVec<VEC * sizeof(R)>::T v;
-    R e[VEC];
-};
 
 // Decode: thread (b, j) updates channels c .. c+VEC-1 of sequence b (VEC * 2
 // or 4 bytes: many threads, little serial work each, since one decode step
@@ -713,6 +884,12 @@ cudaError_t launch_tile(const DenseArgs &a, cudaStream_t stream) {
 template <typename E, int MAXW>
 cudaError_t launch_fwd_t(const DenseArgs &a, bool vec, cudaStream_t stream) {
     if (vec) return launch_tile<E>(a, stream);
+    if (a.x_st == 1 && a.T > 1 && (reinterpret_cast<uintptr_t>(a.x) & 15u) == 0) {
+        // channel-major: a warp per (sequence, channel)
+        const int64_t warps = static_cast<int64_t>(a.batch) * a.dim;
+        return launch_pdl(dense_fwd_cm<E, MAXW>, dim3(static_cast<unsigned>((warps + 7) / 8)),
+                          dim3(256), 0, stream, a);
+    }
     return launch_pdl(dense_fwd_generic<E, MAXW>, dim3(a.batch, (a.dim + 127) / 128), dim3(128),
                       0, stream, a);
 }

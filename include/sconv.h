@@ -300,9 +300,12 @@ sconv_status sconv_extract_windows_paged(
  *                    [0, num_lines) sets SCONV_EFLAG_SLOT, one whose
  *                    query_start_loc entries are out of order or range sets
  *                    SCONV_EFLAG_QUERY_START; such a sequence is skipped.
- * One thread block owns a (sequence, channel block) column and walks it in
- * row order, so the in-place form needs no scratch memory and no ordering
- * between blocks.  Asynchronous; no allocation; CUDA-graph capturable.
+ * One thread block (or warp) owns a (sequence, channel) column and walks it
+ * in row order, so the in-place form needs no scratch memory and no ordering
+ * between blocks.  weight and bias are read before the wait for the kernel
+ * that precedes the call on the stream (programmatic dependent launch), so
+ * that kernel must not write them.  Asynchronous; no allocation; CUDA-graph
+ * capturable.
  */
 sconv_status sconv_causal_conv1d_fwd(
     void *x, int64_t x_stride_t, int64_t x_stride_c, int total_tokens, int dim,
@@ -329,7 +332,8 @@ sconv_status sconv_causal_conv1d_fwd(
  *
  *   x [batch, dim] (strides x_stride_b, x_stride_c); out has x's strides and
  *   is x itself or does not overlap it.  conv_state is required.  Other
- *   arguments and errors as in sconv_causal_conv1d_fwd.
+ *   arguments, errors and the rule on weight and bias as in
+ *   sconv_causal_conv1d_fwd.
  */
 sconv_status sconv_causal_conv1d_update(
     void *x, int64_t x_stride_b, int64_t x_stride_c, int batch, int dim,

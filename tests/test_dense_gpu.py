@@ -102,6 +102,21 @@ def test_fwd_random(seed):
                     with_states=seed % 7 != 6) == 0
 
 
+@pytest.mark.parametrize("W", [2, 3, 4, 5, 8])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_fwd_channel_major(W, dtype):
+    """Channel-major x (token stride 1): the warp-per-channel kernel over
+    sequences longer than its 4 x 128-token load window, starts that are and
+    are not multiples of the 4-token vector, every line length from W-1."""
+    rng = np.random.default_rng(40 + W)
+    lens = np.concatenate([rng.integers(0, 1200, size=5), [1, 2, 129, 512, 513]])
+    L = int(rng.integers(W - 1, 17))
+    d = workloads.dense_conv_inputs(1000 + W, dtype=dtype, dim=37, W=W, state_len=L,
+                                    lens=lens, num_pad=1, x_layout="channel_major",
+                                    state_layout="c_contig" if W % 2 else "k_contig")
+    assert _run_fwd(d, dtype, silu=W != 5, in_place=W != 3) == 0
+
+
 def test_fwd_in_place_equals_out_of_place():
     d = workloads.dense_conv_inputs(801, dtype="bf16", dim=256, W=4, state_len=3,
                                     lens=[700, 3, 0, 129])
