@@ -18,14 +18,15 @@
 //    call: the widest column that still gives the SMs 1.5 blocks each, and
 //    blocks run longest sequence first.
 //  * dense_fwd_cm -- channel-major x (token stride 1): a warp per (sequence,
-//    channel) walks the channel's contiguous tokens, four per lane, with the
-//    taps before a lane's tokens shuffled from the lanes below.
+//    channel) walks the channel's contiguous tokens, one 16-byte vector (8
+//    bf16 or 4 fp32 tokens) per lane, with the taps before a lane's tokens
+//    shuffled from the lanes below.
 //  * dense_fwd_generic -- any other layout: a thread per (sequence, channel)
 //    walks the rows with the taps in registers.
 //  * dense_update -- one token per sequence; shifted or circular line.
 //
 // Every sum runs oldest tap first, starting from the bias, in fp32 FMAs, so
-// the three kernels agree bit for bit on the same token.  A sequence whose
+// all the kernels agree bit for bit on the same token.  A sequence whose
 // line or row range is out of range is skipped and reported through the
 // optional error flag; nothing traps or waits.
 #include "common.cuh"
@@ -646,9 +647,9 @@ __global__ void __launch_bounds__(128) dense_fwd_generic(const __grid_constant__
 }
 
 
-// Decode: thread (b, j) updates channels c .. c+VEC-1 of sequence b (VEC * 2
-// or 4 bytes: many threads, little serial work each, since one decode step
-// is bound by memory latency, not bandwidth).  The block's weights are
+// Decode: thread (b, j) updates channels c .. c+VEC-1 of sequence b, 4 bytes
+// of channels (2 bf16 or 1 fp32): many threads with little serial work each,
+// since one decode step is bound by memory latency, not bandwidth.  The block's weights are
 // staged in shared memory before the wait for the preceding kernel (they
 // are constant).  Every line entry the update needs is read before the
 // first write, so the line costs one memory round trip.  Line access by
