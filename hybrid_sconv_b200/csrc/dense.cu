@@ -649,10 +649,11 @@ __global__ void __launch_bounds__(128) dense_fwd_generic(const __grid_constant__
 
 // Decode: thread (b, j) updates channels c .. c+VEC-1 of sequence b, 4 bytes
 // of channels (2 bf16 or 1 fp32): many threads with little serial work each,
-// since one decode step is bound by memory latency, not bandwidth.  The block's weights are
-// staged in shared memory before the wait for the preceding kernel (they
-// are constant).  Every line entry the update needs is read before the
-// first write, so the line costs one memory round trip.  Line access by
+// since one decode step is bound by memory latency, not bandwidth.  Each
+// thread loads its channels' weights before the wait for the preceding
+// kernel (they are constant; staging the block's weights through shared
+// memory instead cost 1.2 us per launch).  Every line entry the update needs
+// is read before the first write, so the line costs one memory round trip.  Line access by
 // layout (MODE = DenseArgs::st_mode): 0 single elements; 1 one VEC-element
 // vector per entry; 2 the block's whole run of lines (VEC*L contiguous
 // elements per thread) staged through shared memory with 16-byte copies,
@@ -669,18 +670,12 @@ __global__ void __launch_bounds__(128) dense_update(const __grid_constant__ Dens
     const bool active = c < a.dim;
     const int L = a.L, W = a.W;
 
-    // weights of the block's channels, [nch][W]
-    R *wsm = reinterpret_cast<R *>(smem16);
-    {
-        const R *wg = static_cast<const R *>(a.w);
-        for (int j = threadIdx.x; j < nch * W; j += blockDim.x) {
-            const int ch = j / W, k = j - ch * W;
-            wsm[j] = __ldg(wg + static_cast<int64_t>(c0 + ch) * a.w_sc +
-                           static_cast<int64_t>(k) * a.w_sk);
-        }
-    }
+    float wt[MAXW][VEC];
     float acc[VEC];
-    if (active) load_bias<E, VEC>(a, c, acc);
+    if (active) {
+        load_taps<E, VEC, MAXW>(a, c, wt);
+        load_bias<E, VEC>(a, c, acc);
+    }
     if (threadIdx.x == 0 && a.lines) prefetch_l2(a.lines + b);
     pdl_wait();
     pdl_trigger();
@@ -709,8 +704,8 @@ __global__ void __launch_bounds__(128) dense_update(const __grid_constant__ Dens
     const int64_t s = ring ? __ldg(a.seqlens + b) : 0;
     R *st = static_cast<R *>(a.st) + line * a.s_line + static_cast<int64_t>(c) * a.s_c;
 
-    // MODE 2: stage this block's contiguous run of lines after the weights.
-    uint4 *run16 = smem16 + (nch * W * static_cast<int>(sizeof(R)) + 15) / 16;
+    // MODE 2: stage this block's contiguous run of lines.
+    uint4 *run16 = smem16;
     R *mine = reinterpret_cast<R *>(run16) + threadIdx.x * VEC * L;
     int n16 = 0;
     uint4 *grun = nullptr;
@@ -720,7 +715,7 @@ __global__ void __launch_bounds__(128) dense_update(const __grid_constant__ Dens
                                          static_cast<int64_t>(c0) * L);
         for (int j = threadIdx.x; j < n16; j += blockDim.x) run16[j] = grun[j];
     }
-    __syncthreads();  // weights (and lines) staged
+    __syncthreads();  // the block's lines staged (MODE 2)
 
     // Entry i of the thread's VEC channels.
     auto get = [&](int64_t i, R (&e)[VEC]) {
@@ -774,16 +769,14 @@ __global__ void __launch_bounds__(128) dense_update(const __grid_constant__ Dens
                 if (i + 1 < L) get(i + 1, keep[i]);
         }
 
-        const R *wt = wsm + threadIdx.x * VEC * W;
 #pragma unroll
         for (int v = 0; v < VEC; ++v) {
 #pragma unroll
             for (int kk = 0; kk < MAXW - 1; ++kk) {
                 const int k = kk - (MAXW - W);
-                if (k >= 0)
-                    acc[v] = fmaf(raw_to_float(wt[v * W + k]), raw_to_float(tap[kk][v]), acc[v]);
+                if (k >= 0) acc[v] = fmaf(wt[kk][v], raw_to_float(tap[kk][v]), acc[v]);
             }
-            acc[v] = fmaf(raw_to_float(wt[v * W + W - 1]), raw_to_float(xr[v]), acc[v]);
+            acc[v] = fmaf(wt[MAXW - 1][v], raw_to_float(xr[v]), acc[v]);
             if (a.silu) acc[v] = silu<E>(acc[v]);
         }
 
@@ -904,7 +897,7 @@ cudaError_t launch_update_l(const DenseArgs &a, bool vec, cudaStream_t stream) {
     const int per_block = 128 * v;
     const dim3 grid(a.T, (a.dim + per_block - 1) / per_block);
     const int nch = a.dim < per_block ? a.dim : per_block;
-    size_t smem = (static_cast<size_t>(nch) * a.W * sizeof(E) + 15) / 16 * 16;
+    size_t smem = 0;
     if (!vec)
         return launch_pdl(dense_update<E, 1, MAXW, LMAX, 0>, grid, dim3(128), smem, stream, a);
     switch (a.st_mode) {
