@@ -90,18 +90,30 @@ __device__ __forceinline__ unsigned window_blocks(const PagedExtractArgs &a, int
     if (r < 0 || r >= a.num_reqs) return SCONV_EFLAG_REQUEST;
     const int64_t end = __ldg(a.abs_pos + slot);
     const int32_t *bt_row = a.bt + static_cast<int64_t>(r) * a.bt_rs;
+    // One division per slot: (lb, o) = the block and offset of the first
+    // non-negative tap position, then stepped along the window.
+    const int64_t p0 = end - d_conv;
+    int64_t lb = (p0 < 0 ? 0 : p0) / a.N;
+    int64_t o = (p0 < 0 ? 0 : p0) - lb * a.N;
+    int64_t loaded = -1;
+    int32_t b = -1;
 #pragma unroll
     for (int k = 0; k < (DC > 0 ? DC : 8); ++k) {
         blk[k] = -1;
         if (k >= d_conv) continue;
-        const int64_t p = end - d_conv + k;
-        if (p < 0) continue;
-        const int64_t lb = p / a.N;
+        if (p0 + k < 0) continue;
         if (lb >= a.max_blocks) return SCONV_EFLAG_LOGICAL;
-        const int32_t b = __ldg(bt_row + lb);
-        if (b < 0 || b >= a.num_blocks) return SCONV_EFLAG_BLOCK;
+        if (lb != loaded) {
+            b = __ldg(bt_row + lb);
+            loaded = lb;
+            if (b < 0 || b >= a.num_blocks) return SCONV_EFLAG_BLOCK;
+        }
         blk[k] = b;
-        off[k] = p - lb * a.N;
+        off[k] = o;
+        if (++o == a.N) {
+            o = 0;
+            ++lb;
+        }
     }
     return 0;
 }
