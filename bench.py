@@ -955,6 +955,9 @@ def main():
     rank, world, local = dist_setup(args)
     if args.impl == "reference":
         main_reference(args, rank, world)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
         return
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device (the sconv kernels have no CPU path)")
