@@ -4,6 +4,7 @@
 // the CUDA runtime, so a malformed call returns a status and enqueues
 // nothing.  Then it picks the 16-byte pack path when every pointer, stride
 // and lane offset allows it (else the one-element path) and launches.
+#include <limits.h>
 #include <stdint.h>
 
 #include "common.cuh"
@@ -457,6 +458,8 @@ sconv_status sconv_causal_conv1d_fwd(
     if (st != SCONV_OK) return st;
     if (batch == 0) return SCONV_OK;
     if (!query_start_loc) return SCONV_ERR_INVALID;
+    // grids: (sequence, column) blocks, or one warp per (sequence, channel)
+    if (static_cast<int64_t>(batch) * dim / 8 + 1 > INT32_MAX) return SCONV_ERR_UNSUPPORTED;
     a.qsl = query_start_loc;
     a.batch = batch;
     a.lines = cache_indices;
