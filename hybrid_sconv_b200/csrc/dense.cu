@@ -7,7 +7,7 @@
 //  * dense_fwd_tile -- varlen prefill, x token-major in 16-byte channel
 //    packs.  One 256-thread block owns a (sequence, column of PP packs) and
 //    walks it in tiles of TT = 2 * 256 / PP rows: each thread copies two
-//    packs of a tile seven tiles ahead into a shared-memory ring with
+//    packs of a tile three or five tiles ahead into a shared-memory ring with
 //    cp.async (only rows of this sequence, so nothing past its end is read)
 //    and convolves two rows of the current tile.  Each ring stage holds the
 //    W-1 rows before its tile, written while the previous tile is computed;
@@ -37,7 +37,13 @@ namespace {
 
 constexpr int kRowsPerThread = 2;  // rows of a tile each thread convolves
 constexpr int kTileThreads = 256;
-constexpr int kStages = 8;
+// Ring depth of the tiled prefill: 4 stages when the grid runs in several
+// waves of blocks (many sequences: short columns, where a deep ring only
+// fetches ahead of the end), 6 when the blocks fit in about one wave (long
+// columns that must stream at full rate).  Measured on the dense mixed and
+// long prefills: 4 stages 50.2 / 445 us, 6: 51.6 / 419, 8: 52.5 / 420.
+constexpr int kStagesFew = 4;
+constexpr int kStagesMany = 6;
 constexpr int kLptMaxBatch = 64;   // longest-first block order up to this many sequences
 constexpr int kMaxL = SCONV_MAX_STATE_LEN;
 
@@ -294,7 +300,7 @@ __device__ __forceinline__ void silu_pack(float (&acc)[VEC]) {
 // carry.  One barrier per tile: tile s reads carry[s & 1] and writes the
 // next into the other, and the stage refilled at tile s was last read at
 // tile s-1.  WT is the exact tap count (2..4), or 8 for any W up to 8.
-template <typename E, int PP, int WT, int THREADS>
+template <typename E, int PP, int WT, int THREADS, int STAGES>
 __global__ void __launch_bounds__(THREADS) dense_fwd_tile(const __grid_constant__ DenseArgs a, int ncb) {
     constexpr int VEC = 16 / sizeof(E);
     constexpr int RPT = kRowsPerThread;
@@ -302,7 +308,7 @@ __global__ void __launch_bounds__(THREADS) dense_fwd_tile(const __grid_constant_
     constexpr int HALO = WT - 1;
     constexpr int SR = HALO + TT;       // rows of one ring stage
     constexpr int NW = WT - 1 + RPT;    // window rows of one thread
-    extern __shared__ uint4 ring[];     // kStages * SR * PP packs
+    extern __shared__ uint4 ring[];     // STAGES * SR * PP packs
     __shared__ uint4 carry[2][kMaxL * PP];
     __shared__ int order[kLptMaxBatch];
 
@@ -370,19 +376,19 @@ __global__ void __launch_bounds__(THREADS) dense_fwd_tile(const __grid_constant_
             const int r = g + j * (TT / RPT);
             const int row = s * TT + r;
             if (s < ntiles && row < n && cvalid)
-                cp_async16(&ring[((s % kStages) * SR + HALO + r) * PP + p], x + row * a.x_st);
+                cp_async16(&ring[((s % STAGES) * SR + HALO + r) * PP + p], x + row * a.x_st);
         }
         cp_async_commit();
     };
 #pragma unroll
-    for (int s = 0; s < kStages - 1; ++s) issue(s);
+    for (int s = 0; s < STAGES - 1; ++s) issue(s);
 
     const int r0 = g * RPT;
     for (int s = 0; s < ntiles; ++s) {
-        cp_async_wait<kStages - 2>();
+        cp_async_wait<STAGES - 2>();
         __syncthreads();  // tile s, its halo and carry[s & 1] are complete
-        issue(s + kStages - 1);
-        const uint4 *stage = ring + (s % kStages) * SR * PP;  // row -HALO of the tile
+        issue(s + STAGES - 1);
+        const uint4 *stage = ring + (s % STAGES) * SR * PP;  // row -HALO of the tile
         const int nv = min(TT, n - s * TT);
         if (r0 < nv && cvalid) {
             // win[j] holds tile row r0 - (WT-1) + j.
@@ -410,7 +416,7 @@ __global__ void __launch_bounds__(THREADS) dense_fwd_tile(const __grid_constant_
         }
         // The next stage's halo: the last HALO rows of this (full) tile.
         if (ci < HALO && s + 1 < ntiles)
-            ring[((s + 1) % kStages) * SR * PP + ci * PP + p] = stage[(TT + ci) * PP + p];
+            ring[((s + 1) % STAGES) * SR * PP + ci * PP + p] = stage[(TT + ci) * PP + p];
         // Next carry: the last L entries of (carry, the tile's nv rows).
         if (a.st && ci < L) {
             const uint4 *cin = carry[s & 1];
@@ -834,31 +840,40 @@ int pick_pp(int batch, int packs) {
     return 1;
 }
 
-template <typename E, int PP, int WT, int THREADS>
+template <typename E, int PP, int WT, int THREADS, int STAGES>
 cudaError_t launch_tile_pp(const DenseArgs &a, int packs, cudaStream_t stream) {
     constexpr int TT = THREADS / PP * kRowsPerThread;
-    constexpr size_t kSmem = static_cast<size_t>(kStages) * (WT - 1 + TT) * PP * sizeof(uint4);
+    constexpr size_t kSmem = static_cast<size_t>(STAGES) * (WT - 1 + TT) * PP * sizeof(uint4);
     static bool configured = false;
     if (!configured) {
         const cudaError_t e = cudaFuncSetAttribute(
-            dense_fwd_tile<E, PP, WT, THREADS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-            static_cast<int>(kSmem));
+            dense_fwd_tile<E, PP, WT, THREADS, STAGES>,
+            cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
         if (e != cudaSuccess) return e;
         configured = true;
     }
     const int ncb = (packs + PP - 1) / PP;
-    return launch_pdl(dense_fwd_tile<E, PP, WT, THREADS>,
+    return launch_pdl(dense_fwd_tile<E, PP, WT, THREADS, STAGES>,
                       dim3(static_cast<unsigned>(static_cast<int64_t>(a.batch) * ncb)),
                       dim3(THREADS), kSmem, stream, a, ncb);
+}
+
+template <typename E, int PP, int WT>
+cudaError_t launch_tile_s(const DenseArgs &a, int packs, cudaStream_t stream) {
+    // Several waves: 3 resident blocks per SM is what registers allow.
+    const int64_t blocks = static_cast<int64_t>(a.batch) * ((packs + PP - 1) / PP);
+    if (blocks >= 2LL * 3 * sm_count())
+        return launch_tile_pp<E, PP, WT, kTileThreads, kStagesFew>(a, packs, stream);
+    return launch_tile_pp<E, PP, WT, kTileThreads, kStagesMany>(a, packs, stream);
 }
 
 template <typename E, int WT>
 cudaError_t launch_tile_w(const DenseArgs &a, int packs, int pp, cudaStream_t stream) {
     switch (pp) {
-        case 8: return launch_tile_pp<E, 8, WT, kTileThreads>(a, packs, stream);
-        case 4: return launch_tile_pp<E, 4, WT, kTileThreads>(a, packs, stream);
-        case 2: return launch_tile_pp<E, 2, WT, kTileThreads>(a, packs, stream);
-        default: return launch_tile_pp<E, 1, WT, kTileThreads>(a, packs, stream);
+        case 8: return launch_tile_s<E, 8, WT>(a, packs, stream);
+        case 4: return launch_tile_s<E, 4, WT>(a, packs, stream);
+        case 2: return launch_tile_s<E, 2, WT>(a, packs, stream);
+        default: return launch_tile_s<E, 1, WT>(a, packs, stream);
     }
 }
 
