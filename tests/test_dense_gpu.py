@@ -83,6 +83,17 @@ def test_fwd_tile_every_column_width(batch, dim, expect_pp, W):
     assert _run_fwd(d, "bf16", silu=W != 7) == 0
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_fwd_tile_many_sequences(dtype):
+    """More sequences than the longest-first ordering ranks (64): blocks
+    interleave the sequences instead; short and empty sequences, pads."""
+    rng = np.random.default_rng(77)
+    lens = rng.integers(0, 90, size=150)
+    d = workloads.dense_conv_inputs(77, dtype=dtype, dim=64, W=4, state_len=5, lens=lens,
+                                    num_pad=12, num_lines=200)
+    assert _run_fwd(d, dtype, silu=True) == 0
+
+
 @pytest.mark.parametrize("seed", range(16))
 def test_fwd_random(seed):
     rng = np.random.default_rng(700 + seed)
