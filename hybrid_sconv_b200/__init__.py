@@ -19,7 +19,8 @@ _EXPORTS = (
     "scatter_intermediate_ssm", "sconv_causal_conv1d_fwd", "sconv_causal_conv1d_update",
     "sconv_extract_windows",
     "sconv_extract_windows_paged", "sconv_fused", "sconv_fused_streams",
-    "sconv_scatter_intermediate_ssm", "sconv_seq_metadata", "sconv_update",
+    "sconv_scatter_intermediate_ssm", "sconv_seq_metadata", "sconv_seq_metadata_ahead",
+    "sconv_update",
 )
 
 __all__ = list(_EXPORTS)

@@ -73,6 +73,7 @@ _SIGNATURES = {
     "sconv_extract_windows": [
         _P, _I64, _INT, _I64, _I64, _P, _P, _INT, _P, _I64, _INT, _INT, _P],
     "sconv_seq_metadata": [_P, _INT, _INT, _INT, _P, _I64, _P, _I64, _P],
+    "sconv_seq_metadata_ahead": [_P, _INT, _INT, _INT, _P, _I64, _P, _I64, _P],
     "sconv_scatter_intermediate_ssm": [
         _P, _I64, _I64, _I64, _P, _P, _INT, _P, _I64, _INT, _P, _P],
     "sconv_causal_conv1d_fwd": [
@@ -398,11 +399,8 @@ def sconv_extract_windows_paged(cache, block_table, request, abs_positions, real
     return out
 
 
-def sconv_seq_metadata(query_start_loc, num_reqs, num_actual_tokens, seq_idx_out,
-                       query_start_out, num_padded_tokens=None, *, stream=None):
-    """Fill seq_idx_out / query_start_out for every token row in one launch
-    (sconv_seq_metadata, "vllm.models.inkling.nvidia.ops.sconv").  Raises
-    ValueError on the size errors the page names."""
+def _seq_metadata(name, query_start_loc, num_reqs, num_actual_tokens, seq_idx_out,
+                  query_start_out, num_padded_tokens, stream):
     if num_padded_tokens is None:
         num_padded_tokens = num_actual_tokens
     if num_padded_tokens < num_actual_tokens:
@@ -418,11 +416,31 @@ def sconv_seq_metadata(query_start_loc, num_reqs, num_actual_tokens, seq_idx_out
     _vector(seq_idx_out, torch.int32, "seq_idx_out", num_padded_tokens)
     _vector(query_start_out, torch.int32, "query_start_out", num_padded_tokens)
     with torch.cuda.device(d):
-        st = LIB.sconv_seq_metadata(
+        st = getattr(LIB, name)(
             _ptr(query_start_loc), num_reqs, num_actual_tokens, num_padded_tokens,
             _ptr(seq_idx_out), seq_idx_out.shape[0], _ptr(query_start_out),
             query_start_out.shape[0], _stream(d, stream))
-    _check("sconv_seq_metadata", st, value_error=True)
+    _check(name, st, value_error=True)
+
+
+def sconv_seq_metadata(query_start_loc, num_reqs, num_actual_tokens, seq_idx_out,
+                       query_start_out, num_padded_tokens=None, *, stream=None):
+    """Fill seq_idx_out / query_start_out for every token row in one launch
+    (sconv_seq_metadata, "vllm.models.inkling.nvidia.ops.sconv").  Raises
+    ValueError on the size errors the page names."""
+    _seq_metadata("sconv_seq_metadata", query_start_loc, num_reqs, num_actual_tokens,
+                  seq_idx_out, query_start_out, num_padded_tokens, stream)
+
+
+def sconv_seq_metadata_ahead(query_start_loc, num_reqs, num_actual_tokens, seq_idx_out,
+                             query_start_out, num_padded_tokens=None, *, stream=None):
+    """sconv_seq_metadata with the lookup done before the launch waits for
+    the kernels ahead of it on the stream (it still completes after them).
+    The caller guarantees that no kernel enqueued since the stream was last
+    fully ordered writes query_start_loc or touches the two outputs, e.g.
+    one metadata buffer set per step in flight."""
+    _seq_metadata("sconv_seq_metadata_ahead", query_start_loc, num_reqs, num_actual_tokens,
+                  seq_idx_out, query_start_out, num_padded_tokens, stream)
 
 
 def _dense_common(x, weight, bias, states, out, err_flag, states_name):

@@ -497,11 +497,11 @@ sconv_status sconv_causal_conv1d_update(
                : SCONV_ERR_LAUNCH;
 }
 
-sconv_status sconv_seq_metadata(const int32_t *query_start_loc, int num_reqs,
-                                int num_actual_tokens, int num_padded_tokens,
-                                int32_t *seq_idx_out, int64_t seq_idx_cap,
-                                int32_t *query_start_out, int64_t query_start_cap,
-                                cudaStream_t stream) {
+namespace {
+sconv_status seq_metadata(const int32_t *query_start_loc, int num_reqs, int num_actual_tokens,
+                          int num_padded_tokens, int32_t *seq_idx_out, int64_t seq_idx_cap,
+                          int32_t *query_start_out, int64_t query_start_cap, bool ahead,
+                          cudaStream_t stream) {
     if (num_padded_tokens < 0) num_padded_tokens = num_actual_tokens;
     if (num_actual_tokens < 0 || num_reqs < 0) return SCONV_ERR_INVALID;
     if (num_padded_tokens < num_actual_tokens) return SCONV_ERR_INVALID;
@@ -511,10 +511,31 @@ sconv_status sconv_seq_metadata(const int32_t *query_start_loc, int num_reqs,
     if (num_padded_tokens == 0) return SCONV_OK;
     if (!query_start_loc || !seq_idx_out || !query_start_out) return SCONV_ERR_INVALID;
     return sconv::launch_seq_metadata(query_start_loc, num_reqs, num_actual_tokens,
-                                      num_padded_tokens, seq_idx_out, query_start_out,
+                                      num_padded_tokens, seq_idx_out, query_start_out, ahead,
                                       stream) == cudaSuccess
                ? SCONV_OK
                : SCONV_ERR_LAUNCH;
+}
+}  // namespace
+
+sconv_status sconv_seq_metadata(const int32_t *query_start_loc, int num_reqs,
+                                int num_actual_tokens, int num_padded_tokens,
+                                int32_t *seq_idx_out, int64_t seq_idx_cap,
+                                int32_t *query_start_out, int64_t query_start_cap,
+                                cudaStream_t stream) {
+    return seq_metadata(query_start_loc, num_reqs, num_actual_tokens, num_padded_tokens,
+                        seq_idx_out, seq_idx_cap, query_start_out, query_start_cap, false,
+                        stream);
+}
+
+sconv_status sconv_seq_metadata_ahead(const int32_t *query_start_loc, int num_reqs,
+                                      int num_actual_tokens, int num_padded_tokens,
+                                      int32_t *seq_idx_out, int64_t seq_idx_cap,
+                                      int32_t *query_start_out, int64_t query_start_cap,
+                                      cudaStream_t stream) {
+    return seq_metadata(query_start_loc, num_reqs, num_actual_tokens, num_padded_tokens,
+                        seq_idx_out, seq_idx_cap, query_start_out, query_start_cap, true,
+                        stream);
 }
 
 }  // extern "C"

@@ -317,7 +317,8 @@ cudaError_t launch_dense_fwd(const DenseArgs &a, bool bf16_data, bool vec, cudaS
 cudaError_t launch_dense_update(const DenseArgs &a, bool bf16_data, bool vec,
                                 cudaStream_t stream);
 cudaError_t launch_seq_metadata(const int32_t *qsl, int num_reqs, int num_actual, int num_padded,
-                                int32_t *seq_idx, int32_t *query_start, cudaStream_t stream);
+                                int32_t *seq_idx, int32_t *query_start, bool ahead,
+                                cudaStream_t stream);
 
 // Launch with programmatic stream serialization enabled.
 template <typename Kernel, typename... Args>

@@ -4,7 +4,8 @@
 // One thread per token row.  The request is the last r < num_reqs with
 // query_start_loc[r] <= t, found by binary search; when the offsets table
 // is small each block first stages it in shared memory so the search's
-// dependent loads hit shared memory instead of L2.
+// dependent loads hit shared memory instead of L2.  A second entry point
+// runs the same lookup ahead of its wait on the stream.
 #include "common.cuh"
 
 namespace sconv {
@@ -13,6 +14,13 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kSmemReqs = 4096;  // stage query_start_loc when num_reqs <= this
 
+// AHEAD = false waits for the kernels before it on the stream, then works.
+// AHEAD = true works first and waits at its end: its completion, which the
+// next kernel waits for, still follows theirs, while the lookup overlaps
+// them.  It is valid only when none of the kernels that may still be running
+// writes query_start_loc or touches the two outputs (one metadata buffer set
+// per step in flight).
+template <bool AHEAD>
 __global__ void __launch_bounds__(kThreads)
 seq_metadata_kernel(const int32_t *__restrict__ qsl, int num_reqs, int num_actual,
                     int num_padded, int32_t *__restrict__ seq_idx,
@@ -23,43 +31,51 @@ seq_metadata_kernel(const int32_t *__restrict__ qsl, int num_reqs, int num_actua
     // kernel, and it gets this kernel's whole wait to prefetch.  Then pull
     // the offsets table into L2 while the preceding kernel drains.
     pdl_trigger();
-    for (int i = threadIdx.x * 32; i < num_reqs; i += blockDim.x * 32) prefetch_l2(qsl + i);
-    pdl_wait();
+    if (!AHEAD) {
+        for (int i = threadIdx.x * 32; i < num_reqs; i += blockDim.x * 32) prefetch_l2(qsl + i);
+        pdl_wait();
+    }
     if (staged) {
         for (int i = threadIdx.x; i < num_reqs; i += blockDim.x) s_qsl[i] = __ldg(qsl + i);
         __syncthreads();
     }
     const int32_t *q = staged ? s_qsl : qsl;
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
-    if (t >= num_padded) return;
-    if (t >= num_actual) {
-        seq_idx[t] = 0;
-        query_start[t] = 0;
-        return;
+    if (t < num_padded) {
+        if (t >= num_actual) {
+            seq_idx[t] = 0;
+            query_start[t] = 0;
+        } else {
+            // Invariant: the answer lies in [lo, hi]; q[lo] <= t is assumed for lo = 0.
+            int lo = 0, hi = num_reqs - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (q[mid] <= t) lo = mid;
+                else hi = mid - 1;
+            }
+            seq_idx[t] = lo;
+            query_start[t] = q[lo];
+        }
     }
-    // Invariant: the answer lies in [lo, hi]; q[lo] <= t is assumed for lo = 0.
-    int lo = 0, hi = num_reqs - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (q[mid] <= t) lo = mid;
-        else hi = mid - 1;
-    }
-    seq_idx[t] = lo;
-    query_start[t] = q[lo];
+    if (AHEAD) pdl_wait();  // every thread: the grid completes after its predecessor
 }
 
 }  // namespace
 
 cudaError_t launch_seq_metadata(const int32_t *qsl, int num_reqs, int num_actual, int num_padded,
-                                int32_t *seq_idx, int32_t *query_start, cudaStream_t stream) {
+                                int32_t *seq_idx, int32_t *query_start, bool ahead,
+                                cudaStream_t stream) {
     // With no actual tokens the search never runs; one entry keeps the
     // staging loop and the search bounds well defined.
     const int nr = num_reqs > 0 ? num_reqs : 1;
     const int staged = nr <= kSmemReqs ? 1 : 0;
     const size_t smem = staged ? static_cast<size_t>(nr) * sizeof(int32_t) : 0;
     const int blocks = (num_padded + kThreads - 1) / kThreads;
-    return launch_pdl(seq_metadata_kernel, dim3(blocks), dim3(kThreads), smem, stream, qsl, nr,
-                      num_actual, num_padded, seq_idx, query_start, staged);
+    if (ahead)
+        return launch_pdl(seq_metadata_kernel<true>, dim3(blocks), dim3(kThreads), smem, stream,
+                          qsl, nr, num_actual, num_padded, seq_idx, query_start, staged);
+    return launch_pdl(seq_metadata_kernel<false>, dim3(blocks), dim3(kThreads), smem, stream, qsl,
+                      nr, num_actual, num_padded, seq_idx, query_start, staged);
 }
 
 }  // namespace sconv

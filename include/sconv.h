@@ -365,6 +365,30 @@ sconv_status sconv_seq_metadata(
     int num_padded_tokens, int32_t *seq_idx_out, int64_t seq_idx_cap,
     int32_t *query_start_out, int64_t query_start_cap, cudaStream_t stream);
 
+/*
+ * sconv_seq_metadata_ahead -- sconv_seq_metadata (same arguments, results
+ * and errors) with its work moved ahead of its wait on the stream.
+ *
+ *   Every launch of this library may start while the kernel before it on
+ *   the stream still runs (programmatic dependent launch) and waits for
+ *   that kernel's completion before it touches data.  This one reads
+ *   query_start_loc and writes both outputs BEFORE that wait and waits
+ *   only at its end: it still completes after everything before it on the
+ *   stream, so the kernels after it see the usual order, and the lookup
+ *   leaves the critical path of back-to-back decode steps.
+ *
+ *   Precondition (the caller's; nothing checks it): no kernel enqueued
+ *   before this call since the stream was last fully ordered (a host
+ *   synchronisation, the start of a graph replay) writes query_start_loc or
+ *   reads or writes seq_idx_out or query_start_out.  A serving loop meets it
+ *   with one metadata buffer set per step in flight, written only by that
+ *   step's own call.  Otherwise use sconv_seq_metadata.
+ */
+sconv_status sconv_seq_metadata_ahead(
+    const int32_t *query_start_loc, int num_reqs, int num_actual_tokens,
+    int num_padded_tokens, int32_t *seq_idx_out, int64_t seq_idx_cap,
+    int32_t *query_start_out, int64_t query_start_cap, cudaStream_t stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *sconv_status_string(sconv_status status);
 

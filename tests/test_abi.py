@@ -112,9 +112,10 @@ def test_extract_host_validation(lib):
     assert call(rc=0) == 1
 
 
-def test_seq_metadata_host_validation(lib):
+@pytest.mark.parametrize("name", ["sconv_seq_metadata", "sconv_seq_metadata_ahead"])
+def test_seq_metadata_host_validation(lib, name):
     def call(R=3, na=7, npad=10, cap_s=10, cap_q=10):
-        return lib.sconv_seq_metadata(FAKE, R, na, npad, FAKE * 2, cap_s, FAKE * 3, cap_q, 0)
+        return getattr(lib, name)(FAKE, R, na, npad, FAKE * 2, cap_s, FAKE * 3, cap_q, 0)
     assert call(na=0, npad=0) == 0
     assert call(npad=5) == 1           # fewer padded than actual
     assert call(cap_s=9) == 1

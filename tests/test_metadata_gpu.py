@@ -1,5 +1,6 @@
-"""GPU parity of sconv_seq_metadata against the CPU oracle (bit-exact)
-("vllm.models.inkling.nvidia.ops.sconv", sconv_seq_metadata)."""
+"""GPU parity of sconv_seq_metadata and sconv_seq_metadata_ahead against
+the CPU oracle (bit-exact) ("vllm.models.inkling.nvidia.ops.sconv",
+sconv_seq_metadata)."""
 from __future__ import annotations
 
 import numpy as np
@@ -16,14 +17,15 @@ DEV = "cuda"
 def _run(qsl_np, R, n_actual, n_padded, cap=None):
     cap = cap or n_padded
     qsl = torch.from_numpy(qsl_np).to(DEV)
-    si = torch.full((cap,), -7, dtype=torch.int32, device=DEV)
-    qs = torch.full((cap,), -7, dtype=torch.int32, device=DEV)
-    hs().sconv_seq_metadata(qsl, R, n_actual, si, qs, n_padded)
-    torch.cuda.synchronize()
     rsi, rqs = oracle.seq_metadata(qsl_np, R, n_actual, n_padded)
-    np.testing.assert_array_equal(si.cpu().numpy()[:n_padded], rsi)
-    np.testing.assert_array_equal(qs.cpu().numpy()[:n_padded], rqs)
-    assert bool((si[n_padded:] == -7).all() and (qs[n_padded:] == -7).all())
+    for name in ("sconv_seq_metadata", "sconv_seq_metadata_ahead"):
+        si = torch.full((cap,), -7, dtype=torch.int32, device=DEV)
+        qs = torch.full((cap,), -7, dtype=torch.int32, device=DEV)
+        getattr(hs(), name)(qsl, R, n_actual, si, qs, n_padded)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(si.cpu().numpy()[:n_padded], rsi, err_msg=name)
+        np.testing.assert_array_equal(qs.cpu().numpy()[:n_padded], rqs, err_msg=name)
+        assert bool((si[n_padded:] == -7).all() and (qs[n_padded:] == -7).all()), name
 
 
 def _qsl(rng, R, max_len, empty_frac=0.2):

@@ -6,7 +6,9 @@ Pipelining builds step i+1's metadata (sconv_seq_metadata,
 sconv_fused runs; the convolutions keep their order, since step i+1 reads
 as history what step i inserted.  Several batches share one paged cache
 here, so any reordering of the convolutions or a metadata buffer read
-before it is complete would change the bits.
+before it is complete would change the bits.  Each case also runs with
+sconv_seq_metadata_ahead, whose lookup runs before its wait on the stream
+and whose completion must still follow the previous convolution's.
 """
 from __future__ import annotations
 
@@ -31,8 +33,9 @@ def _reset(sets_obj, cache0):
         s["query_start"].fill_(-7)
 
 
+@pytest.mark.parametrize("ahead", [False, True])
 @pytest.mark.parametrize("n", [1, 2, 6])
-def test_pipelined_steps_equal_plain_steps(n):
+def test_pipelined_steps_equal_plain_steps(n, ahead):
     dev = torch.device("cuda", 0)
     sets_obj = bench.DecodeSets(n, 5151, dev, max_hist=64)
     cache0 = raw(sets_obj.cache).clone()
@@ -40,8 +43,19 @@ def test_pipelined_steps_equal_plain_steps(n):
     _reset(sets_obj, cache0)
     for i in range(n):
         sets_obj.step(i)
-    torch.cuda.synchronize()
+        torch.cuda.synchronize()  # fully ordered reference
     plain_cache, plain_outs = _snapshot(sets_obj)
+
+    # back to back on one stream, with the chosen metadata builder
+    sets_obj.ahead = ahead
+    _reset(sets_obj, cache0)
+    for i in range(n):
+        sets_obj.step(i)
+    torch.cuda.synchronize()
+    cache, outs = _snapshot(sets_obj)
+    assert torch.equal(cache, plain_cache)
+    for a, b in zip(outs, plain_outs):
+        assert torch.equal(a, b)
 
     side = torch.cuda.Stream(dev)
     _reset(sets_obj, cache0)
