@@ -13,10 +13,15 @@
 // all completing on one mbarrier.  Tiles flow through a ring of STAGES
 // shared-memory stages, so up to STAGES-1 tiles are in flight while one is
 // computed: the memory system sees a steady stream of bulk copies whatever
-// the register budget of the compute threads.  The grid is persistent: one
-// block per resident slot (SMs x blocks per SM), each taking an equal
-// contiguous share of the (channel block, tile) units, so there is no
-// partial last wave.
+// the register budget of the compute threads.  The grid is persistent: G
+// blocks per channel block, G x (channel blocks) <= the resident slots
+// (SMs x blocks per SM).  Block b keeps channel block b % ncb (its weights
+// stay in registers) and takes the token tiles g, g + G, g + 2G, ... with
+// g = b / ncb, so at any moment the grid works on about G consecutive token
+// tiles across every channel block: a compact band of x, out and the cache
+// rather than one scattered spot per block, which DRAM serves measurably
+// faster (chunked prefill 82.2 -> 77.3 us, long prefill 611 -> 584 us,
+// against equal contiguous shares of the (channel block, tile) units).
 //
 // Compute.  Eight warps per block; warp g owns tokens 4g..4g+3 of the tile
 // and lane l the 16-byte pack of channels c0 + 8l .. c0 + 8l + 7.  Lanes
@@ -180,19 +185,19 @@ enum : int { kSkip = 0, kFast = 1, kSlow = 2 };
 
 template <int W, int STAGES, bool SILU, bool RESID>
 __global__ void __launch_bounds__(kThreads, STAGES <= 3 ? 3 : 2)
-fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ TmaMaps maps,
-                 int64_t units) {
+fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ TmaMaps maps) {
     using L = Layout<W>;
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * L::stage);
     uint64_t *empty = full + STAGES;
 
-    // Work units are (channel block, tile) pairs, channel-block major; this
-    // block takes an equal contiguous share of them.
+    // This block's channel block and its token tiles g, g + G, ...
     const int ntiles = (a.T + kBT - 1) / kBT;
-    const int64_t u_begin = units * blockIdx.x / gridDim.x;
-    const int64_t u_end = units * (blockIdx.x + 1) / gridDim.x;
-    const int my = static_cast<int>(u_end - u_begin);
+    const int ncb = (a.C + kBC - 1) / kBC;
+    const int G = static_cast<int>(gridDim.x) / ncb;  // blocks per channel block
+    const int cb = static_cast<int>(blockIdx.x) % ncb;
+    const int g = static_cast<int>(blockIdx.x) / ncb;
+    const int my = g < ntiles ? (ntiles - g + G - 1) / G : 0;
     if (my <= 0) return;  // whole block
 
     if (threadIdx.x == 0) {
@@ -212,9 +217,8 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
         ++issued;
         const int s = k % STAGES;
         unsigned char *st = smem + s * L::stage;
-        const int64_t u = u_begin + k;
-        const int c0 = static_cast<int>(u / ntiles) * kBC;
-        const int t0 = static_cast<int>(u % ntiles) * kBT;
+        const int c0 = cb * kBC;
+        const int t0 = (g + k * G) * kBT;
         mbar_expect_tx(&full[s], L::stage);
         tma_2d(st, &maps.x, c0, t0 - (W - 1), &full[s]);
         tma_1d(st + L::x_bytes, &maps.pos, t0, &full[s]);
@@ -229,29 +233,21 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
     const int i0 = (threadIdx.x >> 5) * kTokPerWarp;
     const int nv = a.C / 8;
     const int64_t slots_total = a.num_blocks * a.N;
-    int cur_cb = -1;
-    bool active = false;
-    int c = 0;
-    int64_t lane = 0;
+    // This lane's channel pack: its taps and its cache lanes.
+    const int pack_raw = cb * (kBC / 8) + lane_id;
+    const bool active = pack_raw < nv;
+    const int c = (active ? pack_raw : nv - 1) * 8;
+    const int h = c / a.ws;
+    const int64_t lane = static_cast<int64_t>(h) * a.cs1 + a.off_s + (c - h * a.ws);
     uint32_t wr[4][4];
+    load_weights_bf16<W>(a, c, wr);
     bool alive = true;
     int next = 0;  // the next tile this thread waits for
 
     for (int k = 0; k < my; ++k) {
         next = k;
         const int s = k % STAGES;
-        const int64_t u = u_begin + k;
-        const int cb = static_cast<int>(u / ntiles);
-        const int t0 = static_cast<int>(u % ntiles) * kBT;
-        if (cb != cur_cb) {  // entering a new channel block: its taps and cache lanes
-            cur_cb = cb;
-            const int pack_raw = cb * (kBC / 8) + lane_id;
-            active = pack_raw < nv;
-            c = (active ? pack_raw : nv - 1) * 8;
-            const int h = c / a.ws;
-            lane = static_cast<int64_t>(h) * a.cs1 + a.off_s + (c - h * a.ws);
-            load_weights_bf16<W>(a, c, wr);
-        }
+        const int t0 = (g + k * G) * kBT;
         if (!mbar_wait(&full[s], (k / STAGES) & 1)) {  // copies did not arrive in time
             if (a.err && lane_id == 0) atomicOr(a.err, static_cast<int>(SCONV_EFLAG_TIMEOUT));
             alive = false;
@@ -455,12 +451,15 @@ cudaError_t launch_flags(const FusedArgs &a, const TmaMaps &maps, cudaStream_t s
             per_sm = 1;
     });
     if (attr != cudaSuccess) return attr;
+    // G blocks per channel block, as many as the resident slots allow (at
+    // least one, at most one per token tile).
     const int64_t ntiles = (a.T + kBT - 1) / kBT;
-    const int64_t units = ntiles * ((a.C + kBC - 1) / kBC);
-    int64_t grid = static_cast<int64_t>(sms) * per_sm;
-    if (grid > units) grid = units;
-    return launch_pdl(kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem, stream, a,
-                      maps, units);
+    const int64_t ncb = (a.C + kBC - 1) / kBC;
+    int64_t G = static_cast<int64_t>(sms) * per_sm / ncb;
+    if (G < 1) G = 1;
+    if (G > ntiles) G = ntiles;
+    return launch_pdl(kernel, dim3(static_cast<unsigned>(G * ncb)), dim3(kThreads), smem, stream,
+                      a, maps);
 }
 
 template <int W>
