@@ -13,15 +13,17 @@
 // all completing on one mbarrier.  Tiles flow through a ring of STAGES
 // shared-memory stages, so up to STAGES-1 tiles are in flight while one is
 // computed: the memory system sees a steady stream of bulk copies whatever
-// the register budget of the compute threads.  The grid is persistent: G
-// blocks per channel block, G x (channel blocks) <= the resident slots
-// (SMs x blocks per SM).  Block b keeps channel block b % ncb (its weights
-// stay in registers) and takes the token tiles g, g + G, g + 2G, ... with
-// g = b / ncb, so at any moment the grid works on about G consecutive token
-// tiles across every channel block: a compact band of x, out and the cache
-// rather than one scattered spot per block, which DRAM serves measurably
-// faster (chunked prefill 82.2 -> 77.3 us, long prefill 611 -> 584 us,
-// against equal contiguous shares of the (channel block, tile) units).
+// the register budget of the compute threads.  The grid is persistent, one
+// block per resident slot (SMs x blocks per SM).  Work units are (token
+// tile, channel block) pairs numbered token-tile major, u = tile * ncb + cb,
+// and block b takes u = b, b + grid, b + 2 grid, ...: at any moment the grid
+// works on one contiguous run of units, a compact band of x, out and the
+// cache rows, and every block ends within one unit of the others.  DRAM
+// serves that band far faster than one scattered spot per block (chunked
+// prefill 82.2 -> 72.3 us, long prefill 611 -> 530 us, against equal
+// contiguous shares of the units in channel-block-major order).  A block's
+// channel block changes from unit to unit; it reloads its weights (a few
+// lines, L1-resident) only when it does.
 //
 // Compute.  Eight warps per block; warp g owns tokens 4g..4g+3 of the tile
 // and lane l the 16-byte pack of channels c0 + 8l .. c0 + 8l + 7.  Lanes
@@ -192,12 +194,13 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
     uint64_t *empty = full + STAGES;
 
     // This block's channel block and its token tiles g, g + G, ...
+    // This block's units: u = b0, b0 + gstride, ... below ntiles * ncb.
     const int ntiles = (a.T + kBT - 1) / kBT;
     const int ncb = (a.C + kBC - 1) / kBC;
-    const int G = static_cast<int>(gridDim.x) / ncb;  // blocks per channel block
-    const int cb = static_cast<int>(blockIdx.x) % ncb;
-    const int g = static_cast<int>(blockIdx.x) / ncb;
-    const int my = g < ntiles ? (ntiles - g + G - 1) / G : 0;
+    const int64_t units = static_cast<int64_t>(ntiles) * ncb;
+    const int64_t gstride = gridDim.x;
+    const int64_t b0 = blockIdx.x;
+    const int my = b0 < units ? static_cast<int>((units - 1 - b0) / gstride + 1) : 0;
     if (my <= 0) return;  // whole block
 
     if (threadIdx.x == 0) {
@@ -217,8 +220,9 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
         ++issued;
         const int s = k % STAGES;
         unsigned char *st = smem + s * L::stage;
-        const int c0 = cb * kBC;
-        const int t0 = (g + k * G) * kBT;
+        const int64_t u = b0 + k * gstride;
+        const int c0 = static_cast<int>(u % ncb) * kBC;
+        const int t0 = static_cast<int>(u / ncb) * kBT;
         mbar_expect_tx(&full[s], L::stage);
         tma_2d(st, &maps.x, c0, t0 - (W - 1), &full[s]);
         tma_1d(st + L::x_bytes, &maps.pos, t0, &full[s]);
@@ -233,21 +237,29 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
     const int i0 = (threadIdx.x >> 5) * kTokPerWarp;
     const int nv = a.C / 8;
     const int64_t slots_total = a.num_blocks * a.N;
-    // This lane's channel pack: its taps and its cache lanes.
-    const int pack_raw = cb * (kBC / 8) + lane_id;
-    const bool active = pack_raw < nv;
-    const int c = (active ? pack_raw : nv - 1) * 8;
-    const int h = c / a.ws;
-    const int64_t lane = static_cast<int64_t>(h) * a.cs1 + a.off_s + (c - h * a.ws);
+    int cur_cb = -1;
+    bool active = false;
+    int c = 0;
+    int64_t lane = 0;
     uint32_t wr[4][4];
-    load_weights_bf16<W>(a, c, wr);
     bool alive = true;
     int next = 0;  // the next tile this thread waits for
 
     for (int k = 0; k < my; ++k) {
         next = k;
         const int s = k % STAGES;
-        const int t0 = (g + k * G) * kBT;
+        const int64_t u = b0 + k * gstride;
+        const int cb = static_cast<int>(u % ncb);
+        const int t0 = static_cast<int>(u / ncb) * kBT;
+        if (cb != cur_cb) {  // a new channel block: its taps and cache lanes
+            cur_cb = cb;
+            const int pack_raw = cb * (kBC / 8) + lane_id;
+            active = pack_raw < nv;
+            c = (active ? pack_raw : nv - 1) * 8;
+            const int h = c / a.ws;
+            lane = static_cast<int64_t>(h) * a.cs1 + a.off_s + (c - h * a.ws);
+            load_weights_bf16<W>(a, c, wr);
+        }
         if (!mbar_wait(&full[s], (k / STAGES) & 1)) {  // copies did not arrive in time
             if (a.err && lane_id == 0) atomicOr(a.err, static_cast<int>(SCONV_EFLAG_TIMEOUT));
             alive = false;
@@ -451,14 +463,12 @@ cudaError_t launch_flags(const FusedArgs &a, const TmaMaps &maps, cudaStream_t s
             per_sm = 1;
     });
     if (attr != cudaSuccess) return attr;
-    // G blocks per channel block, as many as the resident slots allow (at
-    // least one, at most one per token tile).
+    // One block per resident slot, at most one per unit.
     const int64_t ntiles = (a.T + kBT - 1) / kBT;
     const int64_t ncb = (a.C + kBC - 1) / kBC;
-    int64_t G = static_cast<int64_t>(sms) * per_sm / ncb;
-    if (G < 1) G = 1;
-    if (G > ntiles) G = ntiles;
-    return launch_pdl(kernel, dim3(static_cast<unsigned>(G * ncb)), dim3(kThreads), smem, stream,
+    int64_t grid = static_cast<int64_t>(sms) * per_sm;
+    if (grid > ntiles * ncb) grid = ntiles * ncb;
+    return launch_pdl(kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem, stream,
                       a, maps);
 }
 
