@@ -395,9 +395,9 @@ cudaError_t launch_w(FusedArgs &a, bool one, cudaStream_t stream) {
                     : launch_pdl(fused_token_kernel<E, VEC, MAXW, false, false>, grid,
                                  dim3(s.cv, s.tg), 0, stream, a);
     }
-    if constexpr (sizeof(E) == 2 && VEC == 8) {
+    if constexpr (VEC * sizeof(E) == 16) {
         bool used = false;
-        const cudaError_t e = launch_fused_tma(a, stream, used);
+        const cudaError_t e = launch_fused_tma(a, sizeof(E) == 2, stream, used);
         if (used || e != cudaSuccess) return e;
     }
     // Strip length: a whole number of 32-token metadata chunks, the longest

@@ -3,8 +3,9 @@
 // and per-token metadata staged in shared memory by the Tensor Memory
 // Accelerator, for sm_100a.
 //
-// Tiling.  A tile is kBT = 32 consecutive tokens x kBC = 256 channels
-// (512 bytes of bf16 per row).  One thread of each block issues, per tile,
+// Tiling.  A tile is kBT = 32 consecutive tokens x 512 bytes of a row (256
+// bf16 or 128 fp32 channels, kBC<E>).  One thread of each block issues, per
+// tile,
 //   * a 2-D tensor copy of x rows [t0 - (W-1), t0 + 32) x [c0, c0 + 256)
 //     (the W-1 halo rows before the tile included; rows before 0 and past T
 //     and channels past C arrive as zeros), and
@@ -26,7 +27,8 @@
 // lines, L1-resident) only when it does.
 //
 // Compute.  Eight warps per block; warp g owns tokens 4g..4g+3 of the tile
-// and lane l the 16-byte pack of channels c0 + 8l .. c0 + 8l + 7.  Lanes
+// and lane l the 16-byte pack l of the tile's row (8 bf16 or 4 fp32
+// channels).  W, the tap count 1..8, is a template parameter.  Lanes
 // 0..3 classify the warp's four tokens (ordinary, PAD, or needing cache
 // taps / out of range) and compute their cache insert offsets once; when all
 // four are ordinary -- nearly always in prefill -- one straight-line block
@@ -52,7 +54,8 @@
 namespace sconv {
 namespace {
 
-constexpr int kBC = 256;           // channels per tile
+template <typename E>
+constexpr int kBC = 512 / static_cast<int>(sizeof(E));  // channels per tile
 constexpr int kBT = 32;            // tokens per tile
 constexpr int kThreads = 256;      // 8 warps
 constexpr int kTokPerWarp = kBT / (kThreads / 32);  // 4
@@ -62,7 +65,7 @@ constexpr uint32_t kWaitSpins = 1u << 22;  // bounded mbarrier polls (seconds, n
 template <int W>
 struct Layout {
     static constexpr int rows = kBT + W - 1;
-    static constexpr int x_bytes = rows * kBC * 2;  // multiple of 512: TMA destinations stay 128-B aligned
+    static constexpr int x_bytes = rows * 512;  // multiple of 512: TMA destinations stay 128-B aligned
     static constexpr int stage = x_bytes + kMetaBytes;
 };
 
@@ -70,6 +73,17 @@ template <int W, int STAGES>
 constexpr int kStages_smem() {
     return STAGES * Layout<W>::stage + 2 * STAGES * 8;
 }
+
+// Shared memory for cached weights: room for ncache * W 512-byte lag rows
+// that still leaves two blocks per SM at every W.  Reloading (and, for bf16,
+// re-pairing) the weights at each channel-block switch is cheap up to W = 4
+// (bf16) or 5 (fp32) and costs more than the shared-memory copy beyond (A/B
+// on the chunked prefill shape, us: bf16 W 4 / 5 / 6 / 8: reload 72.4 /
+// 96.1 / 139.0 / 123.4, cached 76.0 / 75.9 / 82.0 / 93.0; fp32 W 4 / 6 / 8:
+// reload 149.2 / 185.5 / 211.3, cached 153.6 / 148.6 / 155.5).
+constexpr int kWeightCacheBytes = 24 * 1024;
+template <typename E, int W>
+constexpr bool kCachesWeights = W > (sizeof(E) == 2 ? 4 : 5);
 
 struct TmaMaps {
     CUtensorMap x, pos, slot, sid, qs;
@@ -125,13 +139,15 @@ __device__ __forceinline__ void tma_1d(void *dst, const CUtensorMap *map, int x,
         : "memory");
 }
 
-using P = Pack<bf16, 8>;
+template <typename E>
+using PackOf = Pack<E, 16 / sizeof(E)>;
 
 // acc += w * tap for one 8-channel pack: eight fp32-accumulating FMAs that
 // take bf16 operands directly (the product of two bf16 values is exact in
 // fp32, so this equals widening both and one fmaf, bit for bit).  w holds
 // the pack's weights for one lag as four bf16 pairs.
-__device__ __forceinline__ void fma_pack(float (&acc)[8], const uint32_t (&w)[4], const P &tap) {
+__device__ __forceinline__ void fma_pack(float (&acc)[8], const uint32_t (&w)[4],
+                                         const Pack<bf16, 8> &tap) {
     const uint32_t q[4] = {tap.u.x, tap.u.y, tap.u.z, tap.u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -144,59 +160,145 @@ __device__ __forceinline__ void fma_pack(float (&acc)[8], const uint32_t (&w)[4]
             : "r"(w[i]), "r"(q[i]));
 }
 
-// The pack's weights as bf16 pairs by lag (wb[d] multiplies position
-// pos - d, weight column W-1-d); lags >= W are zero.
+// The pack's weights by lag (lag d multiplies position pos - d, weight
+// column W-1-d).  With a dense [C, W] weight the pack's VEC*W elements are
+// contiguous and 16-byte aligned: W vector loads.
+template <typename E, int W>
+struct LagWeights;
+
 template <int W>
-__device__ __forceinline__ void load_weights_bf16(const FusedArgs &a, int c, uint32_t (&wb)[4][4]) {
-    const unsigned short *w = static_cast<const unsigned short *>(a.w);
-    unsigned short e[8][4];
-    if (a.w_vec) {  // dense [C, 4]: 32 contiguous elements
-        union {
-            uint4 u[4];
-            unsigned short h[32];
-        } raw;
-        const uint4 *p = reinterpret_cast<const uint4 *>(w + static_cast<int64_t>(c) * 4);
+struct LagWeights<bf16, W> {
+    uint32_t w[W][4];  // bf16 pairs, channel 2i in the low half
+    __device__ __forceinline__ void load(const FusedArgs &a, int c) {
+        const unsigned short *wp = static_cast<const unsigned short *>(a.w);
+        unsigned short e[8][W];
+        if (a.w_vec) {
+            union {
+                uint4 u[W];
+                unsigned short h[8 * W];
+            } raw;
+            const uint4 *p = reinterpret_cast<const uint4 *>(wp + static_cast<int64_t>(c) * W);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) raw.u[q] = __ldg(p + q);
+            for (int q = 0; q < W; ++q) raw.u[q] = __ldg(p + q);
 #pragma unroll
-        for (int v = 0; v < 8; ++v)
+            for (int v = 0; v < 8; ++v)
 #pragma unroll
-            for (int d = 0; d < 4; ++d) e[v][d] = raw.h[v * 4 + 3 - d];
-    } else {
+                for (int d = 0; d < W; ++d) e[v][d] = raw.h[v * W + W - 1 - d];
+        } else {
 #pragma unroll
-        for (int v = 0; v < 8; ++v)
+            for (int v = 0; v < 8; ++v)
 #pragma unroll
-            for (int d = 0; d < 4; ++d)
-                e[v][d] = d < W ? __ldg(w + static_cast<int64_t>(c + v) * a.w_sc +
-                                        static_cast<int64_t>(W - 1 - d) * a.w_sk)
-                                : static_cast<unsigned short>(0);
+                for (int d = 0; d < W; ++d)
+                    e[v][d] = __ldg(wp + static_cast<int64_t>(c + v) * a.w_sc +
+                                    static_cast<int64_t>(W - 1 - d) * a.w_sk);
+        }
+#pragma unroll
+        for (int d = 0; d < W; ++d)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                w[d][i] = static_cast<uint32_t>(e[2 * i][d]) |
+                          (static_cast<uint32_t>(e[2 * i + 1][d]) << 16);
     }
+    __device__ __forceinline__ void fma(float (&acc)[8], int d, const Pack<bf16, 8> &tap) const {
+        fma_pack(acc, w[d], tap);
+    }
+    // Lag d of this lane at wc[d * 32 + lane]: conflict-free 16-byte accesses.
+    __device__ __forceinline__ void to_smem(uint4 *wc, int lane) const {
 #pragma unroll
-    for (int d = 0; d < 4; ++d)
+        for (int d = 0; d < W; ++d) wc[d * 32 + lane] = make_uint4(w[d][0], w[d][1], w[d][2], w[d][3]);
+    }
+    __device__ __forceinline__ void from_smem(const uint4 *wc, int lane) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            wb[d][i] = static_cast<uint32_t>(e[2 * i][d]) | (static_cast<uint32_t>(e[2 * i + 1][d]) << 16);
-}
+        for (int d = 0; d < W; ++d) {
+            const uint4 q = wc[d * 32 + lane];
+            w[d][0] = q.x;
+            w[d][1] = q.y;
+            w[d][2] = q.z;
+            w[d][3] = q.w;
+        }
+    }
+};
+
+template <int W>
+struct LagWeights<float, W> {
+    float w[W][4];
+    __device__ __forceinline__ void load(const FusedArgs &a, int c) {
+        const float *wp = static_cast<const float *>(a.w);
+        if (a.w_vec) {
+            union {
+                uint4 u[W];
+                float f[4 * W];
+            } raw;
+            const uint4 *p = reinterpret_cast<const uint4 *>(wp + static_cast<int64_t>(c) * W);
+#pragma unroll
+            for (int q = 0; q < W; ++q) raw.u[q] = __ldg(p + q);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+#pragma unroll
+                for (int d = 0; d < W; ++d) w[d][v] = raw.f[v * W + W - 1 - d];
+        } else {
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+#pragma unroll
+                for (int d = 0; d < W; ++d)
+                    w[d][v] = __ldg(wp + static_cast<int64_t>(c + v) * a.w_sc +
+                                    static_cast<int64_t>(W - 1 - d) * a.w_sk);
+        }
+    }
+    __device__ __forceinline__ void fma(float (&acc)[4], int d, const Pack<float, 4> &tap) const {
+        float t[4];
+        tap.to_float(t);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[v] = fmaf(w[d][v], t[v], acc[v]);
+    }
+    __device__ __forceinline__ void to_smem(uint4 *wc, int lane) const {
+#pragma unroll
+        for (int d = 0; d < W; ++d)
+            wc[d * 32 + lane] = make_uint4(__float_as_uint(w[d][0]), __float_as_uint(w[d][1]),
+                                           __float_as_uint(w[d][2]), __float_as_uint(w[d][3]));
+    }
+    __device__ __forceinline__ void from_smem(const uint4 *wc, int lane) {
+#pragma unroll
+        for (int d = 0; d < W; ++d) {
+            const uint4 q = wc[d * 32 + lane];
+            w[d][0] = __uint_as_float(q.x);
+            w[d][1] = __uint_as_float(q.y);
+            w[d][2] = __uint_as_float(q.z);
+            w[d][3] = __uint_as_float(q.w);
+        }
+    }
+};
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+// The pack lane l works on in channel block cb (clamped to the last pack
+// for lanes past C, which compute but store nothing).
+__device__ __forceinline__ int cb_pack(int cb, int l, int nv) {
+    const int p = cb * 32 + l;
+    return p < nv ? p : nv - 1;
+}
+
 // What a warp's lane u (< kTokPerWarp) knows about token u of its group.
 enum : int { kSkip = 0, kFast = 1, kSlow = 2 };
 
-template <int W, int STAGES, bool SILU, bool RESID>
+template <typename E, int W, int STAGES, bool SILU, bool RESID>
 __global__ void __launch_bounds__(kThreads, STAGES <= 3 ? 3 : 2)
-fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ TmaMaps maps) {
+fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ TmaMaps maps,
+                 int ncache) {
     using L = Layout<W>;
+    using P = PackOf<E>;
+    constexpr int VEC = 16 / static_cast<int>(sizeof(E));
+    constexpr int BC = kBC<E>;
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * L::stage);
     uint64_t *empty = full + STAGES;
+    uint4 *wcache = reinterpret_cast<uint4 *>(empty + STAGES);  // ncache x W x 32 lanes
 
-    // This block's channel block and its token tiles g, g + G, ...
     // This block's units: u = b0, b0 + gstride, ... below ntiles * ncb.
     const int ntiles = (a.T + kBT - 1) / kBT;
-    const int ncb = (a.C + kBC - 1) / kBC;
+    const int ncb = (a.C + BC - 1) / BC;
     const int64_t units = static_cast<int64_t>(ntiles) * ncb;
     const int64_t gstride = gridDim.x;
     const int64_t b0 = blockIdx.x;
@@ -221,7 +323,7 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
         const int s = k % STAGES;
         unsigned char *st = smem + s * L::stage;
         const int64_t u = b0 + k * gstride;
-        const int c0 = static_cast<int>(u % ncb) * kBC;
+        const int c0 = static_cast<int>(u % ncb) * BC;
         const int t0 = static_cast<int>(u / ncb) * kBT;
         mbar_expect_tx(&full[s], L::stage);
         tma_2d(st, &maps.x, c0, t0 - (W - 1), &full[s]);
@@ -234,14 +336,28 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
         for (int k = 0; k < STAGES && k < my; ++k) issue(k);
 
     const int lane_id = threadIdx.x & 31;
+    // A block's channel block repeats with period ncache (ncache * gstride
+    // is a multiple of ncb); when the host found room, the weights of those
+    // channel blocks are unpacked once into shared memory, so a switch costs
+    // W shared-memory loads instead of W global loads and the unpacking.
+    if (kCachesWeights<E, W> && ncache > 0) {
+        for (int j = threadIdx.x >> 5; j < ncache; j += kThreads / 32) {
+            const int cbj = static_cast<int>((b0 + j * gstride) % ncb);
+            const int pj = cb_pack(cbj, lane_id, a.C / VEC);
+            LagWeights<E, W> t;
+            t.load(a, pj * VEC);
+            t.to_smem(wcache + j * W * 32, lane_id);
+        }
+        __syncthreads();
+    }
     const int i0 = (threadIdx.x >> 5) * kTokPerWarp;
-    const int nv = a.C / 8;
+    const int nv = a.C / VEC;
     const int64_t slots_total = a.num_blocks * a.N;
     int cur_cb = -1;
     bool active = false;
     int c = 0;
     int64_t lane = 0;
-    uint32_t wr[4][4];
+    LagWeights<E, W> wr;
     bool alive = true;
     int next = 0;  // the next tile this thread waits for
 
@@ -253,12 +369,14 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
         const int t0 = static_cast<int>(u / ncb) * kBT;
         if (cb != cur_cb) {  // a new channel block: its taps and cache lanes
             cur_cb = cb;
-            const int pack_raw = cb * (kBC / 8) + lane_id;
-            active = pack_raw < nv;
-            c = (active ? pack_raw : nv - 1) * 8;
+            active = cb * 32 + lane_id < nv;
+            c = cb_pack(cb, lane_id, nv) * VEC;
             const int h = c / a.ws;
             lane = static_cast<int64_t>(h) * a.cs1 + a.off_s + (c - h * a.ws);
-            load_weights_bf16<W>(a, c, wr);
+            if (kCachesWeights<E, W> && ncache > 0)
+                wr.from_smem(wcache + (k % ncache) * W * 32, lane_id);
+            else
+                wr.load(a, c);
         }
         if (!mbar_wait(&full[s], (k / STAGES) & 1)) {  // copies did not arrive in time
             if (a.err && lane_id == 0) atomicOr(a.err, static_cast<int>(SCONV_EFLAG_TIMEOUT));
@@ -301,24 +419,24 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
 #pragma unroll
         for (int r = 0; r < kTokPerWarp + W - 1; ++r) rows[r] = xs[(i0 + r) * 32];
 
-        bf16 *out = static_cast<bf16 *>(a.out);
-        bf16 *cache = static_cast<bf16 *>(a.cache);
+        E *out = static_cast<E *>(a.out);
+        E *cache = static_cast<E *>(a.cache);
         if ((fast_mask & 0xfu) == 0xfu) {
             // The common case: four ordinary tokens, straight-line code.
 #pragma unroll
             for (int uu = 0; uu < kTokPerWarp; ++uu) {
-                float acc[8];
+                float acc[VEC];
 #pragma unroll
-                for (int v = 0; v < 8; ++v) acc[v] = 0.f;
+                for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
 #pragma unroll
-                for (int d = W - 1; d >= 0; --d) fma_pack(acc, wr[d], rows[uu + W - 1 - d]);
+                for (int d = W - 1; d >= 0; --d) wr.fma(acc, d, rows[uu + W - 1 - d]);
                 const int64_t ins_u = __shfl_sync(0xffffffffu, ins, uu);
-                float xc[8];
+                float xc[VEC];
                 rows[uu + W - 1].to_float(xc);
 #pragma unroll
-                for (int v = 0; v < 8; ++v) {
+                for (int v = 0; v < VEC; ++v) {
                     float y = acc[v];
-                    if (SILU) y = silu<bf16>(y);
+                    if (SILU) y = silu<E>(y);
                     if (RESID) y = __fadd_rn(y, xc[v]);  // never contracted into an FMA
                     acc[v] = y;
                 }
@@ -337,12 +455,12 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
                 if (code_u == kSkip) continue;  // PAD row or past T
                 const int i = i0 + uu;
                 const int t = t0 + i;
-                float acc[8];
+                float acc[VEC];
 #pragma unroll
-                for (int v = 0; v < 8; ++v) acc[v] = 0.f;
+                for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
                 if (code_u == kFast) {
 #pragma unroll
-                    for (int d = W - 1; d >= 0; --d) fma_pack(acc, wr[d], rows[uu + W - 1 - d]);
+                    for (int d = W - 1; d >= 0; --d) wr.fma(acc, d, rows[uu + W - 1 - d]);
                 } else {
                     // Taps before the request's first row come from the cache
                     // (zero before position 0), or an index is out of range.
@@ -355,29 +473,33 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
                     if (req < 0 || req >= a.num_reqs) bad |= SCONV_EFLAG_REQUEST;
                     if (q0 < 0 || q0 > t) bad |= SCONV_EFLAG_QUERY_START;
                     if (pos < 0) bad |= SCONV_EFLAG_POSITION;
-                    P ct[W];
+                    // Each cache tap is accumulated as it arrives; a bad
+                    // block-table index adds its flag (the union over all
+                    // taps, as the token kernel reports) and skips the token.
+                    if (!bad) {
 #pragma unroll
-                    for (int d = 1; d < W; ++d)
-                        if (t - d < q0 && pos - d >= 0 && !bad)
-                            bad |= load_cache_tap<bf16, 8>(a, req, pos - d, lane, ct[d]);
+                        for (int d = W - 1; d >= 0; --d) {
+                            if (d == 0 || t - d >= q0) {
+                                wr.fma(acc, d, rows[uu + W - 1 - d]);
+                            } else if (pos - d >= 0) {
+                                P ct;
+                                const unsigned e = load_cache_tap<E, VEC>(a, req, pos - d, lane, ct);
+                                bad |= e;
+                                if (!e) wr.fma(acc, d, ct);
+                            }
+                        }
+                    }
                     if (bad) {
                         if (a.err && active) atomicOr(a.err, static_cast<int>(bad));
                         continue;
                     }
-#pragma unroll
-                    for (int d = W - 1; d >= 0; --d) {
-                        if (d == 0 || t - d >= q0)
-                            fma_pack(acc, wr[d], rows[uu + W - 1 - d]);
-                        else if (pos - d >= 0)
-                            fma_pack(acc, wr[d], ct[d]);
-                    }
                 }
-                float xc[8];
+                float xc[VEC];
                 rows[uu + W - 1].to_float(xc);
 #pragma unroll
-                for (int v = 0; v < 8; ++v) {
+                for (int v = 0; v < VEC; ++v) {
                     float y = acc[v];
-                    if (SILU) y = silu<bf16>(y);
+                    if (SILU) y = silu<E>(y);
                     if (RESID) y = __fadd_rn(y, xc[v]);  // never contracted into an FMA
                     acc[v] = y;
                 }
@@ -441,11 +563,20 @@ bool encode_1d(CUtensorMap *m, CUtensorMapDataType type, const void *base, int64
 
 constexpr int kLaunchStages = 4;
 
-template <int W, bool SILU, bool RESID>
+int gcd_int(int64_t x, int64_t y) {
+    while (y != 0) {
+        const int64_t r = x % y;
+        x = y;
+        y = r;
+    }
+    return static_cast<int>(x);
+}
+
+template <typename E, int W, bool SILU, bool RESID>
 cudaError_t launch_flags(const FusedArgs &a, const TmaMaps &maps, cudaStream_t stream) {
     constexpr int S = kLaunchStages;
-    constexpr int smem = kStages_smem<W, S>();
-    auto kernel = fused_tma_kernel<W, S, SILU, RESID>;
+    constexpr int smem = kStages_smem<W, S>() + (kCachesWeights<E, W> ? kWeightCacheBytes : 0);
+    auto kernel = fused_tma_kernel<E, W, S, SILU, RESID>;
     // Resident blocks per SM and the SM count, once per process and kernel
     // (the grid is a function of the device and of T and C only).
     static std::once_flag once;
@@ -465,41 +596,50 @@ cudaError_t launch_flags(const FusedArgs &a, const TmaMaps &maps, cudaStream_t s
     if (attr != cudaSuccess) return attr;
     // One block per resident slot, at most one per unit.
     const int64_t ntiles = (a.T + kBT - 1) / kBT;
-    const int64_t ncb = (a.C + kBC - 1) / kBC;
+    const int64_t ncb = (a.C + kBC<E> - 1) / kBC<E>;
     int64_t grid = static_cast<int64_t>(sms) * per_sm;
     if (grid > ntiles * ncb) grid = ntiles * ncb;
-    return launch_pdl(kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem, stream,
-                      a, maps);
+    // A block visits ncb / gcd(grid, ncb) channel blocks in turn.
+    const int period = static_cast<int>(ncb / gcd_int(grid, ncb));
+    const int ncache = (kCachesWeights<E, W> && period > 1 &&
+                        period * W * 512 <= kWeightCacheBytes)
+                           ? period
+                           : 0;
+    return launch_pdl(kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads),
+                      static_cast<size_t>(kStages_smem<W, S>() + ncache * W * 512), stream, a,
+                      maps, ncache);
 }
 
-template <int W>
+template <typename E, int W>
 cudaError_t launch_w(const FusedArgs &a, const TmaMaps &maps, cudaStream_t stream) {
     if (a.silu) {
-        return a.resid ? launch_flags<W, true, true>(a, maps, stream)
-                       : launch_flags<W, true, false>(a, maps, stream);
+        return a.resid ? launch_flags<E, W, true, true>(a, maps, stream)
+                       : launch_flags<E, W, true, false>(a, maps, stream);
     }
-    return a.resid ? launch_flags<W, false, true>(a, maps, stream)
-                   : launch_flags<W, false, false>(a, maps, stream);
+    return a.resid ? launch_flags<E, W, false, true>(a, maps, stream)
+                   : launch_flags<E, W, false, false>(a, maps, stream);
 }
 
-}  // namespace
-
-cudaError_t launch_fused_tma(const FusedArgs &a, cudaStream_t stream, bool &used) {
-    used = false;
+template <typename E>
+cudaError_t launch_typed(const FusedArgs &a, cudaStream_t stream, bool &used) {
+    constexpr int e = static_cast<int>(sizeof(E));
     auto al16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
-    if (a.W < 1 || a.W > 4 || a.C < kBC || encode_fn() == nullptr) return cudaSuccess;
-    if (!al16(a.x) || (a.x_rs * 2) % 16 != 0 || !al16(a.positions) || !al16(a.slot) ||
+    if (a.W < 1 || a.W > 8 || a.C < kBC<E> || encode_fn() == nullptr) return cudaSuccess;
+    if (!al16(a.x) || (a.x_rs * e) % 16 != 0 || !al16(a.positions) || !al16(a.slot) ||
         !al16(a.seq_idx) || !al16(a.qstart))
         return cudaSuccess;
     TmaMaps maps;
     {
         const cuuint64_t dim[2] = {static_cast<cuuint64_t>(a.C), static_cast<cuuint64_t>(a.T)};
-        const cuuint64_t stride[1] = {static_cast<cuuint64_t>(a.x_rs) * 2};
-        const cuuint32_t box[2] = {kBC, static_cast<cuuint32_t>(kBT + a.W - 1)};
+        const cuuint64_t stride[1] = {static_cast<cuuint64_t>(a.x_rs) * e};
+        const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBC<E>),
+                                   static_cast<cuuint32_t>(kBT + a.W - 1)};
         const cuuint32_t elem[2] = {1, 1};
-        if (encode_fn()(&maps.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(a.x), dim,
-                        stride, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+        const CUtensorMapDataType type =
+            e == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+        if (encode_fn()(&maps.x, type, 2, const_cast<void *>(a.x), dim, stride, box, elem,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaSuccess;
     }
@@ -510,11 +650,23 @@ cudaError_t launch_fused_tma(const FusedArgs &a, cudaStream_t stream, bool &used
         return cudaSuccess;
     used = true;
     switch (a.W) {
-        case 1: return launch_w<1>(a, maps, stream);
-        case 2: return launch_w<2>(a, maps, stream);
-        case 3: return launch_w<3>(a, maps, stream);
-        default: return launch_w<4>(a, maps, stream);
+        case 1: return launch_w<E, 1>(a, maps, stream);
+        case 2: return launch_w<E, 2>(a, maps, stream);
+        case 3: return launch_w<E, 3>(a, maps, stream);
+        case 4: return launch_w<E, 4>(a, maps, stream);
+        case 5: return launch_w<E, 5>(a, maps, stream);
+        case 6: return launch_w<E, 6>(a, maps, stream);
+        case 7: return launch_w<E, 7>(a, maps, stream);
+        default: return launch_w<E, 8>(a, maps, stream);
     }
+}
+
+}  // namespace
+
+cudaError_t launch_fused_tma(const FusedArgs &a, bool bf16_data, cudaStream_t stream,
+                             bool &used) {
+    used = false;
+    return bf16_data ? launch_typed<bf16>(a, stream, used) : launch_typed<float>(a, stream, used);
 }
 
 }  // namespace sconv

@@ -53,24 +53,33 @@ def test_every_window_length(W, dtype):
 
 
 @pytest.mark.parametrize("W", range(1, 9))
-def test_strip_kernel_every_window_length(W):
-    """Enough token-packs (T*C/8 >= 2^19) for the streamed strip kernel,
-    with request starts, histories and PAD rows inside strips."""
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_prefill_tile_kernel_every_window_length(W, dtype):
+    """Enough token-packs (T*C/VEC >= 2^19) for the prefill form (TMA tiles
+    of 32 tokens x 512 bytes, W-1 halo rows), with request starts,
+    histories and PAD rows inside tiles, for every tap count and both
+    dtypes."""
     rng = np.random.default_rng(100 + W)
-    wl = workloads.build(f"strip_w{W}", dtype="bf16", H=16, D=136, ws=128, off_s=8, W=W, N=16,
-                         hist=rng.integers(0, 30, size=4), new=rng.integers(600, 900, size=4),
-                         act="silu", residual=bool(W % 2), seed=W, num_pad=9, rng=rng)
-    assert wl.T * wl.C // 8 >= 1 << 19
+    H = 16 if dtype == "bf16" else 8
+    wl = workloads.build(f"tile_w{W}_{dtype}", dtype=dtype, H=H, D=136, ws=128, off_s=8, W=W,
+                         N=16, hist=rng.integers(0, 30, size=4),
+                         new=rng.integers(600, 900, size=4), act="silu",
+                         residual=bool(W % 2), seed=W, num_pad=9, rng=rng)
+    vec = 8 if dtype == "bf16" else 4
+    assert wl.T * wl.C // vec >= 1 << 19
     check_small(wl, DEV)
 
 
-def test_unaligned_metadata_takes_the_strip_kernel():
+@pytest.mark.parametrize("W", [4, 5, 8])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_unaligned_metadata_takes_the_strip_kernel(W, dtype):
     """Metadata arrays that start 8 bytes past a 16-byte boundary cannot be
     bulk-copied; the streamed strip kernel serves the same step."""
     rng = np.random.default_rng(11)
-    wl = workloads.build("strip_unaligned", dtype="bf16", H=16, D=128, ws=128, off_s=0, W=4,
-                         N=16, hist=rng.integers(0, 30, size=4), new=rng.integers(600, 900, size=4),
-                         act="silu", residual=True, seed=11, num_pad=5, rng=rng)
+    wl = workloads.build(f"strip_unaligned_w{W}", dtype=dtype, H=16, D=128, ws=128, off_s=0,
+                         W=W, N=16, hist=rng.integers(0, 30, size=4),
+                         new=rng.integers(600, 900, size=4), act="silu", residual=True,
+                         seed=11, num_pad=5, rng=rng)
     t = wl.tensors(DEV)
     for k in ("positions", "slot_mapping"):
         buf = torch.empty(wl.T + 1, dtype=torch.int64, device=DEV)
@@ -212,14 +221,17 @@ def _chunk_inputs(wl, t, a, b):
                 seq_idx=seq_idx.to(DEV), query_start=qs.to(DEV)), rows
 
 
+@pytest.mark.parametrize("H,ws,W", [(8, 64, 4), (16, 128, 4), (16, 128, 7)])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_chunked_prefill_bit_exact_on_gpu(dtype):
+def test_chunked_prefill_bit_exact_on_gpu(dtype, H, ws, W):
     """Prefill split into chunks, each later chunk reading the cache the
     earlier ones wrote, equals one-shot prefill bit for bit (outputs and
-    cache), on the device."""
+    cache), on the device.  With C = 2048 the one-shot step and the larger
+    chunks take the tiled prefill form and the small chunks the token form,
+    so this also checks that both forms produce the same bits."""
     R, L = 4, 700
     rng = np.random.default_rng(9)
-    wl = workloads.build("chunks", dtype=dtype, H=8, D=64, ws=64, off_s=0, W=4, N=16,
+    wl = workloads.build("chunks", dtype=dtype, H=H, D=ws, ws=ws, off_s=0, W=W, N=16,
                          hist=rng.integers(0, 50, size=R), new=np.full(R, L), act="silu",
                          residual=True, seed=9, rng=rng)
     t = wl.tensors(DEV)
