@@ -42,6 +42,12 @@
  *     index out of range is skipped whole (no cache write, no output row)
  *     and, if `err_flag` is not NULL, the matching SCONV_EFLAG_* bits are
  *     OR-ed into *err_flag.  Nothing traps or waits.
+ *   - Every kernel is launched with programmatic dependent launch: it may
+ *     start while the kernel before it on the stream still runs, and waits
+ *     for that kernel to complete before it reads data that kernel may
+ *     write.  weight and bias are the exception: they may be read before
+ *     that wait, so the kernel that precedes a call on the stream must not
+ *     write them.
  *   - Preconditions not checked (behaviour is undefined when broken): the
  *     rows of one request are contiguous in x with positions rising by one;
  *     the non-PAD slots of a call are distinct; no slot written by a call is
