@@ -24,7 +24,9 @@
 //    streamed through a register ring: the x row and metadata of token
 //    t + PF are loaded while token t is computed, so loads are always in
 //    flight and each x element is read from DRAM once (the W-1 halo rows
-//    before the strip come from L2).  Used for prefill.
+//    before the strip come from L2).  Used for the prefill shapes the tiled
+//    form (fused_tma.cu) does not take: metadata or x not 16-byte aligned,
+//    layouts without 16-byte channel packs, C below one tile row.
 //
 // The tap source (x, cache, zero) depends only on the token, so it is
 // uniform across a warp.  The grid of either kernel is a function of T and
@@ -80,9 +82,10 @@ __device__ __forceinline__ void conv_store(const FusedArgs &a, const float (&wr)
 
 // Before the PDL wait, while the preceding kernel drains: pull token t's
 // metadata, its x pack and (for a speculating launch) the pack's weights
-// into L2 (a warp's lanes share t), then go one step further.  The token's metadata and block-table
-// entries are read *speculatively* with L2-only loads (ld.global.cg, so no
-// line enters L1) -- the preceding kernel may still be writing them -- and
+// into L2 (a warp's lanes share t), then go one step further.  The token's
+// metadata and block-table entries are read *speculatively* with L2-only
+// loads (ld.global.cg, so no line enters L1) -- the preceding kernel may
+// still be writing them -- and
 // used only to choose which block-table lines and cache taps to prefetch
 // into L2.  Every speculative index is range-checked before it forms an
 // address.  After the wait the real loads run as usual; a stale value costs
@@ -380,9 +383,12 @@ inline Shape block_shape(int nv, int64_t rows) {
 }
 
 // Speculative prefetching before the PDL wait pays off only when this
-// launch's blocks can be resident while the preceding kernel still runs:
-// a launch of at most a quarter of the GPU's thread slots (148 SMs x 2048).
-inline bool speculate(int64_t threads) { return threads <= 148LL * 512; }
+// launch's blocks can be resident while the preceding kernel still runs: a
+// launch of at most an eighth of the GPU's thread slots (148 SMs x 2048).
+// Measured (A/B, us, with / without): decode 256 x 128 threads 3.51 / 3.93,
+// sconv_update 3.36 / 4.17; two streams in one launch (2 x 256 x 128
+// threads) 4.56 / 4.47; spec decode 512 x 256 threads 7.57 / 6.12.
+inline bool speculate(int64_t threads) { return threads <= 148LL * 256; }
 
 // Strip kernel only when there is enough work to stream: T*C/VEC
 // token-packs above this many.
