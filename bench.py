@@ -444,6 +444,32 @@ def _entry(wl, secs, nbytes, peak):
             "alg_bytes": nbytes, "alg_gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
 
 
+def bench_prefill_shapes(device, stream, peak, reps=50):
+    """The chunked prefill's requests and channel count (T = 16 070, C =
+    4096) in fp32 with W = 4 and in bf16 with W = 8: the tiled prefill form
+    outside the named workloads' dtype and tap count."""
+    import hybrid_sconv_b200 as hs
+    table = {}
+    for tag, dtype, W in (("f32_w4", "f32", 4), ("bf16_w8", "bf16", 8)):
+        rng = np.random.default_rng(1003)
+        hist = rng.integers(0, 2049, size=16)
+        new = rng.integers(1, 2049, size=16)
+        wl = workloads.build(f"chunked_prefill_{tag}", dtype=dtype, H=32, D=128, ws=128,
+                             off_s=0, W=W, N=16, hist=hist, new=new, act="silu",
+                             residual=False, seed=1003, rng=rng)
+        t = wl.tensors(device)
+        out = torch.empty_like(t["x"])
+
+        def f():
+            hs.sconv_fused(t["x"], t["weight"], t["cache"], t["positions"], t["block_table"],
+                           t["seq_idx"], t["slot_mapping"], t["query_start"], out=out,
+                           **wl.kwargs())
+        table[wl.name] = _entry(wl, _kernel_time([f], reps, stream), algorithmic_bytes(wl), peak)
+        del t, out
+        torch.cuda.empty_cache()
+    return table
+
+
 def bench_prefill(name, device, stream, peak, reps=None):
     """One prefill workload (a single set, larger than L2): the fused
     kernel's throughput; for the long prefill also the window extraction
@@ -778,6 +804,7 @@ def per_workload_table(device, stream, peak, sets_obj=None):
         table.update(bench_decode_chain(sets_obj, stream, peak))
     table.update(bench_prefill("chunked_prefill_bf16", device, stream, peak))
     table.update(bench_prefill("long_prefill_bf16", device, stream, peak))
+    table.update(bench_prefill_shapes(device, stream, peak))
     table.update(bench_spec_decode(device, stream, peak))
     table.update(bench_ssm_gather(device, stream, peak))
     table.update(bench_dense(device, stream, peak))
