@@ -39,17 +39,36 @@ __device__ __forceinline__ int clamped_count(const ExtractArgs &a) {
     return rc;
 }
 
+// Before the PDL wait the thread reads real_count and its slot's end
+// position *speculatively* (L2-only loads; the preceding kernel may still be
+// writing them), range-checks them and only prefetches its window's rows
+// into L2.  After the wait real_count and the end position are loaded
+// together, so the gather waits for one L2 round trip before its rows, not
+// two; a stale speculative value costs a useless prefetch, never a wrong
+// result.
 template <typename E, int DC>
 __global__ void __launch_bounds__(256) extract_windows_vec(const __grid_constant__ ExtractArgs a) {
     using R = typename Raw<E>::T;
     constexpr int VEC = Elem<E>::kVec;
     const int slot = blockIdx.x;
-    if (slot >= clamped_count(a)) return;
     const int pack = blockIdx.y * blockDim.x + threadIdx.x;
-    if (pack >= a.conv_dim / VEC) return;
+    const bool in_range = pack < a.conv_dim / VEC;
     const int c = pack * VEC;
-    const int64_t end = __ldg(a.abs_pos + slot);
     const R *src = static_cast<const R *>(a.src);
+    if (in_range && slot < __ldcg(a.real_count)) {
+        const int64_t end = __ldcg(a.abs_pos + slot);
+#pragma unroll
+        for (int k = 0; k < DC; ++k) {
+            const int64_t p = end - DC + k;
+            if (p >= 0 && p < a.seq_len) prefetch_l2(src + p * a.src_ss + c);
+        }
+    }
+    pdl_wait();
+    pdl_trigger();
+    int rc = __ldg(a.real_count);
+    const int64_t end = __ldg(a.abs_pos + slot);  // slot < max_count: always in bounds
+    if (rc > a.max_count) rc = a.max_count;
+    if (slot >= rc || !in_range) return;
 
     union U {
         uint4 u;

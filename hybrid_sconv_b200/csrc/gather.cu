@@ -82,13 +82,12 @@ __global__ void __launch_bounds__(256) scatter_ssm_elem(const __grid_constant__ 
 
 // Resolve slot i's window: the physical block of each tap position (-1 for
 // p < 0).  Returns the SCONV_EFLAG_* bits of an out-of-range index, else 0.
+// r and end are the slot's request and end position, loaded by the caller.
 template <int DC>
-__device__ __forceinline__ unsigned window_blocks(const PagedExtractArgs &a, int slot, int d_conv,
-                                                  int64_t (&blk)[DC > 0 ? DC : 8],
+__device__ __forceinline__ unsigned window_blocks(const PagedExtractArgs &a, int r, int64_t end,
+                                                  int d_conv, int64_t (&blk)[DC > 0 ? DC : 8],
                                                   int64_t (&off)[DC > 0 ? DC : 8]) {
-    const int r = __ldg(a.request + slot);
     if (r < 0 || r >= a.num_reqs) return SCONV_EFLAG_REQUEST;
-    const int64_t end = __ldg(a.abs_pos + slot);
     const int32_t *bt_row = a.bt + static_cast<int64_t>(r) * a.bt_rs;
     // One division per slot: (lb, o) = the block and offset of the first
     // non-negative tap position, then stepped along the window.
@@ -119,30 +118,51 @@ __device__ __forceinline__ unsigned window_blocks(const PagedExtractArgs &a, int
 }
 
 // 16-byte channel packs (VEC elements of raw type R), DC taps per window.
+// Before the PDL wait the thread resolves its window *speculatively*
+// (L2-only loads of real_count, the slot's request and end position and
+// the block-table entries, each range-checked) and prefetches the cache rows
+// into L2; after the wait the same chain runs with ordinary loads, now L2
+// hits.  real_count, the request and the end position are loaded together.
 template <typename R, int DC>
 __global__ void __launch_bounds__(256) extract_paged_vec(const __grid_constant__ PagedExtractArgs a) {
     constexpr int VEC = 16 / sizeof(R);
     const int slot = blockIdx.x;
-    if (threadIdx.x == 0) {
-        prefetch_l2(a.real_count);
-        prefetch_l2(a.request + slot);
-        prefetch_l2(a.abs_pos + slot);
-    }
-    pdl_wait();
-    pdl_trigger();
-    if (slot >= clamp_count(a.real_count, a.max_count)) return;
-    int64_t blk[DC], off[DC];
-    const unsigned bad = window_blocks<DC>(a, slot, DC, blk, off);
-    if (bad) {
-        if (a.err && threadIdx.x == 0 && blockIdx.y == 0) atomicOr(a.err, static_cast<int>(bad));
-        return;
-    }
     const int pack = blockIdx.y * blockDim.x + threadIdx.x;
-    if (pack >= a.H * a.ws / VEC) return;
+    const bool in_range = pack < a.H * a.ws / VEC;
     const int c = pack * VEC;
     const int h = c / a.ws;
     const int64_t lane = static_cast<int64_t>(h) * a.cs1 + a.off_s + (c - h * a.ws);
     const R *cache = static_cast<const R *>(a.cache);
+    if (in_range && slot < __ldcg(a.real_count)) {
+        const int r = __ldcg(a.request + slot);
+        const int64_t end = __ldcg(a.abs_pos + slot);
+        if (r >= 0 && r < a.num_reqs) {
+            const int32_t *bt_row = a.bt + static_cast<int64_t>(r) * a.bt_rs;
+#pragma unroll
+            for (int k = 0; k < DC; ++k) {
+                const int64_t p = end - DC + k;
+                if (p < 0) continue;
+                const int64_t lb = p / a.N;
+                if (lb >= a.max_blocks) break;
+                const int32_t b = __ldcg(bt_row + lb);
+                if (b < 0 || b >= a.num_blocks) break;
+                prefetch_l2(cache + b * a.cs0 + (p - lb * a.N) * a.cs2 + lane);
+            }
+        }
+    }
+    pdl_wait();
+    pdl_trigger();
+    const int rc = clamp_count(a.real_count, a.max_count);
+    const int r = __ldg(a.request + slot);  // slot < max_count: always in bounds
+    const int64_t end = __ldg(a.abs_pos + slot);
+    if (slot >= rc) return;
+    int64_t blk[DC], off[DC];
+    const unsigned bad = window_blocks<DC>(a, r, end, DC, blk, off);
+    if (bad) {
+        if (a.err && threadIdx.x == 0 && blockIdx.y == 0) atomicOr(a.err, static_cast<int>(bad));
+        return;
+    }
+    if (!in_range) return;
     union U {
         uint4 u;
         R e[VEC];
@@ -178,7 +198,8 @@ __global__ void __launch_bounds__(256) extract_paged_elem(const __grid_constant_
     pdl_trigger();
     if (slot >= clamp_count(a.real_count, a.max_count)) return;
     int64_t blk[8], off[8];
-    const unsigned bad = window_blocks<0>(a, slot, a.d_conv, blk, off);
+    const unsigned bad = window_blocks<0>(a, __ldg(a.request + slot), __ldg(a.abs_pos + slot),
+                                          a.d_conv, blk, off);
     if (bad) {
         if (a.err && threadIdx.x == 0 && blockIdx.y == 0) atomicOr(a.err, static_cast<int>(bad));
         return;
