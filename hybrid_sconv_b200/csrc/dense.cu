@@ -682,7 +682,20 @@ __global__ void __launch_bounds__(128) dense_update(const __grid_constant__ Dens
         load_taps<E, VEC, MAXW>(a, c, wt);
         load_bias<E, VEC>(a, c, acc);
     }
-    if (threadIdx.x == 0 && a.lines) prefetch_l2(a.lines + b);
+    // While the preceding kernel drains: the x pack and, from a speculative
+    // read of the line index (L2-only, range-checked), the thread's line
+    // entries into L2.  A stale index costs a useless prefetch only.
+    if (active) {
+        prefetch_l2(static_cast<const R *>(a.x) + static_cast<int64_t>(b) * a.x_st +
+                    static_cast<int64_t>(c) * a.x_sc);
+        const int64_t ls = a.lines ? __ldcg(a.lines + b) : b;
+        if (ls >= 0 && ls < a.num_lines && !(a.lines && ls == a.pad)) {
+            const R *sp = static_cast<const R *>(a.st) + ls * a.s_line +
+                          static_cast<int64_t>(c) * a.s_c;
+            for (int i = 0; i < L; ++i) prefetch_l2(sp + i * a.s_k);
+        }
+    }
+    if (threadIdx.x == 0 && a.seqlens) prefetch_l2(a.seqlens + b);
     pdl_wait();
     pdl_trigger();
     const int64_t line = a.lines ? __ldg(a.lines + b) : b;
