@@ -70,6 +70,28 @@ def test_prefill_tile_kernel_every_window_length(W, dtype):
     check_small(wl, DEV)
 
 
+@pytest.mark.parametrize("dtype,H,W", [
+    ("bf16", 32, 5), ("bf16", 32, 8),   # 16 channel blocks: weights cached, 2 per block
+    ("f32", 16, 6), ("f32", 16, 8),     # the same for fp32 (cached above W = 5)
+    ("bf16", 18, 5),                    # 9 channel blocks: 9 cached weight sets
+    ("bf16", 18, 8),                    # 9 blocks x W 8 exceed the cache: reloaded per switch
+])
+def test_prefill_tile_kernel_channel_block_switches(dtype, H, W):
+    """The tiled prefill form's persistent blocks take (token tile, channel
+    block) units in token-major order, so a block's channel block changes
+    from unit to unit when the grid is not a multiple of the channel-block
+    count: its weights then come from the shared-memory copy made at entry
+    (W above 4 for bf16, above 5 for fp32, when they fit) or are reloaded."""
+    rng = np.random.default_rng(300 + W + H)
+    wl = workloads.build(f"switch_{dtype}_h{H}_w{W}", dtype=dtype, H=H, D=136, ws=128,
+                         off_s=8, W=W, N=16, hist=rng.integers(0, 30, size=4),
+                         new=rng.integers(500, 700, size=4), act="silu", residual=True,
+                         seed=W + H, num_pad=11, rng=rng)
+    vec = 8 if dtype == "bf16" else 4
+    assert wl.T * wl.C // vec >= 1 << 19
+    check_small(wl, DEV)
+
+
 @pytest.mark.parametrize("W", [4, 5, 8])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_unaligned_metadata_takes_the_strip_kernel(W, dtype):
