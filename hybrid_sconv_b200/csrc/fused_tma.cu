@@ -6,7 +6,7 @@
 // Tiling.  A tile is kBT = 32 consecutive tokens x 512 bytes of a row (256
 // bf16 or 128 fp32 channels, kBC<E>).  One thread of each block issues, per
 // tile,
-//   * a 2-D tensor copy of x rows [t0 - (W-1), t0 + 32) x [c0, c0 + 256)
+//   * a 2-D tensor copy of x rows [t0 - (W-1), t0 + 32) x [c0, c0 + kBC<E>)
 //     (the W-1 halo rows before the tile included; rows before 0 and past T
 //     and channels past C arrive as zeros), and
 //   * four 1-D tensor copies of the tile's positions, slot_mapping, seq_idx
@@ -23,8 +23,9 @@
 // serves that band far faster than one scattered spot per block (chunked
 // prefill 82.2 -> 72.3 us, long prefill 611 -> 530 us, against equal
 // contiguous shares of the units in channel-block-major order).  A block's
-// channel block changes from unit to unit; it reloads its weights (a few
-// lines, L1-resident) only when it does.
+// channel block changes from unit to unit; when it does, the block reloads
+// its weights (a few lines, L1-resident) or, for bf16 W > 4 and fp32 W > 5,
+// copies them from the shared-memory set it unpacked at entry.
 //
 // Compute.  Eight warps per block; warp g owns tokens 4g..4g+3 of the tile
 // and lane l the 16-byte pack l of the tile's row (8 bf16 or 4 fp32
