@@ -27,7 +27,6 @@ import hashlib
 import json
 import os
 import platform
-import re
 import statistics
 import subprocess
 import sys
@@ -162,17 +161,18 @@ def kernel_source_hash() -> str:
 
 def profiled_traffic(workload: str):
     """DRAM bytes per launch of the fused kernel from the committed ncu
-    summary, if it was taken on the current kernel source."""
-    path = os.path.join(ROOT, "profiles", f"fused_sconv_{workload}.md")
+    record (profiles/fused_sconv_<workload>.json), if it was taken on the
+    current kernel source; None otherwise."""
+    path = os.path.join(ROOT, "profiles", f"fused_sconv_{workload}.json")
     try:
-        text = open(path).read()
-    except OSError:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
         return None
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
-    s = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
-    if not m or not s or s.group(1) != kernel_source_hash():
+    if rec.get("kernel_source_sha256_16") != kernel_source_hash():
         return None
-    return int(m.group(1))
+    v = rec.get("traffic_bytes_per_launch")
+    return int(v) if v is not None else None
 
 
 # --------------------------------------------------------------------------
@@ -359,15 +359,37 @@ def run_steps_graphs(sets_obj, K, stream, pipeline=False, **step_kw):
         else:
             for i in range(n):
                 sets_obj.step(i, **step_kw)
-    full = capture(lambda: steps(M), stream)
+    full = capture(lambda: steps(M), stream) if K >= M else None
     tail = capture(lambda: steps(K % M), stream) if K % M else None
     return full, tail, K // M
 
 
-def time_region(full, tail, reps, stream, world, sampler=None):
+class L2Flush:
+    """A device buffer larger than L2 (256 MiB), written right before a timed
+    region so that no input of the timed steps is still cached from the
+    warm-up."""
+
+    def __init__(self, device):
+        self.buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=device)
+
+    def __call__(self):
+        self.buf.zero_()
+
+
+# GPU cycles of the spin kernel enqueued before a timed region (about 1 ms at
+# the B200's 1.965 GHz): the device stays busy while the host enqueues the
+# start event and the graph launches, so the region measures the GPU's work
+# and not the host's submission latency.
+HOST_LEAD_CYCLES = 2_000_000
+
+
+def time_region(full, tail, reps, stream, world, sampler=None, flush=None):
     """Seconds for the replays, by CUDA events on the launching stream,
     bracketed by a barrier and a device synchronisation on both sides.
-    With a sampler, also returns the host wall-clock span of the region."""
+    flush: written on the stream before the start event (L2 cold for the
+    timed steps).  A spin kernel precedes the start event so the device does
+    not wait for the host's launches inside the region.  With a sampler,
+    also returns the host wall-clock span of the region."""
     barrier(world)
     torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
@@ -377,6 +399,9 @@ def time_region(full, tail, reps, stream, world, sampler=None):
         time.sleep(1.0)  # nvidia-smi takes a moment before its first reading
     w0 = time.time()
     with torch.cuda.stream(stream):
+        if flush is not None:
+            flush()
+        torch.cuda._sleep(HOST_LEAD_CYCLES)
         start.record()
         replay_steps(full, tail, reps)
         end.record()
@@ -388,6 +413,32 @@ def time_region(full, tail, reps, stream, world, sampler=None):
         time.sleep(0.3)
         sampler.stop()
     return start.elapsed_time(end) / 1e3, (w0, w1)  # seconds
+
+
+def prime(full, tail, stream):
+    """Replay each graph that is about to be timed once, untimed: the first
+    replay of a freshly instantiated graph also uploads it."""
+    with torch.cuda.stream(stream):
+        for g in (full, tail):
+            if g is not None:
+                g.replay()
+    torch.cuda.synchronize()
+
+
+def l2_statement(sets_obj, K):
+    """What the timed region does about L2, computed for this run: which
+    sets the K timed steps read and how many bytes one pass over them
+    touches."""
+    M = len(sets_obj.sets)
+    if K <= M:
+        touched = sum(sets_obj.alg_bytes[:K])
+        return (f"L2 flushed (256 MiB written) before the timed region; the {K} timed steps "
+                f"each read their own input set (none repeats within the region; "
+                f"{touched / 1e6:.0f} MB touched in all)")
+    touched = sum(sets_obj.alg_bytes)
+    verdict = "> 126 MB L2" if touched > L2_BYTES else "NOT above the 126 MB L2"
+    return (f"L2 flushed (256 MiB written) before the timed region; the steps rotate over "
+            f"{M} input sets, each rotation touching {touched / 1e6:.0f} MB {verdict}")
 
 
 def fused_launch_duration(sets_obj, stream, reps=200):
@@ -552,15 +603,17 @@ def bench_spec_decode(device, stream, peak, n_sets=40):
 
 
 def bench_serial_step(sets_obj, stream, peak, reps=200):
-    """The decode step without pipelining, on one stream: metadata then
-    convolution.  With sconv_seq_metadata each step's metadata waits for
-    the previous step's convolution before its lookup; with
-    sconv_seq_metadata_ahead the lookup overlaps that convolution and only
-    the completion waits.  Also the headline's pipelined step with the
-    plain metadata builder, for comparison."""
+    """The headline's pipelined step in steady state (its full graph of all
+    rotating sets replayed many times), and for comparison the step without
+    pipelining, on one stream: metadata then convolution.  With
+    sconv_seq_metadata each step's metadata waits for the previous step's
+    convolution before its lookup; with sconv_seq_metadata_ahead the lookup
+    overlaps that convolution and only the completion waits.  Also the
+    pipelined step with the plain metadata builder."""
     saved = sets_obj.ahead
     res = {}
-    for key, ahead, pipeline in (("decode_step_serial", False, False),
+    for key, ahead, pipeline in (("decode_step_pipelined", True, True),
+                                 ("decode_step_serial", False, False),
                                  ("decode_step_serial_ahead", True, False),
                                  ("decode_step_pipelined_plain_metadata", False, True)):
         sets_obj.ahead = ahead
@@ -908,7 +961,7 @@ def _packed_inputs(sets_obj, keys):
     return packed
 
 
-def e2e(sets_obj, K, stream, world):
+def e2e(sets_obj, K, stream, world, flush):
     """End to end through the public API with host buffers.  Every step
     copies its inputs (x, positions, slot_mapping, block_table,
     query_start_loc) from pinned host memory to the device, builds the
@@ -951,10 +1004,10 @@ def e2e(sets_obj, K, stream, world):
         cur.wait_stream(down)
 
     M = len(sets_obj.sets)
-    full = capture(lambda: steps(M), stream)
+    full = capture(lambda: steps(M), stream) if K >= M else None
     tail = capture(lambda: steps(K % M), stream) if K % M else None
-    replay_steps(full, None, 2)
-    secs = max_over_ranks(time_region(full, tail, K // M, stream, world)[0], world)
+    prime(full, tail, stream)
+    secs = max_over_ranks(time_region(full, tail, K // M, stream, world, flush=flush)[0], world)
     del full, tail
     tokens = sum_over_ranks(float(sets_obj.wls[0].T * K), world)
     return {"value": round(tokens / secs / 1e6, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -965,7 +1018,7 @@ def e2e(sets_obj, K, stream, world):
 
 # --------------------------------------------------------------------------
 
-def config_block(world):
+def config_block(world, l2):
     return {"workload": "decode_bf16: 256 single-token requests over cached histories "
                         "U{1..4096}; H=32, D=128, ws=32, off_s=32, C=1024, W=4, N=16; "
                         "SiLU + residual",
@@ -977,8 +1030,7 @@ def config_block(world):
                           "convolutions run in order, each waiting for the previous one",
             "metadata": "sconv_seq_metadata_ahead: one metadata buffer set per step, so the "
                         "lookup may run before the launch's wait on its predecessors",
-            "l2": "rotating input sets (each touching its own cache blocks), combined "
-                  "footprint > 126 MB L2"}
+            "l2": l2}
 
 
 def main_reference(args, rank, world):
@@ -1023,7 +1075,7 @@ def main_reference(args, rank, world):
             "n_gpus": world, "steps": K, "warmup": W,
             "ms_per_step": round(el / K * 1e3, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_block(1),
+            "config": config_block(1, "oracle on the host: no GPU cache involved"),
             "cpu_baseline": {"value": round(v, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
                              "sample": sample, "host": host_cpu()},
             "e2e": {"value": round(v, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -1067,7 +1119,7 @@ def main():
 
     sets_obj = DecodeSets(args.sets, rank_seed(args.seed, rank), device, args.max_hist,
                           ahead=True)
-    touched = sum(sets_obj.alg_bytes)
+    flush = L2Flush(device)
 
     # warm-up, then exactly K timed steps
     wfull, wtail, wreps = run_steps_graphs(sets_obj, W, stream, pipeline=True)
@@ -1076,8 +1128,9 @@ def main():
     torch.cuda.synchronize()
     del wfull, wtail
     full, tail, reps = run_steps_graphs(sets_obj, K, stream, pipeline=True)
+    prime(full, tail, stream)
     sampler = ClockSampler(local) if rank == 0 else None
-    secs, (w0, w1) = time_region(full, tail, reps, stream, world, sampler)
+    secs, (w0, w1) = time_region(full, tail, reps, stream, world, sampler, flush)
     secs = max_over_ranks(secs, world)
     clocks = None
     if sampler is not None:
@@ -1085,9 +1138,13 @@ def main():
         clocks = ClockSampler.summary(inside, "timed region")
         if len(inside) < 3:
             # The timed region was too short for 100 ms sampling: sample a
-            # separate ~2 s replay of the same graphs instead.
+            # separate ~2 s replay of the same steps instead.
             load = ClockSampler(local)
-            n = max(1, int(2.0 / max(secs / max(reps, 1), 1e-6)))
+            if full is None:
+                full, _, _ = run_steps_graphs(sets_obj, len(sets_obj.sets), stream,
+                                              pipeline=True)
+                prime(full, None, stream)
+            n = max(1, int(2.0 / max(secs / K * len(sets_obj.sets), 1e-6)))
             _, (l0, l1) = time_region(full, None, n, stream, 1, load)
             clocks = ClockSampler.summary(load.samples(l0, l1),
                                           "2 s replay of the step graphs after the timed region")
@@ -1108,9 +1165,9 @@ def main():
         "steps": K, "warmup": W, "ms_per_step": round(secs / K * 1e3, 6),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded generator; random-normal x, weight and cache)",
-        "config": dict(config_block(world), **({} if touched > L2_BYTES and args.max_hist == 4096
-                                                 else {"l2": "NOT defeated: profiling case",
-                                                       "max_hist": args.max_hist})),
+        "config": config_block(world, l2_statement(sets_obj, K) if args.max_hist == 4096
+                               else "NOT a benchmark figure: profiling case "
+                                    f"(histories up to {args.max_hist} tokens)"),
         "hbm_gbs": round(step_bytes / secs / 1e9, 1),
         "gpu_launches": 2 * K,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
@@ -1125,7 +1182,7 @@ def main():
         line["clocks"] = clocks
 
     if not args.no_extras:
-        line["e2e"] = e2e(sets_obj, min(K, 24000), stream, world)
+        line["e2e"] = e2e(sets_obj, min(K, 24000), stream, world, flush)
         if rank == 0:
             line["per_config"] = per_workload_table(device, stream, peak, sets_obj)
         if rank == 0 and world == 1:

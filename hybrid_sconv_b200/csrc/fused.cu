@@ -397,6 +397,12 @@ constexpr int kPF = 4;
 
 template <typename E, int VEC, int MAXW>
 cudaError_t launch_w(FusedArgs &a, bool one, cudaStream_t stream) {
+    // a.w_vec says the weight is a dense, 16-byte aligned [C, W].  The token
+    // and strip kernels address it with the compile-time MAXW, so they take
+    // vector loads only when W == MAXW; the tiled form uses the exact W and
+    // takes them for every W.
+    const int w_vec_exact = a.w_vec;
+    a.w_vec = a.w_vec && a.W == MAXW;
     const int nv = a.C / VEC;
     const int64_t work = static_cast<int64_t>(a.T) * nv;
     if (one || work < kStripMinWork || a.T < 64) {
@@ -416,8 +422,10 @@ cudaError_t launch_w(FusedArgs &a, bool one, cudaStream_t stream) {
                                  dim3(s.cv, s.tg), 0, stream, a);
     }
     if constexpr (VEC * sizeof(E) == 16) {
+        FusedArgs tiled = a;
+        tiled.w_vec = w_vec_exact;
         bool used = false;
-        const cudaError_t e = launch_fused_tma(a, sizeof(E) == 2, stream, used);
+        const cudaError_t e = launch_fused_tma(tiled, sizeof(E) == 2, stream, used);
         if (used || e != cudaSuccess) return e;
     }
     // Strip length: a whole number of 32-token metadata chunks, the longest
@@ -436,11 +444,7 @@ cudaError_t launch_w(FusedArgs &a, bool one, cudaStream_t stream) {
 
 template <typename E, int VEC>
 cudaError_t launch_v(FusedArgs &a, bool one, cudaStream_t stream) {
-    if (a.W <= 4) {
-        a.w_vec = a.w_vec && a.W == 4;
-        return launch_w<E, VEC, 4>(a, one, stream);
-    }
-    a.w_vec = a.w_vec && a.W == 8;
+    if (a.W <= 4) return launch_w<E, VEC, 4>(a, one, stream);
     return launch_w<E, VEC, 8>(a, one, stream);
 }
 

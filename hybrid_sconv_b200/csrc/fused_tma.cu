@@ -61,7 +61,9 @@ constexpr int kBT = 32;            // tokens per tile
 constexpr int kThreads = 256;      // 8 warps
 constexpr int kTokPerWarp = kBT / (kThreads / 32);  // 4
 constexpr int kMetaBytes = kBT * (8 + 8 + 4 + 4);   // positions, slots, seq_idx, query_start
-constexpr uint32_t kWaitSpins = 1u << 22;  // bounded mbarrier polls (seconds, not forever)
+// An mbarrier wait gives up this many nanoseconds of %globaltimer time after
+// it begins (plus at most one try_wait suspension).
+constexpr uint64_t kWaitNs = 1000000000ull;
 
 template <int W>
 struct Layout {
@@ -116,10 +118,22 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
     return done != 0;
 }
 
-// Bounded wait for the phase with the given parity to complete.
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for the phase with the given parity to complete, for at most kWaitNs
+// of wall time: each try_wait may suspend the thread for a system-dependent
+// interval, so the bound is taken from the global nanosecond timer rather
+// than from a count of polls.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kWaitSpins; ++i)
+    if (mbar_test(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    do {
         if (mbar_test(bar, parity)) return true;
+    } while (globaltimer_ns() - t0 < kWaitNs);
     return false;
 }
 

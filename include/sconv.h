@@ -84,7 +84,9 @@ typedef enum sconv_act { SCONV_ACT_NONE = 0, SCONV_ACT_SILU = 1 } sconv_act;
 #define SCONV_EFLAG_QUERY_START 0x10u /* query_start[t] outside [0, t] */
 #define SCONV_EFLAG_POSITION    0x20u /* positions[t] < 0 */
 #define SCONV_EFLAG_TIMEOUT     0x40u /* a block's bulk copies did not arrive within its bounded
-                                         wait; that block wrote nothing further and returned */
+                                         wait (1 s of wall time by the GPU's global timer, plus
+                                         at most one mbarrier try_wait suspension); that block
+                                         wrote nothing further and returned */
 
 #define SCONV_MAX_W 8      /* taps supported by sconv_fused / sconv_update */
 #define SCONV_MAX_STREAMS 4 /* conv streams per sconv_fused_streams call */

@@ -47,6 +47,14 @@ def run_fused(wl, t, out=None, err=None, **kw):
                             t["query_start"], out=out, err_flag=err, **args)
 
 
+def run_update(wl, t, out=None, err=None, **kw):
+    """sconv_update on a decode-form step (token b is request b)."""
+    args = wl.kwargs()
+    args.update(kw)
+    return hs().sconv_update(t["x"], t["weight"], t["cache"], t["positions"],
+                             t["block_table"], t["slot_mapping"], out=out, err_flag=err, **args)
+
+
 def oracle_fused(wl, x, weight, cache, md, **kw):
     args = dict(dtype=wl.dtype, x=x, weight=weight, cache=cache,
                 positions=md["positions"], block_table=md["block_table"],
@@ -90,12 +98,13 @@ def sample_ranges(T, pieces=4, width=1024, seed=0):
     return sorted((s, s + width) for s in starts)
 
 
-def check_full_size(wl, device="cuda", ranges=None, t=None):
+def check_full_size(wl, device="cuda", ranges=None, t=None, run=run_fused):
     """Full-size step: the launch the benchmark times, compared with the
     oracle on sampled token ranges (outputs and the insert of each sampled
     token, element by element), plus size-independent properties over every
     token: each written element holds x, nothing else in the cache changed,
-    PAD rows are untouched."""
+    PAD rows are untouched.  ``run`` launches the step (sconv_fused by
+    default; run_update for a decode-form step)."""
     if t is None:
         t = wl.tensors(device)
     md_cpu = wl.metadata("cpu")
@@ -104,7 +113,7 @@ def check_full_size(wl, device="cuda", ranges=None, t=None):
     cache_before = t["cache"].clone()
     out = workloads.sentinel(tuple(t["x"].shape), wl.dtype, device)
     err = torch.zeros(1, dtype=torch.int32, device=device)
-    run_fused(wl, t, out=out, err=err)
+    run(wl, t, out=out, err=err)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
     got = out.cpu()

@@ -61,3 +61,37 @@ def test_reference_arm_prints_the_contract_line_on_cpu():
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["config"]["workload"].startswith("decode_bf16")
     assert np.isfinite(line["ms_per_step"])
+
+
+class _Sets:
+    def __init__(self, alg_bytes):
+        self.alg_bytes = alg_bytes
+        self.sets = [None] * len(alg_bytes)
+
+
+def test_l2_statement_for_fewer_steps_than_sets():
+    """K timed steps on K distinct sets: the statement says the region is
+    preceded by a flush and counts only the K sets' bytes."""
+    s = bench.l2_statement(_Sets([3_000_000] * 96), 20)
+    assert "flushed" in s and "none repeats" in s and "60 MB" in s
+
+
+def test_l2_statement_for_rotations():
+    big = bench.l2_statement(_Sets([3_000_000] * 96), 500)
+    assert "288 MB > 126 MB L2" in big
+    small = bench.l2_statement(_Sets([1_000_000] * 8), 500)
+    assert "NOT above the 126 MB L2" in small
+
+
+def test_profiled_traffic_reads_the_json_record(tmp_path, monkeypatch):
+    """The roofline's traffic comes from profiles/fused_sconv_<workload>.json
+    and only while its source hash matches the kernel sources."""
+    (tmp_path / "profiles").mkdir()
+    rec = {"traffic_bytes_per_launch": 1234, "kernel_source_sha256_16": "abc"}
+    (tmp_path / "profiles" / "fused_sconv_w.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "abc")
+    assert bench.profiled_traffic("w") == 1234
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "changed")
+    assert bench.profiled_traffic("w") is None
+    assert bench.profiled_traffic("missing") is None

@@ -9,7 +9,7 @@ import torch
 import oracle
 import workloads
 from tests._gpu import (assert_close, check_cache_holds_x, check_full_size, check_small, hs,
-                        oracle_fused, raw, run_fused)
+                        oracle_fused, raw, run_fused, run_update)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -208,6 +208,19 @@ def test_update_equals_fused_bit_exact():
                                      block_table=wl.block_table, slot_mapping=wl.slot_mapping,
                                      write_cache=False, **wl.kwargs())
     assert_close(oracle.to_f64(out_u.cpu(), wl.dtype), ref, wl.dtype, "update")
+
+
+def test_update_full_size_decode():
+    """sconv_update on the full decode workload the benchmark times: 256
+    requests over histories of up to 4096 tokens, a 4.2 GB cache whose
+    element offsets pass 2^31.  The workload is in decode form (token b is
+    request b), so the fused definition with its own metadata is the
+    update's; every token is compared with the oracle, the inserts element
+    by element and the whole cache by the holds-x invariant."""
+    wl = workloads.decode_bf16()
+    ar = np.arange(wl.T)
+    assert np.array_equal(wl.seq_idx, ar) and np.array_equal(wl.query_start, ar)
+    check_full_size(wl, DEV, run=run_update)
 
 
 def test_update_with_pad_rows():
