@@ -84,6 +84,13 @@ def _bind(path: str) -> ctypes.CDLL:
         _P, _P, _I64, _I64, _I64, _I64, _I64,  # states in/out, strides, L, num_lines
         _P, _P, _INT, _I64, _P, _P,            # cache_seqlens, indices, silu, pad, out, state
     ]
+    lib.oracle_resolve_taps.restype = None
+    lib.oracle_resolve_taps.argtypes = [
+        _P, _I64, _I64, _I64,                  # query_start_loc, num_reqs, num_actual, num_padded
+        _P, _P, _P, _I64, _I64, _I64, _I64,    # positions, slots, block_table, bt stride, max_blocks,
+        _INT,                                  #   num_blocks, N; W
+        _P, _P, _P,                            # seq_idx_out, query_start_out, taps
+    ]
     lib.oracle_check_preconditions.restype = _INT
     lib.oracle_check_preconditions.argtypes = [
         _I64, _INT, _I64, _P, _P, _P, _P, _P, _I64, _I64]
@@ -260,6 +267,34 @@ def seq_metadata(query_start_loc, num_reqs, num_actual_tokens, num_padded_tokens
     lib().oracle_seq_metadata(_ptr(qsl), num_reqs, num_actual_tokens,
                               num_padded_tokens, _ptr(si), _ptr(qs))
     return si, qs
+
+
+# Entries of the resolved tap table (see oracle_resolve_taps).
+SRC_X, SRC_ZERO = -2, -1
+
+
+def resolve_taps(*, query_start_loc, num_reqs, num_actual_tokens, positions, slot_mapping,
+                 block_table, num_blocks, block_size, W, num_padded_tokens=None):
+    """Oracle of the per-step tap resolution: returns (seq_idx, query_start,
+    taps) with taps int64 [num_padded, W-1] (lag d in column d-1): -2 for a
+    same-forward x row, -1 for a zero tap, the flat cache slot of a
+    pre-forward tap, or -(flags*256) when the token cannot be resolved.
+    ``query_start_loc`` None is the decode form (token t is request t)."""
+    if num_padded_tokens is None:
+        num_padded_tokens = num_actual_tokens
+    qsl = None if query_start_loc is None else _np(query_start_loc, np.int32)
+    pos = _np(positions, np.int64)
+    slot = _np(slot_mapping, np.int64)
+    bt = _np(block_table, np.int32)
+    if bt.ndim != 2:
+        raise ValueError("block_table must be [num_reqs, max_blocks]")
+    si = np.zeros(num_padded_tokens, np.int32)
+    qs = np.zeros(num_padded_tokens, np.int32)
+    taps = np.zeros((num_padded_tokens, max(W - 1, 0)), np.int64)
+    lib().oracle_resolve_taps(_ptr(qsl), num_reqs, num_actual_tokens, num_padded_tokens,
+                              _ptr(pos), _ptr(slot), _ptr(bt), bt.shape[1], bt.shape[1],
+                              num_blocks, block_size, W, _ptr(si), _ptr(qs), _ptr(taps))
+    return si, qs, taps
 
 
 def extract_windows(*, dtype, src, abs_positions, real_count, out, d_conv):

@@ -223,6 +223,87 @@ void oracle_seq_metadata(const int32_t *query_start_loc, int64_t num_reqs,
 }
 
 /*
+ * oracle_resolve_taps -- the tap-source resolution of [P1] (module
+ * docstring and fused_sconv argument comments) written out per token, so
+ * that it can be done once per step and read by every layer's convolution.
+ *
+ * The token's request r and first x row q0 come from query_start_loc as in
+ * oracle_seq_metadata (last r with query_start_loc[r] <= t), or, when
+ * query_start_loc is NULL (the decode form, token t is request t), r = q0 = t.
+ * For a non-PAD token t < num_actual at position pos, the entry for lag
+ * d = 1..W-1 (the tap at position src = pos - d), taps[t*(W-1) + d-1], is
+ *   -2                 the same-forward tap: x row t - d, when t - d >= q0;
+ *   -1                 the zero tap: src < 0 (and t - d < q0);
+ *   b*N + src % N      otherwise: the flat cache slot of src, with
+ *                      b = block_table[r][src / N] (the block/offset split
+ *                      of a flat slot that slot_mapping uses);
+ *   -(flags * 256)     for every lag, when the token cannot be resolved:
+ *                      flags holds the bounds-policy bits of its own
+ *                      indices (0x02 request >= num_reqs, 0x10 q0 outside
+ *                      [0, t], 0x20 pos < 0) or, when those are clean, the
+ *                      union over its cache taps of 0x04 (src / N >=
+ *                      max_blocks) and 0x08 (block outside [0, num_blocks)).
+ * PAD rows (slot_mapping == -1) and rows [num_actual, num_padded) get -1 at
+ * every lag and are never flagged.  seq_idx_out / query_start_out (either
+ * may be NULL) receive r and q0, and 0 on rows [num_actual, num_padded).
+ */
+#define SRC_X (-2)
+#define SRC_ZERO (-1)
+
+void oracle_resolve_taps(const int32_t *query_start_loc, int64_t num_reqs,
+                         int64_t num_actual, int64_t num_padded,
+                         const int64_t *positions, const int64_t *slot_mapping,
+                         const int32_t *block_table, int64_t bt_row_stride,
+                         int64_t max_blocks, int64_t num_blocks, int64_t N, int W,
+                         int32_t *seq_idx_out, int32_t *query_start_out,
+                         int64_t *taps) {
+    int64_t L = W - 1;
+    for (int64_t t = 0; t < num_padded; ++t) {
+        int64_t r = 0, q0 = 0;
+        for (int64_t d = 1; d <= L; ++d) taps[t * L + d - 1] = SRC_ZERO;
+        if (t < num_actual) {
+            if (query_start_loc) {
+                for (int64_t k = 0; k < num_reqs; ++k)
+                    if (query_start_loc[k] <= t) r = k;
+                q0 = query_start_loc[r];
+            } else {
+                r = t;
+                q0 = t;
+            }
+        }
+        if (seq_idx_out) seq_idx_out[t] = (int32_t)r;
+        if (query_start_out) query_start_out[t] = (int32_t)q0;
+        if (t >= num_actual || slot_mapping[t] == -1) continue;
+
+        int64_t pos = positions[t];
+        int64_t own = 0;
+        if (r >= num_reqs) own |= 0x02;
+        if (q0 < 0 || q0 > t) own |= 0x10;
+        if (pos < 0) own |= 0x20;
+        int64_t flags = own;
+        if (!own) {
+            for (int64_t d = 1; d <= L; ++d) {
+                int64_t src = pos - d;
+                int64_t *e = &taps[t * L + d - 1];
+                if (t - d >= q0) {
+                    *e = SRC_X;            /* same-forward tap ([P1]) */
+                } else if (src < 0) {
+                    *e = SRC_ZERO;         /* before position 0 */
+                } else {
+                    int64_t logical = src / N;
+                    if (logical >= max_blocks) { flags |= 0x04; continue; }
+                    int64_t b = block_table[r * bt_row_stride + logical];
+                    if (b < 0 || b >= num_blocks) { flags |= 0x08; continue; }
+                    *e = b * N + src % N;  /* pre-forward tap via block_table */
+                }
+            }
+        }
+        if (flags)
+            for (int64_t d = 1; d <= L; ++d) taps[t * L + d - 1] = -(flags * 256);
+    }
+}
+
+/*
  * oracle_extract_windows -- [P2] scatter_intermediate_conv: for slot
  * i < real_count, out[i][c][k] = src[abs_positions[i] - d_conv + k][c]
  * (window [pos - d_conv, pos), written transposed), with rows outside

@@ -3,8 +3,8 @@
 Each mutant is a copy of the oracle's C source with one plausible slip
 planted (a reversed or shifted tap, a wrong comparison, a swapped index, a
 dropped term, a transposed write).  It is compiled on the CPU, and the pin
-suites (tests/test_oracle_pins.py and tests/test_oracle_pins_dense.py) are
-run against it in a child process; they must fail for every mutant.  Every planted slip keeps all memory
+suites (tests/test_oracle_pins.py, tests/test_oracle_pins_dense.py and
+tests/test_oracle_pins_taps.py) are run against it in a child process; they must fail for every mutant.  Every planted slip keeps all memory
 accesses inside their buffers, so a mutant fails by assertion, not by crash.
 """
 from __future__ import annotations
@@ -124,7 +124,33 @@ MUTANTS = [
      "                        i = L + TAP_POSITION(0, W, k);",
      "                        i = (W - 1) + TAP_POSITION(0, W, k);"),
 ]
-PIN_FILES = ["test_oracle_pins.py", "test_oracle_pins_dense.py"]
+MUTANTS += [
+    ("resolve_same_forward_strict",
+     "                if (t - d >= q0) {\n                    *e = SRC_X;",
+     "                if (t - d > q0) {\n                    *e = SRC_X;"),
+    ("resolve_offset_div",
+     "                    *e = b * N + src % N;",
+     "                    *e = b * N + (src / N) % N;"),
+    ("resolve_logical_wraps",
+     "                    int64_t logical = src / N;\n                    if (logical >= max_blocks) { flags |= 0x04;",
+     "                    int64_t logical = (src / N) % max_blocks;\n                    if (logical >= max_blocks) { flags |= 0x04;"),
+    ("resolve_block_from_token_position",
+     "                    int64_t b = block_table[r * bt_row_stride + logical];",
+     "                    int64_t b = block_table[r * bt_row_stride + pos / N];"),
+    ("resolve_flags_on_first_lag_only",
+     "            for (int64_t d = 1; d <= L; ++d) taps[t * L + d - 1] = -(flags * 256);",
+     "            for (int64_t d = 1; d <= 1; ++d) taps[t * L + d - 1] = -(flags * 256);"),
+    ("resolve_pad_rows_resolved",
+     "        if (t >= num_actual || slot_mapping[t] == -1) continue;",
+     "        if (t >= num_actual) continue;"),
+    ("resolve_search_strict",
+     "                    if (query_start_loc[k] <= t) r = k;",
+     "                    if (query_start_loc[k] < t) r = k;"),
+    ("resolve_decode_start_zero",
+     "                r = t;\n                q0 = t;",
+     "                r = t;\n                q0 = 0;"),
+]
+PIN_FILES = ["test_oracle_pins.py", "test_oracle_pins_dense.py", "test_oracle_pins_taps.py"]
 
 
 def _run_mutant(tmp, name, old, new):
