@@ -44,6 +44,14 @@ import workloads  # noqa: E402
 METRIC = "fused sconv Mtokens/s and achieved HBM GB/s (% of B200 peak) per config"
 UNIT = "Mtokens/s"
 HEADLINE = "decode_bf16"
+# The headline step: its form (DecodeSets mode) and schedule (see
+# run_steps_graphs), the fastest single-layer decode step measured.
+STEP_MODE = "paged"
+STEP_SCHEDULE = "side"
+STEP_KERNEL = {"paged": "fused_token_kernel (sconv_fused at decode sizes)",
+               "taps": "fused_taps_kernel (sconv_fused_taps)"}
+STEP_CALLS = {"paged": "sconv_seq_metadata_ahead + sconv_fused",
+              "taps": "sconv_seq_metadata_taps_ahead + sconv_fused_taps"}
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 
@@ -120,6 +128,17 @@ def rank_seed(base: int, rank: int) -> int:
 
 # --------------------------------------------------------------------------
 # algorithmic bytes (what one launch must move, no re-reads)
+
+def algorithmic_bytes_taps(wl) -> int:
+    """Bytes of one sconv_fused_taps launch: as algorithmic_bytes, with the
+    per-token metadata being the slot (8 B) and the resolved table row
+    (8 B per lag) instead of 24 B of metadata plus block-table entries."""
+    e, C, W = wl.elem_bytes, wl.C, wl.W
+    live = int((wl.slot_mapping != -1).sum())
+    hist_rows = sum(min(W - 1, int(wl.hist[r])) for r in range(wl.R) if wl.new[r] > 0)
+    return (wl.T * C * e + 2 * live * C * e + hist_rows * C * e + C * W * e
+            + (8 + 8 * (W - 1)) * wl.T)
+
 
 def algorithmic_bytes(wl) -> int:
     """x rows read + inserts + outputs + the distinct pre-forward cache rows
@@ -277,15 +296,22 @@ def replay_steps(graphs_full, graph_tail, reps):
 class DecodeSets:
     """``n`` independent decode batches sharing one weight and one paged
     cache; each has its own requests, histories, block permutation, x,
-    metadata buffers and output."""
+    metadata buffers (seq_idx, query_start and the resolved tap table) and
+    output.
 
-    def __init__(self, n, seed, device, max_hist=4096, ahead=False):
-        # ahead: build each step's metadata with sconv_seq_metadata_ahead,
-        # whose precondition holds because every set has its own buffers and
-        # a graph replay touches each set once.
+    mode "taps" (the benchmark's step): sconv_seq_metadata_taps(_ahead)
+    builds the step's metadata and tap table, sconv_fused_taps convolves.
+    mode "paged": sconv_seq_metadata(_ahead), then sconv_fused reading
+    positions, request metadata and the block table itself."""
+
+    def __init__(self, n, seed, device, max_hist=4096, ahead=False, mode="taps", min_hist=1):
+        # ahead: build each step's metadata with the *_ahead builder, whose
+        # precondition holds because every set has its own buffers and a
+        # graph replay touches each set once.
         self.ahead = ahead
-        self.wls = [workloads.decode_bf16(seed=seed + 7919 * i, max_hist=max_hist)
-                    for i in range(n)]
+        self.mode = mode
+        self.wls = [workloads.decode_bf16(seed=seed + 7919 * i, max_hist=max_hist,
+                                          min_hist=min_hist) for i in range(n)]
         self.device = device
         nb = max(w.num_blocks for w in self.wls)
         w0 = self.wls[0]
@@ -302,21 +328,43 @@ class DecodeSets:
                 "block_table": md["block_table"], "query_start_loc": md["query_start_loc"],
                 "seq_idx": torch.empty(wl.T, dtype=torch.int32, device=device),
                 "query_start": torch.empty(wl.T, dtype=torch.int32, device=device),
+                "taps": torch.empty((wl.T, wl.W - 1), dtype=torch.int64, device=device),
                 "out": torch.empty((wl.T, wl.C), dtype=torch.bfloat16, device=device),
             }
             self.sets.append(s)
         self.alg_bytes = [algorithmic_bytes(wl) for wl in self.wls]
+        self.alg_bytes_taps = [algorithmic_bytes_taps(wl) for wl in self.wls]
 
-    def step(self, i, fused=True, metadata=True):
+    def kernel_alg_bytes(self):
+        """Algorithmic bytes of one convolution launch in this mode."""
+        return self.alg_bytes_taps if self.mode == "taps" else self.alg_bytes
+
+    def step(self, i, fused=True, metadata=True, ready=False):
+        """Metadata build and/or convolution of set i.  ready: the set's
+        metadata was complete before the kernel ahead of the convolution on
+        its stream began (sconv_fused_taps may then read it before its
+        wait)."""
         import hybrid_sconv_b200 as hs
         wl, s = self.wls[i], self.sets[i]
         if metadata:
-            build = hs.sconv_seq_metadata_ahead if self.ahead else hs.sconv_seq_metadata
-            build(s["query_start_loc"], wl.R, wl.T, s["seq_idx"], s["query_start"])
+            if self.mode == "taps":
+                build = (hs.sconv_seq_metadata_taps_ahead if self.ahead
+                         else hs.sconv_seq_metadata_taps)
+                build(s["query_start_loc"], wl.R, wl.T, s["positions"], s["slot_mapping"],
+                      s["block_table"], wl.num_blocks, wl.N, wl.W, seq_idx_out=s["seq_idx"],
+                      query_start_out=s["query_start"], taps_out=s["taps"])
+            else:
+                build = hs.sconv_seq_metadata_ahead if self.ahead else hs.sconv_seq_metadata
+                build(s["query_start_loc"], wl.R, wl.T, s["seq_idx"], s["query_start"])
         if fused:
-            hs.sconv_fused(s["x"], self.weight, self.cache, s["positions"], s["block_table"],
-                           s["seq_idx"], s["slot_mapping"], s["query_start"], out=s["out"],
-                           **wl.kwargs())
+            if self.mode == "taps":
+                hs.sconv_fused_taps(s["x"], self.weight, self.cache, s["slot_mapping"],
+                                    s["taps"], out=s["out"], metadata_ready=ready,
+                                    **wl.kwargs())
+            else:
+                hs.sconv_fused(s["x"], self.weight, self.cache, s["positions"],
+                               s["block_table"], s["seq_idx"], s["slot_mapping"],
+                               s["query_start"], out=s["out"], **wl.kwargs())
 
 
 def pipelined_steps(sets_obj, idxs, side):
@@ -337,6 +385,9 @@ def pipelined_steps(sets_obj, idxs, side):
         main.wait_event(meta_done)
         before = torch.cuda.Event()
         before.record(main)  # everything up to conv(i-1)
+        # Not ready: under stream capture the event join becomes a
+        # programmatic edge, which orders this launch after the builder's
+        # trigger, not after its completion.
         sets_obj.step(i, metadata=False)
         if j + 1 < len(idxs):
             side.wait_event(before)
@@ -347,15 +398,35 @@ def pipelined_steps(sets_obj, idxs, side):
     main.wait_stream(side)
 
 
+def interleaved_steps(sets_obj, idxs):
+    """Steps idxs in order on one stream, each convolution preceded by the
+    NEXT step's metadata build (the set's builder; an *_ahead builder looks
+    up before its wait, beside the convolution ahead of it): metadata(0),
+    metadata(1), conv(0), metadata(2), conv(1), ...  A convolution other
+    than the first reads its table before its wait, since the builder of
+    that table is two launches back, with the previous convolution between
+    them.  Each step still launches both kernels."""
+    sets_obj.step(idxs[0], fused=False)
+    for j, i in enumerate(idxs):
+        if j + 1 < len(idxs):
+            sets_obj.step(idxs[j + 1], fused=False)
+        sets_obj.step(i, metadata=False, ready=j > 0)
+
+
 def run_steps_graphs(sets_obj, K, stream, pipeline=False, **step_kw):
-    """Graphs that together replay exactly K steps over the rotating sets
-    (pipelined: next-step metadata beside the current convolution)."""
+    """Graphs that together replay exactly K steps over the rotating sets.
+    pipeline: False (metadata then convolution, one stream), "side" (next
+    step's metadata on a second stream beside the current convolution) or
+    "interleaved" (next step's metadata ahead of the current convolution on
+    one stream)."""
     M = len(sets_obj.sets)
     side = torch.cuda.Stream(stream.device)
 
     def steps(n):
-        if pipeline:
+        if pipeline == "side":
             pipelined_steps(sets_obj, list(range(n)), side)
+        elif pipeline == "interleaved":
+            interleaved_steps(sets_obj, list(range(n)))
         else:
             for i in range(n):
                 sets_obj.step(i, **step_kw)
@@ -443,11 +514,14 @@ def l2_statement(sets_obj, K):
 
 def fused_launch_duration(sets_obj, stream, reps=200):
     """Average duration of one fused launch: a graph of the fused launches
-    alone (one per rotating set, metadata already built) replayed `reps`
-    times, timed by CUDA events on the launching stream, divided by the
-    number of launches."""
+    alone (one per rotating set, metadata built beforehand, so complete
+    before any of them starts) replayed `reps` times, timed by CUDA events
+    on the launching stream, divided by the number of launches."""
     n = len(sets_obj.sets)
-    g = capture(lambda: [sets_obj.step(i, metadata=False) for i in range(n)], stream)
+    for i in range(n):
+        sets_obj.step(i, fused=False)
+    torch.cuda.synchronize()
+    g = capture(lambda: [sets_obj.step(i, metadata=False, ready=True) for i in range(n)], stream)
     with torch.cuda.stream(stream):  # on the timed stream, finished before timing
         for _ in range(3):
             g.replay()
@@ -577,7 +651,8 @@ def bench_prefill(name, device, stream, peak, reps=None):
 
 def bench_spec_decode(device, stream, peak, n_sets=40):
     """Speculative decode: rotating sets (each 7.5 MB, 40 sets > L2) over one
-    shared cache; the fused kernel's throughput."""
+    shared cache; the convolution launch alone, as sconv_fused and as
+    sconv_fused_taps on tables built beforehand."""
     import hybrid_sconv_b200 as hs
     wls = [workloads.spec_decode_bf16(seed=1004 + 7919 * i) for i in range(n_sets)]
     nb = max(w.num_blocks for w in wls)
@@ -586,50 +661,113 @@ def bench_spec_decode(device, stream, peak, n_sets=40):
     cache = torch.empty((nb, w0.H, w0.N, w0.D), dtype=torch.bfloat16, device=device)
     workloads.fill_normal_(cache, 1.0, g, device)
     weight = workloads.normal((w0.C, w0.W), 0.5, torch.bfloat16, g, device)
-    fns = []
+    fns, tfns = [], []
     for wl in wls:
         md = wl.metadata(device)
         x = workloads.normal((wl.T, wl.C), 1.0, torch.bfloat16, g, device)
         out = torch.empty_like(x)
+        taps = hs.sconv_seq_metadata_taps(md["query_start_loc"], wl.R, wl.T, md["positions"],
+                                          md["slot_mapping"], md["block_table"], wl.num_blocks,
+                                          wl.N, wl.W)
         fns.append(lambda wl=wl, md=md, x=x, out=out: hs.sconv_fused(
             x, weight, cache, md["positions"], md["block_table"], md["seq_idx"],
             md["slot_mapping"], md["query_start"], out=out, **wl.kwargs()))
+        tfns.append(lambda wl=wl, md=md, x=x, out=out, taps=taps: hs.sconv_fused_taps(
+            x, weight, cache, md["slot_mapping"], taps, out=out, metadata_ready=True,
+            **wl.kwargs()))
+    torch.cuda.synchronize()
+    res = {}
     secs = _kernel_time(fns, 200, stream)
-    nbytes = int(np.mean([algorithmic_bytes(w) for w in wls]))
-    res = {"spec_decode_bf16": _entry(w0, secs, nbytes, peak)}
-    del cache, fns
+    res["spec_decode_bf16"] = _entry(w0, secs, int(np.mean([algorithmic_bytes(w) for w in wls])),
+                                     peak)
+    secs = _kernel_time(tfns, 200, stream)
+    res["spec_decode_bf16_fused_taps"] = _entry(
+        w0, secs, int(np.mean([algorithmic_bytes_taps(w) for w in wls])), peak)
+    del cache, fns, tfns
     torch.cuda.empty_cache()
     return res
 
 
 def bench_serial_step(sets_obj, stream, peak, reps=200):
-    """The headline's pipelined step in steady state (its full graph of all
-    rotating sets replayed many times), and for comparison the step without
-    pipelining, on one stream: metadata then convolution.  With
-    sconv_seq_metadata each step's metadata waits for the previous step's
-    convolution before its lookup; with sconv_seq_metadata_ahead the lookup
-    overlaps that convolution and only the completion waits.  Also the
-    pipelined step with the plain metadata builder."""
-    saved = sets_obj.ahead
+    """Decode steps in steady state (a full graph of all rotating sets
+    replayed many times): the headline's pipelined step, and for comparison
+    the other step shapes.  side: the next step's metadata is built on a
+    second stream beside the current convolution (joined by an event);
+    interleaved: one stream, the next step's metadata enqueued ahead of the
+    current convolution; serial: one stream, metadata then convolution.  taps: sconv_seq_metadata_taps + sconv_fused_taps; paged:
+    sconv_seq_metadata + sconv_fused.  With a plain builder each step's
+    metadata waits for the previous step's convolution before its lookup;
+    with an *_ahead builder the lookup overlaps it and only the completion
+    waits."""
+    saved = (sets_obj.ahead, sets_obj.mode)
     res = {}
-    for key, ahead, pipeline in (("decode_step_pipelined", True, True),
-                                 ("decode_step_serial", False, False),
-                                 ("decode_step_serial_ahead", True, False),
-                                 ("decode_step_pipelined_plain_metadata", False, True)):
-        sets_obj.ahead = ahead
+    for key, mode, ahead, pipeline in (
+            ("decode_step_pipelined", STEP_MODE, True, STEP_SCHEDULE),
+            ("decode_step_taps_side", "taps", True, "side"),
+            ("decode_step_taps_interleaved", "taps", True, "interleaved"),
+            ("decode_step_serial_taps", "taps", False, False),
+            ("decode_step_serial_taps_ahead", "taps", True, False),
+            ("decode_step_paged_side", "paged", True, "side"),
+            ("decode_step_paged_interleaved", "paged", True, "interleaved"),
+            ("decode_step_serial", "paged", False, False),
+            ("decode_step_serial_ahead", "paged", True, False),
+            ("decode_step_paged_side_plain_metadata", "paged", False, "side")):
+        sets_obj.ahead, sets_obj.mode = ahead, mode
         full, _, _ = run_steps_graphs(sets_obj, len(sets_obj.sets), stream, pipeline=pipeline)
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                full.replay()
-        torch.cuda.synchronize()
+        prime(full, None, stream)
         secs, _ = time_region(full, None, reps, stream, 1)
         del full
         per = secs / (reps * len(sets_obj.sets))
+        names = {("taps", True): "sconv_seq_metadata_taps_ahead",
+                 ("taps", False): "sconv_seq_metadata_taps",
+                 ("paged", True): "sconv_seq_metadata_ahead",
+                 ("paged", False): "sconv_seq_metadata"}
         res[key] = {"step_us": round(per * 1e6, 3),
                     "mtokens_s": round(sets_obj.wls[0].T / per / 1e6, 2),
-                    "metadata": "sconv_seq_metadata_ahead" if ahead else "sconv_seq_metadata",
-                    "pipelined": pipeline}
-    sets_obj.ahead = saved
+                    "metadata": names[(mode, ahead)],
+                    "conv": "sconv_fused_taps" if mode == "taps" else "sconv_fused",
+                    "schedule": pipeline or "serial"}
+    sets_obj.ahead, sets_obj.mode = saved
+    return res
+
+
+def bench_metadata_kernels(sets_obj, stream, reps=200):
+    """The metadata builders alone, one launch per rotating set back to back:
+    sconv_seq_metadata (request index and start) and
+    sconv_seq_metadata_taps (the same plus the tap table)."""
+    saved = (sets_obj.ahead, sets_obj.mode)
+    res = {}
+    for key, mode in (("decode_bf16_seq_metadata", "paged"),
+                      ("decode_bf16_seq_metadata_taps", "taps")):
+        sets_obj.ahead, sets_obj.mode = False, mode
+        n = len(sets_obj.sets)
+        secs = _kernel_time([lambda i=i: sets_obj.step(i, fused=False) for i in range(n)], reps,
+                            stream)
+        res[key] = {"kernel_us": round(secs * 1e6, 3)}
+    sets_obj.ahead, sets_obj.mode = saved
+    return res
+
+
+def bench_decode_kernels(sets_obj, stream, peak, zero_sets=None):
+    """The convolution launch alone (metadata built beforehand), both forms,
+    on the decode sets and on a batch of the same shape with no history
+    (every token at position 0: no cache taps, so the difference is the
+    cost of the cache trip)."""
+    res = {}
+    for tag, so in (("", sets_obj), ("_zero_history", zero_sets)):
+        if so is None:
+            continue
+        saved = so.mode
+        for mode, kernel in (("taps", "fused_taps_kernel"), ("paged", "fused_token_kernel")):
+            so.mode = mode
+            secs = fused_launch_duration(so, stream)
+            nbytes = float(np.mean(so.kernel_alg_bytes()))
+            gbs = nbytes / secs / 1e9
+            res[f"decode_bf16{tag}_{'fused_taps' if mode == 'taps' else 'fused'}"] = {
+                "kernel_us": round(secs * 1e6, 3), "kernel": kernel,
+                "mtokens_s": round(so.wls[0].T / secs / 1e6, 2), "alg_bytes": int(nbytes),
+                "alg_gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
+        so.mode = saved
     return res
 
 
@@ -648,14 +786,17 @@ def bench_update(sets_obj, stream, peak, reps=200):
 
 
 def bench_streams(sets_obj, stream, peak, reps=200):
-    """Two conv streams of the decode layer in one sconv_fused_streams
-    launch: the workload's stream (lanes 32..63) and a second stream on
-    lanes 0..31, sharing tokens, metadata and cache."""
+    """Two conv streams of the decode layer in one launch: the workload's
+    stream (lanes 32..63) and a second stream on lanes 0..31, sharing
+    tokens, metadata and cache; as sconv_fused_streams and as
+    sconv_fused_streams_taps (tables built beforehand)."""
     import hybrid_sconv_b200 as hs
     wl0 = sets_obj.wls[0]
     g = torch.Generator(device=sets_obj.device).manual_seed(7)
     w2 = workloads.normal((wl0.C, wl0.W), 0.5, torch.bfloat16, g, sets_obj.device)
-    fns = []
+    for i in range(len(sets_obj.sets)):
+        sets_obj.step(i, fused=False)     # seq_idx, query_start (and the table in taps mode)
+    fns, tfns = [], []
     for wl, s in zip(sets_obj.wls, sets_obj.sets):
         x2 = workloads.normal((wl.T, wl.C), 1.0, torch.bfloat16, g, sets_obj.device)
         o2 = torch.empty_like(x2)
@@ -666,28 +807,42 @@ def bench_streams(sets_obj, stream, peak, reps=200):
         fns.append(lambda s=s, streams=streams, wl=wl: hs.sconv_fused_streams(
             streams, sets_obj.cache, s["positions"], s["block_table"], s["seq_idx"],
             s["slot_mapping"], s["query_start"], wl.N))
-    secs = _kernel_time(fns, reps, stream)
-    nbytes = 2 * int(np.mean(sets_obj.alg_bytes)) - 24 * wl0.T  # per-token metadata read once
-    gbs = nbytes / secs / 1e9
-    return {"decode_bf16_two_streams": {
-        "kernel_us": round(secs * 1e6, 3), "streams": 2,
-        "mtokens_s_per_stream": round(wl0.T / secs / 1e6, 2),
-        "stream_mtokens_s": round(2 * wl0.T / secs / 1e6, 2), "alg_bytes": nbytes,
-        "alg_gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}}
+        if sets_obj.mode == "taps":
+            tfns.append(lambda s=s, streams=streams, wl=wl: hs.sconv_fused_streams_taps(
+                streams, sets_obj.cache, s["slot_mapping"], s["taps"], wl.N,
+                metadata_ready=True))
+    torch.cuda.synchronize()
+    res = {}
+    for key, f, nbytes in (("decode_bf16_two_streams", fns,
+                            2 * int(np.mean(sets_obj.alg_bytes)) - 24 * wl0.T),
+                           ("decode_bf16_two_streams_taps", tfns,
+                            2 * int(np.mean(sets_obj.alg_bytes_taps)) - 32 * wl0.T)):
+        if not f:
+            continue
+        secs = _kernel_time(f, reps, stream)
+        gbs = nbytes / secs / 1e9
+        res[key] = {
+            "kernel_us": round(secs * 1e6, 3), "streams": 2,
+            "mtokens_s_per_stream": round(wl0.T / secs / 1e6, 2),
+            "stream_mtokens_s": round(2 * wl0.T / secs / 1e6, 2), "alg_bytes": nbytes,
+            "alg_gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
+    return res
 
 
 def decode_chain_step(hs, sets_obj, i, layers, pdl, side):
     """One decode step through a stack of layers: the metadata build (the
-    set's builder, see DecodeSets), then one sconv_fused per layer (its own
-    cache and weight), layer l+1 convolving layer l's output.  pdl: every
-    launch on the current stream (programmatic dependent launch between
+    set's builder and mode, see DecodeSets), then one convolution per layer
+    (its own cache and weight), layer l+1 convolving layer l's output; in
+    taps mode every layer reads the step's one table, and a layer other
+    than the first reads it before its wait (the layer ahead of it on the
+    stream began only after the builder had finished).  pdl: every launch
+    on the current stream (programmatic dependent launch between
     neighbours).  Otherwise the layers alternate between the current stream
     and `side`, joined by events, so each launch waits for its predecessor
     to finish."""
     wl, s = sets_obj.wls[i], sets_obj.sets[i]
     main = torch.cuda.current_stream()
-    build = hs.sconv_seq_metadata_ahead if sets_obj.ahead else hs.sconv_seq_metadata
-    build(s["query_start_loc"], wl.R, wl.T, s["seq_idx"], s["query_start"])
+    sets_obj.step(i, fused=False)
     x, cur = s["x"], main
     for l, (cache, weight, out) in enumerate(layers):
         target = main if (pdl or l % 2 == 0) else side
@@ -696,8 +851,13 @@ def decode_chain_step(hs, sets_obj, i, layers, pdl, side):
             ev.record(cur)
             target.wait_event(ev)
         with torch.cuda.stream(target):
-            hs.sconv_fused(x, weight, cache, s["positions"], s["block_table"], s["seq_idx"],
-                           s["slot_mapping"], s["query_start"], out=out, **wl.kwargs())
+            if sets_obj.mode == "taps":
+                hs.sconv_fused_taps(x, weight, cache, s["slot_mapping"], s["taps"], out=out,
+                                    metadata_ready=l > 0, **wl.kwargs())
+            else:
+                hs.sconv_fused(x, weight, cache, s["positions"], s["block_table"],
+                               s["seq_idx"], s["slot_mapping"], s["query_start"], out=out,
+                               **wl.kwargs())
         cur, x = target, out
     if cur is not main:
         ev = torch.cuda.Event()
@@ -709,11 +869,12 @@ def bench_decode_chain(sets_obj, stream, peak, n_layers=4, reps=50):
     """The decode workload through a stack of n_layers layers (each its own
     4.2 GB cache and weight; layer l+1 convolves layer l's output, the chain
     a model's decode step runs, without the projections between), over the
-    96 rotating sets.  Timed with every launch on one stream (PDL: a launch
-    becomes resident while its predecessor runs and prefetches its
-    metadata, block-table lines and cache taps before waiting) and with the
-    layers alternating between two streams joined by events (each launch
-    starts only when its predecessor has finished)."""
+    96 rotating sets, in both modes (taps: one table per step read by every
+    layer; paged: every layer resolves its taps itself).  Timed with every
+    launch on one stream (PDL: a launch becomes resident while its
+    predecessor runs and prefetches before waiting) and with the layers
+    alternating between two streams joined by events (each launch starts
+    only when its predecessor has finished)."""
     import hybrid_sconv_b200 as hs
     dev = sets_obj.device
     w0 = sets_obj.wls[0]
@@ -729,21 +890,30 @@ def bench_decode_chain(sets_obj, stream, peak, n_layers=4, reps=50):
         layers.append((cache, weight, torch.zeros((w0.T, w0.C), dtype=torch.bfloat16, device=dev)))
     side = torch.cuda.Stream(dev)
     n = len(sets_obj.sets)
-    res = {}
-    for mode, pdl in (("pdl", True), ("serialised", False)):
-        secs = _kernel_time([lambda i=i: decode_chain_step(hs, sets_obj, i, layers, pdl, side)
-                             for i in range(n)], reps, stream)
-        res[mode] = secs
+    saved = sets_obj.mode
+    table = {}
+    for mode, key in (("taps", f"decode_chain_{n_layers}_layers"),
+                      ("paged", f"decode_chain_{n_layers}_layers_paged")):
+        sets_obj.mode = mode
+        res = {}
+        for kind, pdl in (("pdl", True), ("serialised", False)):
+            res[kind] = _kernel_time([lambda i=i: decode_chain_step(hs, sets_obj, i, layers, pdl,
+                                                                    side)
+                                      for i in range(n)], reps, stream)
+        table[key] = {
+            "step_us_pdl": round(res["pdl"] * 1e6, 3),
+            "step_us_serialised": round(res["serialised"] * 1e6, 3),
+            "layer_us_pdl": round(res["pdl"] * 1e6 / n_layers, 3),
+            "layer_us_serialised": round(res["serialised"] * 1e6 / n_layers, 3),
+            "mtokens_s_layers": round(w0.T * n_layers / res["pdl"] / 1e6, 2),
+            "launches_per_step": 1 + n_layers,
+            "metadata": ("sconv_seq_metadata_taps" if mode == "taps" else "sconv_seq_metadata")
+                        + ("_ahead" if sets_obj.ahead else ""),
+            "conv": "sconv_fused_taps" if mode == "taps" else "sconv_fused"}
+    sets_obj.mode = saved
     del layers
     torch.cuda.empty_cache()
-    return {f"decode_chain_{n_layers}_layers": {
-        "step_us_pdl": round(res["pdl"] * 1e6, 3),
-        "step_us_serialised": round(res["serialised"] * 1e6, 3),
-        "layer_us_pdl": round(res["pdl"] * 1e6 / n_layers, 3),
-        "layer_us_serialised": round(res["serialised"] * 1e6 / n_layers, 3),
-        "mtokens_s_layers": round(w0.T * n_layers / res["pdl"] / 1e6, 2),
-        "launches_per_step": 1 + n_layers,
-        "metadata": "sconv_seq_metadata_ahead" if sets_obj.ahead else "sconv_seq_metadata"}}
+    return table
 
 
 def bench_ssm_gather(device, stream, peak, reps=50):
@@ -848,10 +1018,12 @@ def bench_dense(device, stream, peak):
     return table
 
 
-def per_workload_table(device, stream, peak, sets_obj=None):
+def per_workload_table(device, stream, peak, sets_obj=None, zero_sets=None):
     table = {}
     if sets_obj is not None:
         table.update(bench_serial_step(sets_obj, stream, peak))
+        table.update(bench_decode_kernels(sets_obj, stream, peak, zero_sets))
+        table.update(bench_metadata_kernels(sets_obj, stream))
         table.update(bench_update(sets_obj, stream, peak))
         table.update(bench_streams(sets_obj, stream, peak))
         table.update(bench_decode_chain(sets_obj, stream, peak))
@@ -965,8 +1137,8 @@ def e2e(sets_obj, K, stream, world, flush):
     """End to end through the public API with host buffers.  Every step
     copies its inputs (x, positions, slot_mapping, block_table,
     query_start_loc) from pinned host memory to the device, builds the
-    metadata, runs the fused step and copies its output back to pinned host
-    memory.  The inputs of a step travel as one copy (they sit back to back
+    metadata and tap table, runs the fused step and copies its output back
+    to pinned host memory.  The inputs of a step travel as one copy (they sit back to back
     in one pinned buffer and are used in place on the device), since every
     copy has a fixed cost of microseconds on top of its bytes (measured:
     five copies per step 5.9 Mtok/s, one 9.7, the one copy split over two
@@ -992,11 +1164,12 @@ def e2e(sets_obj, K, stream, world, flush):
             with torch.cuda.stream(up):
                 p["dev"].copy_(p["host"], non_blocking=True)
             cur.wait_stream(up)
-            hs.sconv_seq_metadata(v["query_start_loc"], wl.R, wl.T, s["seq_idx"],
-                                  s["query_start"])
-            hs.sconv_fused(v["x"], sets_obj.weight, sets_obj.cache, v["positions"],
-                           v["block_table"], s["seq_idx"], v["slot_mapping"], s["query_start"],
-                           out=s["out"], **wl.kwargs())
+            hs.sconv_seq_metadata_taps(v["query_start_loc"], wl.R, wl.T, v["positions"],
+                                       v["slot_mapping"], v["block_table"], wl.num_blocks,
+                                       wl.N, wl.W, seq_idx_out=s["seq_idx"],
+                                       query_start_out=s["query_start"], taps_out=s["taps"])
+            hs.sconv_fused_taps(v["x"], sets_obj.weight, sets_obj.cache, v["slot_mapping"],
+                                s["taps"], out=s["out"], **wl.kwargs())
             down.wait_stream(cur)
             with torch.cuda.stream(down):
                 p["out_host"].copy_(s["out"], non_blocking=True)
@@ -1024,12 +1197,13 @@ def config_block(world, l2):
                         "SiLU + residual",
             "global_batch": 256 * world, "seq_len": 1,
             "parallelism": f"dp{world}" if world > 1 else "single",
-            "step": "sconv_seq_metadata_ahead + sconv_fused",
-            "pipelining": "the next step's metadata build runs beside the current "
-                          "step's sconv_fused (engine-style input preparation); the "
-                          "convolutions run in order, each waiting for the previous one",
-            "metadata": "sconv_seq_metadata_ahead: one metadata buffer set per step, so the "
-                        "lookup may run before the launch's wait on its predecessors",
+            "step": STEP_CALLS[STEP_MODE],
+            "pipelining": "the next step's metadata is built on a second stream beside the "
+                          "current step's convolution, as a serving engine prepares step "
+                          "i+1's inputs while step i runs; the convolutions run in order, "
+                          "each waiting for the previous one",
+            "metadata": "one metadata buffer set per step, so the *_ahead builder may look "
+                        "up before the launch's wait on its predecessors",
             "l2": l2}
 
 
@@ -1118,16 +1292,16 @@ def main():
     K, W = args.steps, max(3, args.warmup)
 
     sets_obj = DecodeSets(args.sets, rank_seed(args.seed, rank), device, args.max_hist,
-                          ahead=True)
+                          ahead=True, mode=STEP_MODE)
     flush = L2Flush(device)
 
     # warm-up, then exactly K timed steps
-    wfull, wtail, wreps = run_steps_graphs(sets_obj, W, stream, pipeline=True)
+    wfull, wtail, wreps = run_steps_graphs(sets_obj, W, stream, pipeline=STEP_SCHEDULE)
     with torch.cuda.stream(stream):
         replay_steps(wfull, wtail, wreps)
     torch.cuda.synchronize()
     del wfull, wtail
-    full, tail, reps = run_steps_graphs(sets_obj, K, stream, pipeline=True)
+    full, tail, reps = run_steps_graphs(sets_obj, K, stream, pipeline=STEP_SCHEDULE)
     prime(full, tail, stream)
     sampler = ClockSampler(local) if rank == 0 else None
     secs, (w0, w1) = time_region(full, tail, reps, stream, world, sampler, flush)
@@ -1142,7 +1316,7 @@ def main():
             load = ClockSampler(local)
             if full is None:
                 full, _, _ = run_steps_graphs(sets_obj, len(sets_obj.sets), stream,
-                                              pipeline=True)
+                                              pipeline=STEP_SCHEDULE)
                 prime(full, None, stream)
             n = max(1, int(2.0 / max(secs / K * len(sets_obj.sets), 1e-6)))
             _, (l0, l1) = time_region(full, None, n, stream, 1, load)
@@ -1154,9 +1328,9 @@ def main():
     value = tokens / secs / 1e6
     step_bytes = sum_over_ranks(float(np.mean(sets_obj.alg_bytes)) * K, world)
 
-    # the fused kernel's own average launch duration
+    # the convolution kernel's own average launch duration
     avg = fused_launch_duration(sets_obj, stream)
-    bytes_per_launch = float(np.mean(sets_obj.alg_bytes))
+    bytes_per_launch = float(np.mean(sets_obj.kernel_alg_bytes()))
     achieved = bytes_per_launch / avg / 1e9
     traffic = profiled_traffic(HEADLINE)
 
@@ -1172,7 +1346,8 @@ def main():
         "gpu_launches": 2 * K,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": traffic, "kernel": "fused_token_kernel (sconv_fused, decode sizes)",
+                     "traffic": traffic,
+                     "kernel": STEP_KERNEL[STEP_MODE],
                      "alg_bytes_per_launch": int(bytes_per_launch),
                      "launch_us": round(avg * 1e6, 3),
                      "kernel_source_sha256_16": kernel_source_hash(),
@@ -1184,7 +1359,10 @@ def main():
     if not args.no_extras:
         line["e2e"] = e2e(sets_obj, min(K, 24000), stream, world, flush)
         if rank == 0:
-            line["per_config"] = per_workload_table(device, stream, peak, sets_obj)
+            zero = DecodeSets(args.sets, rank_seed(args.seed, rank) + 1, device, max_hist=0,
+                              min_hist=0)
+            line["per_config"] = per_workload_table(device, stream, peak, sets_obj, zero)
+            del zero
         if rank == 0 and world == 1:
             line["cpu_baseline"] = cpu_baseline(sets_obj)
     if rank == 0:

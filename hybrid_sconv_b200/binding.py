@@ -73,6 +73,16 @@ _SIGNATURES = {
     "sconv_extract_windows": [
         _P, _I64, _INT, _I64, _I64, _P, _P, _INT, _P, _I64, _INT, _INT, _P],
     "sconv_seq_metadata": [_P, _INT, _INT, _INT, _P, _I64, _P, _I64, _P],
+    "sconv_seq_metadata_taps": [
+        _P, _INT, _INT, _INT, _P, _P, _P, _I64, _INT, _I64, _INT, _INT,
+        _P, _I64, _P, _I64, _P, _I64, _P],
+    "sconv_seq_metadata_taps_ahead": [
+        _P, _INT, _INT, _INT, _P, _P, _P, _I64, _INT, _I64, _INT, _INT,
+        _P, _I64, _P, _I64, _P, _I64, _P],
+    "sconv_fused_taps": [
+        ctypes.POINTER(StreamDesc), _INT, _INT, _INT,
+        _P, _I64P, _I64, _INT, _INT, _INT,
+        _P, _P, _INT, _INT, _P, _P],
     "sconv_seq_metadata_ahead": [_P, _INT, _INT, _INT, _P, _I64, _P, _I64, _P],
     "sconv_scatter_intermediate_ssm": [
         _P, _I64, _I64, _I64, _P, _P, _INT, _P, _I64, _INT, _P, _P],
@@ -441,6 +451,145 @@ def sconv_seq_metadata_ahead(query_start_loc, num_reqs, num_actual_tokens, seq_i
     one metadata buffer set per step in flight."""
     _seq_metadata("sconv_seq_metadata_ahead", query_start_loc, num_reqs, num_actual_tokens,
                   seq_idx_out, query_start_out, num_padded_tokens, stream)
+
+
+# Entries of the resolved tap table (SCONV_TAP_* in sconv.h).
+TAP_ZERO, TAP_X = -1, -2
+
+
+def _seq_metadata_taps(name, query_start_loc, num_reqs, num_actual_tokens, positions,
+                       slot_mapping, block_table, num_blocks, block_size, W, seq_idx_out,
+                       query_start_out, taps_out, num_padded_tokens, stream):
+    if num_padded_tokens is None:
+        num_padded_tokens = num_actual_tokens
+    if taps_out is None:
+        taps_out = torch.empty((num_padded_tokens, max(W - 1, 0)), dtype=torch.int64,
+                               device=positions.device)
+    d = _dev(positions, slot_mapping, block_table, query_start_loc, seq_idx_out,
+             query_start_out, taps_out)
+    _vector(positions, torch.int64, "positions", num_actual_tokens)
+    _vector(slot_mapping, torch.int64, "slot_mapping", num_actual_tokens)
+    _want(block_table, torch.int32, "block_table")
+    if block_table.dim() != 2 or block_table.stride(1) != 1:
+        raise ValueError("block_table must be [rows, max_blocks] with unit inner stride")
+    if query_start_loc is not None:
+        _vector(query_start_loc, torch.int32, "query_start_loc", num_reqs + 1)
+    for t, nm in ((seq_idx_out, "seq_idx_out"), (query_start_out, "query_start_out")):
+        if t is not None:
+            _vector(t, torch.int32, nm, num_padded_tokens)
+    _want(taps_out, torch.int64, "taps_out")
+    if not taps_out.is_contiguous():
+        raise ValueError("taps_out must be contiguous")
+    with torch.cuda.device(d):
+        st = getattr(LIB, name)(
+            _ptr(query_start_loc), num_reqs, num_actual_tokens, num_padded_tokens,
+            _ptr(positions), _ptr(slot_mapping), _ptr(block_table), block_table.stride(0),
+            block_table.shape[1], num_blocks, block_size, W,
+            _ptr(seq_idx_out), seq_idx_out.numel() if seq_idx_out is not None else 0,
+            _ptr(query_start_out), query_start_out.numel() if query_start_out is not None else 0,
+            _ptr(taps_out), taps_out.numel(), _stream(d, stream))
+    _check(name, st, value_error=True)
+    return taps_out
+
+
+def sconv_seq_metadata_taps(query_start_loc, num_reqs, num_actual_tokens, positions,
+                            slot_mapping, block_table, num_blocks, block_size, W, *,
+                            seq_idx_out=None, query_start_out=None, taps_out=None,
+                            num_padded_tokens=None, stream=None):
+    """sconv_seq_metadata plus every token's pre-forward taps resolved into
+    a [num_padded, W-1] int64 table (sconv_seq_metadata_taps in sconv.h):
+    TAP_X for a same-forward x row, TAP_ZERO before position 0, the flat
+    cache slot of a pre-forward tap, or -(flags << 8) for a token that cannot
+    be resolved.  ``query_start_loc`` None is the decode form (token t is
+    request t, ``num_reqs`` the block-table rows).  seq_idx_out /
+    query_start_out are written when given.  Returns the table."""
+    return _seq_metadata_taps("sconv_seq_metadata_taps", query_start_loc, num_reqs,
+                              num_actual_tokens, positions, slot_mapping, block_table,
+                              num_blocks, block_size, W, seq_idx_out, query_start_out, taps_out,
+                              num_padded_tokens, stream)
+
+
+def sconv_seq_metadata_taps_ahead(query_start_loc, num_reqs, num_actual_tokens, positions,
+                                  slot_mapping, block_table, num_blocks, block_size, W, *,
+                                  seq_idx_out=None, query_start_out=None, taps_out=None,
+                                  num_padded_tokens=None, stream=None):
+    """sconv_seq_metadata_taps with its work done before the launch waits
+    for the kernels ahead of it on the stream (same precondition as
+    sconv_seq_metadata_ahead, extended to positions, slot_mapping, the block
+    table and the table)."""
+    return _seq_metadata_taps("sconv_seq_metadata_taps_ahead", query_start_loc, num_reqs,
+                              num_actual_tokens, positions, slot_mapping, block_table,
+                              num_blocks, block_size, W, seq_idx_out, query_start_out, taps_out,
+                              num_padded_tokens, stream)
+
+
+def sconv_fused_streams_taps(streams, cache, slot_mapping, taps, block_size, *,
+                             metadata_ready=False, err_flag=None, stream=None):
+    """The fused step of sconv_fused_streams with every token's taps read
+    from a table of sconv_seq_metadata_taps (sconv_fused_taps in sconv.h).
+    ``streams`` as in sconv_fused_streams.  metadata_ready=True lets the
+    launch read slot_mapping and the table before waiting for the kernels
+    it depends on; the caller guarantees the precondition sconv.h states
+    (e.g. another call of this library, not an *_ahead builder, between
+    the builder and this call on one stream; an event join from another
+    stream does not suffice under graph capture).  Returns the outputs."""
+    if not 1 <= len(streams) <= MAX_STREAMS:
+        raise ValueError(f"1..{MAX_STREAMS} streams per call")
+    x0 = streams[0]["x"]
+    dt = _float_common(x0, streams[0]["weight"], cache)
+    T = x0.shape[0]
+    W = streams[0]["weight"].shape[1]
+    outs = []
+    descs = (StreamDesc * len(streams))()
+    for i, sd in enumerate(streams):
+        x, w = sd["x"], sd["weight"]
+        _float_common(x, w, cache)
+        if x.shape[0] != T or w.shape[1] != W:
+            raise ValueError("all streams share T and W")
+        out = sd.get("out")
+        if out is None:
+            out = torch.empty_like(x)
+        if out.dtype != x.dtype or tuple(out.shape) != tuple(x.shape) or (T and out.stride(1) != 1):
+            raise ValueError("out must be [T, C] like x with unit channel stride")
+        outs.append(out)
+        descs[i] = StreamDesc(_ptr(x), x.stride(0), _ptr(w), w.stride(0), w.stride(1), _ptr(out),
+                              out.stride(0), sd["off_s"], sd["ws"], _act(sd.get("activation")),
+                              int(bool(sd.get("use_residual", True))))
+    if T == 0:
+        return outs
+    d = _dev(x0, cache, slot_mapping, taps, err_flag, *[sd["x"] for sd in streams],
+             *[sd["weight"] for sd in streams], *outs)
+    _vector(slot_mapping, torch.int64, "slot_mapping", T)
+    if W > 1:
+        _want(taps, torch.int64, "taps")
+        if taps.dim() != 2 or taps.shape[0] < T or taps.shape[1] != W - 1 or \
+                not taps.is_contiguous():
+            raise ValueError("taps must be a contiguous [>= T, W-1] int64 table")
+    if err_flag is not None:
+        _vector(err_flag, torch.int32, "err_flag", 1)
+    if cache.shape[2] != block_size:
+        raise ValueError("cache.shape[2] must equal block_size")
+    nb, H, N, D = cache.shape
+    cs = (ctypes.c_int64 * 4)(*cache.stride())
+    with torch.cuda.device(d):
+        st = LIB.sconv_fused_taps(
+            descs, len(streams), T, W, _ptr(cache), cs, nb, H, N, D, _ptr(slot_mapping),
+            _ptr(taps) if W > 1 else 0, int(bool(metadata_ready)), dt, _ptr(err_flag),
+            _stream(d, stream))
+    _check("sconv_fused_taps", st)
+    return outs
+
+
+def sconv_fused_taps(x, weight, cache, slot_mapping, taps, off_s, ws, block_size,
+                     activation=None, use_residual=True, *, out=None, metadata_ready=False,
+                     err_flag=None, stream=None):
+    """sconv_fused with the tap sources read from a table built by
+    sconv_seq_metadata_taps for the same step (one conv stream).  Same
+    result as sconv_fused on the metadata the table was built from."""
+    return sconv_fused_streams_taps(
+        [dict(x=x, weight=weight, off_s=off_s, ws=ws, activation=activation,
+              use_residual=use_residual, out=out)], cache, slot_mapping, taps, block_size,
+        metadata_ready=metadata_ready, err_flag=err_flag, stream=stream)[0]
 
 
 def _dense_common(x, weight, bias, states, out, err_flag, states_name):

@@ -33,7 +33,7 @@ sconv_status check_fused(const void *x, int64_t x_rs, int T, int C, const void *
                          const int64_t *slot_mapping, const int32_t *block_table, int64_t bt_rs,
                          int num_reqs, int max_blocks, int off_s, int ws, sconv_act act,
                          int use_residual, sconv_dtype dt, void *out, int64_t out_rs,
-                         int32_t *err_flag, FusedArgs &a, bool &vec) {
+                         int32_t *err_flag, FusedArgs &a, bool &vec, bool paged = true) {
     if (dt != SCONV_F32 && dt != SCONV_BF16) return SCONV_ERR_UNSUPPORTED;
     if (W < 1) return SCONV_ERR_INVALID;
     if (W > SCONV_MAX_W) return SCONV_ERR_UNSUPPORTED;
@@ -41,11 +41,15 @@ sconv_status check_fused(const void *x, int64_t x_rs, int T, int C, const void *
     if (C < 1 || H < 1 || N < 1 || D < 1 || ws < 1 || off_s < 0) return SCONV_ERR_INVALID;
     if (static_cast<int64_t>(off_s) + ws > D) return SCONV_ERR_INVALID;
     if (static_cast<int64_t>(H) * ws != C) return SCONV_ERR_INVALID;
-    if (num_blocks < 1 || num_reqs < 1 || max_blocks < 1) return SCONV_ERR_INVALID;
-    if (!x || !weight || !cache || !cs || !positions || !slot_mapping || !block_table || !out)
+    if (num_blocks < 1) return SCONV_ERR_INVALID;
+    if (!x || !weight || !cache || !cs || !slot_mapping || !out) return SCONV_ERR_INVALID;
+    // paged: the call reads positions and the block table itself (every
+    // form but sconv_fused_taps, whose taps come resolved)
+    if (paged && (num_reqs < 1 || max_blocks < 1 || !positions || !block_table ||
+                  bt_rs < max_blocks))
         return SCONV_ERR_INVALID;
     if (cs[3] != 1 || cs[0] < 1 || cs[1] < 1 || cs[2] < 1) return SCONV_ERR_INVALID;
-    if (x_rs < C || out_rs < C || bt_rs < max_blocks) return SCONV_ERR_INVALID;
+    if (x_rs < C || out_rs < C) return SCONV_ERR_INVALID;
     if (w_sc < 0 || w_sk < 0) return SCONV_ERR_INVALID;
 
     const int64_t e = elem_size(dt);
@@ -94,6 +98,7 @@ sconv_status check_fused(const void *x, int64_t x_rs, int T, int C, const void *
     a.out = out;
     a.out_rs = out_rs;
     a.err = err_flag;
+    a.taps = nullptr;
     return SCONV_OK;
 }
 
@@ -281,6 +286,50 @@ sconv_status sconv_fused_streams(const sconv_stream_desc *streams, int n_streams
     }
     return sconv::launch_fused_streams(a, n_streams, dt == SCONV_BF16, vec_all, stream) ==
                    cudaSuccess
+               ? SCONV_OK
+               : SCONV_ERR_LAUNCH;
+}
+
+sconv_status sconv_fused_taps(const sconv_stream_desc *streams, int n_streams, int T, int W,
+                              void *cache, const int64_t cache_strides[4], int64_t num_blocks,
+                              int H, int N, int D, const int64_t *slot_mapping,
+                              const int64_t *taps, int metadata_ready, sconv_dtype dt,
+                              int32_t *err_flag, cudaStream_t stream) {
+    if (T < 0 || n_streams < 1 || !streams) return SCONV_ERR_INVALID;
+    if (n_streams > SCONV_MAX_STREAMS) return SCONV_ERR_UNSUPPORTED;
+    if (T == 0) return SCONV_OK;
+    if (W > 1 && !taps) return SCONV_ERR_INVALID;
+    FusedArgs a[SCONV_MAX_STREAMS];
+    bool vec_all = true;
+    const int64_t e = elem_size(dt);
+    const int64_t taps_bytes = static_cast<int64_t>(T) * (W > 1 ? W - 1 : 0) * 8;
+    for (int i = 0; i < n_streams; ++i) {
+        const sconv_stream_desc &d = streams[i];
+        bool vec = false;
+        const sconv_status st = check_fused(
+            d.x, d.x_row_stride, T, H * d.ws, d.weight, d.w_stride_c, d.w_stride_k, W, cache,
+            cache_strides, num_blocks, H, N, D, nullptr, slot_mapping, nullptr, 0, 0, 0,
+            d.off_s, d.ws, d.act, d.use_residual, dt, d.out, d.out_row_stride, err_flag, a[i],
+            vec, false);
+        if (st != SCONV_OK) return st;
+        a[i].taps = taps;
+        vec_all = vec_all && vec;
+        const int64_t out_bytes =
+            ((static_cast<int64_t>(T) - 1) * d.out_row_stride + H * d.ws) * e;
+        if (taps_bytes && overlaps(d.out, out_bytes, taps, taps_bytes)) return SCONV_ERR_INVALID;
+        for (int j = 0; j < i; ++j) {
+            const sconv_stream_desc &o = streams[j];
+            if (d.off_s < o.off_s + o.ws && o.off_s < d.off_s + d.ws) return SCONV_ERR_INVALID;
+            const int64_t o_out = ((static_cast<int64_t>(T) - 1) * o.out_row_stride + H * o.ws) * e;
+            const int64_t o_x = ((static_cast<int64_t>(T) - 1) * o.x_row_stride + H * o.ws) * e;
+            const int64_t d_x = ((static_cast<int64_t>(T) - 1) * d.x_row_stride + H * d.ws) * e;
+            if (overlaps(d.out, out_bytes, o.out, o_out) || overlaps(d.out, out_bytes, o.x, o_x) ||
+                overlaps(o.out, o_out, d.x, d_x))
+                return SCONV_ERR_INVALID;
+        }
+    }
+    return sconv::launch_fused_taps(a, n_streams, dt == SCONV_BF16, vec_all,
+                                    metadata_ready != 0, stream) == cudaSuccess
                ? SCONV_OK
                : SCONV_ERR_LAUNCH;
 }
@@ -517,6 +566,76 @@ sconv_status seq_metadata(const int32_t *query_start_loc, int num_reqs, int num_
                : SCONV_ERR_LAUNCH;
 }
 }  // namespace
+
+namespace {
+sconv_status seq_metadata_taps(const int32_t *qsl, int num_reqs, int num_actual,
+                               int num_padded, const int64_t *positions,
+                               const int64_t *slot_mapping, const int32_t *block_table,
+                               int64_t bt_rs, int max_blocks, int64_t num_blocks, int N, int W,
+                               int32_t *seq_idx_out, int64_t seq_idx_cap,
+                               int32_t *query_start_out, int64_t query_start_cap,
+                               int64_t *taps_out, int64_t taps_cap, bool ahead,
+                               cudaStream_t stream) {
+    if (num_padded < 0) num_padded = num_actual;
+    if (num_actual < 0 || num_reqs < 0 || num_padded < num_actual) return SCONV_ERR_INVALID;
+    if (W < 1) return SCONV_ERR_INVALID;
+    if (W > SCONV_MAX_W) return SCONV_ERR_UNSUPPORTED;
+    if (N < 1 || num_blocks < 1 || max_blocks < 1 || bt_rs < max_blocks) return SCONV_ERR_INVALID;
+    if (num_actual > 0 && num_reqs < 1) return SCONV_ERR_INVALID;
+    if ((seq_idx_out && num_padded > seq_idx_cap) ||
+        (query_start_out && num_padded > query_start_cap))
+        return SCONV_ERR_INVALID;
+    if (static_cast<int64_t>(num_padded) * (W - 1) > taps_cap) return SCONV_ERR_INVALID;
+    if (num_padded == 0) return SCONV_OK;
+    if ((W > 1 && !taps_out) || (num_actual > 0 && (!positions || !slot_mapping || !block_table)))
+        return SCONV_ERR_INVALID;
+    if (W == 1 && !seq_idx_out && !query_start_out) return SCONV_OK;  // nothing to write
+    sconv::TapResolveArgs a = {};
+    a.qsl = qsl;
+    a.num_reqs = num_reqs;
+    a.num_actual = num_actual;
+    a.num_padded = num_padded;
+    a.positions = positions;
+    a.slot = slot_mapping;
+    a.bt = block_table;
+    a.bt_rs = bt_rs;
+    a.max_blocks = max_blocks;
+    a.num_blocks = num_blocks;
+    a.N = N;
+    a.W = W;
+    a.seq_idx = seq_idx_out;
+    a.qstart = query_start_out;
+    a.taps = taps_out;
+    return sconv::launch_seq_metadata_taps(a, ahead, stream) == cudaSuccess ? SCONV_OK
+                                                                            : SCONV_ERR_LAUNCH;
+}
+}  // namespace
+
+sconv_status sconv_seq_metadata_taps(const int32_t *query_start_loc, int num_reqs,
+                                     int num_actual_tokens, int num_padded_tokens,
+                                     const int64_t *positions, const int64_t *slot_mapping,
+                                     const int32_t *block_table, int64_t bt_row_stride,
+                                     int max_blocks, int64_t num_blocks, int N, int W,
+                                     int32_t *seq_idx_out, int64_t seq_idx_cap,
+                                     int32_t *query_start_out, int64_t query_start_cap,
+                                     int64_t *taps_out, int64_t taps_cap, cudaStream_t stream) {
+    return seq_metadata_taps(query_start_loc, num_reqs, num_actual_tokens, num_padded_tokens,
+                             positions, slot_mapping, block_table, bt_row_stride, max_blocks,
+                             num_blocks, N, W, seq_idx_out, seq_idx_cap, query_start_out,
+                             query_start_cap, taps_out, taps_cap, false, stream);
+}
+
+sconv_status sconv_seq_metadata_taps_ahead(
+    const int32_t *query_start_loc, int num_reqs, int num_actual_tokens, int num_padded_tokens,
+    const int64_t *positions, const int64_t *slot_mapping, const int32_t *block_table,
+    int64_t bt_row_stride, int max_blocks, int64_t num_blocks, int N, int W,
+    int32_t *seq_idx_out, int64_t seq_idx_cap, int32_t *query_start_out,
+    int64_t query_start_cap, int64_t *taps_out, int64_t taps_cap, cudaStream_t stream) {
+    return seq_metadata_taps(query_start_loc, num_reqs, num_actual_tokens, num_padded_tokens,
+                             positions, slot_mapping, block_table, bt_row_stride, max_blocks,
+                             num_blocks, N, W, seq_idx_out, seq_idx_cap, query_start_out,
+                             query_start_cap, taps_out, taps_cap, true, stream);
+}
 
 sconv_status sconv_seq_metadata(const int32_t *query_start_loc, int num_reqs,
                                 int num_actual_tokens, int num_padded_tokens,

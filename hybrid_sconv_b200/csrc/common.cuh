@@ -226,6 +226,23 @@ struct FusedArgs {
     int64_t out_rs;
     int32_t *err;
     int strip;        // tokens per thread in the strip kernel
+    const int64_t *taps;  // resolved tap table [T, W-1] (sconv_fused_taps only)
+};
+
+// The per-step tap resolution (sconv_seq_metadata_taps).
+struct TapResolveArgs {
+    const int32_t *qsl;       // [num_reqs + 1], or nullptr: token t is request t
+    int num_reqs, num_actual, num_padded;
+    const int64_t *positions, *slot;
+    const int32_t *bt;
+    int64_t bt_rs;
+    int max_blocks;
+    int64_t num_blocks;
+    int N, W;
+    FastDiv divN;
+    int32_t *seq_idx, *qstart;  // either may be nullptr
+    int64_t *taps;              // [num_padded, W-1]
+    int staged;                 // query_start_loc staged in shared memory
 };
 
 struct ExtractArgs {
@@ -320,6 +337,11 @@ cudaError_t launch_dense_update(const DenseArgs &a, bool bf16_data, bool vec,
 cudaError_t launch_seq_metadata(const int32_t *qsl, int num_reqs, int num_actual, int num_padded,
                                 int32_t *seq_idx, int32_t *query_start, bool ahead,
                                 cudaStream_t stream);
+cudaError_t launch_seq_metadata_taps(TapResolveArgs &a, bool ahead, cudaStream_t stream);
+// Several streams (n >= 1) of one layer with their taps read from a resolved
+// table; `ready`: slot_mapping and the table may be read before the wait.
+cudaError_t launch_fused_taps(FusedArgs *s, int n, bool bf16_data, bool vec, bool ready,
+                              cudaStream_t stream);
 
 // Launch with programmatic stream serialization enabled.
 template <typename Kernel, typename... Args>

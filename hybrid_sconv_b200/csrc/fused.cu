@@ -46,9 +46,9 @@ constexpr int kThreads = 256;
 // tap_of(d, use) returns the tap at lag d and sets `use` false for a tap
 // that is zero (before position 0).
 template <typename E, int VEC, int MAXW, typename TapFn>
-__device__ __forceinline__ void conv_store(const FusedArgs &a, const float (&wr)[MAXW][VEC],
-                                           TapFn tap_of, const Pack<E, VEC> &cur, int t, int c,
-                                           int64_t slot, int64_t lane) {
+__device__ __forceinline__ void conv_store_at(const FusedArgs &a, const float (&wr)[MAXW][VEC],
+                                              TapFn tap_of, const Pack<E, VEC> &cur, E *out,
+                                              E *ins) {
     float acc[VEC];
 #pragma unroll
     for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
@@ -74,10 +74,19 @@ __device__ __forceinline__ void conv_store(const FusedArgs &a, const float (&wr)
     }
     Pack<E, VEC> o;
     o.from_float(acc);
-    o.store(static_cast<E *>(a.out) + static_cast<int64_t>(t) * a.out_rs + c);
+    o.store(out);
+    cur.store(ins);
+}
+
+template <typename E, int VEC, int MAXW, typename TapFn>
+__device__ __forceinline__ void conv_store(const FusedArgs &a, const float (&wr)[MAXW][VEC],
+                                           TapFn tap_of, const Pack<E, VEC> &cur, int t, int c,
+                                           int64_t slot, int64_t lane) {
     int64_t blk, off;
     split_n(a, slot, a.slots32 != 0, blk, off);
-    cur.store(static_cast<E *>(a.cache) + blk * a.cs0 + off * a.cs2 + lane);
+    conv_store_at<E, VEC, MAXW>(a, wr, tap_of, cur,
+                                static_cast<E *>(a.out) + static_cast<int64_t>(t) * a.out_rs + c,
+                                static_cast<E *>(a.cache) + blk * a.cs0 + off * a.cs2 + lane);
 }
 
 // Before the PDL wait, while the preceding kernel drains: pull token t's
@@ -204,13 +213,23 @@ struct StreamSet {
     int y0[SCONV_MAX_STREAMS + 1];  // first y block of each stream, y0[n] = total
 };
 
+// Runs f(args of stream si) with si a compile-time index in each branch, so
+// the stream's fields are read from the parameter bank at fixed offsets (an
+// index computed from blockIdx would turn every field read into an indexed
+// load).
+template <typename F>
+__device__ __forceinline__ void with_stream(const StreamSet &m, int si, F f) {
+    static_assert(SCONV_MAX_STREAMS == 4, "one branch per stream");
+    switch (si) {
+        case 0: f(m.s[0]); break;
+        case 1: f(m.s[1]); break;
+        case 2: f(m.s[2]); break;
+        default: f(m.s[3]); break;
+    }
+}
+
 template <typename E, int VEC, int MAXW, bool SPEC>
-__global__ void __launch_bounds__(kThreads) fused_streams_kernel(const __grid_constant__ StreamSet m) {
-    int si = 0;
-    while (si + 1 < m.n && static_cast<int>(blockIdx.y) >= m.y0[si + 1]) ++si;
-    const FusedArgs &a = m.s[si];
-    const int pack = (blockIdx.y - m.y0[si]) * blockDim.x + threadIdx.x;
-    const int t = blockIdx.x * blockDim.y + threadIdx.y;
+__device__ __forceinline__ void streams_body(const FusedArgs &a, int pack, int t) {
     const bool in_range = pack < a.C / VEC && t < a.T;
     float wr[MAXW][VEC];
     if (in_range) {
@@ -220,6 +239,173 @@ __global__ void __launch_bounds__(kThreads) fused_streams_kernel(const __grid_co
     pdl_wait();
     pdl_trigger();
     if (in_range) token_body<E, VEC, MAXW, false, !SPEC>(a, pack, t, wr);
+}
+
+template <typename E, int VEC, int MAXW, bool SPEC>
+__global__ void __launch_bounds__(kThreads) fused_streams_kernel(const __grid_constant__ StreamSet m) {
+    int si = 0;
+    while (si + 1 < m.n && static_cast<int>(blockIdx.y) >= m.y0[si + 1]) ++si;
+    const int pack = (blockIdx.y - m.y0[si]) * blockDim.x + threadIdx.x;
+    const int t = blockIdx.x * blockDim.y + threadIdx.y;
+    with_stream(m, si, [&](const FusedArgs &a) { streams_body<E, VEC, MAXW, SPEC>(a, pack, t); });
+}
+
+// ---------------------------------------------------------------------------
+// The fused step with resolved taps (sconv_fused_taps).  A token's tap
+// sources come from one row of the table sconv_seq_metadata_taps built for
+// the step: SCONV_TAP_X (x row t - d), SCONV_TAP_ZERO, a flat cache slot, or
+// a failure code carrying SCONV_EFLAG_* bits.  The kernel reads no
+// positions, request metadata or block table, so a token's taps are one
+// dependent access after its slot and table row -- and with READY those are
+// read before the PDL wait (the caller guarantees no kernel still running
+// writes them), the x rows and cache taps are prefetched into L2 there, and
+// after the wait only the x and cache loads remain.
+
+template <int MAXW>
+__device__ __forceinline__ void load_tap_row(const FusedArgs &a, int t, int64_t (&src)[MAXW]) {
+    const int64_t *row = a.taps + static_cast<int64_t>(t) * (a.W - 1);
+#pragma unroll
+    for (int d = 1; d < MAXW; ++d) src[d] = d < a.W ? __ldg(row + d - 1) : SCONV_TAP_ZERO;
+}
+
+// SCONV_EFLAG_* bits of a non-PAD token: those its table row carries (an
+// entry that is neither a valid slot, SCONV_TAP_X on a row of this call,
+// SCONV_TAP_ZERO nor a failure code counts as SCONV_EFLAG_BLOCK), or, for a
+// slot out of range, SCONV_EFLAG_SLOT with the row's request, query-start
+// and position bits -- the bits sconv_fused reports for the same token.
+template <int MAXW>
+__device__ __forceinline__ unsigned tap_row_flags(const FusedArgs &a, int t, int64_t slot,
+                                                  const int64_t (&src)[MAXW]) {
+    const int64_t limit = a.num_blocks * a.N;
+    unsigned f = 0;
+#pragma unroll
+    for (int d = 1; d < MAXW; ++d) {
+        if (d >= a.W) continue;
+        const int64_t e = src[d];
+        if (e >= 0) {
+            if (e >= limit) f |= SCONV_EFLAG_BLOCK;
+        } else if (e == SCONV_TAP_X) {
+            if (t - d < 0) f |= SCONV_EFLAG_QUERY_START;
+        } else if (e != SCONV_TAP_ZERO) {
+            const unsigned bits =
+                e <= -256 ? static_cast<unsigned>((~static_cast<uint64_t>(e) + 1) >> 8) & 0x3fu
+                          : 0u;
+            f |= bits ? bits : SCONV_EFLAG_BLOCK;
+        }
+    }
+    if (slot < 0 || slot >= limit)
+        f = SCONV_EFLAG_SLOT |
+            (f & (SCONV_EFLAG_REQUEST | SCONV_EFLAG_QUERY_START | SCONV_EFLAG_POSITION));
+    return f;
+}
+
+// One token-pack of the resolved-tap form (pack, token t).  With READY the
+// slot and table row are read before the PDL wait and the token's cache taps
+// prefetched into L2 there; after the wait come the checks, the tap loads,
+// the arithmetic and the two stores.  (Measured: this straight-line shape
+// beats a form that carries precomputed addresses across the wait, 3.2 ->
+// 2.4 us per decode launch.)  Without READY the table row is read
+// speculatively before the wait with L2-only loads (the kernel that writes
+// it may still be running), range-checked and used only to choose which
+// cache taps to prefetch; the real reads follow the wait.
+template <typename E, int VEC, int MAXW, bool READY>
+__device__ __forceinline__ void taps_body(const FusedArgs &a, int pack, int t) {
+    using P = Pack<E, VEC>;
+    const bool in_range = pack < a.C / VEC && t < a.T;
+    const int c = pack * VEC;
+    const int h = c / a.ws;
+    const int64_t lane = static_cast<int64_t>(h) * a.cs1 + a.off_s + (c - h * a.ws);
+    const E *x = static_cast<const E *>(a.x);
+    const E *cache = static_cast<const E *>(a.cache);
+
+    float wr[MAXW][VEC];
+    int64_t slot = -1;
+    int64_t src[MAXW];
+    if (in_range) {
+        load_weights<E, VEC, MAXW>(a, c, wr);
+        prefetch_l2(x + static_cast<int64_t>(t) * a.x_rs + c);
+        if (READY) {
+            slot = __ldg(a.slot + t);
+            load_tap_row<MAXW>(a, t, src);
+            const int64_t limit = a.num_blocks * a.N;
+#pragma unroll
+            for (int d = 1; d < MAXW; ++d) {
+                if (src[d] >= 0 && src[d] < limit) {
+                    int64_t blk, off;
+                    split_n(a, src[d], a.slots32 != 0, blk, off);
+                    prefetch_l2(cache + blk * a.cs0 + off * a.cs2 + lane);
+                }
+            }
+        } else {
+            const int64_t *row = a.taps + static_cast<int64_t>(t) * (a.W - 1);
+            const int64_t limit = a.num_blocks * a.N;
+#pragma unroll
+            for (int d = 1; d < MAXW; ++d) {
+                if (d >= a.W) continue;
+                const int64_t e = __ldcg(row + d - 1);
+                if (e >= 0 && e < limit) {
+                    int64_t blk, off;
+                    split_n(a, e, a.slots32 != 0, blk, off);
+                    prefetch_l2(cache + blk * a.cs0 + off * a.cs2 + lane);
+                }
+            }
+        }
+    }
+    pdl_wait();
+    pdl_trigger();
+    if (!in_range) return;
+    if (!READY) {
+        slot = __ldg(a.slot + t);
+        load_tap_row<MAXW>(a, t, src);
+    }
+    if (slot == -1) return;  // PAD row
+    const unsigned bad = tap_row_flags<MAXW>(a, t, slot, src);
+    if (bad) {
+        if (a.err) atomicOr(a.err, static_cast<int>(bad));
+        return;
+    }
+    P tap[MAXW];
+    bool use[MAXW];
+    tap[0].load_nc(x + static_cast<int64_t>(t) * a.x_rs + c);
+    use[0] = true;
+#pragma unroll
+    for (int d = 1; d < MAXW; ++d) {
+        use[d] = false;
+        if (src[d] >= 0) {
+            int64_t blk, off;
+            split_n(a, src[d], a.slots32 != 0, blk, off);
+            tap[d].load_nc(cache + blk * a.cs0 + off * a.cs2 + lane);
+            use[d] = true;
+        } else if (src[d] == SCONV_TAP_X) {
+            tap[d].load_nc(x + static_cast<int64_t>(t - d) * a.x_rs + c);
+            use[d] = true;
+        }
+    }
+    conv_store<E, VEC, MAXW>(
+        a, wr,
+        [&](int d, bool &u) {
+            u = use[d];
+            return tap[d];
+        },
+        tap[0], t, c, slot, lane);
+}
+
+// One conv stream: the arguments are a plain kernel parameter.
+template <typename E, int VEC, int MAXW, bool READY>
+__global__ void __launch_bounds__(kThreads) fused_taps_kernel(const __grid_constant__ FusedArgs a) {
+    taps_body<E, VEC, MAXW, READY>(a, blockIdx.y * blockDim.x + threadIdx.x,
+                                   blockIdx.x * blockDim.y + threadIdx.y);
+}
+
+// Several streams of one layer in one launch: the grid's y blocks are the
+// streams' channel blocks laid end to end.
+template <typename E, int VEC, int MAXW, bool READY>
+__global__ void __launch_bounds__(kThreads) fused_taps_streams_kernel(const __grid_constant__ StreamSet m) {
+    int si = 0;
+    while (si + 1 < m.n && static_cast<int>(blockIdx.y) >= m.y0[si + 1]) ++si;
+    const int pack = (blockIdx.y - m.y0[si]) * blockDim.x + threadIdx.x;
+    const int t = blockIdx.x * blockDim.y + threadIdx.y;
+    with_stream(m, si, [&](const FusedArgs &a) { taps_body<E, VEC, MAXW, READY>(a, pack, t); });
 }
 
 // Ring of x rows: Q >= PF + MAXW slots, a power of two.
@@ -476,6 +662,39 @@ cudaError_t launch_streams_v(FusedArgs *s, int n, cudaStream_t stream) {
     return launch_streams_t<E, VEC, 8>(s, n, stream);
 }
 
+template <typename E, int VEC, int MAXW>
+cudaError_t launch_taps_t(FusedArgs *s, int n, bool ready, cudaStream_t stream) {
+    StreamSet m;
+    m.n = n;
+    int nv_max = 0;
+    for (int i = 0; i < n; ++i) nv_max = s[i].C / VEC > nv_max ? s[i].C / VEC : nv_max;
+    const Shape sh = block_shape(nv_max, s[0].T);
+    m.y0[0] = 0;
+    for (int i = 0; i < n; ++i) {
+        s[i].w_vec = s[i].w_vec && s[i].W == MAXW;
+        m.s[i] = s[i];
+        m.y0[i + 1] = m.y0[i] + (s[i].C / VEC + sh.cv - 1) / sh.cv;
+    }
+    for (int i = n; i < SCONV_MAX_STREAMS; ++i) m.s[i] = s[0];  // never selected
+    dim3 grid(static_cast<unsigned>((s[0].T + sh.tg - 1) / sh.tg), static_cast<unsigned>(m.y0[n]));
+    const dim3 block(sh.cv, sh.tg);
+    if (n == 1)
+        return ready ? launch_pdl(fused_taps_kernel<E, VEC, MAXW, true>, grid, block, 0, stream,
+                                  m.s[0])
+                     : launch_pdl(fused_taps_kernel<E, VEC, MAXW, false>, grid, block, 0, stream,
+                                  m.s[0]);
+    return ready ? launch_pdl(fused_taps_streams_kernel<E, VEC, MAXW, true>, grid, block, 0,
+                              stream, m)
+                 : launch_pdl(fused_taps_streams_kernel<E, VEC, MAXW, false>, grid, block, 0,
+                              stream, m);
+}
+
+template <typename E, int VEC>
+cudaError_t launch_taps_v(FusedArgs *s, int n, bool ready, cudaStream_t stream) {
+    if (s[0].W <= 4) return launch_taps_t<E, VEC, 4>(s, n, ready, stream);
+    return launch_taps_t<E, VEC, 8>(s, n, ready, stream);
+}
+
 }  // namespace
 
 cudaError_t launch_fused_streams(FusedArgs *s, int n, bool bf16_data, bool vec,
@@ -499,6 +718,20 @@ cudaError_t launch_fused_streams(FusedArgs *s, int n, bool bf16_data, bool vec,
     if (bf16_data)
         return vec ? launch_streams_v<bf16, 8>(s, n, stream) : launch_streams_v<bf16, 1>(s, n, stream);
     return vec ? launch_streams_v<float, 4>(s, n, stream) : launch_streams_v<float, 1>(s, n, stream);
+}
+
+cudaError_t launch_fused_taps(FusedArgs *s, int n, bool bf16_data, bool vec, bool ready,
+                              cudaStream_t stream) {
+    for (int i = 0; i < n; ++i) {
+        s[i].divN = FastDiv::make(static_cast<uint32_t>(s[i].N));
+        s[i].slots32 = s[i].num_blocks * s[i].N < (1ll << 31);
+        s[i].strip = 1;
+    }
+    if (bf16_data)
+        return vec ? launch_taps_v<bf16, 8>(s, n, ready, stream)
+                   : launch_taps_v<bf16, 1>(s, n, ready, stream);
+    return vec ? launch_taps_v<float, 4>(s, n, ready, stream)
+               : launch_taps_v<float, 1>(s, n, ready, stream);
 }
 
 cudaError_t launch_fused(FusedArgs &a, bool bf16_data, bool vec, bool one, cudaStream_t stream) {

@@ -88,6 +88,20 @@ typedef enum sconv_act { SCONV_ACT_NONE = 0, SCONV_ACT_SILU = 1 } sconv_act;
                                          at most one mbarrier try_wait suspension); that block
                                          wrote nothing further and returned */
 
+/*
+ * Entries of the resolved tap table that sconv_seq_metadata_taps writes and
+ * sconv_fused_taps reads: one int64 per token and lag d = 1..W-1 (the tap at
+ * position pos - d), in row t at column d - 1:
+ *   >= 0             the flat cache slot block * N + offset of a pre-forward
+ *                    tap (the block/offset split slot_mapping uses);
+ *   SCONV_TAP_ZERO   a tap before position 0 (zero);
+ *   SCONV_TAP_X      a same-forward tap: x row t - d of the same call;
+ *   <= -256          the token cannot be resolved; bits 8.. of the negated
+ *                    entry are its SCONV_EFLAG_* bits (the same at every lag).
+ */
+#define SCONV_TAP_ZERO (-1)
+#define SCONV_TAP_X    (-2)
+
 #define SCONV_MAX_W 8      /* taps supported by sconv_fused / sconv_update */
 #define SCONV_MAX_STREAMS 4 /* conv streams per sconv_fused_streams call */
 #define SCONV_MAX_DCONV 8  /* window length supported by sconv_extract_windows */
@@ -396,6 +410,121 @@ sconv_status sconv_seq_metadata_ahead(
     const int32_t *query_start_loc, int num_reqs, int num_actual_tokens,
     int num_padded_tokens, int32_t *seq_idx_out, int64_t seq_idx_cap,
     int32_t *query_start_out, int64_t query_start_cap, cudaStream_t stream);
+
+/*
+ * sconv_seq_metadata_taps -- sconv_seq_metadata together with the resolution
+ * of every token's pre-forward taps into a table, in one launch.  The
+ * resolution is the tap rule of the vllm sconv page (module docstring and
+ * fused_sconv): a tap inside the current forward is read from x, an earlier
+ * one from the cache through block_table[req, src / N] at offset src % N, a
+ * tap before position 0 is zero.  Done once per step, the table serves every
+ * layer whose cache shares the block table and block size, and lets
+ * sconv_fused_taps reach a token's taps in one dependent memory access
+ * instead of three (metadata, block table, cache).
+ *
+ *   query_start_loc  [num_reqs + 1] int32 as in sconv_seq_metadata, or NULL
+ *                    for the decode form: token t is request t.
+ *   num_reqs         the requests (query_start_loc given) or the rows of
+ *                    block_table (decode form; a token t >= num_reqs is
+ *                    flagged SCONV_EFLAG_REQUEST).
+ *   positions        [num_actual_tokens] int64 absolute positions.
+ *   slot_mapping     [num_actual_tokens] int64; a PAD row (-1) is resolved
+ *                    to SCONV_TAP_ZERO at every lag and never flagged.
+ *   block_table      [num_reqs, max_blocks] int32, row stride bt_row_stride.
+ *   num_blocks, N    the cache's block count and block size.
+ *   W                taps, 1..SCONV_MAX_W (W == 1: no table, taps_out may be NULL).
+ *   seq_idx_out, query_start_out   as in sconv_seq_metadata (request index
+ *                    and its first row; t for both in the decode form);
+ *                    either may be NULL and is then not written.
+ *   taps_out         [num_padded_tokens, W - 1] int64, row-major, entries as
+ *                    SCONV_TAP_* describes; taps_cap is its element capacity.
+ *                    Rows [num_actual, num_padded) get SCONV_TAP_ZERO.
+ * A token whose own indices are out of range (request, query start,
+ * position < 0) gets those bits at every lag; otherwise, if a pre-forward
+ * tap lies past the table (src / N >= max_blocks) or on a block outside
+ * [0, num_blocks), it gets the union of those bits.
+ * Returns SCONV_ERR_INVALID (enqueuing nothing) for negative counts,
+ * num_padded_tokens < num_actual_tokens, capacities too small, a missing
+ * pointer that is needed, bt_row_stride < max_blocks, or num_reqs < 1 while
+ * num_actual_tokens > 0; SCONV_ERR_UNSUPPORTED for W outside 1..8.
+ * num_padded_tokens < 0 means num_actual_tokens; 0 rows enqueue nothing.
+ */
+sconv_status sconv_seq_metadata_taps(
+    const int32_t *query_start_loc, int num_reqs, int num_actual_tokens,
+    int num_padded_tokens, const int64_t *positions, const int64_t *slot_mapping,
+    const int32_t *block_table, int64_t bt_row_stride, int max_blocks, int64_t num_blocks,
+    int N, int W, int32_t *seq_idx_out, int64_t seq_idx_cap, int32_t *query_start_out,
+    int64_t query_start_cap, int64_t *taps_out, int64_t taps_cap, cudaStream_t stream);
+
+/*
+ * sconv_seq_metadata_taps_ahead -- sconv_seq_metadata_taps (same arguments,
+ * results and errors) with its work moved ahead of its wait on the stream,
+ * as sconv_seq_metadata_ahead does for sconv_seq_metadata, and under the
+ * same precondition, extended to every buffer it reads and writes: no
+ * kernel enqueued before this call since the stream was last fully ordered
+ * writes query_start_loc, positions, slot_mapping or block_table, or reads
+ * or writes the three outputs.
+ */
+sconv_status sconv_seq_metadata_taps_ahead(
+    const int32_t *query_start_loc, int num_reqs, int num_actual_tokens,
+    int num_padded_tokens, const int64_t *positions, const int64_t *slot_mapping,
+    const int32_t *block_table, int64_t bt_row_stride, int max_blocks, int64_t num_blocks,
+    int N, int W, int32_t *seq_idx_out, int64_t seq_idx_cap, int32_t *query_start_out,
+    int64_t query_start_cap, int64_t *taps_out, int64_t taps_cap, cudaStream_t stream);
+
+/*
+ * sconv_fused_taps -- the fused step of sconv_fused_streams (one or more
+ * conv streams of a layer; n_streams == 1 is plain sconv_fused) with every
+ * token's tap sources read from the table sconv_seq_metadata_taps built for
+ * the same step, instead of from positions, seq_idx, query_start and the
+ * block table ("vllm.models.inkling.nvidia.ops.sconv", fused_sconv).  The
+ * outputs, cache inserts and err_flag bits are bit for bit those of
+ * sconv_fused_streams on the metadata the table was built from.
+ *
+ *   streams, n_streams, T, W, cache, cache_strides, num_blocks, H, N, D, dt:
+ *                    as in sconv_fused_streams.
+ *   slot_mapping     [T] int64 as in sconv_fused.
+ *   taps             [T, W - 1] int64 table built with the same W and N;
+ *                    may be NULL when W == 1.  Must not overlap any out.
+ *   metadata_ready   0: slot_mapping and taps are read after the wait for
+ *                    the kernels this launch depends on (always valid;
+ *                    before the wait the table may be read speculatively,
+ *                    only to prefetch cache taps into L2).
+ *                    1: they are read BEFORE that wait, and each token's x
+ *                    rows and cache taps are prefetched into L2 there, so
+ *                    that after the wait a token's loads are one dependent
+ *                    access.  A launch of this library may begin as soon as
+ *                    every kernel it depends on has signalled its
+ *                    dependents, which every kernel here except the *_ahead
+ *                    builders does after its own wait.  Precondition of 1
+ *                    (the caller's; nothing checks it): every kernel that
+ *                    writes slot_mapping or taps has completed before any
+ *                    kernel this launch depends on could signal it.  Valid
+ *                    patterns: the tables were complete before the stream
+ *                    (or the graph replay) last started from a fully
+ *                    ordered state; or at least one call of this library
+ *                    other than the *_ahead builders runs on this stream
+ *                    between the builder and this call, and this call
+ *                    depends on nothing else.  NOT sufficient: a builder on
+ *                    another stream joined by an event -- under stream
+ *                    capture that edge becomes programmatic like the
+ *                    stream's own, and orders this launch only after the
+ *                    builder signals, which is at its start.
+ *   err_flag         optional: a skipped token sets the bits its table row
+ *                    carries, or SCONV_EFLAG_SLOT (with the row's request,
+ *                    query-start and position bits) for a slot out of range;
+ *                    an entry that is neither a slot below num_blocks * N,
+ *                    SCONV_TAP_X on a row of this call, SCONV_TAP_ZERO nor a
+ *                    failure code sets SCONV_EFLAG_BLOCK.
+ * The form is built for decode-size steps (one thread per 16-byte channel
+ * pack of a token); prefill-size steps are served by sconv_fused.
+ * T == 0 returns SCONV_OK and enqueues nothing.
+ */
+sconv_status sconv_fused_taps(
+    const sconv_stream_desc *streams, int n_streams, int T, int W,
+    void *cache, const int64_t cache_strides[4], int64_t num_blocks, int H, int N, int D,
+    const int64_t *slot_mapping, const int64_t *taps, int metadata_ready, sconv_dtype dt,
+    int32_t *err_flag, cudaStream_t stream);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *sconv_status_string(sconv_status status);

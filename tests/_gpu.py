@@ -65,15 +65,16 @@ def oracle_fused(wl, x, weight, cache, md, **kw):
     return oracle.fused(**args)
 
 
-def check_small(wl, device="cuda", t=None, md_cpu=None):
+def check_small(wl, device="cuda", t=None, md_cpu=None, run=run_fused):
     """Full comparison of one step: every output row, every cache byte, and
-    the untouched PAD rows.  Returns the GPU out tensor."""
+    the untouched PAD rows.  ``run(wl, t, out=...)`` launches the step
+    (sconv_fused by default).  Returns the GPU out tensor."""
     if t is None:
         t = wl.tensors(device)
     md_cpu = md_cpu or wl.metadata("cpu")
     cache_before = t["cache"].cpu()
     out = workloads.sentinel(tuple(t["x"].shape), wl.dtype, device)
-    run_fused(wl, t, out=out)
+    run(wl, t, out=out)
     torch.cuda.synchronize()
     ref, state, cache_ref, skipped = oracle_fused(wl, t["x"].cpu(), t["weight"].cpu(),
                                                   cache_before, md_cpu)

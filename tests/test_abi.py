@@ -243,3 +243,51 @@ def test_dense_entry_points_host_validation(lib):
     assert upd(L=17) == 2
     assert upd(W=9) == 2
     assert upd(dt=9) == 2
+
+
+@pytest.mark.parametrize("name", ["sconv_seq_metadata_taps", "sconv_seq_metadata_taps_ahead"])
+def test_seq_metadata_taps_host_validation(lib, name):
+    """Size, capacity and pointer errors of the tap resolution are rejected
+    before any launch."""
+    def call(qsl=FAKE, R=3, na=7, npad=10, pos=FAKE * 4, slot=FAKE * 5, bt=FAKE * 6, bt_rs=4,
+             MB=4, nb=8, N=16, W=4, si=FAKE * 2, cap_s=10, qs=FAKE * 3, cap_q=10, taps=FAKE * 7,
+             cap_t=30):
+        return getattr(lib, name)(qsl, R, na, npad, pos, slot, bt, bt_rs, MB, nb, N, W, si,
+                                  cap_s, qs, cap_q, taps, cap_t, 0)
+    assert call(na=0, npad=0) == 0
+    assert call(npad=5) == 1            # fewer padded than actual rows
+    assert call(cap_s=9) == 1
+    assert call(cap_q=9) == 1
+    assert call(cap_t=29) == 1          # 10 rows x 3 lags do not fit
+    assert call(W=0) == 1
+    assert call(W=9) == 2
+    assert call(R=0) == 1
+    assert call(bt_rs=3) == 1
+    assert call(N=0) == 1
+    assert call(taps=0) == 1            # a table is needed for W > 1
+    assert call(pos=0) == 1
+    assert call(W=1, taps=0, cap_t=0, si=0, qs=0) == 0   # nothing to write
+
+
+def test_fused_taps_host_validation(lib):
+    """sconv_fused_taps needs a table for W > 1, rejects an output that
+    overlaps it, and applies the stream checks of sconv_fused_streams."""
+    from hybrid_sconv_b200.binding import StreamDesc
+
+    def desc(x, out, off_s, ws=4):
+        return StreamDesc(x, 8, FAKE + 4096, 4, 1, out, 8, off_s, ws, 0, 1)
+
+    def call(descs, T=4, W=4, taps=FAKE * 2048, slot=FAKE, ready=1, cs=None, dt=1):
+        arr = (StreamDesc * len(descs))(*descs)
+        return lib.sconv_fused_taps(arr, len(descs), T, W, FAKE * 64,
+                                    cs or _strides(512, 256, 16, 1), 8, 2, 16, 16, slot, taps,
+                                    ready, dt, 0, 0)
+    ok = desc(FAKE, FAKE * 512, 0)
+    assert call([ok], T=0) == 0
+    assert call([ok], taps=0) == 1                      # W > 1 without a table
+    assert call([ok], slot=0) == 1
+    assert call([ok], taps=FAKE * 512 + 8) == 1         # table inside the output
+    assert call([ok, desc(FAKE * 2, FAKE * 1024, 2)]) == 1   # lane ranges overlap
+    assert call([ok], W=9) == 2
+    assert call([ok], cs=_strides(512, 256, 16, 2)) == 1    # D stride must be 1
+    assert call([ok], dt=7) == 2

@@ -95,3 +95,14 @@ def test_profiled_traffic_reads_the_json_record(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "changed")
     assert bench.profiled_traffic("w") is None
     assert bench.profiled_traffic("missing") is None
+
+
+def test_algorithmic_bytes_taps_by_hand():
+    """One request, 2 new tokens after 9 cached ones, W = 4, C = 8, bf16: x,
+    insert and out of both tokens, three history rows, the weights, and per
+    token the slot (8 B) and a table row of three 8-byte entries."""
+    wl = workloads.build("h", dtype="bf16", H=1, D=8, ws=8, off_s=0, W=4, N=4, hist=[9],
+                         new=[2], act=None, residual=False, seed=3)
+    C, e = 8, 2
+    expect = 2 * C * e + 2 * 2 * C * e + 3 * C * e + C * 4 * e + (8 + 24) * 2
+    assert bench.algorithmic_bytes_taps(wl) == expect

@@ -1,14 +1,17 @@
 """The benchmark's pipelined decode steps compute exactly what the plain
 sequence of steps computes.
 
-Pipelining builds step i+1's metadata (sconv_seq_metadata,
-"vllm.models.inkling.nvidia.ops.sconv") on a second stream while step i's
-sconv_fused runs; the convolutions keep their order, since step i+1 reads
-as history what step i inserted.  Several batches share one paged cache
-here, so any reordering of the convolutions or a metadata buffer read
-before it is complete would change the bits.  Each case also runs with
-sconv_seq_metadata_ahead, whose lookup runs before its wait on the stream
-and whose completion must still follow the previous convolution's.
+Pipelining builds step i+1's metadata (sconv_seq_metadata, or
+sconv_seq_metadata_taps with the tap table, "vllm.models.inkling.nvidia.ops.sconv")
+beside step i's convolution: on a second stream joined by an event
+("side"), or enqueued ahead of it on the same stream ("interleaved", where
+the convolution then reads its table before its wait).  The convolutions
+keep their order, since step i+1 reads as history what step i inserted.
+Several batches share one paged cache here, so any reordering of the
+convolutions or a metadata buffer read before it is complete would change
+the bits.  Each case also runs with the *_ahead builders, whose lookup
+runs before their wait on the stream and whose completion must still
+follow the previous convolution's.
 """
 from __future__ import annotations
 
@@ -31,13 +34,15 @@ def _reset(sets_obj, cache0):
         raw(s["out"]).fill_(-1)
         s["seq_idx"].fill_(-7)
         s["query_start"].fill_(-7)
+        s["taps"].fill_(-7)
 
 
+@pytest.mark.parametrize("mode", ["taps", "paged"])
 @pytest.mark.parametrize("ahead", [False, True])
 @pytest.mark.parametrize("n", [1, 2, 6])
-def test_pipelined_steps_equal_plain_steps(n, ahead):
+def test_pipelined_steps_equal_plain_steps(n, ahead, mode):
     dev = torch.device("cuda", 0)
-    sets_obj = bench.DecodeSets(n, 5151, dev, max_hist=64)
+    sets_obj = bench.DecodeSets(n, 5151, dev, max_hist=64, mode=mode)
     cache0 = raw(sets_obj.cache).clone()
 
     _reset(sets_obj, cache0)
@@ -66,16 +71,26 @@ def test_pipelined_steps_equal_plain_steps(n, ahead):
     for a, b in zip(outs, plain_outs):
         assert torch.equal(a, b)
 
-    # the same from the benchmark's graphs (two rounds over the batches)
-    stream = torch.cuda.Stream(dev)
     _reset(sets_obj, cache0)
-    full, tail, reps = bench.run_steps_graphs(sets_obj, n, stream, pipeline=True)
-    _reset(sets_obj, cache0)
-    with torch.cuda.stream(stream):
-        bench.replay_steps(full, tail, reps)
+    bench.interleaved_steps(sets_obj, list(range(n)))
     torch.cuda.synchronize()
     cache, outs = _snapshot(sets_obj)
     assert torch.equal(cache, plain_cache)
     for a, b in zip(outs, plain_outs):
         assert torch.equal(a, b)
-    del full, tail
+
+    # the same from the benchmark's graphs, replayed twice
+    stream = torch.cuda.Stream(dev)
+    for schedule in ("side", "interleaved"):
+        _reset(sets_obj, cache0)
+        full, tail, reps = bench.run_steps_graphs(sets_obj, n, stream, pipeline=schedule)
+        for _ in range(2):
+            _reset(sets_obj, cache0)
+            with torch.cuda.stream(stream):
+                bench.replay_steps(full, tail, reps)
+            torch.cuda.synchronize()
+            cache, outs = _snapshot(sets_obj)
+            assert torch.equal(cache, plain_cache), schedule
+            for a, b in zip(outs, plain_outs):
+                assert torch.equal(a, b), schedule
+        del full, tail

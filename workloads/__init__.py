@@ -221,12 +221,14 @@ def tiny_prefill_f32(seed=1001) -> Workload:
                  deal_per_request=4, num_blocks=8)
 
 
-def decode_bf16(seed=1002, R=256, max_hist=4096) -> Workload:
+def decode_bf16(seed=1002, R=256, max_hist=4096, min_hist=1) -> Workload:
     """256 single-token requests over histories of U{1..4096} cached tokens;
     H=32, D=128, stream 2 of 4 (ws=32, off_s=32), C=1024, W=4, N=16; cache
-    filled with N(0,1); weight~N(0,0.5); SiLU, residual on."""
+    filled with N(0,1); weight~N(0,0.5); SiLU, residual on.  min_hist =
+    max_hist = 0 gives the same batch shape with no history (every token at
+    position 0, no cache taps)."""
     rng = np.random.default_rng(seed)
-    hist = rng.integers(1, max_hist + 1, size=R)
+    hist = rng.integers(min_hist, max_hist + 1, size=R)
     return build("decode_bf16", dtype="bf16", H=32, D=128, ws=32, off_s=32, W=4, N=16,
                  hist=hist, new=np.ones(R, np.int64), act="silu", residual=True,
                  seed=seed, rng=rng)
