@@ -1137,8 +1137,8 @@ def e2e(sets_obj, K, stream, world, flush):
     """End to end through the public API with host buffers.  Every step
     copies its inputs (x, positions, slot_mapping, block_table,
     query_start_loc) from pinned host memory to the device, builds the
-    metadata and tap table, runs the fused step and copies its output back
-    to pinned host memory.  The inputs of a step travel as one copy (they sit back to back
+    metadata (and, in taps mode, the tap table), runs the fused step and
+    copies its output back to pinned host memory.  The inputs of a step travel as one copy (they sit back to back
     in one pinned buffer and are used in place on the device), since every
     copy has a fixed cost of microseconds on top of its bytes (measured:
     five copies per step 5.9 Mtok/s, one 9.7, the one copy split over two
@@ -1164,12 +1164,20 @@ def e2e(sets_obj, K, stream, world, flush):
             with torch.cuda.stream(up):
                 p["dev"].copy_(p["host"], non_blocking=True)
             cur.wait_stream(up)
-            hs.sconv_seq_metadata_taps(v["query_start_loc"], wl.R, wl.T, v["positions"],
-                                       v["slot_mapping"], v["block_table"], wl.num_blocks,
-                                       wl.N, wl.W, seq_idx_out=s["seq_idx"],
-                                       query_start_out=s["query_start"], taps_out=s["taps"])
-            hs.sconv_fused_taps(v["x"], sets_obj.weight, sets_obj.cache, v["slot_mapping"],
-                                s["taps"], out=s["out"], **wl.kwargs())
+            if sets_obj.mode == "taps":
+                hs.sconv_seq_metadata_taps(v["query_start_loc"], wl.R, wl.T, v["positions"],
+                                           v["slot_mapping"], v["block_table"], wl.num_blocks,
+                                           wl.N, wl.W, seq_idx_out=s["seq_idx"],
+                                           query_start_out=s["query_start"],
+                                           taps_out=s["taps"])
+                hs.sconv_fused_taps(v["x"], sets_obj.weight, sets_obj.cache, v["slot_mapping"],
+                                    s["taps"], out=s["out"], **wl.kwargs())
+            else:
+                hs.sconv_seq_metadata(v["query_start_loc"], wl.R, wl.T, s["seq_idx"],
+                                      s["query_start"])
+                hs.sconv_fused(v["x"], sets_obj.weight, sets_obj.cache, v["positions"],
+                               v["block_table"], s["seq_idx"], v["slot_mapping"],
+                               s["query_start"], out=s["out"], **wl.kwargs())
             down.wait_stream(cur)
             with torch.cuda.stream(down):
                 p["out_host"].copy_(s["out"], non_blocking=True)
