@@ -69,7 +69,8 @@ def parse_args():
     p.add_argument("--only", choices=["chunked_prefill_bf16", "long_prefill_bf16",
                                       "spec_decode_bf16", "dense", "dense_prefill_bf16",
                                       "dense_long_prefill_bf16", "dense_decode_bf16",
-                                      "decode_chain"],
+                                      "decode_chain", "chunked_prefill_f32_w4",
+                                      "chunked_prefill_bf16_w8"],
                    help="time just this workload's kernels and print its table row")
     p.add_argument("--max-hist", type=int, default=4096,
                    help="longest cached history of the decode requests (smaller only for "
@@ -367,32 +368,39 @@ class DecodeSets:
                                s["query_start"], out=s["out"], **wl.kwargs())
 
 
-def pipelined_steps(sets_obj, idxs, side):
-    """Steps idxs in order, each metadata build + sconv_fused over its
+def pipelined_steps(sets_obj, idxs, side, carry=None):
+    """Steps idxs in order, each metadata build + convolution over its
     batch, with the next step's metadata built beside the current step's
     convolution, as a serving engine prepares step i+1's inputs while step
     i runs: metadata(i+1) goes to `side` once conv(i-1) has finished (its
     buffers are the next batch's own), and conv(i+1) waits for both
     conv(i) (its cache inserts are the next step's history) and
-    metadata(i+1).  Each step still launches both kernels."""
+    metadata(i+1).  carry: the index of the step after idxs; then the first
+    step's metadata is taken as already built (by the call before this one)
+    and the last build is for step `carry` -- still one build and one
+    convolution per step, as in a serving loop's steady state."""
     main = torch.cuda.current_stream()
     side.wait_stream(main)
-    with torch.cuda.stream(side):
-        sets_obj.step(idxs[0], fused=False)
-    meta_done = torch.cuda.Event()
-    meta_done.record(side)
+    meta_done = None
+    if carry is None:
+        with torch.cuda.stream(side):
+            sets_obj.step(idxs[0], fused=False)
+        meta_done = torch.cuda.Event()
+        meta_done.record(side)
+    nxt = list(idxs[1:]) + ([] if carry is None else [carry])
     for j, i in enumerate(idxs):
-        main.wait_event(meta_done)
+        if meta_done is not None:
+            main.wait_event(meta_done)
         before = torch.cuda.Event()
         before.record(main)  # everything up to conv(i-1)
         # Not ready: under stream capture the event join becomes a
         # programmatic edge, which orders this launch after the builder's
         # trigger, not after its completion.
         sets_obj.step(i, metadata=False)
-        if j + 1 < len(idxs):
+        if j < len(nxt):
             side.wait_event(before)
             with torch.cuda.stream(side):
-                sets_obj.step(idxs[j + 1], fused=False)
+                sets_obj.step(nxt[j], fused=False)
             meta_done = torch.cuda.Event()
             meta_done.record(side)
     main.wait_stream(side)
@@ -413,18 +421,21 @@ def interleaved_steps(sets_obj, idxs):
         sets_obj.step(i, metadata=False, ready=j > 0)
 
 
-def run_steps_graphs(sets_obj, K, stream, pipeline=False, **step_kw):
+def run_steps_graphs(sets_obj, K, stream, pipeline=False, carry=False, **step_kw):
     """Graphs that together replay exactly K steps over the rotating sets.
     pipeline: False (metadata then convolution, one stream), "side" (next
     step's metadata on a second stream beside the current convolution) or
     "interleaved" (next step's metadata ahead of the current convolution on
-    one stream)."""
+    one stream).  carry (with "side"): each graph takes its first step's
+    metadata as built by whatever ran before it and builds the metadata of
+    the step after its last (see pipelined_steps); carry_prologue() builds
+    the first one before the first replay."""
     M = len(sets_obj.sets)
     side = torch.cuda.Stream(stream.device)
 
     def steps(n):
         if pipeline == "side":
-            pipelined_steps(sets_obj, list(range(n)), side)
+            pipelined_steps(sets_obj, list(range(n)), side, n % M if carry else None)
         elif pipeline == "interleaved":
             interleaved_steps(sets_obj, list(range(n)))
         else:
@@ -433,6 +444,14 @@ def run_steps_graphs(sets_obj, K, stream, pipeline=False, **step_kw):
     full = capture(lambda: steps(M), stream) if K >= M else None
     tail = capture(lambda: steps(K % M), stream) if K % M else None
     return full, tail, K // M
+
+
+def carry_prologue(sets_obj, stream):
+    """The metadata of set 0, built before the first replay of carry graphs
+    (the build a previous window of the serving loop would have made)."""
+    with torch.cuda.stream(stream):
+        sets_obj.step(0, fused=False)
+    torch.cuda.synchronize()
 
 
 class L2Flush:
@@ -569,13 +588,18 @@ def _entry(wl, secs, nbytes, peak):
             "alg_bytes": nbytes, "alg_gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
 
 
-def bench_prefill_shapes(device, stream, peak, reps=50):
+PREFILL_SHAPES = (("f32_w4", "f32", 4), ("bf16_w8", "bf16", 8))
+
+
+def bench_prefill_shapes(device, stream, peak, reps=50, only=None):
     """The chunked prefill's requests and channel count (T = 16 070, C =
     4096) in fp32 with W = 4 and in bf16 with W = 8: the tiled prefill form
-    outside the named workloads' dtype and tap count."""
+    outside the named workloads' dtype and tap count.  only: one tag."""
     import hybrid_sconv_b200 as hs
     table = {}
-    for tag, dtype, W in (("f32_w4", "f32", 4), ("bf16_w8", "bf16", 8)):
+    for tag, dtype, W in PREFILL_SHAPES:
+        if only is not None and tag != only:
+            continue
         rng = np.random.default_rng(1003)
         hist = rng.integers(0, 2049, size=16)
         new = rng.integers(1, 2049, size=16)
@@ -1110,6 +1134,71 @@ def host_cpu() -> dict:
 # --------------------------------------------------------------------------
 # e2e: the public API with host buffers
 
+class MappedOut:
+    """Pinned host memory mapped into the device's address space
+    (cudaHostAlloc with cudaHostAllocMapped), presented with the tensor
+    interface the binding reads (data_ptr, shape, stride, dtype, device):
+    the fused kernel stores a step's output straight into host memory, so
+    the result crosses to the host without a copy-engine transfer.  The
+    device address comes from cudaHostGetDevicePointer; both calls' return
+    codes are checked and any failure raises before a kernel sees the
+    buffer."""
+
+    _rt = None
+
+    @classmethod
+    def runtime(cls):
+        if cls._rt is None:
+            import ctypes
+            rt = ctypes.CDLL("libcudart.so.12")  # the runtime torch and libsconv share
+            rt.cudaHostAlloc.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_size_t,
+                                         ctypes.c_uint]
+            rt.cudaHostGetDevicePointer.argtypes = [ctypes.POINTER(ctypes.c_void_p),
+                                                    ctypes.c_void_p, ctypes.c_uint]
+            rt.cudaFreeHost.argtypes = [ctypes.c_void_p]
+            cls._rt = rt
+        return cls._rt
+
+    def __init__(self, shape, dtype, device):
+        import ctypes
+        rt = self.runtime()
+        self.shape = torch.Size(shape)
+        self.dtype = dtype
+        self.device = torch.device(device)
+        self.nbytes = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+        host = ctypes.c_void_p()
+        err = rt.cudaHostAlloc(ctypes.byref(host), self.nbytes, 2)  # cudaHostAllocMapped
+        if err != 0:
+            raise RuntimeError(f"cudaHostAlloc(mapped) failed: {err}")
+        dev = ctypes.c_void_p()
+        err = rt.cudaHostGetDevicePointer(ctypes.byref(dev), host, 0)
+        if err != 0 or not dev.value:
+            rt.cudaFreeHost(host)
+            raise RuntimeError(f"cudaHostGetDevicePointer failed: {err}")
+        self.host_ptr, self.dev_ptr = host.value, dev.value
+
+    def data_ptr(self):
+        return self.dev_ptr
+
+    def dim(self):
+        return len(self.shape)
+
+    def stride(self, i=None):
+        st = (self.shape[1], 1)
+        return st if i is None else st[i]
+
+    def host_view(self):
+        """A CPU tensor over the same bytes (valid until free())."""
+        import ctypes
+        buf = (ctypes.c_uint8 * self.nbytes).from_address(self.host_ptr)
+        return torch.frombuffer(buf, dtype=self.dtype).view(self.shape)
+
+    def free(self):
+        if self.host_ptr:
+            self.runtime().cudaFreeHost(self.host_ptr)
+            self.host_ptr = self.dev_ptr = 0
+
+
 def _packed_inputs(sets_obj, keys):
     """Per set, one pinned host buffer and one device buffer holding all of
     a step's inputs back to back (each 256-byte aligned), and device views
@@ -1137,50 +1226,70 @@ def e2e(sets_obj, K, stream, world, flush):
     """End to end through the public API with host buffers.  Every step
     copies its inputs (x, positions, slot_mapping, block_table,
     query_start_loc) from pinned host memory to the device, builds the
-    metadata (and, in taps mode, the tap table), runs the fused step and
-    copies its output back to pinned host memory.  The inputs of a step travel as one copy (they sit back to back
-    in one pinned buffer and are used in place on the device), since every
-    copy has a fixed cost of microseconds on top of its bytes (measured:
-    five copies per step 5.9 Mtok/s, one 9.7, the one copy split over two
-    or three streams 8.4 / 7.7).  As a
-    serving engine does, upload, kernels and download run on their own
-    streams (joined by events), so step i+1's upload and step i-1's
-    download overlap step i's kernels; each step still moves all of its own
-    bytes."""
+    metadata (and, in taps mode, the tap table) and runs the fused step,
+    whose output lands in host memory: the fused kernel stores it straight
+    into mapped pinned host memory (MappedOut), so the copy engine carries
+    only the uploads, or, where host memory cannot be mapped, a copy-engine
+    download on its own stream follows.  The inputs of a step travel as one
+    copy (they sit back to back in one pinned buffer and are used in place
+    on the device), since every copy has a fixed cost of microseconds on top
+    of its bytes (measured: five copies per step 5.9 Mtok/s, one 9.7).  As a
+    serving engine does, uploads and kernels run on their own streams
+    (joined by events), so step i+1's upload overlaps step i's kernels;
+    each step still moves all of its own bytes."""
     import hybrid_sconv_b200 as hs
     keys = ("x", "positions", "slot_mapping", "block_table", "query_start_loc")
     packed = _packed_inputs(sets_obj, keys)
     h2d = packed[0]["h2d"]
     d2h = packed[0]["out_host"].numel() * packed[0]["out_host"].element_size()
+    try:
+        mapped = [MappedOut(tuple(s["out"].shape), s["out"].dtype, s["out"].device)
+                  for s in sets_obj.sets]
+    except (OSError, RuntimeError):
+        mapped = None
     up, down = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def kernels(i, out):
+        wl, s, v = sets_obj.wls[i], sets_obj.sets[i], packed[i]["views"]
+        if sets_obj.mode == "taps":
+            hs.sconv_seq_metadata_taps(v["query_start_loc"], wl.R, wl.T, v["positions"],
+                                       v["slot_mapping"], v["block_table"], wl.num_blocks,
+                                       wl.N, wl.W, seq_idx_out=s["seq_idx"],
+                                       query_start_out=s["query_start"], taps_out=s["taps"])
+            hs.sconv_fused_taps(v["x"], sets_obj.weight, sets_obj.cache, v["slot_mapping"],
+                                s["taps"], out=out, **wl.kwargs())
+        else:
+            hs.sconv_seq_metadata(v["query_start_loc"], wl.R, wl.T, s["seq_idx"],
+                                  s["query_start"])
+            hs.sconv_fused(v["x"], sets_obj.weight, sets_obj.cache, v["positions"],
+                           v["block_table"], s["seq_idx"], v["slot_mapping"], s["query_start"],
+                           out=out, **wl.kwargs())
+
+    if mapped:
+        # One step of set 0 into device memory, then the same step into the
+        # mapped buffer (a step never reads its own inserts, so the history
+        # is the same): the bytes must agree.
+        packed[0]["dev"].copy_(packed[0]["host"])
+        kernels(0, sets_obj.sets[0]["out"])
+        kernels(0, mapped[0])
+        torch.cuda.synchronize()
+        assert torch.equal(mapped[0].host_view().view(torch.int16),
+                           sets_obj.sets[0]["out"].cpu().view(torch.int16)), "mapped output"
 
     def steps(n):
         cur = torch.cuda.current_stream()
         up.wait_stream(cur)
         down.wait_stream(cur)
         for i in range(n):
-            wl, s, p = sets_obj.wls[i], sets_obj.sets[i], packed[i]
-            v = p["views"]
+            s, p = sets_obj.sets[i], packed[i]
             with torch.cuda.stream(up):
                 p["dev"].copy_(p["host"], non_blocking=True)
             cur.wait_stream(up)
-            if sets_obj.mode == "taps":
-                hs.sconv_seq_metadata_taps(v["query_start_loc"], wl.R, wl.T, v["positions"],
-                                           v["slot_mapping"], v["block_table"], wl.num_blocks,
-                                           wl.N, wl.W, seq_idx_out=s["seq_idx"],
-                                           query_start_out=s["query_start"],
-                                           taps_out=s["taps"])
-                hs.sconv_fused_taps(v["x"], sets_obj.weight, sets_obj.cache, v["slot_mapping"],
-                                    s["taps"], out=s["out"], **wl.kwargs())
-            else:
-                hs.sconv_seq_metadata(v["query_start_loc"], wl.R, wl.T, s["seq_idx"],
-                                      s["query_start"])
-                hs.sconv_fused(v["x"], sets_obj.weight, sets_obj.cache, v["positions"],
-                               v["block_table"], s["seq_idx"], v["slot_mapping"],
-                               s["query_start"], out=s["out"], **wl.kwargs())
-            down.wait_stream(cur)
-            with torch.cuda.stream(down):
-                p["out_host"].copy_(s["out"], non_blocking=True)
+            kernels(i, mapped[i] if mapped else s["out"])
+            if not mapped:
+                down.wait_stream(cur)
+                with torch.cuda.stream(down):
+                    p["out_host"].copy_(s["out"], non_blocking=True)
         cur.wait_stream(up)
         cur.wait_stream(down)
 
@@ -1190,11 +1299,17 @@ def e2e(sets_obj, K, stream, world, flush):
     prime(full, tail, stream)
     secs = max_over_ranks(time_region(full, tail, K // M, stream, world, flush=flush)[0], world)
     del full, tail
+    torch.cuda.synchronize()
+    if mapped:
+        for m in mapped:
+            m.free()
     tokens = sum_over_ranks(float(sets_obj.wls[0].T * K), world)
     return {"value": round(tokens / secs / 1e6, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": K,
-            "launch": "cuda_graph; one packed upload, kernels and download per step on three "
-                      "streams"}
+            "launch": "cuda_graph; one packed upload per step on its own stream, kernels on "
+                      "another",
+            "d2h": ("the fused kernel stores the step's output in mapped pinned host memory"
+                    if mapped else "copy-engine download on a third stream")}
 
 
 # --------------------------------------------------------------------------
@@ -1209,7 +1324,10 @@ def config_block(world, l2):
             "pipelining": "the next step's metadata is built on a second stream beside the "
                           "current step's convolution, as a serving engine prepares step "
                           "i+1's inputs while step i runs; the convolutions run in order, "
-                          "each waiting for the previous one",
+                          "each waiting for the previous one; the timed region holds K "
+                          "convolutions and K metadata builds (the first step's metadata "
+                          "comes from the step before the region, the last build is for the "
+                          "step after it)",
             "metadata": "one metadata buffer set per step, so the *_ahead builder may look "
                         "up before the launch's wait on its predecessors",
             "l2": l2}
@@ -1288,6 +1406,9 @@ def main():
         elif args.only == "decode_chain":
             sets_obj = DecodeSets(args.sets, rank_seed(args.seed, rank), device, args.max_hist)
             row = bench_decode_chain(sets_obj, stream, peak)
+        elif args.only in ("chunked_prefill_f32_w4", "chunked_prefill_bf16_w8"):
+            row = bench_prefill_shapes(device, stream, peak, reps=max(3, args.steps),
+                                       only=args.only[len("chunked_prefill_"):])
         elif args.only == "dense_decode_bf16":
             row = bench_dense_decode(device, stream, peak, nsets=args.sets,
                                      reps=max(3, args.steps))
@@ -1303,14 +1424,20 @@ def main():
                           ahead=True, mode=STEP_MODE)
     flush = L2Flush(device)
 
-    # warm-up, then exactly K timed steps
-    wfull, wtail, wreps = run_steps_graphs(sets_obj, W, stream, pipeline=STEP_SCHEDULE)
+    # warm-up, then exactly K timed steps (each step's metadata built during
+    # the step before it; set 0's by the prologue for the first replay)
+    carry_prologue(sets_obj, stream)
+    wfull, wtail, wreps = run_steps_graphs(sets_obj, W, stream, pipeline=STEP_SCHEDULE,
+                                           carry=True)
     with torch.cuda.stream(stream):
         replay_steps(wfull, wtail, wreps)
     torch.cuda.synchronize()
     del wfull, wtail
-    full, tail, reps = run_steps_graphs(sets_obj, K, stream, pipeline=STEP_SCHEDULE)
+    carry_prologue(sets_obj, stream)
+    full, tail, reps = run_steps_graphs(sets_obj, K, stream, pipeline=STEP_SCHEDULE,
+                                        carry=True)
     prime(full, tail, stream)
+    carry_prologue(sets_obj, stream)
     sampler = ClockSampler(local) if rank == 0 else None
     secs, (w0, w1) = time_region(full, tail, reps, stream, world, sampler, flush)
     secs = max_over_ranks(secs, world)
@@ -1324,7 +1451,7 @@ def main():
             load = ClockSampler(local)
             if full is None:
                 full, _, _ = run_steps_graphs(sets_obj, len(sets_obj.sets), stream,
-                                              pipeline=STEP_SCHEDULE)
+                                              pipeline=STEP_SCHEDULE, carry=True)
                 prime(full, None, stream)
             n = max(1, int(2.0 / max(secs / K * len(sets_obj.sets), 1e-6)))
             _, (l0, l1) = time_region(full, None, n, stream, 1, load)

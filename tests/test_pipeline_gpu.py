@@ -79,13 +79,20 @@ def test_pipelined_steps_equal_plain_steps(n, ahead, mode):
     for a, b in zip(outs, plain_outs):
         assert torch.equal(a, b)
 
-    # the same from the benchmark's graphs, replayed twice
+    # the same from the benchmark's graphs, replayed twice; with carry the
+    # first step's metadata comes from the prologue and the graph's last
+    # build is for the step after it
     stream = torch.cuda.Stream(dev)
-    for schedule in ("side", "interleaved"):
+    for schedule, carry in (("side", False), ("interleaved", False), ("side", True)):
         _reset(sets_obj, cache0)
-        full, tail, reps = bench.run_steps_graphs(sets_obj, n, stream, pipeline=schedule)
+        if carry:
+            bench.carry_prologue(sets_obj, stream)
+        full, tail, reps = bench.run_steps_graphs(sets_obj, n, stream, pipeline=schedule,
+                                                  carry=carry)
         for _ in range(2):
             _reset(sets_obj, cache0)
+            if carry:
+                bench.carry_prologue(sets_obj, stream)
             with torch.cuda.stream(stream):
                 bench.replay_steps(full, tail, reps)
             torch.cuda.synchronize()
