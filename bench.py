@@ -46,12 +46,14 @@ UNIT = "Mtokens/s"
 HEADLINE = "decode_bf16"
 # The headline step: its form (DecodeSets mode) and schedule (see
 # run_steps_graphs), the fastest single-layer decode step measured.
-STEP_MODE = "paged"
-STEP_SCHEDULE = "side"
+STEP_MODE = "taps"
+STEP_SCHEDULE = "next"
 STEP_KERNEL = {"paged": "fused_token_kernel (sconv_fused at decode sizes)",
-               "taps": "fused_taps_kernel (sconv_fused_taps)"}
+               "taps": "fused_taps_next_kernel (sconv_fused_taps_next: this step's "
+                       "convolution and the next step's tap table in one launch)"}
 STEP_CALLS = {"paged": "sconv_seq_metadata_ahead + sconv_fused",
-              "taps": "sconv_seq_metadata_taps_ahead + sconv_fused_taps"}
+              "taps": "sconv_fused_taps_next (one launch: this step's convolution and the "
+                      "next step's metadata and tap table)"}
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 
@@ -141,6 +143,22 @@ def algorithmic_bytes_taps(wl) -> int:
             + (8 + 8 * (W - 1)) * wl.T)
 
 
+def algorithmic_bytes_resolve(wl) -> int:
+    """Bytes of one step's tap resolution: positions and slots read (16 B
+    per token), query_start_loc (4 B per request + 4), the distinct
+    block-table entries of the pre-forward taps (4 B each), and seq_idx,
+    query_start and the table row written (8 + 8 (W-1) B per token)."""
+    W, N = wl.W, wl.N
+    bt_entries = 0
+    for r in range(wl.R):
+        if wl.new[r] == 0:
+            continue
+        h = int(wl.hist[r])
+        rows = min(W - 1, h)
+        bt_entries += len({p // N for p in range(h - rows, h)})
+    return 16 * wl.T + 4 * (wl.R + 1) + 4 * bt_entries + (8 + 8 * (W - 1)) * wl.T
+
+
 def algorithmic_bytes(wl) -> int:
     """x rows read + inserts + outputs + the distinct pre-forward cache rows
     of each request (min(W-1, history) rows of C elements) + weights + 24 B
@@ -170,10 +188,11 @@ def measured_hbm_peak():
 
 
 def kernel_source_hash() -> str:
-    """Hash of the sources of the fused token kernel (the one the decode
-    workload runs), to tell whether a committed ncu summary is current."""
+    """Hash of the sources of the decode step's kernels (fused.cu and the
+    headers it includes), to tell whether a committed ncu record is
+    current."""
     h = hashlib.sha256()
-    for name in ("fused.cu", "fused_common.cuh", "common.cuh"):
+    for name in ("fused.cu", "fused_common.cuh", "common.cuh", "taps_resolve.cuh"):
         with open(os.path.join(ROOT, "hybrid_sconv_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -335,9 +354,30 @@ class DecodeSets:
             self.sets.append(s)
         self.alg_bytes = [algorithmic_bytes(wl) for wl in self.wls]
         self.alg_bytes_taps = [algorithmic_bytes_taps(wl) for wl in self.wls]
+        # one sconv_fused_taps_next launch: set i's convolution, set i+1's table
+        self.alg_bytes_next = [algorithmic_bytes_taps(wl) +
+                               algorithmic_bytes_resolve(self.wls[(i + 1) % n])
+                               for i, wl in enumerate(self.wls)]
 
-    def kernel_alg_bytes(self):
-        """Algorithmic bytes of one convolution launch in this mode."""
+    def step_next(self, i, j):
+        """Set i's convolution and set j's tap table in one launch
+        (sconv_fused_taps_next; taps mode)."""
+        import hybrid_sconv_b200 as hs
+        wl, s, wn, sn = self.wls[i], self.sets[i], self.wls[j], self.sets[j]
+        hs.sconv_fused_taps_next(
+            s["x"], self.weight, self.cache, s["slot_mapping"], s["taps"], out=s["out"],
+            next_step=dict(query_start_loc=sn["query_start_loc"], num_reqs=wn.R,
+                           num_actual_tokens=wn.T, positions=sn["positions"],
+                           slot_mapping=sn["slot_mapping"], block_table=sn["block_table"],
+                           seq_idx_out=sn["seq_idx"], query_start_out=sn["query_start"],
+                           taps_out=sn["taps"]),
+            **wl.kwargs())
+
+    def kernel_alg_bytes(self, schedule=None):
+        """Algorithmic bytes of one convolution launch in this mode (with the
+        next step's table build for the "next" schedule)."""
+        if schedule == "next":
+            return self.alg_bytes_next
         return self.alg_bytes_taps if self.mode == "taps" else self.alg_bytes
 
     def step(self, i, fused=True, metadata=True, ready=False):
@@ -421,12 +461,22 @@ def interleaved_steps(sets_obj, idxs):
         sets_obj.step(i, metadata=False, ready=j > 0)
 
 
+def next_steps(sets_obj, idxs, carry):
+    """Steps idxs in order, one launch each: the step's convolution and the
+    next step's tap table (sconv_fused_taps_next), the last one building
+    step `carry`'s; the first step's table comes from before.  One table
+    build and one convolution per step."""
+    for i, j in zip(idxs, list(idxs[1:]) + [carry]):
+        sets_obj.step_next(i, j)
+
+
 def run_steps_graphs(sets_obj, K, stream, pipeline=False, carry=False, **step_kw):
     """Graphs that together replay exactly K steps over the rotating sets.
     pipeline: False (metadata then convolution, one stream), "side" (next
     step's metadata on a second stream beside the current convolution) or
     "interleaved" (next step's metadata ahead of the current convolution on
-    one stream).  carry (with "side"): each graph takes its first step's
+    one stream) or "next" (one sconv_fused_taps_next launch per step, which
+    always carries).  carry (with "side"): each graph takes its first step's
     metadata as built by whatever ran before it and builds the metadata of
     the step after its last (see pipelined_steps); carry_prologue() builds
     the first one before the first replay."""
@@ -434,7 +484,9 @@ def run_steps_graphs(sets_obj, K, stream, pipeline=False, carry=False, **step_kw
     side = torch.cuda.Stream(stream.device)
 
     def steps(n):
-        if pipeline == "side":
+        if pipeline == "next":
+            next_steps(sets_obj, list(range(n)), n % M)
+        elif pipeline == "side":
             pipelined_steps(sets_obj, list(range(n)), side, n % M if carry else None)
         elif pipeline == "interleaved":
             interleaved_steps(sets_obj, list(range(n)))
@@ -529,6 +581,21 @@ def l2_statement(sets_obj, K):
     verdict = "> 126 MB L2" if touched > L2_BYTES else "NOT above the 126 MB L2"
     return (f"L2 flushed (256 MiB written) before the timed region; the steps rotate over "
             f"{M} input sets, each rotation touching {touched / 1e6:.0f} MB {verdict}")
+
+
+def step_launch_duration(sets_obj, stream, reps=200):
+    """Average duration of one launch of the headline step's kernel: with
+    the "next" schedule the step is one launch, so a graph of the full
+    rotation of steps (after the prologue) replayed `reps` times; otherwise
+    the convolution launches alone (fused_launch_duration)."""
+    if STEP_SCHEDULE != "next":
+        return fused_launch_duration(sets_obj, stream, reps)
+    carry_prologue(sets_obj, stream)
+    full, _, _ = run_steps_graphs(sets_obj, len(sets_obj.sets), stream, pipeline="next")
+    prime(full, None, stream)
+    secs, _ = time_region(full, None, reps, stream, 1)
+    del full
+    return secs / (reps * len(sets_obj.sets))
 
 
 def fused_launch_duration(sets_obj, stream, reps=200):
@@ -727,6 +794,7 @@ def bench_serial_step(sets_obj, stream, peak, reps=200):
     res = {}
     for key, mode, ahead, pipeline in (
             ("decode_step_pipelined", STEP_MODE, True, STEP_SCHEDULE),
+            ("decode_step_taps_next", "taps", True, "next"),
             ("decode_step_taps_side", "taps", True, "side"),
             ("decode_step_taps_interleaved", "taps", True, "interleaved"),
             ("decode_step_serial_taps", "taps", False, False),
@@ -737,6 +805,8 @@ def bench_serial_step(sets_obj, stream, peak, reps=200):
             ("decode_step_serial_ahead", "paged", True, False),
             ("decode_step_paged_side_plain_metadata", "paged", False, "side")):
         sets_obj.ahead, sets_obj.mode = ahead, mode
+        if pipeline == "next":
+            carry_prologue(sets_obj, stream)
         full, _, _ = run_steps_graphs(sets_obj, len(sets_obj.sets), stream, pipeline=pipeline)
         prime(full, None, stream)
         secs, _ = time_region(full, None, reps, stream, 1)
@@ -748,8 +818,10 @@ def bench_serial_step(sets_obj, stream, peak, reps=200):
                  ("paged", False): "sconv_seq_metadata"}
         res[key] = {"step_us": round(per * 1e6, 3),
                     "mtokens_s": round(sets_obj.wls[0].T / per / 1e6, 2),
-                    "metadata": names[(mode, ahead)],
-                    "conv": "sconv_fused_taps" if mode == "taps" else "sconv_fused",
+                    "metadata": ("built by the previous launch (sconv_fused_taps_next)"
+                                 if pipeline == "next" else names[(mode, ahead)]),
+                    "conv": ("sconv_fused_taps_next" if pipeline == "next" else
+                             "sconv_fused_taps" if mode == "taps" else "sconv_fused"),
                     "schedule": pipeline or "serial"}
     sets_obj.ahead, sets_obj.mode = saved
     return res
@@ -1463,9 +1535,9 @@ def main():
     value = tokens / secs / 1e6
     step_bytes = sum_over_ranks(float(np.mean(sets_obj.alg_bytes)) * K, world)
 
-    # the convolution kernel's own average launch duration
-    avg = fused_launch_duration(sets_obj, stream)
-    bytes_per_launch = float(np.mean(sets_obj.kernel_alg_bytes()))
+    # the step kernel's own average launch duration
+    avg = step_launch_duration(sets_obj, stream)
+    bytes_per_launch = float(np.mean(sets_obj.kernel_alg_bytes(STEP_SCHEDULE)))
     achieved = bytes_per_launch / avg / 1e9
     traffic = profiled_traffic(HEADLINE)
 
@@ -1478,7 +1550,7 @@ def main():
                                else "NOT a benchmark figure: profiling case "
                                     f"(histories up to {args.max_hist} tokens)"),
         "hbm_gbs": round(step_bytes / secs / 1e9, 1),
-        "gpu_launches": 2 * K,
+        "gpu_launches": (1 if STEP_SCHEDULE == "next" else 2) * K,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": traffic,

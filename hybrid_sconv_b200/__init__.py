@@ -21,7 +21,8 @@ _EXPORTS = (
     "sconv_extract_windows_paged", "sconv_fused", "sconv_fused_streams",
     "sconv_scatter_intermediate_ssm", "sconv_seq_metadata", "sconv_seq_metadata_ahead",
     "sconv_update", "sconv_seq_metadata_taps", "sconv_seq_metadata_taps_ahead",
-    "sconv_fused_taps", "sconv_fused_streams_taps", "TAP_X", "TAP_ZERO",
+    "sconv_fused_taps", "sconv_fused_streams_taps", "sconv_fused_taps_next", "TAP_X",
+    "TAP_ZERO",
 )
 
 __all__ = list(_EXPORTS)

@@ -49,6 +49,15 @@ class StreamDesc(ctypes.Structure):
                 ("ws", _INT), ("act", _INT), ("use_residual", _INT)]
 
 
+class TapsBuild(ctypes.Structure):
+    """sconv_taps_build of sconv.h (one step's tap resolution)."""
+    _fields_ = [("query_start_loc", _P), ("num_reqs", _INT), ("num_actual_tokens", _INT),
+                ("num_padded_tokens", _INT), ("positions", _P), ("slot_mapping", _P),
+                ("block_table", _P), ("bt_row_stride", _I64), ("max_blocks", _INT),
+                ("seq_idx_out", _P), ("seq_idx_cap", _I64), ("query_start_out", _P),
+                ("query_start_cap", _I64), ("taps_out", _P), ("taps_cap", _I64)]
+
+
 _SIGNATURES = {
     "sconv_fused": [
         _P, _I64, _INT, _INT, _P, _I64, _I64, _INT,
@@ -83,6 +92,10 @@ _SIGNATURES = {
         ctypes.POINTER(StreamDesc), _INT, _INT, _INT,
         _P, _I64P, _I64, _INT, _INT, _INT,
         _P, _P, _INT, _INT, _P, _P],
+    "sconv_fused_taps_next": [
+        ctypes.POINTER(StreamDesc), _INT, _INT, _INT,
+        _P, _I64P, _I64, _INT, _INT, _INT,
+        _P, _P, _INT, _P, ctypes.POINTER(TapsBuild), _P],
     "sconv_seq_metadata_ahead": [_P, _INT, _INT, _INT, _P, _I64, _P, _I64, _P],
     "sconv_scatter_intermediate_ssm": [
         _P, _I64, _I64, _I64, _P, _P, _INT, _P, _I64, _INT, _P, _P],
@@ -578,6 +591,74 @@ def sconv_fused_streams_taps(streams, cache, slot_mapping, taps, block_size, *,
             _stream(d, stream))
     _check("sconv_fused_taps", st)
     return outs
+
+
+def sconv_fused_taps_next(x, weight, cache, slot_mapping, taps, off_s, ws, block_size,
+                          activation=None, use_residual=True, *, next_step, out=None,
+                          err_flag=None, stream=None):
+    """One decode-loop step in one launch (sconv_fused_taps_next in
+    sconv.h): this step's fused convolution reading ``taps`` (after the
+    launch's wait), and the next step's tap table built by extra blocks of
+    the same launch.  ``next_step`` is a dict with the arguments of
+    sconv_seq_metadata_taps for that step: query_start_loc (or None),
+    num_reqs, num_actual_tokens, positions, slot_mapping, block_table,
+    taps_out, and optionally seq_idx_out, query_start_out,
+    num_padded_tokens.  Returns ``out``."""
+    dt = _float_common(x, weight, cache)
+    T, C = x.shape
+    W = weight.shape[1]
+    if out is None:
+        out = torch.empty_like(x)
+    n = next_step
+    npad = n.get("num_padded_tokens")
+    npad = n["num_actual_tokens"] if npad is None else npad
+    bt = n["block_table"]
+    _want(bt, torch.int32, "next block_table")
+    if bt.dim() != 2 or bt.stride(1) != 1:
+        raise ValueError("next block_table must be [rows, max_blocks] with unit inner stride")
+    _vector(n["positions"], torch.int64, "next positions", n["num_actual_tokens"])
+    _vector(n["slot_mapping"], torch.int64, "next slot_mapping", n["num_actual_tokens"])
+    if n.get("query_start_loc") is not None:
+        _vector(n["query_start_loc"], torch.int32, "next query_start_loc", n["num_reqs"] + 1)
+    for k in ("seq_idx_out", "query_start_out"):
+        if n.get(k) is not None:
+            _vector(n[k], torch.int32, k, npad)
+    tout = n["taps_out"]
+    _want(tout, torch.int64, "taps_out")
+    if not tout.is_contiguous():
+        raise ValueError("taps_out must be contiguous")
+    d = _dev(x, weight, cache, slot_mapping, taps, out, err_flag, bt, n["positions"],
+             n["slot_mapping"], tout)
+    if T:
+        _vector(slot_mapping, torch.int64, "slot_mapping", T)
+        if out.dtype != x.dtype or tuple(out.shape) != (T, C) or out.stride(1) != 1:
+            raise ValueError("out must be [T, C] like x with unit channel stride")
+    if W > 1 and T:
+        _want(taps, torch.int64, "taps")
+        if taps.dim() != 2 or taps.shape[0] < T or taps.shape[1] != W - 1 or \
+                not taps.is_contiguous():
+            raise ValueError("taps must be a contiguous [>= T, W-1] int64 table")
+    if err_flag is not None:
+        _vector(err_flag, torch.int32, "err_flag", 1)
+    if cache.shape[2] != block_size:
+        raise ValueError("cache.shape[2] must equal block_size")
+    nb, H, N, D = cache.shape
+    cs = (ctypes.c_int64 * 4)(*cache.stride())
+    desc = (StreamDesc * 1)(StreamDesc(_ptr(x), x.stride(0), _ptr(weight), weight.stride(0),
+                                       weight.stride(1), _ptr(out), out.stride(0), off_s, ws,
+                                       _act(activation), int(bool(use_residual))))
+    si, qs = n.get("seq_idx_out"), n.get("query_start_out")
+    build = TapsBuild(_ptr(n.get("query_start_loc")), n["num_reqs"], n["num_actual_tokens"],
+                      npad, _ptr(n["positions"]), _ptr(n["slot_mapping"]), _ptr(bt),
+                      bt.stride(0), bt.shape[1], _ptr(si), si.numel() if si is not None else 0,
+                      _ptr(qs), qs.numel() if qs is not None else 0, _ptr(tout), tout.numel())
+    with torch.cuda.device(d):
+        st = LIB.sconv_fused_taps_next(
+            desc, 1, T, W, _ptr(cache), cs, nb, H, N, D, _ptr(slot_mapping),
+            _ptr(taps) if (W > 1 and T) else 0, dt, _ptr(err_flag), ctypes.byref(build),
+            _stream(d, stream))
+    _check("sconv_fused_taps_next", st)
+    return out
 
 
 def sconv_fused_taps(x, weight, cache, slot_mapping, taps, off_s, ws, block_size,

@@ -290,17 +290,16 @@ sconv_status sconv_fused_streams(const sconv_stream_desc *streams, int n_streams
                : SCONV_ERR_LAUNCH;
 }
 
-sconv_status sconv_fused_taps(const sconv_stream_desc *streams, int n_streams, int T, int W,
-                              void *cache, const int64_t cache_strides[4], int64_t num_blocks,
-                              int H, int N, int D, const int64_t *slot_mapping,
-                              const int64_t *taps, int metadata_ready, sconv_dtype dt,
-                              int32_t *err_flag, cudaStream_t stream) {
-    if (T < 0 || n_streams < 1 || !streams) return SCONV_ERR_INVALID;
-    if (n_streams > SCONV_MAX_STREAMS) return SCONV_ERR_UNSUPPORTED;
-    if (T == 0) return SCONV_OK;
+}  // extern "C"
+
+namespace {
+// Shared checks of sconv_fused_taps and sconv_fused_taps_next (T > 0).
+sconv_status check_taps_call(const sconv_stream_desc *streams, int n_streams, int T, int W,
+                             void *cache, const int64_t cache_strides[4], int64_t num_blocks,
+                             int H, int N, int D, const int64_t *slot_mapping, const int64_t *taps,
+                             sconv_dtype dt, int32_t *err_flag, FusedArgs *a, bool &vec_all) {
     if (W > 1 && !taps) return SCONV_ERR_INVALID;
-    FusedArgs a[SCONV_MAX_STREAMS];
-    bool vec_all = true;
+    vec_all = true;
     const int64_t e = elem_size(dt);
     const int64_t taps_bytes = static_cast<int64_t>(T) * (W > 1 ? W - 1 : 0) * 8;
     for (int i = 0; i < n_streams; ++i) {
@@ -328,6 +327,26 @@ sconv_status sconv_fused_taps(const sconv_stream_desc *streams, int n_streams, i
                 return SCONV_ERR_INVALID;
         }
     }
+    return SCONV_OK;
+}
+}  // namespace
+
+extern "C" {
+
+sconv_status sconv_fused_taps(const sconv_stream_desc *streams, int n_streams, int T, int W,
+                              void *cache, const int64_t cache_strides[4], int64_t num_blocks,
+                              int H, int N, int D, const int64_t *slot_mapping,
+                              const int64_t *taps, int metadata_ready, sconv_dtype dt,
+                              int32_t *err_flag, cudaStream_t stream) {
+    if (T < 0 || n_streams < 1 || !streams) return SCONV_ERR_INVALID;
+    if (n_streams > SCONV_MAX_STREAMS) return SCONV_ERR_UNSUPPORTED;
+    if (T == 0) return SCONV_OK;
+    FusedArgs a[SCONV_MAX_STREAMS];
+    bool vec_all = true;
+    const sconv_status st = check_taps_call(streams, n_streams, T, W, cache, cache_strides,
+                                            num_blocks, H, N, D, slot_mapping, taps, dt, err_flag,
+                                            a, vec_all);
+    if (st != SCONV_OK) return st;
     return sconv::launch_fused_taps(a, n_streams, dt == SCONV_BF16, vec_all,
                                     metadata_ready != 0, stream) == cudaSuccess
                ? SCONV_OK
@@ -568,14 +587,16 @@ sconv_status seq_metadata(const int32_t *query_start_loc, int num_reqs, int num_
 }  // namespace
 
 namespace {
-sconv_status seq_metadata_taps(const int32_t *qsl, int num_reqs, int num_actual,
-                               int num_padded, const int64_t *positions,
-                               const int64_t *slot_mapping, const int32_t *block_table,
-                               int64_t bt_rs, int max_blocks, int64_t num_blocks, int N, int W,
-                               int32_t *seq_idx_out, int64_t seq_idx_cap,
-                               int32_t *query_start_out, int64_t query_start_cap,
-                               int64_t *taps_out, int64_t taps_cap, bool ahead,
-                               cudaStream_t stream) {
+// Checks of a tap resolution; on SCONV_OK fills `a`, and `empty` says there
+// is nothing to write.
+sconv_status resolve_args(const int32_t *qsl, int num_reqs, int num_actual, int num_padded,
+                          const int64_t *positions, const int64_t *slot_mapping,
+                          const int32_t *block_table, int64_t bt_rs, int max_blocks,
+                          int64_t num_blocks, int N, int W, int32_t *seq_idx_out,
+                          int64_t seq_idx_cap, int32_t *query_start_out,
+                          int64_t query_start_cap, int64_t *taps_out, int64_t taps_cap,
+                          sconv::TapResolveArgs &a, bool &empty) {
+    empty = true;
     if (num_padded < 0) num_padded = num_actual;
     if (num_actual < 0 || num_reqs < 0 || num_padded < num_actual) return SCONV_ERR_INVALID;
     if (W < 1) return SCONV_ERR_INVALID;
@@ -590,7 +611,7 @@ sconv_status seq_metadata_taps(const int32_t *qsl, int num_reqs, int num_actual,
     if ((W > 1 && !taps_out) || (num_actual > 0 && (!positions || !slot_mapping || !block_table)))
         return SCONV_ERR_INVALID;
     if (W == 1 && !seq_idx_out && !query_start_out) return SCONV_OK;  // nothing to write
-    sconv::TapResolveArgs a = {};
+    a = sconv::TapResolveArgs{};
     a.qsl = qsl;
     a.num_reqs = num_reqs;
     a.num_actual = num_actual;
@@ -606,10 +627,80 @@ sconv_status seq_metadata_taps(const int32_t *qsl, int num_reqs, int num_actual,
     a.seq_idx = seq_idx_out;
     a.qstart = query_start_out;
     a.taps = taps_out;
+    empty = false;
+    return SCONV_OK;
+}
+
+sconv_status seq_metadata_taps(const int32_t *qsl, int num_reqs, int num_actual,
+                               int num_padded, const int64_t *positions,
+                               const int64_t *slot_mapping, const int32_t *block_table,
+                               int64_t bt_rs, int max_blocks, int64_t num_blocks, int N, int W,
+                               int32_t *seq_idx_out, int64_t seq_idx_cap,
+                               int32_t *query_start_out, int64_t query_start_cap,
+                               int64_t *taps_out, int64_t taps_cap, bool ahead,
+                               cudaStream_t stream) {
+    sconv::TapResolveArgs a;
+    bool empty = true;
+    const sconv_status st = resolve_args(qsl, num_reqs, num_actual, num_padded, positions,
+                                         slot_mapping, block_table, bt_rs, max_blocks, num_blocks,
+                                         N, W, seq_idx_out, seq_idx_cap, query_start_out,
+                                         query_start_cap, taps_out, taps_cap, a, empty);
+    if (st != SCONV_OK || empty) return st;
     return sconv::launch_seq_metadata_taps(a, ahead, stream) == cudaSuccess ? SCONV_OK
                                                                             : SCONV_ERR_LAUNCH;
 }
 }  // namespace
+
+sconv_status sconv_fused_taps_next(const sconv_stream_desc *streams, int n_streams, int T, int W,
+                                   void *cache, const int64_t cache_strides[4],
+                                   int64_t num_blocks, int H, int N, int D,
+                                   const int64_t *slot_mapping, const int64_t *taps,
+                                   sconv_dtype dt, int32_t *err_flag,
+                                   const sconv_taps_build *next, cudaStream_t stream) {
+    if (T < 0 || n_streams < 1 || !streams || !next) return SCONV_ERR_INVALID;
+    if (n_streams > SCONV_MAX_STREAMS) return SCONV_ERR_UNSUPPORTED;
+    sconv::TapResolveArgs nx;
+    bool empty = true;
+    sconv_status st = resolve_args(
+        next->query_start_loc, next->num_reqs, next->num_actual_tokens,
+        next->num_padded_tokens, next->positions, next->slot_mapping, next->block_table,
+        next->bt_row_stride, next->max_blocks, num_blocks, N, W, next->seq_idx_out,
+        next->seq_idx_cap, next->query_start_out, next->query_start_cap, next->taps_out,
+        next->taps_cap, nx, empty);
+    if (st != SCONV_OK) return st;
+    if (T == 0) {
+        if (empty) return SCONV_OK;
+        return sconv::launch_seq_metadata_taps(nx, true, stream) == cudaSuccess
+                   ? SCONV_OK
+                   : SCONV_ERR_LAUNCH;
+    }
+    FusedArgs a[SCONV_MAX_STREAMS];
+    bool vec_all = true;
+    st = check_taps_call(streams, n_streams, T, W, cache, cache_strides, num_blocks, H, N, D,
+                         slot_mapping, taps, dt, err_flag, a, vec_all);
+    if (st != SCONV_OK) return st;
+    if (!empty && next->taps_out && W > 1) {
+        const int64_t nb = static_cast<int64_t>(nx.num_padded) * (W - 1) * 8;
+        const int64_t tb = static_cast<int64_t>(T) * (W - 1) * 8;
+        if (overlaps(next->taps_out, nb, taps, tb)) return SCONV_ERR_INVALID;
+        const int64_t e = elem_size(dt);
+        for (int i = 0; i < n_streams; ++i) {
+            const sconv_stream_desc &d = streams[i];
+            const int64_t out_bytes =
+                ((static_cast<int64_t>(T) - 1) * d.out_row_stride + H * d.ws) * e;
+            if (overlaps(next->taps_out, nb, d.out, out_bytes)) return SCONV_ERR_INVALID;
+        }
+    }
+    if (empty)
+        return sconv::launch_fused_taps(a, n_streams, dt == SCONV_BF16, vec_all, false, stream) ==
+                       cudaSuccess
+                   ? SCONV_OK
+                   : SCONV_ERR_LAUNCH;
+    return sconv::launch_fused_taps_next(a, n_streams, dt == SCONV_BF16, vec_all, nx, stream) ==
+                   cudaSuccess
+               ? SCONV_OK
+               : SCONV_ERR_LAUNCH;
+}
 
 sconv_status sconv_seq_metadata_taps(const int32_t *query_start_loc, int num_reqs,
                                      int num_actual_tokens, int num_padded_tokens,

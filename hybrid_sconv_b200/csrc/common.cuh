@@ -342,6 +342,10 @@ cudaError_t launch_seq_metadata_taps(TapResolveArgs &a, bool ahead, cudaStream_t
 // table; `ready`: slot_mapping and the table may be read before the wait.
 cudaError_t launch_fused_taps(FusedArgs *s, int n, bool bf16_data, bool vec, bool ready,
                               cudaStream_t stream);
+// The same (taps read after the wait) with the next step's table built by
+// extra blocks of the same launch.
+cudaError_t launch_fused_taps_next(FusedArgs *s, int n, bool bf16_data, bool vec,
+                                   TapResolveArgs &next, cudaStream_t stream);
 
 // Launch with programmatic stream serialization enabled.
 template <typename Kernel, typename... Args>

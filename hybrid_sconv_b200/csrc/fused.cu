@@ -36,6 +36,7 @@
 #include "common.cuh"
 #include "fused_common.cuh"
 #include "sconv.h"
+#include "taps_resolve.cuh"
 
 namespace sconv {
 namespace {
@@ -408,6 +409,50 @@ __global__ void __launch_bounds__(kThreads) fused_taps_streams_kernel(const __gr
     with_stream(m, si, [&](const FusedArgs &a) { taps_body<E, VEC, MAXW, READY>(a, pack, t); });
 }
 
+// The fused step with the NEXT step's table built in the same launch
+// (sconv_fused_taps_next): blocks with blockIdx.x < gx convolve this step
+// (its table read after the wait, speculatively prefetched before it);
+// blocks beyond build the next step's table from the next step's inputs,
+// which no running kernel writes, so they neither wait nor hold back the
+// launch of this grid's dependents (they signal at entry).  The next launch
+// still waits for this whole grid before it reads that table.
+template <bool DECODE_NEXT, int MAXW>
+__device__ __forceinline__ void build_next(const TapResolveArgs &nx, int gx) {
+    extern __shared__ int32_t s_qsl[];
+    pdl_trigger();
+    if (blockIdx.y != 0) return;  // one row of build blocks
+    const int nthr = blockDim.x * blockDim.y;
+    const int tid = threadIdx.y * blockDim.x + threadIdx.x;
+    resolve_block<DECODE_NEXT, MAXW>(nx, (blockIdx.x - gx) * nthr + tid, tid, nthr, s_qsl);
+}
+
+template <typename E, int VEC, int MAXW, bool DECODE_NEXT>
+__global__ void __launch_bounds__(kThreads)
+fused_taps_next_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ TapResolveArgs nx,
+                       int gx) {
+    if (static_cast<int>(blockIdx.x) >= gx) {
+        build_next<DECODE_NEXT, MAXW>(nx, gx);
+        return;
+    }
+    taps_body<E, VEC, MAXW, false>(a, blockIdx.y * blockDim.x + threadIdx.x,
+                                   blockIdx.x * blockDim.y + threadIdx.y);
+}
+
+template <typename E, int VEC, int MAXW, bool DECODE_NEXT>
+__global__ void __launch_bounds__(kThreads)
+fused_taps_streams_next_kernel(const __grid_constant__ StreamSet m,
+                               const __grid_constant__ TapResolveArgs nx, int gx) {
+    if (static_cast<int>(blockIdx.x) >= gx) {
+        build_next<DECODE_NEXT, MAXW>(nx, gx);
+        return;
+    }
+    int si = 0;
+    while (si + 1 < m.n && static_cast<int>(blockIdx.y) >= m.y0[si + 1]) ++si;
+    const int pack = (blockIdx.y - m.y0[si]) * blockDim.x + threadIdx.x;
+    const int t = blockIdx.x * blockDim.y + threadIdx.y;
+    with_stream(m, si, [&](const FusedArgs &a) { taps_body<E, VEC, MAXW, false>(a, pack, t); });
+}
+
 // Ring of x rows: Q >= PF + MAXW slots, a power of two.
 template <int PF, int MAXW>
 struct Ring {
@@ -689,6 +734,45 @@ cudaError_t launch_taps_t(FusedArgs *s, int n, bool ready, cudaStream_t stream) 
                               stream, m);
 }
 
+template <typename E, int VEC, int MAXW>
+cudaError_t launch_taps_next_t(FusedArgs *s, int n, TapResolveArgs &nx, cudaStream_t stream) {
+    StreamSet m;
+    m.n = n;
+    int nv_max = 0;
+    for (int i = 0; i < n; ++i) nv_max = s[i].C / VEC > nv_max ? s[i].C / VEC : nv_max;
+    const Shape sh = block_shape(nv_max, s[0].T);
+    m.y0[0] = 0;
+    for (int i = 0; i < n; ++i) {
+        s[i].w_vec = s[i].w_vec && s[i].W == MAXW;
+        m.s[i] = s[i];
+        m.y0[i + 1] = m.y0[i] + (s[i].C / VEC + sh.cv - 1) / sh.cv;
+    }
+    for (int i = n; i < SCONV_MAX_STREAMS; ++i) m.s[i] = s[0];  // never selected
+    const int gx = (s[0].T + sh.tg - 1) / sh.tg;
+    const int threads = sh.cv * sh.tg;
+    const int bx = (nx.num_padded + threads - 1) / threads;  // build blocks
+    size_t smem = 0;
+    resolve_staging(nx, smem);
+    const dim3 grid(static_cast<unsigned>(gx + bx), static_cast<unsigned>(m.y0[n]));
+    const dim3 block(sh.cv, sh.tg);
+    const bool dec = nx.qsl == nullptr;
+    if (n == 1)
+        return dec ? launch_pdl(fused_taps_next_kernel<E, VEC, MAXW, true>, grid, block, smem,
+                                stream, m.s[0], nx, gx)
+                   : launch_pdl(fused_taps_next_kernel<E, VEC, MAXW, false>, grid, block, smem,
+                                stream, m.s[0], nx, gx);
+    return dec ? launch_pdl(fused_taps_streams_next_kernel<E, VEC, MAXW, true>, grid, block, smem,
+                            stream, m, nx, gx)
+               : launch_pdl(fused_taps_streams_next_kernel<E, VEC, MAXW, false>, grid, block,
+                            smem, stream, m, nx, gx);
+}
+
+template <typename E, int VEC>
+cudaError_t launch_taps_next_v(FusedArgs *s, int n, TapResolveArgs &nx, cudaStream_t stream) {
+    if (s[0].W <= 4) return launch_taps_next_t<E, VEC, 4>(s, n, nx, stream);
+    return launch_taps_next_t<E, VEC, 8>(s, n, nx, stream);
+}
+
 template <typename E, int VEC>
 cudaError_t launch_taps_v(FusedArgs *s, int n, bool ready, cudaStream_t stream) {
     if (s[0].W <= 4) return launch_taps_t<E, VEC, 4>(s, n, ready, stream);
@@ -732,6 +816,20 @@ cudaError_t launch_fused_taps(FusedArgs *s, int n, bool bf16_data, bool vec, boo
                    : launch_taps_v<bf16, 1>(s, n, ready, stream);
     return vec ? launch_taps_v<float, 4>(s, n, ready, stream)
                : launch_taps_v<float, 1>(s, n, ready, stream);
+}
+
+cudaError_t launch_fused_taps_next(FusedArgs *s, int n, bool bf16_data, bool vec,
+                                   TapResolveArgs &next, cudaStream_t stream) {
+    for (int i = 0; i < n; ++i) {
+        s[i].divN = FastDiv::make(static_cast<uint32_t>(s[i].N));
+        s[i].slots32 = s[i].num_blocks * s[i].N < (1ll << 31);
+        s[i].strip = 1;
+    }
+    if (bf16_data)
+        return vec ? launch_taps_next_v<bf16, 8>(s, n, next, stream)
+                   : launch_taps_next_v<bf16, 1>(s, n, next, stream);
+    return vec ? launch_taps_next_v<float, 4>(s, n, next, stream)
+               : launch_taps_next_v<float, 1>(s, n, next, stream);
 }
 
 cudaError_t launch_fused(FusedArgs &a, bool bf16_data, bool vec, bool one, cudaStream_t stream) {

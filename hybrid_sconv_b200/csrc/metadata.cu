@@ -9,6 +9,7 @@
 // also resolves every token's pre-forward taps into a table.
 #include "common.cuh"
 #include "sconv.h"
+#include "taps_resolve.cuh"
 
 namespace sconv {
 namespace {
@@ -62,117 +63,23 @@ seq_metadata_kernel(const int32_t *__restrict__ qsl, int num_reqs, int num_actua
     if (AHEAD) pdl_wait();  // every thread: the grid completes after its predecessor
 }
 
-// Tap resolution, one thread per token row ("vllm.models.inkling.nvidia.ops.sconv",
-// module docstring: a tap in the current forward comes from x, an earlier
-// one from the cache through block_table[req, src / N] at offset src % N, a
-// tap before position 0 is zero).  The request and its first row come from
-// the same binary search as above, or are the token itself in the decode
-// form.  Row t of the table holds, for lag d = 1..W-1, SCONV_TAP_X,
-// SCONV_TAP_ZERO, the flat cache slot b*N + src % N, or -(bits << 8) at every
-// lag when the token cannot be resolved.  A thread issues its W-1
-// block-table loads together, so the lookup is two dependent accesses
-// (positions and query_start_loc, then the block table).
+// The standalone tap resolution (taps_resolve.cuh), one thread per token.
 template <bool AHEAD, bool DECODE, int MAXW>
 __global__ void __launch_bounds__(kThreads) seq_metadata_taps_kernel(const TapResolveArgs a) {
     extern __shared__ int32_t s_qsl[];
     pdl_trigger();  // as in seq_metadata_kernel
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
-    const bool live = t < a.num_actual;
     if (!AHEAD) {
         if (!DECODE)
             for (int i = threadIdx.x * 32; i < a.num_reqs; i += blockDim.x * 32)
                 prefetch_l2(a.qsl + i);
-        if (live && (threadIdx.x & 15) == 0) {
+        if (t < a.num_actual && (threadIdx.x & 15) == 0) {
             prefetch_l2(a.positions + t);
             prefetch_l2(a.slot + t);
         }
         pdl_wait();
     }
-    int64_t pos = 0, slot = -1;
-    if (live) {
-        pos = __ldg(a.positions + t);
-        slot = __ldg(a.slot + t);
-    }
-    if (!DECODE && a.staged) {
-        for (int i = threadIdx.x; i < a.num_reqs; i += blockDim.x) s_qsl[i] = __ldg(a.qsl + i);
-        __syncthreads();
-    }
-    if (t < a.num_padded) {
-        int r = 0, q0 = 0;
-        if (live) {
-            if (DECODE) {
-                r = t;
-                q0 = t;
-            } else {
-                const int32_t *q = a.staged ? s_qsl : a.qsl;
-                int lo = 0, hi = a.num_reqs - 1;
-                while (lo < hi) {
-                    const int mid = (lo + hi + 1) >> 1;
-                    if (q[mid] <= t) lo = mid;
-                    else hi = mid - 1;
-                }
-                r = lo;
-                q0 = q[lo];
-            }
-        }
-        if (a.seq_idx) a.seq_idx[t] = r;
-        if (a.qstart) a.qstart[t] = q0;
-
-        int64_t e[MAXW];
-#pragma unroll
-        for (int d = 1; d < MAXW; ++d) e[d] = SCONV_TAP_ZERO;
-        if (live && slot != -1) {
-            unsigned flags = 0;
-            if (r >= a.num_reqs) flags |= SCONV_EFLAG_REQUEST;
-            if (q0 < 0 || q0 > t) flags |= SCONV_EFLAG_QUERY_START;
-            if (pos < 0) flags |= SCONV_EFLAG_POSITION;
-            if (!flags) {
-                const int32_t *row = a.bt + static_cast<int64_t>(r) * a.bt_rs;
-                int32_t blk[MAXW];
-                int64_t off[MAXW];
-                bool need[MAXW];
-#pragma unroll
-                for (int d = 1; d < MAXW; ++d) {  // issue every block-table load first
-                    need[d] = false;
-                    if (d >= a.W) continue;
-                    const int64_t src = pos - d;
-                    if (t - d >= q0) {
-                        e[d] = SCONV_TAP_X;
-                    } else if (src >= 0) {
-                        int64_t lb;
-                        if (src < (1ll << 31)) {
-                            const uint32_t q = a.divN.div(static_cast<uint32_t>(src));
-                            lb = q;
-                            off[d] = src - static_cast<int64_t>(q) * a.N;
-                        } else {
-                            lb = src / a.N;
-                            off[d] = src - lb * a.N;
-                        }
-                        if (lb >= a.max_blocks) {
-                            flags |= SCONV_EFLAG_LOGICAL;
-                        } else {
-                            blk[d] = __ldg(row + lb);
-                            need[d] = true;
-                        }
-                    }
-                }
-#pragma unroll
-                for (int d = 1; d < MAXW; ++d) {
-                    if (!need[d]) continue;
-                    if (blk[d] < 0 || blk[d] >= a.num_blocks) flags |= SCONV_EFLAG_BLOCK;
-                    else e[d] = static_cast<int64_t>(blk[d]) * a.N + off[d];
-                }
-            }
-            if (flags) {
-#pragma unroll
-                for (int d = 1; d < MAXW; ++d) e[d] = -static_cast<int64_t>(flags) * 256;
-            }
-        }
-        int64_t *out = a.taps + static_cast<int64_t>(t) * (a.W - 1);
-#pragma unroll
-        for (int d = 1; d < MAXW; ++d)
-            if (d < a.W) out[d - 1] = e[d];
-    }
+    resolve_block<DECODE, MAXW>(a, t, threadIdx.x, blockDim.x, s_qsl);
     if (AHEAD) pdl_wait();  // every thread: the grid completes after its predecessor
 }
 
@@ -189,10 +96,9 @@ cudaError_t launch_taps_w(const TapResolveArgs &a, size_t smem, cudaStream_t str
 }  // namespace
 
 cudaError_t launch_seq_metadata_taps(TapResolveArgs &a, bool ahead, cudaStream_t stream) {
-    a.divN = FastDiv::make(static_cast<uint32_t>(a.N));
+    size_t smem = 0;
+    resolve_staging(a, smem);
     const bool decode = a.qsl == nullptr;
-    a.staged = !decode && a.num_reqs <= kSmemReqs ? 1 : 0;
-    const size_t smem = a.staged ? static_cast<size_t>(a.num_reqs) * sizeof(int32_t) : 0;
     if (ahead)
         return decode ? launch_taps_w<true, true>(a, smem, stream)
                       : launch_taps_w<true, false>(a, smem, stream);

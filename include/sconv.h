@@ -526,6 +526,57 @@ sconv_status sconv_fused_taps(
     const int64_t *slot_mapping, const int64_t *taps, int metadata_ready, sconv_dtype dt,
     int32_t *err_flag, cudaStream_t stream);
 
+/*
+ * One step's tap resolution for sconv_fused_taps_next: the arguments of
+ * sconv_seq_metadata_taps for that step, with num_blocks, N and W taken from
+ * the sconv_fused_taps_next call.
+ */
+typedef struct sconv_taps_build {
+    const int32_t *query_start_loc;   /* [num_reqs + 1], or NULL (decode form) */
+    int num_reqs, num_actual_tokens, num_padded_tokens; /* num_padded < 0: num_actual */
+    const int64_t *positions;         /* [num_actual_tokens] */
+    const int64_t *slot_mapping;      /* [num_actual_tokens] */
+    const int32_t *block_table;       /* [num_reqs, max_blocks] */
+    int64_t bt_row_stride;
+    int max_blocks;
+    int32_t *seq_idx_out;             /* may be NULL */
+    int64_t seq_idx_cap;
+    int32_t *query_start_out;         /* may be NULL */
+    int64_t query_start_cap;
+    int64_t *taps_out;                /* [num_padded_tokens, W - 1] */
+    int64_t taps_cap;
+} sconv_taps_build;
+
+/*
+ * sconv_fused_taps_next -- one decode-loop step in one launch: the fused
+ * step of sconv_fused_taps for this step (metadata_ready 0: its table is read
+ * after the wait for the kernels this launch depends on) and, by extra
+ * blocks of the same launch, the tap resolution of sconv_seq_metadata_taps
+ * for the NEXT step (`next`).  Those blocks read only the next step's inputs
+ * and write only its outputs, so they start at once, never wait and do not
+ * hold back the launch of the calls that follow; a following call still
+ * waits for this whole launch before it reads the table built here.  So a
+ * loop of calls, each building the table the next one reads, keeps the
+ * tap resolution off the dependent path of its convolutions, with one launch
+ * per step (the first step's table comes from sconv_seq_metadata_taps).
+ *
+ *   every argument up to err_flag: as in sconv_fused_taps.
+ *   next     the next step's resolution; must not be NULL.  Its taps_out
+ *            must not overlap `taps` or any out; the same preconditions as
+ *            sconv_seq_metadata_taps_ahead apply to its buffers (no kernel
+ *            that may still be running writes its inputs or touches its
+ *            outputs).
+ * Errors: those of sconv_fused_taps and of sconv_seq_metadata_taps for
+ * `next`.  T == 0 is allowed (the launch then only builds the next table);
+ * T == 0 with next->num_padded_tokens == 0 returns SCONV_OK and enqueues
+ * nothing.
+ */
+sconv_status sconv_fused_taps_next(
+    const sconv_stream_desc *streams, int n_streams, int T, int W,
+    void *cache, const int64_t cache_strides[4], int64_t num_blocks, int H, int N, int D,
+    const int64_t *slot_mapping, const int64_t *taps, sconv_dtype dt, int32_t *err_flag,
+    const sconv_taps_build *next, cudaStream_t stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *sconv_status_string(sconv_status status);
 

@@ -291,3 +291,25 @@ def test_fused_taps_host_validation(lib):
     assert call([ok], W=9) == 2
     assert call([ok], cs=_strides(512, 256, 16, 2)) == 1    # D stride must be 1
     assert call([ok], dt=7) == 2
+
+
+def test_fused_taps_next_host_validation(lib):
+    """The combined step checks both its convolution arguments and the next
+    step's resolution, and rejects a next table that overlaps this step's
+    table or output, before any launch."""
+    from hybrid_sconv_b200.binding import StreamDesc, TapsBuild
+
+    def call(T=4, W=4, taps=FAKE * 2048, next_taps=FAKE * 4096, npad=8, nq=FAKE * 8,
+             nnull=False):
+        d = (StreamDesc * 1)(StreamDesc(FAKE, 8, FAKE + 4096, 4, 1, FAKE * 512, 8, 0, 4, 0, 1))
+        b = TapsBuild(nq, 2, npad, npad, FAKE * 16, FAKE * 24, FAKE * 32, 4, 4, 0, 0, 0, 0,
+                      next_taps, npad * (W - 1))
+        return lib.sconv_fused_taps_next(d, 1, T, W, FAKE * 64, _strides(512, 256, 16, 1), 8,
+                                         2, 16, 16, FAKE, taps, 1, 0,
+                                         None if nnull else ctypes.byref(b), 0)
+    assert call(nnull=True) == 1                      # next is required
+    assert call(T=0, npad=0) == 0                     # nothing to do
+    assert call(taps=0) == 1                          # this step's table is needed
+    assert call(next_taps=FAKE * 2048 + 8) == 1       # next table overlaps this one
+    assert call(next_taps=FAKE * 512 + 8) == 1        # next table inside the output
+    assert call(W=9) == 2

@@ -106,3 +106,13 @@ def test_algorithmic_bytes_taps_by_hand():
     C, e = 8, 2
     expect = 2 * C * e + 2 * 2 * C * e + 3 * C * e + C * 4 * e + (8 + 24) * 2
     assert bench.algorithmic_bytes_taps(wl) == expect
+
+
+def test_algorithmic_bytes_resolve_by_hand():
+    """One request, 2 new tokens after 9 cached ones, W = 4, N = 4: per
+    token 16 B read (position, slot) and 8 + 24 B written (seq_idx,
+    query_start, table row); query_start_loc 2 entries; the three history
+    rows (positions 6, 7, 8) lie in two logical blocks."""
+    wl = workloads.build("h", dtype="bf16", H=1, D=8, ws=8, off_s=0, W=4, N=4, hist=[9],
+                         new=[2], act=None, residual=False, seed=3)
+    assert bench.algorithmic_bytes_resolve(wl) == 16 * 2 + 4 * 2 + 4 * 2 + 32 * 2

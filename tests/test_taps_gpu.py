@@ -347,3 +347,134 @@ def test_interleaved_graph_equals_plain_steps():
             assert torch.equal(raw(r), raw(s["out"]))
         assert torch.equal(raw(cache), raw(ref_cache))
     del graph
+
+
+def _next_dict(wl, md, taps_out, decode_form=False, si=None, qs=None):
+    return dict(query_start_loc=None if decode_form else md["query_start_loc"],
+                num_reqs=wl.block_table.shape[0] if decode_form else wl.R,
+                num_actual_tokens=wl.T, positions=md["positions"],
+                slot_mapping=md["slot_mapping"], block_table=md["block_table"],
+                taps_out=taps_out, seq_idx_out=si, query_start_out=qs)
+
+
+@pytest.mark.parametrize("decode_form", [False, True])
+def test_fused_taps_next_one_call(decode_form):
+    """One launch: this step's convolution (bit for bit sconv_fused_taps on
+    the same table, and the oracle's step within tolerance) and the next
+    step's table (bit for bit the oracle's resolution)."""
+    a = workloads.decode_bf16(seed=41, R=96, max_hist=900)
+    b = workloads.spec_decode_bf16(seed=42, max_hist=700) if not decode_form else \
+        workloads.decode_bf16(seed=43, R=80, max_hist=500)
+    ta = a.tensors(DEV)
+    # one cache serves both steps: the next step's taps are resolved against it
+    nb = max(a.num_blocks, b.num_blocks)
+    big = torch.empty((nb, a.H, a.N, a.D), dtype=torch.bfloat16, device=DEV)
+    workloads.fill_normal_(big, 1.0, torch.Generator(device=DEV).manual_seed(41), DEV)
+    big[:a.num_blocks].copy_(ta["cache"])
+    ta["cache"] = big
+    mdb = b.metadata(DEV)
+    _, _, taps_a = resolve(a, ta)
+    torch.cuda.synchronize()
+    cache0 = ta["cache"].clone()
+    ref = hs().sconv_fused_taps(ta["x"], ta["weight"], ta["cache"], ta["slot_mapping"], taps_a,
+                                **a.kwargs())
+    torch.cuda.synchronize()
+    ref_cache = ta["cache"].clone()
+    ta["cache"].copy_(cache0)
+    taps_b = torch.full((b.T, b.W - 1), -7, dtype=torch.int64, device=DEV)
+    si = torch.full((b.T,), -7, dtype=torch.int32, device=DEV)
+    qs = torch.full((b.T,), -7, dtype=torch.int32, device=DEV)
+    out = hs().sconv_fused_taps_next(ta["x"], ta["weight"], ta["cache"], ta["slot_mapping"],
+                                     taps_a, next_step=_next_dict(b, mdb, taps_b, decode_form,
+                                                                  si, qs), **a.kwargs())
+    torch.cuda.synchronize()
+    assert torch.equal(raw(out), raw(ref))
+    assert torch.equal(raw(ta["cache"]), raw(ref_cache))
+    rsi, rqs, rtaps = oracle_resolve(b, decode_form=decode_form)
+    np.testing.assert_array_equal(taps_b.cpu().numpy(), rtaps)
+    np.testing.assert_array_equal(si.cpu().numpy(), rsi)
+    np.testing.assert_array_equal(qs.cpu().numpy(), rqs)
+    refo, state, _, _ = oracle_fused(a, ta["x"].cpu(), ta["weight"].cpu(), cache0.cpu(),
+                                     a.metadata("cpu"), write_cache=False)
+    rows = state == 1
+    assert_close(oracle.to_f64(out.cpu(), "bf16")[rows], refo[rows], "bf16", "fused_taps_next")
+
+
+def test_fused_taps_next_build_only():
+    """T == 0: the launch only builds the next step's table."""
+    b = workloads.decode_bf16(seed=44, R=33, max_hist=200)
+    mdb = b.metadata(DEV)
+    x = torch.empty((0, b.C), dtype=torch.bfloat16, device=DEV)
+    w = torch.zeros((b.C, b.W), dtype=torch.bfloat16, device=DEV)
+    cache = torch.zeros((b.num_blocks, b.H, b.N, b.D), dtype=torch.bfloat16, device=DEV)
+    taps_b = torch.full((b.T, b.W - 1), -7, dtype=torch.int64, device=DEV)
+    hs().sconv_fused_taps_next(x, w, cache, torch.empty(0, dtype=torch.int64, device=DEV), None,
+                               next_step=_next_dict(b, mdb, taps_b), **b.kwargs())
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(taps_b.cpu().numpy(), oracle_resolve(b)[2])
+
+
+def test_fused_taps_next_loop_graph_equals_plain_steps():
+    """A decode loop of one launch per step, each building the next step's
+    table, captured in a graph and replayed with every table reset (the
+    first from the standalone builder), equals the plain sequence of
+    sconv_fused steps on one shared cache, bit for bit."""
+    wls = [workloads.decode_bf16(seed=600 + i, R=64, max_hist=600) for i in range(6)]
+    nb = max(w.num_blocks for w in wls)
+    w0 = wls[0]
+    g = torch.Generator(device="cpu").manual_seed(6)
+    cache = torch.empty((nb, w0.H, w0.N, w0.D), dtype=torch.bfloat16, device=DEV)
+    workloads.fill_normal_(cache, 1.0, torch.Generator(device=DEV).manual_seed(6), DEV)
+    weight = workloads.normal((w0.C, w0.W), 0.5, torch.bfloat16, g, "cpu").to(DEV)
+    sets = []
+    for wl in wls:
+        md = wl.metadata(DEV)
+        md["x"] = workloads.normal((wl.T, wl.C), 1.0, torch.bfloat16, g, "cpu").to(DEV)
+        md["out"] = torch.empty_like(md["x"])
+        md["taps"] = torch.empty((wl.T, wl.W - 1), dtype=torch.int64, device=DEV)
+        sets.append(md)
+    cache0 = cache.clone()
+    ref = [hs().sconv_fused(s["x"], weight, cache, s["positions"], s["block_table"],
+                            s["seq_idx"], s["slot_mapping"], s["query_start"], **wl.kwargs())
+           for wl, s in zip(wls, sets)]
+    torch.cuda.synchronize()
+    ref_cache = cache.clone()
+
+    def steps():
+        for i, (wl, s) in enumerate(zip(wls, sets)):
+            j = (i + 1) % len(wls)
+            hs().sconv_fused_taps_next(s["x"], weight, cache, s["slot_mapping"], s["taps"],
+                                       out=s["out"],
+                                       next_step=_next_dict(wls[j], sets[j], sets[j]["taps"]),
+                                       **wl.kwargs())
+
+    def reset():
+        cache.copy_(cache0)
+        for s in sets:
+            s["out"].fill_(0)
+            s["taps"].fill_(-7)
+        wl, s = wls[0], sets[0]
+        hs().sconv_seq_metadata_taps(s["query_start_loc"], wl.R, wl.T, s["positions"],
+                                     s["slot_mapping"], s["block_table"], wl.num_blocks, wl.N,
+                                     wl.W, taps_out=s["taps"])
+        torch.cuda.synchronize()
+
+    main = torch.cuda.Stream()
+    reset()
+    with torch.cuda.stream(main):
+        steps()
+    torch.cuda.synchronize()
+    for r, s in zip(ref, sets):
+        assert torch.equal(raw(r), raw(s["out"]))
+    assert torch.equal(raw(cache), raw(ref_cache))
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=main):
+        steps()
+    for _ in range(2):
+        reset()
+        graph.replay()
+        torch.cuda.synchronize()
+        for r, s in zip(ref, sets):
+            assert torch.equal(raw(r), raw(s["out"]))
+        assert torch.equal(raw(cache), raw(ref_cache))
+    del graph
