@@ -525,7 +525,21 @@ class L2Flush:
 HOST_LEAD_CYCLES = 2_000_000
 
 
-def time_region(full, tail, reps, stream, world, sampler=None, flush=None):
+class nvtx_range:
+    """An NVTX range around a phase of the benchmark (host-side markers for
+    a timeline profiler; they add nothing to the device's work)."""
+
+    def __init__(self, name):
+        self.name = name
+
+    def __enter__(self):
+        torch.cuda.nvtx.range_push(self.name)
+
+    def __exit__(self, *exc):
+        torch.cuda.nvtx.range_pop()
+
+
+def time_region(full, tail, reps, stream, world, sampler=None, flush=None, label="timed"):
     """Seconds for the replays, by CUDA events on the launching stream,
     bracketed by a barrier and a device synchronisation on both sides.
     flush: written on the stream before the start event (L2 cold for the
@@ -540,7 +554,7 @@ def time_region(full, tail, reps, stream, world, sampler=None, flush=None):
         sampler.start()
         time.sleep(1.0)  # nvidia-smi takes a moment before its first reading
     w0 = time.time()
-    with torch.cuda.stream(stream):
+    with torch.cuda.stream(stream), nvtx_range(label):
         if flush is not None:
             flush()
         torch.cuda._sleep(HOST_LEAD_CYCLES)
@@ -1501,7 +1515,7 @@ def main():
     carry_prologue(sets_obj, stream)
     wfull, wtail, wreps = run_steps_graphs(sets_obj, W, stream, pipeline=STEP_SCHEDULE,
                                            carry=True)
-    with torch.cuda.stream(stream):
+    with torch.cuda.stream(stream), nvtx_range("warm-up"):
         replay_steps(wfull, wtail, wreps)
     torch.cuda.synchronize()
     del wfull, wtail
@@ -1511,7 +1525,8 @@ def main():
     prime(full, tail, stream)
     carry_prologue(sets_obj, stream)
     sampler = ClockSampler(local) if rank == 0 else None
-    secs, (w0, w1) = time_region(full, tail, reps, stream, world, sampler, flush)
+    secs, (w0, w1) = time_region(full, tail, reps, stream, world, sampler, flush,
+                                 label=f"timed decode steps (K={K})")
     secs = max_over_ranks(secs, world)
     clocks = None
     if sampler is not None:
@@ -1564,14 +1579,17 @@ def main():
         line["clocks"] = clocks
 
     if not args.no_extras:
-        line["e2e"] = e2e(sets_obj, min(K, 24000), stream, world, flush)
+        with nvtx_range("e2e"):
+            line["e2e"] = e2e(sets_obj, min(K, 24000), stream, world, flush)
         if rank == 0:
-            zero = DecodeSets(args.sets, rank_seed(args.seed, rank) + 1, device, max_hist=0,
-                              min_hist=0)
-            line["per_config"] = per_workload_table(device, stream, peak, sets_obj, zero)
-            del zero
+            with nvtx_range("per-configuration table"):
+                zero = DecodeSets(args.sets, rank_seed(args.seed, rank) + 1, device, max_hist=0,
+                                  min_hist=0)
+                line["per_config"] = per_workload_table(device, stream, peak, sets_obj, zero)
+                del zero
         if rank == 0 and world == 1:
-            line["cpu_baseline"] = cpu_baseline(sets_obj)
+            with nvtx_range("cpu baseline"):
+                line["cpu_baseline"] = cpu_baseline(sets_obj)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
