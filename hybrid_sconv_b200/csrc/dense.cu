@@ -6,17 +6,17 @@
 //
 //  * dense_fwd_tile -- varlen prefill, x token-major in 16-byte channel
 //    packs.  One 256-thread block owns a (sequence, column of PP packs) and
-//    walks it in tiles of TT = 2 * 256 / PP rows: each thread copies two
-//    packs of a tile three or five tiles ahead into a shared-memory ring with
-//    cp.async (only rows of this sequence, so nothing past its end is read)
-//    and convolves two rows of the current tile.  Each ring stage holds the
-//    W-1 rows before its tile, written while the previous tile is computed;
-//    the column's last L inputs ride along in a carry that starts as the
-//    state line and ends as the new line.  No block re-reads x rows that
-//    another block may already have overwritten, so the in-place form needs
-//    no scratch memory and no ordering between blocks.  PP is chosen per
-//    call: the widest column that still gives the SMs 1.5 blocks each, and
-//    blocks run longest sequence first.
+//    walks it in tiles of TT = 2 * 256 / PP rows, which one thread brings
+//    into a shared-memory ring by tensor copy four or five tiles ahead;
+//    per-stage mbarriers pace the copies and the eight warps, with no
+//    block-wide barrier per tile.  Each thread convolves two rows of the
+//    current tile.  Each ring stage holds the W-1 rows before its tile,
+//    written while the previous tile is computed; the new state line is
+//    read from the last two tiles at the end.  No block re-reads x rows
+//    that another block may already have overwritten, so the in-place form
+//    needs no scratch memory and no ordering between blocks.  PP is chosen
+//    per call: the widest column that still gives the SMs 1.5 blocks each,
+//    and blocks run longest sequence first.
 //  * dense_fwd_cm -- channel-major x (token stride 1): a warp per (sequence,
 //    channel) walks the channel's contiguous tokens, one 16-byte vector (8
 //    bf16 or 4 fp32 tokens) per lane, with the taps before a lane's tokens
@@ -28,21 +28,26 @@
 // Every sum runs oldest tap first, starting from the bias, in fp32 FMAs, so
 // all the kernels agree bit for bit on the same token.  A sequence whose
 // line or row range is out of range is skipped and reported through the
-// optional error flag; nothing traps or waits.
+// optional error flag; nothing traps, and the tiled prefill's mbarrier
+// waits are bounded in time (SCONV_EFLAG_TIMEOUT).
+#include <mutex>
+
 #include "common.cuh"
 #include "sconv.h"
+#include "tma.cuh"
 
 namespace sconv {
 namespace {
 
 constexpr int kRowsPerThread = 2;  // rows of a tile each thread convolves
 constexpr int kTileThreads = 256;
-// Ring depth of the tiled prefill: 4 stages when the grid runs in several
+// Ring depth of the tiled prefill: 5 stages when the grid runs in several
 // waves of blocks (many sequences: short columns, where a deep ring only
 // fetches ahead of the end), 6 when the blocks fit in about one wave (long
 // columns that must stream at full rate).  Measured on the dense mixed and
-// long prefills: 4 stages 50.2 / 445 us, 6: 51.6 / 419, 8: 52.5 / 420.
-constexpr int kStagesFew = 4;
+// long prefills (us): 4 / 6 stages 49.7 / 404, 5 / 5: 49.3 / 425, 6 / 8:
+// 49.4 / 405.
+constexpr int kStagesFew = 5;
 constexpr int kStagesMany = 6;
 constexpr int kLptMaxBatch = 64;   // longest-first block order up to this many sequences
 constexpr int kMaxL = SCONV_MAX_STATE_LEN;
@@ -98,18 +103,6 @@ __device__ __forceinline__ uint16_t float_to_raw<bf16>(float f) {
 template <>
 __device__ __forceinline__ uint32_t float_to_raw<float>(float f) {
     return __float_as_uint(f);
-}
-
-__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
-    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void flag(int32_t *err, unsigned bits) {
@@ -293,27 +286,78 @@ __device__ __forceinline__ void silu_pack(float (&acc)[VEC]) {
 // short ones fill the tail), else sequences interleave.  A tile is TT rows;
 // thread (g, p) = (threadIdx.x / PP, threadIdx.x % PP) convolves rows
 // g*RPT .. g*RPT+RPT-1 of pack p from a register window of W-1+RPT rows.
-// Each ring stage holds HALO = WT-1 rows ahead of its tile: the rows before
-// the tile, written into the stage while the previous tile is computed (the
-// first from the state line), so every tap is a plain shared-memory read.
-// The last L inputs (the new state line) ride along in a double-buffered
-// carry.  One barrier per tile: tile s reads carry[s & 1] and writes the
-// next into the other, and the stage refilled at tile s was last read at
-// tile s-1.  WT is the exact tap count (2..4), or 8 for any W up to 8.
+//
+// Tiles arrive by tensor copy: thread 0 issues each tile's TT x PP-pack box
+// into a ring stage and the copy completes on the stage's `full` mbarrier;
+// each warp releases the stage on its `empty` mbarrier when it is done, and
+// thread 0 refills the stage of tile s-1 (once all eight warps released it)
+// after tile s, so a warp never waits for the others to finish the tile it
+// is on and no block-wide barrier runs per tile.  Each stage keeps the WT-1
+// rows before its tile (the halo) just below the tile's rows: only warp 0
+// reads them (the first rows of a tile), and warp 0 writes them, from the
+// last rows of the previous tile (the first from the state line), so every
+// tap is a plain shared-memory read and the halo needs only warp-level
+// ordering.  The new state line, the last L inputs, is read at the end from
+// the last two tiles' stages (TT >= L) and the old line kept in shared
+// memory.  Copies cover whole tiles and may read rows past the sequence's
+// end (another sequence's, possibly being rewritten in place by its own
+// block, or zeros past T); those rows are never used.  Rows of this
+// sequence are copied before this block writes them, and never re-read, so
+// the in-place form needs no scratch memory and no ordering between blocks.
+// WT is the exact tap count (2..4), or 8 for any W up to 8.
+template <int PP, int WT, int THREADS, int STAGES>
+struct TileLayout {
+    static constexpr int TT = THREADS / PP * kRowsPerThread;
+    static constexpr int HALO = WT - 1;
+    static constexpr int row_bytes = PP * 16;
+    // The tile's rows start on a 128-byte boundary (the copy's destination);
+    // the halo rows sit just below them.
+    static constexpr int tile_off = (HALO * row_bytes + 127) / 128 * 128;
+    static constexpr int halo_off = tile_off - HALO * row_bytes;
+    static constexpr int stage = tile_off + TT * row_bytes;
+    static constexpr int tile_bytes = TT * row_bytes;
+    // A copy box holds at most 256 rows.
+    static constexpr int boxes = TT > 256 ? TT / 256 : 1;
+    static constexpr int box_rows = TT / boxes;
+    static constexpr int bars = STAGES * stage;  // full[STAGES], empty[STAGES]
+    static constexpr int line0 = bars + 2 * STAGES * 8;
+    static constexpr int order = line0 + kMaxL * PP * 16;
+    static constexpr int smem = order + kLptMaxBatch * 4;
+};
+
 template <typename E, int PP, int WT, int THREADS, int STAGES>
-__global__ void __launch_bounds__(THREADS) dense_fwd_tile(const __grid_constant__ DenseArgs a, int ncb) {
+__global__ void __launch_bounds__(THREADS)
+dense_fwd_tile(const __grid_constant__ DenseArgs a, const __grid_constant__ CUtensorMap xmap,
+               int ncb) {
+    using Lay = TileLayout<PP, WT, THREADS, STAGES>;
+    using namespace tma;
     constexpr int VEC = 16 / sizeof(E);
     constexpr int RPT = kRowsPerThread;
-    constexpr int TT = THREADS / PP * RPT;
-    constexpr int HALO = WT - 1;
-    constexpr int SR = HALO + TT;       // rows of one ring stage
-    constexpr int NW = WT - 1 + RPT;    // window rows of one thread
-    extern __shared__ uint4 ring[];     // STAGES * SR * PP packs
-    __shared__ uint4 carry[2][kMaxL * PP];
-    __shared__ int order[kLptMaxBatch];
+    constexpr int TT = Lay::TT;
+    constexpr int HALO = Lay::HALO;
+    constexpr int NW = WT - 1 + RPT;  // window rows of one thread
+    // The threads whose windows reach into the halo are all in warp 0.
+    static_assert((HALO + RPT - 1) / RPT * PP <= 32, "halo readers must be warp 0");
+    static_assert(TT >= kMaxL, "the new line must lie in the last two tiles");
+    static_assert(STAGES >= 3, "the halo stage must differ from the refilled one");
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + Lay::bars);
+    uint64_t *empty = full + STAGES;
+    uint4 *line0 = reinterpret_cast<uint4 *>(smem + Lay::line0);  // the old line, L x PP
+    int *order = reinterpret_cast<int *>(smem + Lay::order);
+    // Row -HALO of stage k: the halo, then the tile's TT rows, PP packs each.
+    auto rows = [&](int k) { return reinterpret_cast<uint4 *>(smem + k * Lay::stage + Lay::halo_off); };
 
     pdl_wait();
     pdl_trigger();
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int k = 0; k < STAGES; ++k) {
+            mbar_init(&full[k], 1);
+            mbar_init(&empty[k], THREADS / 32);
+        }
+        mbar_init_fence();
+    }
     int b, y;
     if (a.batch <= kLptMaxBatch) {
         // Rank sequences by length, longest first (ties by index).
@@ -327,13 +371,16 @@ __global__ void __launch_bounds__(THREADS) dense_fwd_tile(const __grid_constant_
             }
             order[rank] = t;
         }
-        __syncthreads();
+        __syncthreads();  // the ranking and the barriers
         b = order[blockIdx.x / ncb];
         y = blockIdx.x % ncb;
     } else {
+        __syncthreads();  // the barriers
         b = blockIdx.x % a.batch;
         y = blockIdx.x / a.batch;
     }
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
     const int p = threadIdx.x % PP;
     const int g = threadIdx.x / PP;
     const int c = (y * PP + p) * VEC;
@@ -345,17 +392,34 @@ __global__ void __launch_bounds__(THREADS) dense_fwd_tile(const __grid_constant_
     bool from;
     if (!sequence_setup(a, b, threadIdx.x == 0 && y == 0, q0, n, line, from)) return;
     const int L = a.L;
-    const int ci = threadIdx.x / PP;  // carry entry / halo row this thread maintains
+    const int ntiles = (n + TT - 1) / TT;
+    const int cx = y * PP * VEC;  // the column's first channel
 
-    // The history: the line (or zeros) is the first carry, and its last
-    // HALO entries are the first stage's halo (zeros before the line).
+    // Thread 0 is the producer: it puts tile j in stage j % STAGES.
+    int issued = 0;  // tiles issued (thread 0)
+    auto issue = [&](int j) {
+        const int k = j % STAGES;
+        unsigned char *dst = smem + k * Lay::stage + Lay::tile_off;
+        mbar_expect_tx(&full[k], Lay::tile_bytes);
+#pragma unroll
+        for (int bx = 0; bx < Lay::boxes; ++bx)
+            copy_2d(dst + bx * Lay::box_rows * Lay::row_bytes, &xmap, cx,
+                    q0 + j * TT + bx * Lay::box_rows, &full[k]);
+        issued = j + 1;
+    };
+    if (threadIdx.x == 0)
+        for (int j = 0; j < STAGES && j < ntiles; ++j) issue(j);
+
+    // The history: the old line (or zeros), and its last HALO entries as the
+    // first tile's halo (zeros before the line).
+    const int ci = threadIdx.x / PP;  // line entry / halo row this thread sets up
     if (a.st && ci < L)
-        carry[0][ci * PP + p] = cvalid ? line_pack<E, VEC>(a, line, c, ci, from)
-                                       : make_uint4(0u, 0u, 0u, 0u);
+        line0[ci * PP + p] = cvalid ? line_pack<E, VEC>(a, line, c, ci, from)
+                                    : make_uint4(0u, 0u, 0u, 0u);
     if (ci < HALO) {
         const int e = L - HALO + ci;
-        ring[ci * PP + p] = (cvalid && a.st && e >= 0) ? line_pack<E, VEC>(a, line, c, e, from)
-                                                       : make_uint4(0u, 0u, 0u, 0u);
+        rows(0)[ci * PP + p] = (cvalid && a.st && e >= 0) ? line_pack<E, VEC>(a, line, c, e, from)
+                                                          : make_uint4(0u, 0u, 0u, 0u);
     }
 
     TileWeights<E, WT> wt;
@@ -364,31 +428,27 @@ __global__ void __launch_bounds__(THREADS) dense_fwd_tile(const __grid_constant_
         wt.load(a, c);
         load_bias<E, VEC>(a, c, bias);
     }
+    __syncthreads();  // the old line and the first halo
 
-    const E *x = static_cast<const E *>(a.x) + static_cast<int64_t>(q0) * a.x_st + c;
     E *out = static_cast<E *>(a.out) + static_cast<int64_t>(q0) * a.x_st + c;
-    const int ntiles = (n + TT - 1) / TT;
-    // Copies: thread (g, p) fetches rows g + j * TT / RPT of pack p, so a
-    // warp's copies cover whole rows.
-    auto issue = [&](int s) {
-#pragma unroll
-        for (int j = 0; j < RPT; ++j) {
-            const int r = g + j * (TT / RPT);
-            const int row = s * TT + r;
-            if (s < ntiles && row < n && cvalid)
-                cp_async16(&ring[((s % STAGES) * SR + HALO + r) * PP + p], x + row * a.x_st);
-        }
-        cp_async_commit();
-    };
-#pragma unroll
-    for (int s = 0; s < STAGES - 1; ++s) issue(s);
-
     const int r0 = g * RPT;
+    bool alive = true;
+    int next = 0;  // tiles this thread has waited for
     for (int s = 0; s < ntiles; ++s) {
-        cp_async_wait<STAGES - 2>();
-        __syncthreads();  // tile s, its halo and carry[s & 1] are complete
-        issue(s + STAGES - 1);
-        const uint4 *stage = ring + (s % STAGES) * SR * PP;  // row -HALO of the tile
+        const int k = s % STAGES;
+        const bool ok = mbar_wait(&full[k], (s / STAGES) & 1);
+        if (!__all_sync(0xffffffffu, ok)) {  // the copy did not arrive in time
+            if (lane == 0) flag(a.err, SCONV_EFLAG_TIMEOUT);
+            alive = false;
+            break;
+        }
+        next = s + 1;
+        const uint4 *stage = rows(k);  // row -HALO of the tile
+        // Warp 0: the next tile's halo, the last HALO rows of this (full) tile.
+        if (warp == 0 && s + 1 < ntiles) {
+            uint4 *h = rows((s + 1) % STAGES);
+            for (int i = lane; i < HALO * PP; i += 32) h[i] = stage[TT * PP + i];
+        }
         const int nv = min(TT, n - s * TT);
         if (r0 < nv && cvalid) {
             // win[j] holds tile row r0 - (WT-1) + j.
@@ -414,21 +474,44 @@ __global__ void __launch_bounds__(THREADS) dense_fwd_tile(const __grid_constant_
                 o.store(orow + u * a.x_st);
             }
         }
-        // The next stage's halo: the last HALO rows of this (full) tile.
-        if (ci < HALO && s + 1 < ntiles)
-            ring[((s + 1) % STAGES) * SR * PP + ci * PP + p] = stage[(TT + ci) * PP + p];
-        // Next carry: the last L entries of (carry, the tile's nv rows).
-        if (a.st && ci < L) {
-            const uint4 *cin = carry[s & 1];
-            const int src = nv + ci;
-            carry[(s + 1) & 1][ci * PP + p] =
-                src >= L ? stage[(HALO + src - L) * PP + p] : cin[src * PP + p];
+        // This warp is done with the stage (and warp 0's halo writes are
+        // ordered before its next tile's reads).
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[k]);
+        // Warp 0: refill the stage of tile s-1 once every warp released it.
+        if (warp == 0) {
+            bool fine = true;
+            if (lane == 0 && s >= 1 && s - 1 + STAGES < ntiles) {
+                const int j = s - 1;
+                fine = mbar_wait(&empty[j % STAGES], (j / STAGES) & 1);
+                if (fine) issue(j + STAGES);
+            }
+            if (!__shfl_sync(0xffffffffu, fine, 0)) {
+                if (lane == 0) flag(a.err, SCONV_EFLAG_TIMEOUT);
+                alive = false;
+                break;
+            }
         }
     }
-    cp_async_wait<0>();
-    // Each thread stores the carry entry it wrote itself: no barrier needed.
-    if (a.st && ci < L && cvalid)
-        store_line_pack<E, VEC>(a, line, c, ci, carry[ntiles & 1][ci * PP + p]);
+    if (!alive) {
+        // Let the copies issued and not waited for land before the block's
+        // shared memory is released (each wait bounded); store nothing more.
+        if (threadIdx.x == 0)
+            for (int j = next; j < issued; ++j) mbar_wait(&full[j % STAGES], (j / STAGES) & 1);
+        return;
+    }
+    // The new line: entry ci is input n + ci of (old line, the n rows).
+    if (a.st && ci < L && cvalid) {
+        const int i = n + ci;
+        uint4 v;
+        if (i < L) {
+            v = line0[i * PP + p];
+        } else {
+            const int r = i - L;  // a row of the last two tiles
+            v = rows((r / TT) % STAGES)[(HALO + r % TT) * PP + p];
+        }
+        store_line_pack<E, VEC>(a, line, c, ci, v);
+    }
 }
 
 // Prefill, channel-major x (token stride 1).  Warp (b, c) walks channel c of
@@ -854,58 +937,93 @@ int pick_pp(int batch, int packs) {
 }
 
 template <typename E, int PP, int WT, int THREADS, int STAGES>
-cudaError_t launch_tile_pp(const DenseArgs &a, int packs, cudaStream_t stream) {
-    constexpr int TT = THREADS / PP * kRowsPerThread;
-    constexpr size_t kSmem = static_cast<size_t>(STAGES) * (WT - 1 + TT) * PP * sizeof(uint4);
-    static bool configured = false;
-    if (!configured) {
-        const cudaError_t e = cudaFuncSetAttribute(
-            dense_fwd_tile<E, PP, WT, THREADS, STAGES>,
-            cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+cudaError_t launch_tile_pp(const DenseArgs &a, const CUtensorMap &map, int packs,
+                           cudaStream_t stream) {
+    constexpr int kSmem = TileLayout<PP, WT, THREADS, STAGES>::smem;
+    auto kernel = dense_fwd_tile<E, PP, WT, THREADS, STAGES>;
+    static std::once_flag once;
+    static cudaError_t attr = cudaSuccess;
+    std::call_once(once, [&] {
+        attr = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    });
+    if (attr != cudaSuccess) return attr;
     const int ncb = (packs + PP - 1) / PP;
-    return launch_pdl(dense_fwd_tile<E, PP, WT, THREADS, STAGES>,
-                      dim3(static_cast<unsigned>(static_cast<int64_t>(a.batch) * ncb)),
-                      dim3(THREADS), kSmem, stream, a, ncb);
+    return launch_pdl(kernel, dim3(static_cast<unsigned>(static_cast<int64_t>(a.batch) * ncb)),
+                      dim3(THREADS), static_cast<size_t>(kSmem), stream, a, map, ncb);
 }
 
 template <typename E, int PP, int WT>
-cudaError_t launch_tile_s(const DenseArgs &a, int packs, cudaStream_t stream) {
+cudaError_t launch_tile_s(const DenseArgs &a, const CUtensorMap &map, int packs,
+                          cudaStream_t stream) {
     // Several waves: 3 resident blocks per SM is what registers allow.
     const int64_t blocks = static_cast<int64_t>(a.batch) * ((packs + PP - 1) / PP);
     if (blocks >= 2LL * 3 * sm_count())
-        return launch_tile_pp<E, PP, WT, kTileThreads, kStagesFew>(a, packs, stream);
-    return launch_tile_pp<E, PP, WT, kTileThreads, kStagesMany>(a, packs, stream);
+        return launch_tile_pp<E, PP, WT, kTileThreads, kStagesFew>(a, map, packs, stream);
+    return launch_tile_pp<E, PP, WT, kTileThreads, kStagesMany>(a, map, packs, stream);
 }
 
 template <typename E, int WT>
-cudaError_t launch_tile_w(const DenseArgs &a, int packs, int pp, cudaStream_t stream) {
+cudaError_t launch_tile_w(const DenseArgs &a, const CUtensorMap &map, int packs, int pp,
+                          cudaStream_t stream) {
     switch (pp) {
-        case 8: return launch_tile_s<E, 8, WT>(a, packs, stream);
-        case 4: return launch_tile_s<E, 4, WT>(a, packs, stream);
-        case 2: return launch_tile_s<E, 2, WT>(a, packs, stream);
-        default: return launch_tile_s<E, 1, WT>(a, packs, stream);
+        case 8: return launch_tile_s<E, 8, WT>(a, map, packs, stream);
+        case 4: return launch_tile_s<E, 4, WT>(a, map, packs, stream);
+        case 2: return launch_tile_s<E, 2, WT>(a, map, packs, stream);
+        default: return launch_tile_s<E, 1, WT>(a, map, packs, stream);
     }
 }
 
+// The tensor map of x for a column of pp packs: rows of dim channels (a
+// stride of x_st elements), boxes of pp packs x min(TT, 256) rows.  Rows
+// past T and channels past dim arrive as zeros.  False when the driver
+// offers no encoder or rejects the layout.
 template <typename E>
-cudaError_t launch_tile(const DenseArgs &a, cudaStream_t stream) {
+bool encode_tile_map(const DenseArgs &a, int pp, CUtensorMap &map) {
+    constexpr int VEC = 16 / sizeof(E);
+    constexpr int64_t e = sizeof(E);
+    if (tma::encode_fn() == nullptr) return false;
+    const int tt = kTileThreads / pp * kRowsPerThread;
+    const cuuint64_t dim[2] = {static_cast<cuuint64_t>(a.dim),
+                               static_cast<cuuint64_t>(a.T > 1 ? a.T : 1)};
+    // With one row the stride is never used; any legal value will do.
+    const int64_t row = a.T > 1 ? a.x_st * e : (a.dim * e + 15) / 16 * 16;
+    const cuuint64_t stride[1] = {static_cast<cuuint64_t>(row)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(pp * VEC),
+                               static_cast<cuuint32_t>(tt > 256 ? 256 : tt)};
+    const cuuint32_t elem[2] = {1, 1};
+    const CUtensorMapDataType type =
+        e == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    return tma::encode_fn()(&map, type, 2, const_cast<void *>(a.x), dim, stride, box, elem,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The tiled prefill; `used` false (nothing launched) when x has no tensor
+// map, for the caller to take another kernel.
+template <typename E>
+cudaError_t launch_tile(const DenseArgs &a, cudaStream_t stream, bool &used) {
     constexpr int VEC = 16 / sizeof(E);
     const int packs = a.dim / VEC;
     const int pp = pick_pp(a.batch, packs);
+    CUtensorMap map;
+    used = encode_tile_map<E>(a, pp, map);
+    if (!used) return cudaSuccess;
     switch (a.W) {
-        case 2: return launch_tile_w<E, 2>(a, packs, pp, stream);
-        case 3: return launch_tile_w<E, 3>(a, packs, pp, stream);
-        case 4: return launch_tile_w<E, 4>(a, packs, pp, stream);
-        default: return launch_tile_w<E, 8>(a, packs, pp, stream);
+        case 2: return launch_tile_w<E, 2>(a, map, packs, pp, stream);
+        case 3: return launch_tile_w<E, 3>(a, map, packs, pp, stream);
+        case 4: return launch_tile_w<E, 4>(a, map, packs, pp, stream);
+        default: return launch_tile_w<E, 8>(a, map, packs, pp, stream);
     }
 }
 
 template <typename E, int MAXW>
 cudaError_t launch_fwd_t(const DenseArgs &a, bool vec, cudaStream_t stream) {
-    if (vec) return launch_tile<E>(a, stream);
+    if (vec) {
+        bool used = false;
+        const cudaError_t e = launch_tile<E>(a, stream, used);
+        if (used) return e;
+    }
     if (a.x_st == 1 && a.T > 1 && (reinterpret_cast<uintptr_t>(a.x) & 15u) == 0) {
         // channel-major: a warp per (sequence, channel)
         const int64_t warps = static_cast<int64_t>(a.batch) * a.dim;

@@ -42,18 +42,17 @@
 // Every wait on an mbarrier is bounded; a block whose copies do not arrive
 // in time sets SCONV_EFLAG_TIMEOUT, waits (bounded) for its other copies and
 // returns without writing anything for that tile.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include <atomic>
-#include <mutex>
 
 #include "common.cuh"
 #include "fused_common.cuh"
 #include "sconv.h"
+#include "tma.cuh"
 
 namespace sconv {
 namespace {
+
+using namespace tma;
 
 template <typename E>
 constexpr int kBC = 512 / static_cast<int>(sizeof(E));  // channels per tile
@@ -61,9 +60,6 @@ constexpr int kBT = 32;            // tokens per tile
 constexpr int kThreads = 256;      // 8 warps
 constexpr int kTokPerWarp = kBT / (kThreads / 32);  // 4
 constexpr int kMetaBytes = kBT * (8 + 8 + 4 + 4);   // positions, slots, seq_idx, query_start
-// An mbarrier wait gives up this many nanoseconds of %globaltimer time after
-// it begins (plus at most one try_wait suspension).
-constexpr uint64_t kWaitNs = 1000000000ull;
 
 template <int W>
 struct Layout {
@@ -91,68 +87,6 @@ constexpr bool kCachesWeights = W > (sizeof(E) == 2 ? 4 : 5);
 struct TmaMaps {
     CUtensorMap x, pos, slot, sid, qs;
 };
-
-__device__ __forceinline__ uint32_t smem_addr(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count));
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
-                 "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(smem_addr(bar)), "r"(parity)
-        : "memory");
-    return done != 0;
-}
-
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Wait for the phase with the given parity to complete, for at most kWaitNs
-// of wall time: each try_wait may suspend the thread for a system-dependent
-// interval, so the bound is taken from the global nanosecond timer rather
-// than from a count of polls.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
-    if (mbar_test(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    do {
-        if (mbar_test(bar, parity)) return true;
-    } while (globaltimer_ns() - t0 < kWaitNs);
-    return false;
-}
-
-__device__ __forceinline__ void tma_2d(void *dst, const CUtensorMap *map, int x, int y,
-                                       uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ void tma_1d(void *dst, const CUtensorMap *map, int x, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.1d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2}], [%3];" ::"r"(smem_addr(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(smem_addr(bar))
-        : "memory");
-}
 
 template <typename E>
 using PackOf = Pack<E, 16 / sizeof(E)>;
@@ -284,10 +218,6 @@ struct LagWeights<float, W> {
     }
 };
 
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
-
 // The pack lane l works on in channel block cb (clamped to the last pack
 // for lanes past C, which compute but store nothing).
 __device__ __forceinline__ int cb_pack(int cb, int l, int nv) {
@@ -326,7 +256,7 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kThreads / 32);
         }
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        mbar_init_fence();
     }
     __syncthreads();
     pdl_wait();  // inputs may come from the previous kernel in the stream
@@ -341,11 +271,11 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
         const int c0 = static_cast<int>(u % ncb) * BC;
         const int t0 = static_cast<int>(u / ncb) * kBT;
         mbar_expect_tx(&full[s], L::stage);
-        tma_2d(st, &maps.x, c0, t0 - (W - 1), &full[s]);
-        tma_1d(st + L::x_bytes, &maps.pos, t0, &full[s]);
-        tma_1d(st + L::x_bytes + kBT * 8, &maps.slot, t0, &full[s]);
-        tma_1d(st + L::x_bytes + kBT * 16, &maps.sid, t0, &full[s]);
-        tma_1d(st + L::x_bytes + kBT * 20, &maps.qs, t0, &full[s]);
+        copy_2d(st, &maps.x, c0, t0 - (W - 1), &full[s]);
+        copy_1d(st + L::x_bytes, &maps.pos, t0, &full[s]);
+        copy_1d(st + L::x_bytes + kBT * 8, &maps.slot, t0, &full[s]);
+        copy_1d(st + L::x_bytes + kBT * 16, &maps.sid, t0, &full[s]);
+        copy_1d(st + L::x_bytes + kBT * 20, &maps.qs, t0, &full[s]);
     };
     if (threadIdx.x == 0)
         for (int k = 0; k < STAGES && k < my; ++k) issue(k);
@@ -548,21 +478,6 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
         // its shared memory is released (each wait bounded).
         for (int j = next; j < issued; ++j) mbar_wait(&full[j % STAGES], (j / STAGES) & 1);
     }
-}
-
-// cuTensorMapEncodeTiled, fetched from the driver once (no link to libcuda).
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
 }
 
 bool encode_1d(CUtensorMap *m, CUtensorMapDataType type, const void *base, int64_t n) {

@@ -322,6 +322,9 @@ sconv_status sconv_extract_windows_paged(
  *                    [0, num_lines) sets SCONV_EFLAG_SLOT, one whose
  *                    query_start_loc entries are out of order or range sets
  *                    SCONV_EFLAG_QUERY_START; such a sequence is skipped.
+ *                    The token-major tiled form (x_stride_c == 1, 16-byte
+ *                    aligned rows) sets SCONV_EFLAG_TIMEOUT when a tile's
+ *                    copy does not arrive within its bounded wait.
  * One thread block (or warp) owns a (sequence, channel) column and walks it
  * in row order, so the in-place form needs no scratch memory and no ordering
  * between blocks.  weight and bias are read before the wait for the kernel
