@@ -498,12 +498,72 @@ def run_steps_graphs(sets_obj, K, stream, pipeline=False, carry=False, **step_kw
     return full, tail, K // M
 
 
-def carry_prologue(sets_obj, stream):
-    """The metadata of set 0, built before the first replay of carry graphs
-    (the build a previous window of the serving loop would have made)."""
+def carry_prologue(sets_obj, stream, i=0):
+    """The metadata of set i (0 unless given), built before the first replay
+    of carry graphs (the build a previous window of the serving loop would
+    have made)."""
     with torch.cuda.stream(stream):
-        sets_obj.step(0, fused=False)
+        sets_obj.step(i, fused=False)
     torch.cuda.synchronize()
+
+
+# Untimed steps at the head of the timed graph: the serving loop's steps
+# before the measured window, so the first timed step starts with the
+# launch pipeline already running, as every later one does.
+LEAD_STEPS = 4
+# Up to this many timed steps go into one graph with the lead steps and the
+# two event nodes; longer runs replay graphs of one rotation each between
+# events on the stream (each graph boundary then costs a launch gap, about
+# 1 % of a rotation).
+EVENT_GRAPH_MAX_STEPS = 768
+
+
+class StepEvents:
+    """The start and end of a timed window of steps inside one captured
+    graph.  start() records an event node on a branch off the step chain,
+    after the last untimed step: it is recorded when that step completes,
+    while the first timed step follows that step on the chain exactly as
+    every step follows its predecessor (its launch and its work before its
+    wait may overlap the step before, as in the serving loop).  end()
+    joins the branch and records an event node after the last timed step
+    completes.  The interval is then K step periods of the running loop,
+    with nothing of the graph's own launch in it."""
+
+    def __init__(self, device):
+        self.begin = torch.cuda.Event(enable_timing=True, external=True)
+        self.finish = torch.cuda.Event(enable_timing=True, external=True)
+        self.branch = torch.cuda.Stream(device)
+
+    def start(self):
+        self.branch.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(self.branch):
+            self.begin.record()
+
+    def end(self):
+        torch.cuda.current_stream().wait_stream(self.branch)
+        self.finish.record()
+
+    def seconds(self):
+        return self.begin.elapsed_time(self.finish) / 1e3
+
+
+def timed_steps_graph(sets_obj, K, stream, lead=LEAD_STEPS):
+    """One graph of `lead` untimed one-launch steps (the sets before set 0
+    in the rotation), then exactly K timed steps (sets 0, 1, ... mod M)
+    between the StepEvents marks.  carry_prologue(sets_obj, stream, idx)
+    with the returned idx builds the first lead step's table before each
+    replay."""
+    M = len(sets_obj.sets)
+    lead_idx = [(M - lead + i) % M for i in range(lead)]
+    timed_idx = [i % M for i in range(K)]
+    marks = StepEvents(stream.device)
+
+    def body():
+        next_steps(sets_obj, lead_idx, timed_idx[0])
+        marks.start()
+        next_steps(sets_obj, timed_idx, K % M)
+        marks.end()
+    return capture(body, stream), marks, lead_idx[0]
 
 
 class L2Flush:
@@ -571,6 +631,32 @@ def time_region(full, tail, reps, stream, world, sampler=None, flush=None, label
     return start.elapsed_time(end) / 1e3, (w0, w1)  # seconds
 
 
+def time_graph_events(graph, marks, stream, world, sampler=None, flush=None, label="timed"):
+    """Seconds between the StepEvents marks of one replay of graph,
+    bracketed by a barrier and a device synchronisation on both sides;
+    flush and the spin kernel as in time_region.  With a sampler, also
+    returns the host wall-clock span of the replay."""
+    barrier(world)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(1.0)
+    w0 = time.time()
+    with torch.cuda.stream(stream), nvtx_range(label):
+        if flush is not None:
+            flush()
+        torch.cuda._sleep(HOST_LEAD_CYCLES)
+        graph.replay()
+    torch.cuda.synchronize()
+    w1 = time.time()
+    barrier(world)
+    torch.cuda.synchronize()
+    if sampler:
+        time.sleep(0.3)
+        sampler.stop()
+    return marks.seconds(), (w0, w1)
+
+
 def prime(full, tail, stream):
     """Replay each graph that is about to be timed once, untimed: the first
     replay of a freshly instantiated graph also uploads it."""
@@ -588,9 +674,11 @@ def l2_statement(sets_obj, K):
     M = len(sets_obj.sets)
     if K <= M:
         touched = sum(sets_obj.alg_bytes[:K])
+        lead = (f"; the {LEAD_STEPS} untimed steps ahead of them read other sets"
+                if K + LEAD_STEPS <= M and K <= EVENT_GRAPH_MAX_STEPS else "")
         return (f"L2 flushed (256 MiB written) before the timed region; the {K} timed steps "
                 f"each read their own input set (none repeats within the region; "
-                f"{touched / 1e6:.0f} MB touched in all)")
+                f"{touched / 1e6:.0f} MB touched in all){lead}")
     touched = sum(sets_obj.alg_bytes)
     verdict = "> 126 MB L2" if touched > L2_BYTES else "NOT above the 126 MB L2"
     return (f"L2 flushed (256 MiB written) before the timed region; the steps rotate over "
@@ -1362,11 +1450,11 @@ def e2e(sets_obj, K, stream, world, flush):
         assert torch.equal(mapped[0].host_view().view(torch.int16),
                            sets_obj.sets[0]["out"].cpu().view(torch.int16)), "mapped output"
 
-    def steps(n):
+    def steps(idxs):
         cur = torch.cuda.current_stream()
         up.wait_stream(cur)
         down.wait_stream(cur)
-        for i in range(n):
+        for i in idxs:
             s, p = sets_obj.sets[i], packed[i]
             with torch.cuda.stream(up):
                 p["dev"].copy_(p["host"], non_blocking=True)
@@ -1379,12 +1467,29 @@ def e2e(sets_obj, K, stream, world, flush):
         cur.wait_stream(up)
         cur.wait_stream(down)
 
+    # As for the headline: up to EVENT_GRAPH_MAX_STEPS, LEAD_STEPS untimed
+    # steps and then the K timed steps between two event-record nodes of
+    # one graph; beyond, graphs of one rotation replayed between events.
     M = len(sets_obj.sets)
-    full = capture(lambda: steps(M), stream) if K >= M else None
-    tail = capture(lambda: steps(K % M), stream) if K % M else None
-    prime(full, tail, stream)
-    secs = max_over_ranks(time_region(full, tail, K // M, stream, world, flush=flush)[0], world)
-    del full, tail
+    if K <= EVENT_GRAPH_MAX_STEPS:
+        marks = StepEvents(stream.device)
+
+        def body():
+            steps([(M - LEAD_STEPS + i) % M for i in range(LEAD_STEPS)])
+            marks.start()
+            steps([i % M for i in range(K)])
+            marks.end()
+        graph = capture(body, stream)
+        prime(graph, None, stream)
+        secs = time_graph_events(graph, marks, stream, world, flush=flush)[0]
+        del graph
+    else:
+        full = capture(lambda: steps(range(M)), stream) if K >= M else None
+        tail = capture(lambda: steps(range(K % M)), stream) if K % M else None
+        prime(full, tail, stream)
+        secs = time_region(full, tail, K // M, stream, world, flush=flush)[0]
+        del full, tail
+    secs = max_over_ranks(secs, world)
     torch.cuda.synchronize()
     if mapped:
         for m in mapped:
@@ -1400,23 +1505,31 @@ def e2e(sets_obj, K, stream, world, flush):
 
 # --------------------------------------------------------------------------
 
-def config_block(world, l2):
-    return {"workload": "decode_bf16: 256 single-token requests over cached histories "
+def config_block(world, l2, K=None):
+    block = {"workload": "decode_bf16: 256 single-token requests over cached histories "
                         "U{1..4096}; H=32, D=128, ws=32, off_s=32, C=1024, W=4, N=16; "
                         "SiLU + residual",
             "global_batch": 256 * world, "seq_len": 1,
             "parallelism": f"dp{world}" if world > 1 else "single",
             "step": STEP_CALLS[STEP_MODE],
-            "pipelining": "the next step's metadata is built on a second stream beside the "
-                          "current step's convolution, as a serving engine prepares step "
-                          "i+1's inputs while step i runs; the convolutions run in order, "
-                          "each waiting for the previous one; the timed region holds K "
-                          "convolutions and K metadata builds (the first step's metadata "
-                          "comes from the step before the region, the last build is for the "
-                          "step after it)",
+            "pipelining": "each step is one launch that convolves this step and, in "
+                          "extra blocks, builds the next step's metadata and tap table, as "
+                          "a serving engine prepares step i+1's inputs while step i runs; "
+                          "the convolutions run in order, each waiting for the previous "
+                          "one; the timed region holds K convolutions and K table builds "
+                          "(the first step's table comes from the step before the region, "
+                          "the last build is for the step after it)",
             "metadata": "one metadata buffer set per step, so the *_ahead builder may look "
                         "up before the launch's wait on its predecessors",
             "l2": l2}
+    if K is not None:
+        block["timing"] = (f"one graph replay: {LEAD_STEPS} untimed steps, then the K timed "
+                           "steps; CUDA events recorded by graph nodes when the last untimed "
+                           "step and the last timed step complete (device time)"
+                           if K <= EVENT_GRAPH_MAX_STEPS else
+                           "graphs of one rotation of steps replayed between CUDA events on "
+                           "the launching stream (device time)")
+    return block
 
 
 def main_reference(args, rank, world):
@@ -1519,14 +1632,24 @@ def main():
         replay_steps(wfull, wtail, wreps)
     torch.cuda.synchronize()
     del wfull, wtail
-    carry_prologue(sets_obj, stream)
-    full, tail, reps = run_steps_graphs(sets_obj, K, stream, pipeline=STEP_SCHEDULE,
-                                        carry=True)
-    prime(full, tail, stream)
-    carry_prologue(sets_obj, stream)
     sampler = ClockSampler(local) if rank == 0 else None
-    secs, (w0, w1) = time_region(full, tail, reps, stream, world, sampler, flush,
-                                 label=f"timed decode steps (K={K})")
+    if K <= EVENT_GRAPH_MAX_STEPS:
+        graph, marks, first = timed_steps_graph(sets_obj, K, stream)
+        carry_prologue(sets_obj, stream, first)
+        prime(graph, None, stream)
+        carry_prologue(sets_obj, stream, first)
+        secs, (w0, w1) = time_graph_events(graph, marks, stream, world, sampler, flush,
+                                           label=f"timed decode steps (K={K})")
+        del graph
+    else:
+        carry_prologue(sets_obj, stream)
+        full, tail, reps = run_steps_graphs(sets_obj, K, stream, pipeline=STEP_SCHEDULE,
+                                            carry=True)
+        prime(full, tail, stream)
+        carry_prologue(sets_obj, stream)
+        secs, (w0, w1) = time_region(full, tail, reps, stream, world, sampler, flush,
+                                     label=f"timed decode steps (K={K})")
+        del full, tail
     secs = max_over_ranks(secs, world)
     clocks = None
     if sampler is not None:
@@ -1536,15 +1659,15 @@ def main():
             # The timed region was too short for 100 ms sampling: sample a
             # separate ~2 s replay of the same steps instead.
             load = ClockSampler(local)
-            if full is None:
-                full, _, _ = run_steps_graphs(sets_obj, len(sets_obj.sets), stream,
-                                              pipeline=STEP_SCHEDULE, carry=True)
-                prime(full, None, stream)
+            carry_prologue(sets_obj, stream)
+            full, _, _ = run_steps_graphs(sets_obj, len(sets_obj.sets), stream,
+                                          pipeline=STEP_SCHEDULE, carry=True)
+            prime(full, None, stream)
             n = max(1, int(2.0 / max(secs / K * len(sets_obj.sets), 1e-6)))
             _, (l0, l1) = time_region(full, None, n, stream, 1, load)
             clocks = ClockSampler.summary(load.samples(l0, l1),
                                           "2 s replay of the step graphs after the timed region")
-    del full, tail
+            del full
     T = sets_obj.wls[0].T
     tokens = sum_over_ranks(float(T * K), world)
     value = tokens / secs / 1e6
@@ -1563,7 +1686,7 @@ def main():
         "data": "synthetic (seeded generator; random-normal x, weight and cache)",
         "config": config_block(world, l2_statement(sets_obj, K) if args.max_hist == 4096
                                else "NOT a benchmark figure: profiling case "
-                                    f"(histories up to {args.max_hist} tokens)"),
+                                    f"(histories up to {args.max_hist} tokens)", K),
         "hbm_gbs": round(step_bytes / secs / 1e9, 1),
         "gpu_launches": (1 if STEP_SCHEDULE == "next" else 2) * K,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,

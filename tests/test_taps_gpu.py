@@ -349,6 +349,81 @@ def test_interleaved_graph_equals_plain_steps():
     del graph
 
 
+def test_stale_table_rewritten_under_the_convolution():
+    """Without metadata_ready the convolution reads its table row before its
+    wait only as a guess, to prefetch the cache taps it names; the taps it
+    uses follow the row read after the wait.  Each step's table here first
+    holds ANOTHER step's table (valid cache slots, wrong ones), then the
+    builder rewrites it and the convolution follows at once on the same
+    stream, so its early reads may see either.  Replayed from a graph
+    several times, outputs and cache equal the plain sconv_fused steps bit
+    for bit."""
+    wls = [workloads.decode_bf16(seed=520 + i, R=64, max_hist=600) for i in range(6)]
+    nb = max(w.num_blocks for w in wls)
+    w0 = wls[0]
+    g = torch.Generator(device="cpu").manual_seed(5)
+    cache = torch.empty((nb, w0.H, w0.N, w0.D), dtype=torch.bfloat16, device=DEV)
+    workloads.fill_normal_(cache, 1.0, torch.Generator(device=DEV).manual_seed(5), DEV)
+    weight = workloads.normal((w0.C, w0.W), 0.5, torch.bfloat16, g, "cpu").to(DEV)
+    sets = []
+    for wl in wls:
+        md = wl.metadata(DEV)
+        md["x"] = workloads.normal((wl.T, wl.C), 1.0, torch.bfloat16, g, "cpu").to(DEV)
+        md["out"] = torch.empty_like(md["x"])
+        md["taps"] = torch.empty((wl.T, wl.W - 1), dtype=torch.int64, device=DEV)
+        sets.append(md)
+    # Another step's real table for each step, all entries valid slots here.
+    stale = []
+    for i in range(len(wls)):
+        j = (i + 1) % len(wls)
+        _, _, tj = resolve(wls[j], sets[j], decode_form=True, with_metadata=False)
+        stale.append(tj)
+    assert all(s.shape == stale[0].shape for s in stale)
+    cache0 = cache.clone()
+    ref = [hs().sconv_fused(s["x"], weight, cache, s["positions"], s["block_table"],
+                            s["seq_idx"], s["slot_mapping"], s["query_start"], **wl.kwargs())
+           for wl, s in zip(wls, sets)]
+    torch.cuda.synchronize()
+    ref_cache = cache.clone()
+
+    def steps():
+        for i, (wl, s) in enumerate(zip(wls, sets)):
+            s["taps"].copy_(stale[i])
+            hs().sconv_seq_metadata_taps(None, wl.block_table.shape[0], wl.T, s["positions"],
+                                        s["slot_mapping"], s["block_table"], wl.num_blocks,
+                                        wl.N, wl.W, taps_out=s["taps"])
+            hs().sconv_fused_taps(s["x"], weight, cache, s["slot_mapping"], s["taps"],
+                                  out=s["out"], metadata_ready=False, **wl.kwargs())
+
+    def check():
+        for r, s in zip(ref, sets):
+            assert torch.equal(raw(r), raw(s["out"]))
+        assert torch.equal(raw(cache), raw(ref_cache))
+
+    def reset():
+        cache.copy_(cache0)
+        for s in sets:
+            s["out"].fill_(0)
+
+    main = torch.cuda.Stream()
+    reset()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(main):
+        steps()
+    torch.cuda.synchronize()
+    check()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=main):
+        steps()
+    for _ in range(8):
+        reset()
+        torch.cuda.synchronize()
+        graph.replay()
+        torch.cuda.synchronize()
+        check()
+    del graph
+
+
 def _next_dict(wl, md, taps_out, decode_form=False, si=None, qs=None):
     return dict(query_start_loc=None if decode_form else md["query_start_loc"],
                 num_reqs=wl.block_table.shape[0] if decode_form else wl.R,
