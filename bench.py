@@ -72,7 +72,7 @@ def parse_args():
                                       "spec_decode_bf16", "dense", "dense_prefill_bf16",
                                       "dense_long_prefill_bf16", "dense_decode_bf16",
                                       "decode_chain", "chunked_prefill_f32_w4",
-                                      "chunked_prefill_bf16_w8"],
+                                      "chunked_prefill_bf16_w8", "chunked_prefill_taps"],
                    help="time just this workload's kernels and print its table row")
     p.add_argument("--max-hist", type=int, default=4096,
                    help="longest cached history of the decode requests (smaller only for "
@@ -760,6 +760,53 @@ def _entry(wl, secs, nbytes, peak):
 PREFILL_SHAPES = (("f32_w4", "f32", 4), ("bf16_w8", "bf16", 8))
 
 
+def prefill_shape_workload(tag, dtype, W):
+    """The chunked prefill's requests (seed 1003: 16 requests, cached
+    prefixes U{0..2048}, new tokens U{1..2048}) and channel count in another
+    dtype or tap count."""
+    rng = np.random.default_rng(1003)
+    hist = rng.integers(0, 2049, size=16)
+    new = rng.integers(1, 2049, size=16)
+    return workloads.build(f"chunked_prefill_{tag}", dtype=dtype, H=32, D=128, ws=128,
+                           off_s=0, W=W, N=16, hist=hist, new=new, act="silu",
+                           residual=False, seed=1003, rng=rng)
+
+
+def bench_prefill_taps(device, stream, peak, reps=50):
+    """The chunked prefill (W 4) and its W 8 shape in the resolved-tap form:
+    the step's table built once (sconv_seq_metadata_taps, shared by every
+    layer of a step; timed alone too), then sconv_fused_taps with the table
+    ready, which runs the TMA-pipelined kernel with the table rows in its
+    tiles.  One set each (134 MB of x, larger than L2)."""
+    import hybrid_sconv_b200 as hs
+    table = {}
+    for name, wl in (("chunked_prefill_bf16", workloads.chunked_prefill_bf16()),
+                     ("chunked_prefill_bf16_w8", prefill_shape_workload("bf16_w8", "bf16", 8))):
+        t = wl.tensors(device)
+        out = torch.empty_like(t["x"])
+        taps = torch.empty((wl.T, wl.W - 1), dtype=torch.int64, device=device)
+
+        def build():
+            hs.sconv_seq_metadata_taps(t["query_start_loc"], wl.R, wl.T, t["positions"],
+                                       t["slot_mapping"], t["block_table"], wl.num_blocks,
+                                       wl.N, wl.W, taps_out=taps)
+
+        def conv():
+            hs.sconv_fused_taps(t["x"], t["weight"], t["cache"], t["slot_mapping"], taps,
+                                out=out, metadata_ready=True, **wl.kwargs())
+        with torch.cuda.stream(stream):
+            build()
+        torch.cuda.synchronize()
+        table[f"{name}_fused_taps"] = _entry(wl, _kernel_time([conv], reps, stream),
+                                             algorithmic_bytes_taps(wl), peak)
+        table[f"{name}_seq_metadata_taps"] = {
+            "kernel_us": round(_kernel_time([build], reps, stream) * 1e6, 3),
+            "alg_bytes": algorithmic_bytes_resolve(wl)}
+        del t, out, taps
+        torch.cuda.empty_cache()
+    return table
+
+
 def bench_prefill_shapes(device, stream, peak, reps=50, only=None):
     """The chunked prefill's requests and channel count (T = 16 070, C =
     4096) in fp32 with W = 4 and in bf16 with W = 8: the tiled prefill form
@@ -769,12 +816,7 @@ def bench_prefill_shapes(device, stream, peak, reps=50, only=None):
     for tag, dtype, W in PREFILL_SHAPES:
         if only is not None and tag != only:
             continue
-        rng = np.random.default_rng(1003)
-        hist = rng.integers(0, 2049, size=16)
-        new = rng.integers(1, 2049, size=16)
-        wl = workloads.build(f"chunked_prefill_{tag}", dtype=dtype, H=32, D=128, ws=128,
-                             off_s=0, W=W, N=16, hist=hist, new=new, act="silu",
-                             residual=False, seed=1003, rng=rng)
+        wl = prefill_shape_workload(tag, dtype, W)
         t = wl.tensors(device)
         out = torch.empty_like(t["x"])
 
@@ -1228,6 +1270,7 @@ def per_workload_table(device, stream, peak, sets_obj=None, zero_sets=None):
     table.update(bench_prefill("chunked_prefill_bf16", device, stream, peak))
     table.update(bench_prefill("long_prefill_bf16", device, stream, peak))
     table.update(bench_prefill_shapes(device, stream, peak))
+    table.update(bench_prefill_taps(device, stream, peak))
     table.update(bench_spec_decode(device, stream, peak))
     table.update(bench_ssm_gather(device, stream, peak))
     table.update(bench_dense(device, stream, peak))
@@ -1605,6 +1648,8 @@ def main():
         elif args.only == "decode_chain":
             sets_obj = DecodeSets(args.sets, rank_seed(args.seed, rank), device, args.max_hist)
             row = bench_decode_chain(sets_obj, stream, peak)
+        elif args.only == "chunked_prefill_taps":
+            row = bench_prefill_taps(device, stream, peak, reps=max(3, args.steps))
         elif args.only in ("chunked_prefill_f32_w4", "chunked_prefill_bf16_w8"):
             row = bench_prefill_shapes(device, stream, peak, reps=max(3, args.steps),
                                        only=args.only[len("chunked_prefill_"):])

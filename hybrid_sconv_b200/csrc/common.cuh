@@ -326,6 +326,10 @@ cudaError_t launch_fused_streams(FusedArgs *s, int n, bool bf16_data, bool vec,
 // nothing) when the call does not meet its layout requirements.
 cudaError_t launch_fused_tma(const FusedArgs &a, bool bf16_data, cudaStream_t stream,
                              bool &used);
+// The same kernel in the resolved-tap form (a.taps and a.slot in place of
+// the paged metadata); `used` as for launch_fused_tma.
+cudaError_t launch_fused_tma_taps(const FusedArgs &a, bool bf16_data, cudaStream_t stream,
+                                  bool &used);
 cudaError_t launch_extract(const ExtractArgs &a, bool bf16_data, bool vec, cudaStream_t stream);
 cudaError_t launch_scatter_ssm(const SsmArgs &a, int elem_bytes, bool vec, cudaStream_t stream);
 cudaError_t launch_extract_paged(const PagedExtractArgs &a, bool bf16_data, bool vec,

@@ -820,6 +820,15 @@ cudaError_t launch_fused_taps(FusedArgs *s, int n, bool bf16_data, bool vec, boo
         s[i].slots32 = s[i].num_blocks * s[i].N < (1ll << 31);
         s[i].strip = 1;
     }
+    // Prefill sizes of one stream: the TMA-pipelined kernel, which reads the
+    // tile's table rows with its x rows (the same bits as the token form).
+    const int vec_n = bf16_data ? 8 : 4;
+    if (n == 1 && vec && s[0].T >= 64 &&
+        static_cast<int64_t>(s[0].T) * (s[0].C / vec_n) >= kStripMinWork) {
+        bool used = false;
+        const cudaError_t e = launch_fused_tma_taps(s[0], bf16_data, stream, used);
+        if (used || e != cudaSuccess) return e;
+    }
     if (bf16_data)
         return vec ? launch_taps_v<bf16, 8>(s, n, ready, stream)
                    : launch_taps_v<bf16, 1>(s, n, ready, stream);

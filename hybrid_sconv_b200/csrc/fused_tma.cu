@@ -61,16 +61,21 @@ constexpr int kThreads = 256;      // 8 warps
 constexpr int kTokPerWarp = kBT / (kThreads / 32);  // 4
 constexpr int kMetaBytes = kBT * (8 + 8 + 4 + 4);   // positions, slots, seq_idx, query_start
 
-template <int W>
+// A stage: the x rows, then the tile's metadata -- positions, slots,
+// seq_idx and query_start, or, with TAPS, the slots and the tokens' rows of
+// the resolved tap table (W-1 int64 each).  Every part starts on a 128-byte
+// boundary.
+template <int W, bool TAPS = false>
 struct Layout {
     static constexpr int rows = kBT + W - 1;
     static constexpr int x_bytes = rows * 512;  // multiple of 512: TMA destinations stay 128-B aligned
-    static constexpr int stage = x_bytes + kMetaBytes;
+    static constexpr int meta = TAPS ? kBT * 8 * W : kMetaBytes;
+    static constexpr int stage = x_bytes + meta;
 };
 
-template <int W, int STAGES>
+template <int W, int STAGES, bool TAPS = false>
 constexpr int kStages_smem() {
-    return STAGES * Layout<W>::stage + 2 * STAGES * 8;
+    return STAGES * Layout<W, TAPS>::stage + 2 * STAGES * 8;
 }
 
 // Shared memory for cached weights: room for ncache * W 512-byte lag rows
@@ -85,7 +90,7 @@ template <typename E, int W>
 constexpr bool kCachesWeights = W > (sizeof(E) == 2 ? 4 : 5);
 
 struct TmaMaps {
-    CUtensorMap x, pos, slot, sid, qs;
+    CUtensorMap x, pos, slot, sid, qs, tab;  // tab: the resolved tap table (TAPS)
 };
 
 template <typename E>
@@ -218,6 +223,37 @@ struct LagWeights<float, W> {
     }
 };
 
+// SCONV_EFLAG_* bits of a non-PAD token of the resolved-tap form from its
+// table row (W-1 entries, lag d at row[d-1]) and slot: the bits the token
+// form (sconv_fused_taps) reports for the same token -- the row's failure
+// codes, SCONV_EFLAG_BLOCK for a slot past the cache or an entry that is no
+// valid code, SCONV_EFLAG_QUERY_START for an x row before the call's first,
+// and for a slot out of range SCONV_EFLAG_SLOT with the row's request,
+// query-start and position bits.
+template <int W>
+__device__ __forceinline__ unsigned tab_flags(const int64_t *row, int t, int64_t slot,
+                                              int64_t slots_total) {
+    unsigned f = 0;
+#pragma unroll
+    for (int d = 1; d < W; ++d) {
+        const int64_t e = row[d - 1];
+        if (e >= 0) {
+            if (e >= slots_total) f |= SCONV_EFLAG_BLOCK;
+        } else if (e == SCONV_TAP_X) {
+            if (t - d < 0) f |= SCONV_EFLAG_QUERY_START;
+        } else if (e != SCONV_TAP_ZERO) {
+            const unsigned bits =
+                e <= -256 ? static_cast<unsigned>((~static_cast<uint64_t>(e) + 1) >> 8) & 0x3fu
+                          : 0u;
+            f |= bits ? bits : SCONV_EFLAG_BLOCK;
+        }
+    }
+    if (slot < 0 || slot >= slots_total)
+        f = SCONV_EFLAG_SLOT |
+            (f & (SCONV_EFLAG_REQUEST | SCONV_EFLAG_QUERY_START | SCONV_EFLAG_POSITION));
+    return f;
+}
+
 // The pack lane l works on in channel block cb (clamped to the last pack
 // for lanes past C, which compute but store nothing).
 __device__ __forceinline__ int cb_pack(int cb, int l, int nv) {
@@ -228,11 +264,11 @@ __device__ __forceinline__ int cb_pack(int cb, int l, int nv) {
 // What a warp's lane u (< kTokPerWarp) knows about token u of its group.
 enum : int { kSkip = 0, kFast = 1, kSlow = 2 };
 
-template <typename E, int W, int STAGES, bool SILU, bool RESID>
+template <typename E, int W, int STAGES, bool SILU, bool RESID, bool TAPS = false>
 __global__ void __launch_bounds__(kThreads, STAGES <= 3 ? 3 : 2)
 fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ TmaMaps maps,
                  int ncache) {
-    using L = Layout<W>;
+    using L = Layout<W, TAPS>;
     using P = PackOf<E>;
     constexpr int VEC = 16 / static_cast<int>(sizeof(E));
     constexpr int BC = kBC<E>;
@@ -272,10 +308,15 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
         const int t0 = static_cast<int>(u / ncb) * kBT;
         mbar_expect_tx(&full[s], L::stage);
         copy_2d(st, &maps.x, c0, t0 - (W - 1), &full[s]);
-        copy_1d(st + L::x_bytes, &maps.pos, t0, &full[s]);
-        copy_1d(st + L::x_bytes + kBT * 8, &maps.slot, t0, &full[s]);
-        copy_1d(st + L::x_bytes + kBT * 16, &maps.sid, t0, &full[s]);
-        copy_1d(st + L::x_bytes + kBT * 20, &maps.qs, t0, &full[s]);
+        if constexpr (TAPS) {
+            copy_1d(st + L::x_bytes, &maps.slot, t0, &full[s]);
+            if constexpr (W > 1) copy_1d(st + L::x_bytes + kBT * 8, &maps.tab, t0 * (W - 1), &full[s]);
+        } else {
+            copy_1d(st + L::x_bytes, &maps.pos, t0, &full[s]);
+            copy_1d(st + L::x_bytes + kBT * 8, &maps.slot, t0, &full[s]);
+            copy_1d(st + L::x_bytes + kBT * 16, &maps.sid, t0, &full[s]);
+            copy_1d(st + L::x_bytes + kBT * 20, &maps.qs, t0, &full[s]);
+        }
     };
     if (threadIdx.x == 0)
         for (int k = 0; k < STAGES && k < my; ++k) issue(k);
@@ -331,14 +372,34 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
         const unsigned char *st = smem + s * L::stage;
         const P *xs = reinterpret_cast<const P *>(st) + lane_id;  // row r at xs[r * 32]
         const int64_t *mpos = reinterpret_cast<const int64_t *>(st + L::x_bytes);
-        const int64_t *mslot = mpos + kBT;
+        const int64_t *mslot = TAPS ? mpos : mpos + kBT;
         const int32_t *msid = reinterpret_cast<const int32_t *>(st + L::x_bytes + kBT * 16);
         const int32_t *mqs = msid + kBT;
+        const int64_t *mtab = mslot + kBT;  // TAPS: token i's table row at mtab[i * (W-1)]
 
         // Lanes 0..3 classify the group's tokens and address their inserts.
         int code = kSkip;
         int64_t ins = 0;
-        if (lane_id < kTokPerWarp) {
+        if (TAPS && lane_id < kTokPerWarp) {
+            // Ordinary: every tap an x row of this call; otherwise the
+            // general path (cache taps, zero taps or an index error).
+            const int i = i0 + lane_id;
+            const int t = t0 + i;
+            const int64_t slot = mslot[i];
+            if (t < a.T && slot != -1) {
+                const int64_t *row = mtab + i * (W - 1);
+                bool all_x = true;
+#pragma unroll
+                for (int d = 1; d < W; ++d) all_x = all_x && row[d - 1] == SCONV_TAP_X;
+                const bool bad = tab_flags<W>(row, t, slot, slots_total) != 0;
+                code = (!bad && all_x) ? kFast : kSlow;
+                if (slot >= 0 && slot < slots_total) {
+                    int64_t blk, off;
+                    split_n(a, slot, a.slots32 != 0, blk, off);
+                    ins = blk * a.cs0 + off * a.cs2;
+                }
+            }
+        } else if (!TAPS && lane_id < kTokPerWarp) {
             const int i = i0 + lane_id;
             const int t = t0 + i;
             const int64_t slot = mslot[i];
@@ -406,6 +467,30 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
                 if (code_u == kFast) {
 #pragma unroll
                     for (int d = W - 1; d >= 0; --d) wr.fma(acc, d, rows[uu + W - 1 - d]);
+                } else if constexpr (TAPS) {
+                    // Each tap from its table entry: an x row of the tile, a
+                    // cache slot, or zero; the entries come from shared
+                    // memory, so every cache tap is one dependent trip.
+                    const int64_t *row = mtab + i * (W - 1);
+                    const unsigned bad = tab_flags<W>(row, t, mslot[i], slots_total);
+                    if (bad) {
+                        if (a.err && active) atomicOr(a.err, static_cast<int>(bad));
+                        continue;
+                    }
+#pragma unroll
+                    for (int d = W - 1; d >= 1; --d) {
+                        const int64_t e = row[d - 1];
+                        if (e == SCONV_TAP_X) {
+                            wr.fma(acc, d, rows[uu + W - 1 - d]);
+                        } else if (e >= 0) {
+                            int64_t blk, off;
+                            split_n(a, e, a.slots32 != 0, blk, off);
+                            P ct;
+                            ct.load_nc(cache + blk * a.cs0 + off * a.cs2 + lane);
+                            wr.fma(acc, d, ct);
+                        }
+                    }
+                    wr.fma(acc, 0, rows[uu + W - 1]);
                 } else {
                     // Taps before the request's first row come from the cache
                     // (zero before position 0), or an index is out of range.
@@ -480,9 +565,10 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
     }
 }
 
-bool encode_1d(CUtensorMap *m, CUtensorMapDataType type, const void *base, int64_t n) {
+bool encode_1d(CUtensorMap *m, CUtensorMapDataType type, const void *base, int64_t n,
+               unsigned box_elems = kBT) {
     const cuuint64_t dim[1] = {static_cast<cuuint64_t>(n)};
-    const cuuint32_t box[1] = {kBT};
+    const cuuint32_t box[1] = {box_elems};
     const cuuint32_t elem[1] = {1};
     const cuuint64_t no_strides[1] = {0};  // rank 1 has no strides, but the array must exist
     return encode_fn()(m, type, 1, const_cast<void *>(base), dim, no_strides, box, elem,
@@ -502,11 +588,12 @@ int gcd_int(int64_t x, int64_t y) {
     return static_cast<int>(x);
 }
 
-template <typename E, int W, bool SILU, bool RESID>
+template <typename E, int W, bool SILU, bool RESID, bool TAPS>
 cudaError_t launch_flags(const FusedArgs &a, const TmaMaps &maps, cudaStream_t stream) {
     constexpr int S = kLaunchStages;
-    constexpr int smem = kStages_smem<W, S>() + (kCachesWeights<E, W> ? kWeightCacheBytes : 0);
-    auto kernel = fused_tma_kernel<E, W, S, SILU, RESID>;
+    constexpr int smem =
+        kStages_smem<W, S, TAPS>() + (kCachesWeights<E, W> ? kWeightCacheBytes : 0);
+    auto kernel = fused_tma_kernel<E, W, S, SILU, RESID, TAPS>;
     // Resident blocks per SM and the SM count, once per process and kernel
     // (the grid is a function of the device and of T and C only).
     static std::once_flag once;
@@ -536,27 +623,30 @@ cudaError_t launch_flags(const FusedArgs &a, const TmaMaps &maps, cudaStream_t s
                            ? period
                            : 0;
     return launch_pdl(kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads),
-                      static_cast<size_t>(kStages_smem<W, S>() + ncache * W * 512), stream, a,
-                      maps, ncache);
+                      static_cast<size_t>(kStages_smem<W, S, TAPS>() + ncache * W * 512),
+                      stream, a, maps, ncache);
 }
 
-template <typename E, int W>
+template <typename E, int W, bool TAPS>
 cudaError_t launch_w(const FusedArgs &a, const TmaMaps &maps, cudaStream_t stream) {
     if (a.silu) {
-        return a.resid ? launch_flags<E, W, true, true>(a, maps, stream)
-                       : launch_flags<E, W, true, false>(a, maps, stream);
+        return a.resid ? launch_flags<E, W, true, true, TAPS>(a, maps, stream)
+                       : launch_flags<E, W, true, false, TAPS>(a, maps, stream);
     }
-    return a.resid ? launch_flags<E, W, false, true>(a, maps, stream)
-                   : launch_flags<E, W, false, false>(a, maps, stream);
+    return a.resid ? launch_flags<E, W, false, true, TAPS>(a, maps, stream)
+                   : launch_flags<E, W, false, false, TAPS>(a, maps, stream);
 }
 
-template <typename E>
+// TAPS: the resolved-tap form (a.taps, a.slot; no positions, block table,
+// seq_idx or query_start).
+template <typename E, bool TAPS>
 cudaError_t launch_typed(const FusedArgs &a, cudaStream_t stream, bool &used) {
     constexpr int e = static_cast<int>(sizeof(E));
     auto al16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
     if (a.W < 1 || a.W > 8 || a.C < kBC<E> || encode_fn() == nullptr) return cudaSuccess;
-    if (!al16(a.x) || (a.x_rs * e) % 16 != 0 || !al16(a.positions) || !al16(a.slot) ||
-        !al16(a.seq_idx) || !al16(a.qstart))
+    if (!al16(a.x) || (a.x_rs * e) % 16 != 0 || !al16(a.slot)) return cudaSuccess;
+    if (TAPS ? !al16(a.taps)
+             : (!al16(a.positions) || !al16(a.seq_idx) || !al16(a.qstart)))
         return cudaSuccess;
     TmaMaps maps;
     {
@@ -573,21 +663,28 @@ cudaError_t launch_typed(const FusedArgs &a, cudaStream_t stream, bool &used) {
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaSuccess;
     }
-    if (!encode_1d(&maps.pos, CU_TENSOR_MAP_DATA_TYPE_INT64, a.positions, a.T) ||
-        !encode_1d(&maps.slot, CU_TENSOR_MAP_DATA_TYPE_INT64, a.slot, a.T) ||
-        !encode_1d(&maps.sid, CU_TENSOR_MAP_DATA_TYPE_INT32, a.seq_idx, a.T) ||
-        !encode_1d(&maps.qs, CU_TENSOR_MAP_DATA_TYPE_INT32, a.qstart, a.T))
+    if (TAPS) {
+        if (!encode_1d(&maps.slot, CU_TENSOR_MAP_DATA_TYPE_INT64, a.slot, a.T) ||
+            (a.W > 1 && !encode_1d(&maps.tab, CU_TENSOR_MAP_DATA_TYPE_INT64, a.taps,
+                                   static_cast<int64_t>(a.T) * (a.W - 1),
+                                   static_cast<unsigned>(kBT * (a.W - 1)))))
+            return cudaSuccess;
+    } else if (!encode_1d(&maps.pos, CU_TENSOR_MAP_DATA_TYPE_INT64, a.positions, a.T) ||
+               !encode_1d(&maps.slot, CU_TENSOR_MAP_DATA_TYPE_INT64, a.slot, a.T) ||
+               !encode_1d(&maps.sid, CU_TENSOR_MAP_DATA_TYPE_INT32, a.seq_idx, a.T) ||
+               !encode_1d(&maps.qs, CU_TENSOR_MAP_DATA_TYPE_INT32, a.qstart, a.T)) {
         return cudaSuccess;
+    }
     used = true;
     switch (a.W) {
-        case 1: return launch_w<E, 1>(a, maps, stream);
-        case 2: return launch_w<E, 2>(a, maps, stream);
-        case 3: return launch_w<E, 3>(a, maps, stream);
-        case 4: return launch_w<E, 4>(a, maps, stream);
-        case 5: return launch_w<E, 5>(a, maps, stream);
-        case 6: return launch_w<E, 6>(a, maps, stream);
-        case 7: return launch_w<E, 7>(a, maps, stream);
-        default: return launch_w<E, 8>(a, maps, stream);
+        case 1: return launch_w<E, 1, TAPS>(a, maps, stream);
+        case 2: return launch_w<E, 2, TAPS>(a, maps, stream);
+        case 3: return launch_w<E, 3, TAPS>(a, maps, stream);
+        case 4: return launch_w<E, 4, TAPS>(a, maps, stream);
+        case 5: return launch_w<E, 5, TAPS>(a, maps, stream);
+        case 6: return launch_w<E, 6, TAPS>(a, maps, stream);
+        case 7: return launch_w<E, 7, TAPS>(a, maps, stream);
+        default: return launch_w<E, 8, TAPS>(a, maps, stream);
     }
 }
 
@@ -596,7 +693,15 @@ cudaError_t launch_typed(const FusedArgs &a, cudaStream_t stream, bool &used) {
 cudaError_t launch_fused_tma(const FusedArgs &a, bool bf16_data, cudaStream_t stream,
                              bool &used) {
     used = false;
-    return bf16_data ? launch_typed<bf16>(a, stream, used) : launch_typed<float>(a, stream, used);
+    return bf16_data ? launch_typed<bf16, false>(a, stream, used)
+                     : launch_typed<float, false>(a, stream, used);
+}
+
+cudaError_t launch_fused_tma_taps(const FusedArgs &a, bool bf16_data, cudaStream_t stream,
+                                  bool &used) {
+    used = false;
+    return bf16_data ? launch_typed<bf16, true>(a, stream, used)
+                     : launch_typed<float, true>(a, stream, used);
 }
 
 }  // namespace sconv

@@ -519,8 +519,14 @@ sconv_status sconv_seq_metadata_taps_ahead(
  *                    an entry that is neither a slot below num_blocks * N,
  *                    SCONV_TAP_X on a row of this call, SCONV_TAP_ZERO nor a
  *                    failure code sets SCONV_EFLAG_BLOCK.
- * The form is built for decode-size steps (one thread per 16-byte channel
- * pack of a token); prefill-size steps are served by sconv_fused.
+ * Decode-size steps run one thread per 16-byte channel pack of a token.
+ * Prefill-size steps of one stream (16-byte aligned x and slot_mapping
+ * and taps rows, T >= 64 and T * C / (16 / element size) >= 2^19) run the
+ * TMA-pipelined kernel of sconv_fused, whose tiles carry the tokens' table
+ * rows instead of their paged metadata; every read then follows the wait
+ * (metadata_ready changes nothing there), the outputs, inserts and index
+ * bits are the same, and err_flag may also get SCONV_EFLAG_TIMEOUT (a
+ * tile's copies did not arrive within the bounded wait).
  * T == 0 returns SCONV_OK and enqueues nothing.
  */
 sconv_status sconv_fused_taps(

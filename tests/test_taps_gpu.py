@@ -133,15 +133,84 @@ def test_fused_taps_every_window_length(W, dtype):
 
 
 @pytest.mark.parametrize("name,decode_form", [("decode_bf16", False), ("decode_bf16", True),
-                                              ("spec_decode_bf16", False)])
+                                              ("spec_decode_bf16", False),
+                                              ("chunked_prefill_bf16", False)])
 def test_fused_taps_full_size(name, decode_form):
-    """The decode and speculative-decode workloads at full size (caches of
-    4.2 / 2.1 GB, element offsets past 2^31): every token against the
+    """The decode, speculative-decode and chunked-prefill workloads at full
+    size (decode caches of 4.2 / 2.1 GB, element offsets past 2^31; the
+    prefill through the TMA-pipelined form): sampled tokens against the
     oracle, inserts element by element, the whole cache by the holds-x
     invariant, PAD rows untouched."""
     wl = workloads.NAMED[name]()
     check_full_size(wl, DEV, run=lambda wl_, t_, out, err: run_taps(
         wl_, t_, out=out, err=err, decode_form=decode_form))
+
+
+def _tiled_case(W, dtype, seed, num_pad=9, residual=True):
+    """A step large enough for the TMA-pipelined form (T x C/VEC >= 2^19):
+    six requests, some with long cached prefixes, some with none, and PAD
+    rows; C = 4096."""
+    rng = np.random.default_rng(seed)
+    T_min = 1100 if dtype == "bf16" else 600
+    new = rng.integers(T_min // 5, T_min // 3, size=6)  # T >= 1.2 T_min
+    hist = np.array([0, 3, 700, 1, 0, 2000])
+    return workloads.build(f"tiled_taps_w{W}_{dtype}", dtype=dtype, H=32, D=128, ws=128,
+                           off_s=0, W=W, N=16, hist=hist, new=new, act="silu",
+                           residual=residual, seed=seed, num_pad=num_pad, rng=rng)
+
+
+@pytest.mark.parametrize("W", range(1, 9))
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_fused_taps_tiled_every_window_length(W, dtype):
+    """At prefill sizes the resolved-tap form runs the TMA-pipelined kernel
+    (the table rows travel with the tile): every output row and cache byte
+    against the oracle, PAD rows untouched, and every byte equal to
+    sconv_fused's on the same step."""
+    wl = _tiled_case(W, dtype, 900 + 10 * W + (dtype == "f32"), residual=W % 2 == 0)
+    assert wl.T * wl.C // (8 if dtype == "bf16" else 4) >= 1 << 19
+    t = wl.tensors(DEV)
+    cache0 = t["cache"].clone()
+    ref_out = workloads.sentinel((wl.T, wl.C), wl.dtype, DEV)
+    run_fused(wl, t, out=ref_out)
+    ref_cache = t["cache"].clone()
+    t["cache"].copy_(cache0)
+    out = check_small(wl, DEV, t=t, run=lambda wl_, t_, out: run_taps(wl_, t_, out=out))
+    assert torch.equal(raw(out), raw(ref_out))
+    assert torch.equal(raw(t["cache"]), raw(ref_cache))
+
+
+def test_fused_taps_tiled_foreign_entries_are_checked():
+    """The TMA-pipelined resolved-tap form checks a table not made by the
+    resolver as the token form does: the tokens with an entry past the
+    cache, a bad code or an x row before the call are skipped with
+    SCONV_EFLAG_BLOCK / SCONV_EFLAG_QUERY_START, a token carrying the
+    resolver's failure code reports its bits, and nothing else changes."""
+    wl = _tiled_case(4, "bf16", 950, num_pad=0)
+    t = wl.tensors(DEV)
+    _, _, taps = resolve(wl, t)
+    torch.cuda.synchronize()
+    good = taps.clone()
+    taps[5, 0] = wl.num_blocks * wl.N          # slot past the cache
+    taps[37, 1] = -7                           # not a code
+    taps[0, 2] = hs().TAP_X                    # x row -3 of this call
+    taps[600, :] = -(0x04 * 256)               # the resolver's LOGICAL failure
+    out = workloads.sentinel((wl.T, wl.C), wl.dtype, DEV)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    cache0 = t["cache"].clone()
+    hs().sconv_fused_taps(t["x"], t["weight"], t["cache"], t["slot_mapping"], taps, out=out,
+                          err_flag=err, **wl.kwargs())
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0x04 | 0x08 | 0x10
+    bad_rows = [0, 5, 37, 600]
+    assert bool((raw(out)[bad_rows] == -1).all())
+    ref = workloads.sentinel((wl.T, wl.C), wl.dtype, DEV)
+    c2 = cache0.clone()
+    hs().sconv_fused_taps(t["x"], t["weight"], c2, t["slot_mapping"], good, out=ref,
+                          **wl.kwargs())
+    torch.cuda.synchronize()
+    keep = torch.ones(wl.T, dtype=torch.bool)
+    keep[bad_rows] = False
+    assert torch.equal(raw(out)[keep.to(DEV)], raw(ref)[keep.to(DEV)])
 
 
 def test_fused_taps_equals_update_on_decode_form():
