@@ -34,10 +34,14 @@
 // taps / out of range) and compute their cache insert offsets once; when all
 // four are ordinary -- nearly always in prefill -- one straight-line block
 // convolves them from the W+3 shared-memory rows they need (16-byte loads,
-// conflict-free: a warp reads one contiguous 512-byte row).  Otherwise each
-// token takes the general path, where taps that precede the token's request
-// come from the cache through the block table.  Outputs and cache inserts
-// are 16-byte stores straight to global memory.
+// conflict-free: a warp reads one contiguous 512-byte row).  When the
+// other tokens of a warp are the opening tokens of one request, the
+// request's last W-1 cached rows replace the x rows before it in the
+// warp's register window, in one round of loads, and the same block
+// convolves them.  Otherwise each token takes the general path, where taps
+// that precede the token's request come from the cache through the block
+// table, one after another.  Outputs and cache inserts are 16-byte stores
+// straight to global memory.
 //
 // Every wait on an mbarrier is bounded; a block whose copies do not arrive
 // in time sets SCONV_EFLAG_TIMEOUT, waits (bounded) for its other copies and
@@ -454,8 +458,61 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
                 }
             }
         } else {
+            // Staged route: when the group's slow tokens all open one
+            // request (first row q0g, its first position p0g >= W-1, the
+            // positions consecutive, every index valid), their cache taps
+            // are the request's last W-1 cached rows.  Those rows replace,
+            // in the register window, the x rows before q0g -- once the
+            // group's tokens of the previous request are done with them --
+            // in one round of loads, and the request's tokens then take the
+            // straight-line path.  Otherwise every token takes the general
+            // path below.
+            bool staged = false;
+            int split = 0, q0g = 0, reqg = 0;
+            int64_t p0g = 0;
+            if constexpr (!TAPS) {
+                bool ok = true, any = false;
+#pragma unroll
+                for (int uu = 0; uu < kTokPerWarp; ++uu) {
+                    if (__shfl_sync(0xffffffffu, code, uu) != kSlow) continue;
+                    const int i = i0 + uu;
+                    const int t = t0 + i;
+                    const int64_t slot = mslot[i];
+                    const int64_t pos = mpos[i];
+                    const int req = msid[i];
+                    const int q0 = mqs[i];
+                    if (slot < 0 || slot >= slots_total || req < 0 || req >= a.num_reqs ||
+                        q0 < 0 || q0 > t || pos < 0)
+                        ok = false;
+                    if (!any) {
+                        any = true;
+                        q0g = q0;
+                        reqg = req;
+                        p0g = pos - (t - q0);
+                    } else if (q0 != q0g || req != reqg || pos - (t - q0) != p0g) {
+                        ok = false;
+                    }
+                }
+                if (ok && any && p0g >= W - 1) {
+                    bool fine = true;
+#pragma unroll
+                    for (int m = 1; m < W; ++m) {
+                        int64_t lb, off;
+                        split_n(a, p0g - m, p0g - m < (1ll << 31), lb, off);
+                        if (lb >= a.max_blocks) {
+                            fine = false;
+                        } else {
+                            const int32_t b = __ldg(a.bt + static_cast<int64_t>(reqg) * a.bt_rs + lb);
+                            fine = fine && b >= 0 && b < a.num_blocks;
+                        }
+                    }
+                    staged = fine;
+                    split = q0g - (t0 + i0) > 0 ? q0g - (t0 + i0) : 0;
+                }
+            }
 #pragma unroll
             for (int uu = 0; uu < kTokPerWarp; ++uu) {
+                if (staged && uu >= split) continue;  // taken below
                 const int code_u = __shfl_sync(0xffffffffu, code, uu);
                 const int64_t ins_u = __shfl_sync(0xffffffffu, ins, uu);
                 if (code_u == kSkip) continue;  // PAD row or past T
@@ -538,6 +595,49 @@ fused_tma_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ Tm
                 if (active) {
                     o.store(out + static_cast<int64_t>(t) * a.out_rs + c);
                     rows[uu + W - 1].store(cache + ins_u + lane);
+                }
+            }
+            if (staged) {
+                // Window row k holds x row t0 - (W-1) + i0 + k; the rows
+                // q0g - m (m = 1..W-1) become the cache rows of positions
+                // p0g - m (their block-table entries checked above).
+                const int ur = q0g - (t0 + i0);
+#pragma unroll
+                for (int k = 0; k < kTokPerWarp + W - 1; ++k) {
+                    const int m = ur + W - 1 - k;
+                    if (k >= split && m >= 1 && m <= W - 1) {
+                        int64_t lb, off;
+                        split_n(a, p0g - m, p0g - m < (1ll << 31), lb, off);
+                        const int32_t b = __ldg(a.bt + static_cast<int64_t>(reqg) * a.bt_rs + lb);
+                        rows[k].load_nc(cache + static_cast<int64_t>(b) * a.cs0 + off * a.cs2 + lane);
+                    }
+                }
+#pragma unroll
+                for (int uu = 0; uu < kTokPerWarp; ++uu) {
+                    if (uu < split) continue;
+                    const int code_u = __shfl_sync(0xffffffffu, code, uu);
+                    const int64_t ins_u = __shfl_sync(0xffffffffu, ins, uu);
+                    if (code_u == kSkip) continue;
+                    float acc[VEC];
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
+#pragma unroll
+                    for (int d = W - 1; d >= 0; --d) wr.fma(acc, d, rows[uu + W - 1 - d]);
+                    float xc[VEC];
+                    rows[uu + W - 1].to_float(xc);
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) {
+                        float y = acc[v];
+                        if (SILU) y = silu<E>(y);
+                        if (RESID) y = __fadd_rn(y, xc[v]);  // never contracted into an FMA
+                        acc[v] = y;
+                    }
+                    P o;
+                    o.from_float(acc);
+                    if (active) {
+                        o.store(out + static_cast<int64_t>(t0 + i0 + uu) * a.out_rs + c);
+                        rows[uu + W - 1].store(cache + ins_u + lane);
+                    }
                 }
             }
         }
