@@ -431,8 +431,10 @@ __device__ __forceinline__ void build_next(const TapResolveArgs &nx, int gx) {
     resolve_block<DECODE_NEXT, MAXW>(nx, (blockIdx.x - gx) * nthr + tid, tid, nthr, s_qsl);
 }
 
+constexpr int kNextThreads = 512;  // block size of the one-stream step at decode sizes
+
 template <typename E, int VEC, int MAXW, bool DECODE_NEXT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kNextThreads)
 fused_taps_next_kernel(const __grid_constant__ FusedArgs a, const __grid_constant__ TapResolveArgs nx,
                        int gx) {
     if (static_cast<int>(blockIdx.x) >= gx) {
@@ -745,11 +747,13 @@ cudaError_t launch_taps_next_t(FusedArgs *s, int n, TapResolveArgs &nx, cudaStre
     m.n = n;
     int nv_max = 0;
     for (int i = 0; i < n; ++i) nv_max = s[i].C / VEC > nv_max ? s[i].C / VEC : nv_max;
-    // Full-size blocks (kThreads) even for few rows: measured on the decode
-    // step (256 tokens x 128 packs), 128 blocks of 256 threads 2.79 us per
-    // launch against 256 blocks of 128 threads 2.90.
+    // Large blocks even for few rows: measured on the decode step (256
+    // tokens x 128 packs, us per launch), 256 blocks of 128 threads 2.90,
+    // 128 of 256 2.79, 64 of 512 (one stream) 2.785 against 2.827 in
+    // another session.  Several streams keep kThreads.
     Shape sh = block_shape(nv_max, s[0].T);
-    if (sh.cv * sh.tg < kThreads) sh.tg = kThreads / sh.cv;
+    const int want = n == 1 ? kNextThreads : kThreads;
+    if (sh.cv * sh.tg < want) sh.tg = want / sh.cv;
     m.y0[0] = 0;
     for (int i = 0; i < n; ++i) {
         s[i].w_vec = s[i].w_vec && s[i].W == MAXW;
