@@ -548,11 +548,11 @@ class StepEvents:
 
 
 def timed_steps_graph(sets_obj, K, stream, lead=LEAD_STEPS):
-    """One graph of `lead` untimed one-launch steps (the sets before set 0
-    in the rotation), then exactly K timed steps (sets 0, 1, ... mod M)
-    between the StepEvents marks.  carry_prologue(sets_obj, stream, idx)
-    with the returned idx builds the first lead step's table before each
-    replay."""
+    """For the one-launch schedule ("next"): one graph of `lead` untimed
+    steps (the sets before set 0 in the rotation), then exactly K timed
+    steps (sets 0, 1, ... mod M) between the StepEvents marks.
+    carry_prologue(sets_obj, stream, idx) with the returned idx builds the
+    first lead step's table before each replay."""
     M = len(sets_obj.sets)
     lead_idx = [(M - lead + i) % M for i in range(lead)]
     timed_idx = [i % M for i in range(K)]
@@ -1569,7 +1569,7 @@ def config_block(world, l2, K=None):
         block["timing"] = (f"one graph replay: {LEAD_STEPS} untimed steps, then the K timed "
                            "steps; CUDA events recorded by graph nodes when the last untimed "
                            "step and the last timed step complete (device time)"
-                           if K <= EVENT_GRAPH_MAX_STEPS else
+                           if K <= EVENT_GRAPH_MAX_STEPS and STEP_SCHEDULE == "next" else
                            "graphs of one rotation of steps replayed between CUDA events on "
                            "the launching stream (device time)")
     return block
@@ -1678,7 +1678,7 @@ def main():
     torch.cuda.synchronize()
     del wfull, wtail
     sampler = ClockSampler(local) if rank == 0 else None
-    if K <= EVENT_GRAPH_MAX_STEPS:
+    if K <= EVENT_GRAPH_MAX_STEPS and STEP_SCHEDULE == "next":
         graph, marks, first = timed_steps_graph(sets_obj, K, stream)
         carry_prologue(sets_obj, stream, first)
         prime(graph, None, stream)
