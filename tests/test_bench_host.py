@@ -76,6 +76,22 @@ def test_l2_statement_for_fewer_steps_than_sets():
     assert "flushed" in s and "none repeats" in s and "60 MB" in s
 
 
+def test_l2_statement_names_the_untimed_lead_steps():
+    """Short runs time K steps after LEAD_STEPS untimed ones in the same
+    graph; the statement says those read other sets."""
+    s = bench.l2_statement(_Sets([3_000_000] * 96), 20)
+    assert f"the {bench.LEAD_STEPS} untimed steps ahead of them read other sets" in s
+    assert "untimed" not in bench.l2_statement(_Sets([3_000_000] * 96), 95)
+
+
+def test_config_timing_says_which_form_ran():
+    short = bench.config_block(1, "l2", 20)["timing"]
+    assert "untimed steps" in short and "graph nodes" in short
+    long = bench.config_block(1, "l2", bench.EVENT_GRAPH_MAX_STEPS + 1)["timing"]
+    assert "rotation" in long
+    assert "timing" not in bench.config_block(1, "l2")
+
+
 def test_l2_statement_for_rotations():
     big = bench.l2_statement(_Sets([3_000_000] * 96), 500)
     assert "288 MB > 126 MB L2" in big
