@@ -748,6 +748,8 @@ cudaError_t launch_typed(const FusedArgs &a, cudaStream_t stream, bool &used) {
     if (TAPS ? !al16(a.taps)
              : (!al16(a.positions) || !al16(a.seq_idx) || !al16(a.qstart)))
         return cudaSuccess;
+    // The table's tile coordinate t0 * (W-1) is a 32-bit copy coordinate.
+    if (TAPS && static_cast<int64_t>(a.T) * (a.W - 1) >= (1ll << 31)) return cudaSuccess;
     TmaMaps maps;
     {
         const cuuint64_t dim[2] = {static_cast<cuuint64_t>(a.C), static_cast<cuuint64_t>(a.T)};
