@@ -983,6 +983,8 @@ bool encode_tile_map(const DenseArgs &a, int pp, CUtensorMap &map) {
     constexpr int64_t e = sizeof(E);
     if (tma::encode_fn() == nullptr) return false;
     const int tt = kTileThreads / pp * kRowsPerThread;
+    // Tile row coordinates (up to T + TT) are 32-bit copy coordinates.
+    if (static_cast<int64_t>(a.T) + tt >= (1ll << 31)) return false;
     const cuuint64_t dim[2] = {static_cast<cuuint64_t>(a.dim),
                                static_cast<cuuint64_t>(a.T > 1 ? a.T : 1)};
     // With one row the stride is never used; any legal value will do.
